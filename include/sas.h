@@ -1,0 +1,166 @@
+/*
+ * sas.h -- C ABI of libsas: SAS gated block-sparse causal attention on B200.
+ *
+ * SAS ("Simple Attention Sparsification via End-to-End Optimization of Context
+ * Ranking", arXiv 2609.13141) splits the context into contiguous blocks of
+ * `block_size` tokens. For a query at position p, the block holding p is the
+ * always-retained current block and the C = floor(p / block_size) blocks
+ * before it are the historical candidates. A selector gives one score per
+ * historical block; the gate is the softmax of those scores
+ * (log g_i = s_i - log sum_j exp s_j) and the current block keeps g_0 = 1.
+ * A hard top-K keeps K historical blocks, and log g of each kept block is added
+ * to every logit q.k/sqrt(d) of its tokens inside the attention softmax:
+ *   o = softmax(q K_S^T / sqrt(d) + log g_S) V_S.
+ * Sources: dimensionstp.github.io SAS study note, 1-1 (block-sparse attention
+ * eq.), 1-2 (TopK eq.), 2-1 (gate eq.), 2-2 (gated attention eq. and the
+ * multiplicative identity), 3-1 (per-query-group selection), 3-7 (decode path);
+ * papers.paperslantern.ai arXiv text, 3 (preliminaries: blocks, selected
+ * token set), 4 (gate position, normalised gate, training scope, ablation
+ * discussion).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Notation: B batch, T query rows per (b, head), Hq query heads, Hkv KV
+ *    heads, G = Hq / Hkv query heads per KV group, d head_dim, b block_size,
+ *    K top_k, NB = ceil((q_offset + T) / b), p = q_offset + t, C = floor(p / b).
+ *  - One block selection per (batch, KV head, query row), shared by the G
+ *    query heads of the group; query head h belongs to KV head h / G.
+ *  - K counts historical blocks only: a row attends to at most (K + 1) * b
+ *    tokens (K kept blocks plus the causal part of the current block).
+ *  - Ties between equal scores go to the lower block index; -0.0 ties +0.0;
+ *    -inf is a valid score (gate 0, ranked last). NaN and +inf scores are
+ *    outside the contract. The kept indices are stored in ascending order.
+ *  - All tensors are dense, row-major, in the layouts given per argument, and
+ *    live in DEVICE memory unless stated. Every pointer must be 16-byte
+ *    aligned. The caller owns and allocates every buffer, including the
+ *    workspace; libsas allocates and frees nothing and keeps no state.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *    default stream) and does not synchronise the host.
+ *  - Errors: argument, shape, alignment and workspace checks run first and
+ *    return a status without launching anything and without touching any
+ *    buffer. A failed launch returns SAS_ERR_CUDA (from cudaGetLastError).
+ *    Faults inside a running kernel are reported by the CUDA runtime on a
+ *    later synchronisation, not by these calls.
+ *  - Supported: d in {64, 128}; b in {32, 64}; Hq % Hkv == 0; G <= 8;
+ *    1 <= K <= 64. Training calls (fwd/bwd) need q_offset == 0 and T % b == 0.
+ *    dtype BF16 or FP32 for q/k/v/o/dO/dq/dk/dv; scores and all statistics are
+ *    always float32.
+ */
+#ifndef SAS_H_
+#define SAS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SAS_OK = 0,
+    SAS_ERR_INVALID_ARG = 1,   /* null pointer, bad shape, inconsistent sizes */
+    SAS_ERR_UNSUPPORTED = 2,   /* valid but outside the supported ranges above */
+    SAS_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned */
+    SAS_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required */
+    SAS_ERR_CUDA = 5           /* a CUDA launch or runtime call failed */
+} sas_status;
+
+typedef enum { SAS_DT_BF16 = 0, SAS_DT_FP32 = 1 } sas_dtype;
+
+/* SOFTMAX: log g_i = s_i - log sum_{j<C} exp s_j (the method's normalised gate).
+ * NONE: every log-gate is 0 and the score gradient is 0 (plain block-sparse). */
+typedef enum { SAS_GATE_SOFTMAX = 0, SAS_GATE_NONE = 1 } sas_gate;
+
+typedef enum { SAS_OP_TOPK = 0, SAS_OP_FWD = 1, SAS_OP_BWD = 2, SAS_OP_DECODE = 3 } sas_op;
+
+typedef struct {
+    int32_t batch;         /* B */
+    int32_t seq_len;       /* T (training); 1 for decode */
+    int32_t q_offset;      /* position of row 0: 0 for training, N - 1 for decode */
+    int32_t n_q_heads;     /* Hq */
+    int32_t n_kv_heads;    /* Hkv */
+    int32_t head_dim;      /* d */
+    int32_t block_size;    /* b */
+    int32_t top_k;         /* K, historical blocks kept per row */
+    float softmax_scale;   /* scale on q.k; <= 0 selects 1/sqrt(d). The log-gate is added unscaled. */
+    int32_t dtype;         /* sas_dtype of q/k/v/o/dO/dq/dk/dv */
+    int32_t gate;          /* sas_gate */
+} sas_desc;
+
+/* Bytes of device workspace `op` needs for this shape (0 if none). The caller
+ * allocates it and passes it to the call; its contents need not be
+ * initialised and are not meaningful afterwards. */
+sas_status sas_workspace_size(int32_t op, const sas_desc* desc, size_t* bytes);
+
+/* Gate normaliser and hard top-K (study note 1-2 TopK eq., 2-1 gate eq.;
+ * arXiv text 4, normalised gate).
+ *   scores     [B, Hkv, T, NB] float32, in: block scores; row t reads [0, C).
+ *   idx        [B, Hkv, T, K] int32, out: kept blocks ascending, -1 padded.
+ *   gate_logit [B, Hkv, T, K] float32, out: log g of each kept block
+ *              (s_i - score_lse under SOFTMAX, 0 under NONE), 0 in padding.
+ *   score_lse  [B, Hkv, T] float32, out: log sum_{i<C} exp s_i (-inf if C = 0).
+ *   n_sel      [B, Hkv, T] int32, out: min(K, C).
+ * Any q_offset >= 0 is allowed (decode rows use T = 1, q_offset = N - 1). */
+sas_status sas_block_topk(const sas_desc* desc, const float* scores, int32_t* idx,
+                          float* gate_logit, float* score_lse, int32_t* n_sel, void* stream);
+
+/* Gated block-sparse causal attention forward (study note 2-2 gated attention
+ * eq.; arXiv text 4, inner log-space gate, sparse training scope).
+ *   q [B, Hq, T, d], k and v [B, Hkv, T, d] (dtype), in.
+ *   idx, gate_logit, n_sel: as written by sas_block_topk for this desc, in.
+ *   o [B, Hq, T, d] (dtype), out; attn_lse [B, Hq, T] float32, out: the
+ *   natural-log log-sum-exp of each row's gated logits (kept for backward).
+ *   ws: device workspace of at least sas_workspace_size(SAS_OP_FWD) bytes. */
+sas_status sas_gated_attn_fwd(const sas_desc* desc, const void* q, const void* k, const void* v,
+                              const int32_t* idx, const float* gate_logit, const int32_t* n_sel,
+                              void* o, float* attn_lse, void* ws, size_t ws_bytes, void* stream);
+
+/* Backward of sas_gated_attn_fwd, including the score gradient through the
+ * gate (study note 2-2, 3-6 "keeps the selector gradient"; arXiv text 4,
+ * gradient of the normalised gate: d log g_i / d s_k = [i = k] - g_k).
+ *   q, k, v, o, attn_lse: the forward's inputs and outputs, in.
+ *   dO [B, Hq, T, d] (dtype), in: upstream gradient of o.
+ *   scores, score_lse, idx, gate_logit, n_sel: the top-K inputs/outputs, in.
+ *   dq [B, Hq, T, d], dk and dv [B, Hkv, T, d] (dtype), out (overwritten).
+ *   dscores [B, Hkv, T, NB] float32, out (overwritten): dL/ds; 0 for i >= C
+ *   and everywhere under SAS_GATE_NONE. For i < C:
+ *   dscores_i = [i kept] * Gsum_i - g_i * sum_{k kept} Gsum_k, where Gsum_i is
+ *   the sum of dL/dlogit over the block's tokens and the group's G heads.
+ *   ws: at least sas_workspace_size(SAS_OP_BWD) bytes. */
+sas_status sas_gated_attn_bwd(const sas_desc* desc, const void* q, const void* k, const void* v,
+                              const void* o, const void* dO, const float* attn_lse,
+                              const float* scores, const float* score_lse, const int32_t* idx,
+                              const float* gate_logit, const int32_t* n_sel, void* dq, void* dk,
+                              void* dv, float* dscores, void* ws, size_t ws_bytes, void* stream);
+
+/* Budgeted sparse decode of one new token per (batch, query head) over a KV
+ * cache (study note 3-7 inference path, steps 2-4; 5-6 efficiency).
+ * desc: seq_len = 1, q_offset = N - 1 where N is the cache length including
+ * the new token; the current block is floor((N - 1) / b) and is causal.
+ *   q [B, Hq, d] (dtype), in.
+ *   k_cache, v_cache [B, Hkv, cache_stride_tokens, d] (dtype), in; tokens
+ *   [0, N) are valid; cache_stride_tokens >= N.
+ *   idx, gate_logit, n_sel [B, Hkv, 1, K] / [B, Hkv, 1]: from sas_block_topk
+ *   with the same desc; idx == NULL selects dense decode over every token
+ *   [0, N) with no gate (gate_logit and n_sel are then ignored).
+ *   o [B, Hq, d] (dtype), out.
+ *   ws: at least sas_workspace_size(SAS_OP_DECODE) bytes. */
+sas_status sas_sparse_decode(const sas_desc* desc, const void* q, const void* k_cache,
+                             const void* v_cache, int64_t cache_stride_tokens, const int32_t* idx,
+                             const float* gate_logit, const int32_t* n_sel, void* o, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/* Diagnostics (no counterpart on the pages): number of device-side waits for
+ * an asynchronous copy that gave up after their ~1 s bound since the library
+ * was loaded; 0 in normal operation. A kernel whose wait gave up leaves NaN in
+ * its output instead of hanging. Synchronises the current device. */
+sas_status sas_device_timeouts(uint32_t* count);
+
+/* Static, NUL-terminated description of a status code (never NULL). */
+const char* sas_status_string(sas_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAS_H_ */

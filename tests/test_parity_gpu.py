@@ -1,0 +1,339 @@
+"""GPU parity: every CUDA output against the oracle, on the same seeded inputs.
+
+Tolerances (stated by the method's accuracy targets): top-K indices and counts
+bit-exact; gate logits and normalisers within fp32 rounding; fp32 paths within
+1e-4 absolute; bf16 outputs within 1e-2 absolute; bf16 gradients within 2e-2
+normwise relative (max |diff| / max |ref| per tensor).
+
+Small workloads are compared element by element everywhere; the full-size
+workloads in the benchmark's launch configuration are compared on sampled
+rows, key blocks and KV groups that the oracle computes one by one.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tests import gpu_util as U
+from trainable_block_sparse_topk_b200 import api, binding as B, synth
+
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+TOL_FP32 = 1e-4
+TOL_BF16_O = 1e-2
+TOL_BF16_GRAD = 2e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    from trainable_block_sparse_topk_b200.build import build
+    build()
+    oracle.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    yield
+    assert B.sas_device_timeouts() == 0
+
+
+def check_topk_rows(w, x, out, rows_by_group, top_k=None, q_offset=0, T=None):
+    K = w.top_k if top_k is None else top_k
+    T = w.seq if T is None else T
+    for (b, g), ts in rows_by_group.items():
+        d = oracle.Desc(batch=1, seq_len=T, n_q_heads=w.group, n_kv_heads=1, head_dim=w.head_dim,
+                        block_size=w.block_size, top_k=K, q_offset=q_offset)
+        s = x[b:b + 1, g:g + 1].numpy()
+        idx, gl, lse, nsel = oracle.topk(d, s, ts)
+        gi = out["idx"][b, g, ts].numpy()
+        np.testing.assert_array_equal(gi, idx)
+        np.testing.assert_array_equal(out["nsel"][b, g, ts].numpy(), nsel)
+        glg = out["gl"][b, g, ts].numpy().astype(np.float64)
+        for r in range(len(ts)):
+            n = nsel[r]
+            np.testing.assert_allclose(glg[r, :n], gl[r, :n], atol=2e-5, rtol=1e-6)
+        sl = out["slse"][b, g, ts].numpy().astype(np.float64)
+        fin = np.isfinite(lse)
+        np.testing.assert_allclose(sl[fin], lse[fin], atol=2e-5, rtol=1e-6)
+        assert np.all(np.isneginf(sl[~fin]))
+
+
+# ------------------------------------------------------------------ top-K ---
+
+def test_topk_golden_ties():
+    with open(os.path.join(GOLDEN, "topk_ties.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        svals = [float(v) for v in c["s"]]
+        C, K, bs = len(svals), c["K"], 32
+        N = C * bs + 1
+        s = torch.zeros(1, 1, 1, -(-N // bs))
+        s[0, 0, 0, :C] = torch.tensor(svals) if C else s[0, 0, 0, :0]
+        d = B.make_desc(batch=1, seq_len=1, q_offset=N - 1, n_q_heads=1, n_kv_heads=1, head_dim=64,
+                        block_size=bs, top_k=K)
+        sel = api.block_topk(d, s.cuda())
+        assert sel.idx[0, 0, 0].cpu().tolist() == c["idx"], c["name"]
+        assert int(sel.n_sel[0, 0, 0]) == min(C, K)
+
+
+@pytest.mark.parametrize("ncand,K", [(31, 4), (127, 15), (500, 31), (2047, 63), (8191, 31), (8191, 64)])
+def test_topk_ties_random(ncand, K):
+    """Rows full of exact ties (small integers, +-0.0, -inf) at every row length
+    the kernel variants cover, against the oracle's brute-force sort."""
+    rng = np.random.default_rng(ncand + K)
+    bs, rows = 64, 8
+    N = ncand * bs + 1
+    NB = -(-N // bs)
+    s = rng.integers(-2, 3, size=(2, rows // 2, 1, NB)).astype(np.float32)
+    s[rng.random(s.shape) < 0.1] = -np.inf
+    s[rng.random(s.shape) < 0.1] = -0.0
+    s[0, 0, 0, :] = 1.0                       # one all-equal row
+    st = torch.from_numpy(s)
+    d = B.make_desc(batch=2, seq_len=1, q_offset=N - 1, n_q_heads=rows // 2, n_kv_heads=rows // 2,
+                    head_dim=64, block_size=bs, top_k=K)
+    sel = api.block_topk(d, st.cuda())
+    out = {"idx": sel.idx.cpu(), "gl": sel.gate_logit.cpu(), "slse": sel.score_lse.cpu(), "nsel": sel.n_sel.cpu()}
+    w = synth.Workload("ties", "decode", 2, N, rows // 2, rows // 2, 64, bs, K, "fp32", 0, 1.0)
+    grp = {(b, g): [0] for b in range(2) for g in range(rows // 2)}
+    check_topk_rows(w, st, out, grp, top_k=K, q_offset=N - 1, T=1)
+
+
+@pytest.mark.parametrize("name", ["tiny", "qwen4b", "qwen14b"])
+def test_topk_train_workloads(name):
+    w = synth.workload(name)
+    x = synth.train_scores(w)
+    d = U.train_desc(w)
+    sel = api.block_topk(d, x.cuda())
+    out = {"idx": sel.idx.cpu(), "gl": sel.gate_logit.cpu(), "slse": sel.score_lse.cpu(), "nsel": sel.n_sel.cpu()}
+    if name == "tiny":
+        grp = {(0, 0): list(range(w.seq))}
+    else:
+        grp = U.by_group(U.sample_rows(w, 3000, seed=11))
+        # plus every row of one whole group
+        grp.setdefault((w.batch - 1, w.n_kv_heads - 1), [])
+        grp[(w.batch - 1, w.n_kv_heads - 1)] = list(range(w.seq))
+    check_topk_rows(w, x, out, {k: sorted(set(v)) for k, v in grp.items()})
+
+
+# ------------------------------------------------------------ tiny (fp32) ---
+
+@pytest.fixture(scope="module")
+def tiny_run():
+    w = synth.workload("tiny")
+    return (w,) + U.run_train(w)
+
+
+def test_tiny_fwd_bwd_fp32_full(tiny_run):
+    """Every output of the fp32 path within 1e-4 of the oracle."""
+    w, x, out = tiny_run
+    d = U.group_desc(w)
+    a = U.group_arrays(x, w, 0, 0)
+    o, lse = oracle.fwd(d, a["q"], a["k"], a["v"], a["s"])
+    G = w.group
+    go = out["o"][0].numpy().transpose(1, 0, 2)          # [T, G, d]
+    np.testing.assert_allclose(go, o, atol=TOL_FP32, rtol=0)
+    np.testing.assert_allclose(out["lse"][0].numpy().T, lse, atol=TOL_FP32, rtol=0)
+    r = oracle.bwd(d, a["q"], a["k"], a["v"], a["s"], a["dO"])
+    np.testing.assert_allclose(out["dq"][0].numpy().transpose(1, 0, 2), r["dq"], atol=TOL_FP32, rtol=0)
+    np.testing.assert_allclose(out["dk"].numpy(), r["dk"], atol=TOL_FP32, rtol=0)
+    np.testing.assert_allclose(out["dv"].numpy(), r["dv"], atol=TOL_FP32, rtol=0)
+    np.testing.assert_allclose(out["ds"][0, 0].numpy(), r["ds"], atol=TOL_FP32, rtol=0)
+    assert G == 2
+
+
+@pytest.mark.parametrize("over", [dict(gate="none"), dict(top_k=16, gate="none"), dict(top_k=1),
+                                  dict(top_k=16)])
+def test_tiny_variants_fp32(over):
+    """Gate off, K >= C (dense), K = 1, and K >= C with the gate, all elementwise."""
+    w = synth.workload("tiny")
+    gate = over.get("gate", "softmax")
+    K = over.get("top_k", w.top_k)
+    x, out = U.run_train(w, gate=gate, top_k=K)
+    d = U.group_desc(w, gate=oracle.GATE_NONE if gate == "none" else oracle.GATE_SOFTMAX, top_k=K)
+    a = U.group_arrays(x, w, 0, 0)
+    o, lse = oracle.fwd(d, a["q"], a["k"], a["v"], a["s"])
+    np.testing.assert_allclose(out["o"][0].numpy().transpose(1, 0, 2), o, atol=TOL_FP32, rtol=0)
+    r = oracle.bwd(d, a["q"], a["k"], a["v"], a["s"], a["dO"])
+    np.testing.assert_allclose(out["dq"][0].numpy().transpose(1, 0, 2), r["dq"], atol=TOL_FP32, rtol=0)
+    np.testing.assert_allclose(out["dk"].numpy(), r["dk"], atol=TOL_FP32, rtol=0)
+    np.testing.assert_allclose(out["dv"].numpy(), r["dv"], atol=TOL_FP32, rtol=0)
+    np.testing.assert_allclose(out["ds"][0, 0].numpy(), r["ds"], atol=TOL_FP32, rtol=0)
+
+
+@pytest.mark.parametrize("shape", [
+    dict(batch=2, seq=256, n_q_heads=8, n_kv_heads=1, head_dim=64, block_size=32, top_k=3, dtype="bf16"),
+    dict(batch=1, seq=384, n_q_heads=5, n_kv_heads=1, head_dim=128, block_size=64, top_k=2, dtype="bf16"),
+    dict(batch=1, seq=320, n_q_heads=3, n_kv_heads=3, head_dim=128, block_size=32, top_k=5, dtype="fp32"),
+    dict(batch=2, seq=192, n_q_heads=4, n_kv_heads=2, head_dim=64, block_size=64, top_k=1, dtype="fp32"),
+])
+def test_small_shapes_elementwise(shape):
+    """Ragged small problems over the supported ranges (G = 1..8, d 64/128,
+    block 32/64, both dtypes), every element against the oracle."""
+    w = synth.Workload("small", "train", shape["batch"], shape["seq"], shape["n_q_heads"], shape["n_kv_heads"],
+                       shape["head_dim"], shape["block_size"], shape["top_k"], shape["dtype"], 99, 0.5,
+                       score_kind="gauss")
+    x, out = U.run_train(w)
+    bf = w.dtype == "bf16"
+    for b in range(w.batch):
+        for g in range(w.n_kv_heads):
+            d = U.group_desc(w)
+            a = U.group_arrays(x, w, b, g)
+            o, _ = oracle.fwd(d, a["q"], a["k"], a["v"], a["s"])
+            G = w.group
+            go = out["o"][b, g * G:(g + 1) * G].float().numpy().transpose(1, 0, 2)
+            np.testing.assert_allclose(go, o, atol=TOL_BF16_O if bf else TOL_FP32, rtol=0)
+            r = oracle.bwd(d, a["q"], a["k"], a["v"], a["s"], a["dO"])
+            gdq = out["dq"][b, g * G:(g + 1) * G].float().numpy().transpose(1, 0, 2)
+            gdk = out["dk"][b:b + 1, g:g + 1].float().numpy()
+            gdv = out["dv"][b:b + 1, g:g + 1].float().numpy()
+            gds = out["ds"][b, g].numpy()
+            if bf:
+                for got, ref in ((gdq, r["dq"]), (gdk, r["dk"]), (gdv, r["dv"]), (gds, r["ds"])):
+                    assert U.normwise(got, ref) <= TOL_BF16_GRAD
+            else:
+                for got, ref in ((gdq, r["dq"]), (gdk, r["dk"]), (gdv, r["dv"]), (gds, r["ds"])):
+                    np.testing.assert_allclose(got, ref, atol=TOL_FP32, rtol=0)
+
+
+# ------------------------------------------------------ full-size bf16 runs ---
+
+@pytest.fixture(scope="module", params=["qwen4b", "qwen14b"])
+def big_run(request):
+    w = synth.workload(request.param)
+    x, out = U.run_train(w)
+    return w, x, out
+
+
+def test_big_rows_fwd_dq_ds(big_run):
+    """Sampled rows: o within 1e-2, dq and the score gradient within 2e-2."""
+    w, x, out = big_run
+    G = w.group
+    rows = U.sample_rows(w, 400 if w.name == "qwen4b" else 150, seed=3)
+    got_o, ref_o, got_dq, ref_dq, got_ds, ref_ds = [], [], [], [], [], []
+    for (b, g), ts in U.by_group(rows).items():
+        ts = np.array(sorted(set(ts)), dtype=np.int64)
+        d = U.group_desc(w)
+        a = U.group_arrays(x, w, b, g)
+        o, _ = oracle.fwd(d, a["q"], a["k"], a["v"], a["s"], ts)
+        r = U.parallel_oracle_bwd(d, a, ts)
+        got_o.append(out["o"][b, g * G:(g + 1) * G][:, ts].float().numpy().transpose(1, 0, 2))
+        ref_o.append(o)
+        got_dq.append(out["dq"][b, g * G:(g + 1) * G][:, ts].float().numpy().transpose(1, 0, 2))
+        ref_dq.append(r["dq"])
+        got_ds.append(out["ds"][b, g][ts].numpy())
+        ref_ds.append(r["ds"])
+    go, ro = np.concatenate(got_o), np.concatenate(ref_o)
+    assert np.abs(go - ro).max() <= TOL_BF16_O
+    assert U.normwise(np.concatenate(got_dq), np.concatenate(ref_dq)) <= TOL_BF16_GRAD
+    assert U.normwise(np.concatenate(got_ds), np.concatenate(ref_ds)) <= TOL_BF16_GRAD
+
+
+def test_big_key_blocks_dk_dv(big_run):
+    """Sampled key blocks: dk, dv of block j from every row that attends it."""
+    w, x, out = big_run
+    nT = w.seq // w.block_size
+    picks = [(0, 0, 1), (w.batch - 1, w.n_kv_heads - 1, nT - 2), (0, w.n_kv_heads // 2, nT // 2)]
+    if w.name == "qwen14b":
+        picks[2] = (w.batch - 1, 1, nT - 40)
+    bs = w.block_size
+    for b, g, j in picks:
+        rows = U.rows_touching_block(w, x, b, g, j, oracle.GATE_SOFTMAX)
+        d = U.group_desc(w)
+        a = U.group_arrays(x, w, b, g)
+        r = U.parallel_oracle_bwd(d, a, rows, chunks=16)
+        ref_dk = r["dk"][0, 0, j * bs:(j + 1) * bs]
+        ref_dv = r["dv"][0, 0, j * bs:(j + 1) * bs]
+        got_dk = out["dk"][b, g, j * bs:(j + 1) * bs].float().numpy()
+        got_dv = out["dv"][b, g, j * bs:(j + 1) * bs].float().numpy()
+        assert U.normwise(got_dk, ref_dk) <= TOL_BF16_GRAD, (b, g, j)
+        assert U.normwise(got_dv, ref_dv) <= TOL_BF16_GRAD, (b, g, j)
+
+
+# ------------------------------------------------------------------ decode ---
+
+def decode_check(w, kc, vc, q, s, N, K, groups, dense=False, gate="softmax"):
+    d = U.decode_desc(w, N, top_k=K, gate=gate)
+    qd = q.to(U.dev_dtype(w)).cuda()
+    sel = None if dense else api.block_topk(d, s.cuda())
+    o = api.sparse_decode(d, qd, kc, vc, sel).float().cpu().numpy()
+    G = w.group
+    worst = 0.0
+    for b, g in groups:
+        od = oracle.Desc(batch=1, seq_len=1, q_offset=N - 1, n_q_heads=G, n_kv_heads=1, head_dim=w.head_dim,
+                         block_size=w.block_size, top_k=K,
+                         gate=oracle.GATE_NONE if gate == "none" else oracle.GATE_SOFTMAX)
+        kk = synth.decode_cache_slice(w, "k", b, g)[:N].numpy()[None, None]
+        vv = synth.decode_cache_slice(w, "v", b, g)[:N].numpy()[None, None]
+        ref = oracle.decode(od, q[b:b + 1, g * G:(g + 1) * G].numpy(), kk, vv,
+                            None if dense else s[b:b + 1, g:g + 1].numpy())
+        worst = max(worst, float(np.abs(o[b, g * G:(g + 1) * G] - ref[0]).max()))
+    assert worst <= TOL_BF16_O, worst
+    return worst
+
+
+@pytest.fixture(scope="module")
+def decode_ws():
+    w = synth.workload("decode")
+    kc, vc = U.build_decode_cache(w)
+    q = synth.decode_q(w)
+    s = synth.decode_scores(w, q)
+    yield w, kc, vc, q, s
+    del kc, vc
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("K", [15, 31, 63])
+def test_decode_budgets(decode_ws, K):
+    w, kc, vc, q, s = decode_ws
+    groups = [(0, g) for g in range(w.n_kv_heads)]
+    decode_check(w, kc, vc, q, s, w.seq, K, groups)
+
+
+@pytest.mark.parametrize("N", [1, 63, 64, 65, 100000])
+def test_decode_ragged_lengths(decode_ws, N):
+    """Cache lengths that leave a partial (or single-token) current block and
+    rows with fewer candidates than K; the cache stride stays the full length."""
+    w, kc, vc, q, _ = decode_ws
+    NB = -(-N // w.block_size)
+    s = torch.randn(1, w.n_kv_heads, 1, NB, generator=torch.Generator().manual_seed(N))
+    groups = [(0, g) for g in (0, 3, 7)]
+    decode_check(w, kc, vc, q, s, N, 31, groups)
+    decode_check(w, kc, vc, q, s, N, 31, groups, gate="none")
+
+
+def test_decode_dense(decode_ws):
+    w, kc, vc, q, s = decode_ws
+    decode_check(w, kc, vc, q, s, w.seq, 31, [(0, 0), (0, 5)], dense=True)
+
+
+@pytest.mark.parametrize("batch", [1, 8])
+def test_long_decode(batch):
+    """524288-token cache, budget 2048: sparse on sampled groups, dense too."""
+    w = synth.workload("long", batch=batch)
+    kc, vc = U.build_decode_cache(w)
+    q = synth.decode_q(w)
+    s = synth.decode_scores(w, q)
+    groups = [(0, 0), (batch - 1, w.n_kv_heads - 1)] + ([(3, 2)] if batch > 3 else [])
+    decode_check(w, kc, vc, q, s, w.seq, w.top_k, groups)
+    decode_check(w, kc, vc, q, s, w.seq, w.top_k, groups[:1], dense=True)
+    del kc, vc
+    torch.cuda.empty_cache()
+
+
+def test_autograd_function_matches_abi():
+    """The autograd wrapper returns exactly what the direct calls return."""
+    w = synth.workload("tiny")
+    x, out = U.run_train(w)
+    d = U.train_desc(w)
+    q = x["q"].cuda().requires_grad_()
+    k = x["k"].cuda().requires_grad_()
+    v = x["v"].cuda().requires_grad_()
+    s = x["scores"].cuda().requires_grad_()
+    o = api.SASAttention.apply(q, k, v, s, d)
+    o.backward(x["dO"].cuda())
+    assert torch.equal(o.detach().cpu(), out["o"])
+    assert torch.equal(q.grad.cpu(), out["dq"]) or torch.allclose(q.grad.cpu(), out["dq"], atol=1e-6)
+    assert torch.allclose(s.grad.cpu(), out["ds"], atol=1e-6)
+    assert math.isfinite(float(o.sum()))

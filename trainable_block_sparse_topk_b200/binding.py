@@ -1,0 +1,158 @@
+"""ctypes binding of libsas (include/sas.h), one Python function per C entry point.
+
+Argument marshalling only: each function checks that the torch tensors it is
+given live on the GPU, are contiguous and have the expected dtype, then passes
+their device pointers and the current CUDA stream to the C function of the same
+name and raises SasError on a non-OK status. All computation happens in the
+library's CUDA kernels; there is no other implementation behind these names.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from .build import LIB
+
+SAS_OK, SAS_ERR_INVALID_ARG, SAS_ERR_UNSUPPORTED, SAS_ERR_MISALIGNED, SAS_ERR_WORKSPACE, SAS_ERR_CUDA = range(6)
+SAS_DT_BF16, SAS_DT_FP32 = 0, 1
+SAS_GATE_SOFTMAX, SAS_GATE_NONE = 0, 1
+SAS_OP_TOPK, SAS_OP_FWD, SAS_OP_BWD, SAS_OP_DECODE = range(4)
+
+
+class SasError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: {sas_status_string(status)} (status {status})")
+        self.status = status
+
+
+class sas_desc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("seq_len", ctypes.c_int32), ("q_offset", ctypes.c_int32),
+                ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("block_size", ctypes.c_int32), ("top_k", ctypes.c_int32), ("softmax_scale", ctypes.c_float),
+                ("dtype", ctypes.c_int32), ("gate", ctypes.c_int32)]
+
+    @property
+    def group(self) -> int:
+        return self.n_q_heads // self.n_kv_heads
+
+    @property
+    def n_blocks(self) -> int:
+        return -(-(self.q_offset + self.seq_len) // self.block_size)
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == SAS_DT_FP32 else torch.bfloat16
+
+
+def make_desc(batch, seq_len, n_q_heads, n_kv_heads, head_dim, block_size, top_k, q_offset=0,
+              softmax_scale=0.0, dtype="bf16", gate="softmax") -> sas_desc:
+    dt = {"bf16": SAS_DT_BF16, "fp32": SAS_DT_FP32}[dtype] if isinstance(dtype, str) else int(dtype)
+    gt = {"softmax": SAS_GATE_SOFTMAX, "none": SAS_GATE_NONE}[gate] if isinstance(gate, str) else int(gate)
+    return sas_desc(batch, seq_len, q_offset, n_q_heads, n_kv_heads, head_dim, block_size, top_k,
+                    softmax_scale, dt, gt)
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libsas.so; raises if it has not been built (there is no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB):
+            raise RuntimeError(f"libsas.so not found at {LIB}: build it with "
+                               "`python -m trainable_block_sparse_topk_b200.build`")
+        L = ctypes.CDLL(LIB)
+        P, D = ctypes.c_void_p, ctypes.POINTER(sas_desc)
+        L.sas_workspace_size.argtypes = [ctypes.c_int32, D, ctypes.POINTER(ctypes.c_size_t)]
+        L.sas_block_topk.argtypes = [D, P, P, P, P, P, P]
+        L.sas_gated_attn_fwd.argtypes = [D, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.sas_gated_attn_bwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.sas_sparse_decode.argtypes = [D, P, P, P, ctypes.c_int64, P, P, P, P, P, ctypes.c_size_t, P]
+        L.sas_status_string.argtypes = [ctypes.c_int]
+        L.sas_status_string.restype = ctypes.c_char_p
+        L.sas_device_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+        for f in ("sas_workspace_size", "sas_block_topk", "sas_gated_attn_fwd", "sas_gated_attn_bwd",
+                  "sas_sparse_decode", "sas_device_timeouts"):
+            getattr(L, f).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _dev(t: torch.Tensor | None, name: str, dtype=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn: str, st: int) -> None:
+    if st != SAS_OK:
+        raise SasError(fn, st)
+
+
+def sas_status_string(status: int) -> str:
+    return lib().sas_status_string(int(status)).decode()
+
+
+def sas_workspace_size(op: int, desc: sas_desc) -> int:
+    n = ctypes.c_size_t(0)
+    _check("sas_workspace_size", lib().sas_workspace_size(int(op), ctypes.byref(desc), ctypes.byref(n)))
+    return int(n.value)
+
+
+def sas_block_topk(desc, scores, idx, gate_logit, score_lse, n_sel, stream=None) -> None:
+    f32, i32 = torch.float32, torch.int32
+    _check("sas_block_topk", lib().sas_block_topk(
+        ctypes.byref(desc), _dev(scores, "scores", f32), _dev(idx, "idx", i32),
+        _dev(gate_logit, "gate_logit", f32), _dev(score_lse, "score_lse", f32), _dev(n_sel, "n_sel", i32),
+        _stream(stream)))
+
+
+def sas_gated_attn_fwd(desc, q, k, v, idx, gate_logit, n_sel, o, attn_lse, ws, stream=None) -> None:
+    dt, f32, i32 = desc.torch_dtype, torch.float32, torch.int32
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("sas_gated_attn_fwd", lib().sas_gated_attn_fwd(
+        ctypes.byref(desc), _dev(q, "q", dt), _dev(k, "k", dt), _dev(v, "v", dt), _dev(idx, "idx", i32),
+        _dev(gate_logit, "gate_logit", f32), _dev(n_sel, "n_sel", i32), _dev(o, "o", dt),
+        _dev(attn_lse, "attn_lse", f32), _dev(ws, "ws"), nbytes, _stream(stream)))
+
+
+def sas_gated_attn_bwd(desc, q, k, v, o, dO, attn_lse, scores, score_lse, idx, gate_logit, n_sel,
+                       dq, dk, dv, dscores, ws, stream=None) -> None:
+    dt, f32, i32 = desc.torch_dtype, torch.float32, torch.int32
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("sas_gated_attn_bwd", lib().sas_gated_attn_bwd(
+        ctypes.byref(desc), _dev(q, "q", dt), _dev(k, "k", dt), _dev(v, "v", dt), _dev(o, "o", dt),
+        _dev(dO, "dO", dt), _dev(attn_lse, "attn_lse", f32), _dev(scores, "scores", f32),
+        _dev(score_lse, "score_lse", f32), _dev(idx, "idx", i32), _dev(gate_logit, "gate_logit", f32),
+        _dev(n_sel, "n_sel", i32), _dev(dq, "dq", dt), _dev(dk, "dk", dt), _dev(dv, "dv", dt),
+        _dev(dscores, "dscores", f32), _dev(ws, "ws"), nbytes, _stream(stream)))
+
+
+def sas_sparse_decode(desc, q, k_cache, v_cache, cache_stride_tokens, idx, gate_logit, n_sel, o, ws,
+                      stream=None) -> None:
+    dt, f32, i32 = desc.torch_dtype, torch.float32, torch.int32
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("sas_sparse_decode", lib().sas_sparse_decode(
+        ctypes.byref(desc), _dev(q, "q", dt), _dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
+        int(cache_stride_tokens), _dev(idx, "idx", i32), _dev(gate_logit, "gate_logit", f32),
+        _dev(n_sel, "n_sel", i32), _dev(o, "o", dt), _dev(ws, "ws"), nbytes, _stream(stream)))
+
+
+def sas_device_timeouts() -> int:
+    c = ctypes.c_uint32(0)
+    _check("sas_device_timeouts", lib().sas_device_timeouts(ctypes.byref(c)))
+    return int(c.value)

@@ -1,0 +1,485 @@
+// attn_simt.cu -- gated block-sparse attention on CUDA cores (exact fp32 math).
+//
+// This path serves the fp32 dtype (no TF32 anywhere, for 1e-4 parity) and any
+// shape the tensor-core kernels do not take. Its arithmetic follows the
+// method's definition (SAS study note 2-2 gated-attention eq.; arXiv text 4):
+//   a_j = scale * q . k_j + log g_blk(j)   over the kept blocks' tokens,
+//   a_j = scale * q . k_j                  over the current block, j <= p,
+//   o = softmax(a) V,
+// and the backward recomputes P = exp(a - lse):
+//   dV_j += P_j dO, dP_j = dO . v_j, dS_j = P_j (dP_j - D), D = dO . o,
+//   dQ = scale sum_j dS_j k_j, dK_j += scale dS_j q,
+//   Gsum[row, slot] = sum over the G heads and the block's tokens of dS
+// (the gradient w.r.t. the block's log-gate, study note 3-6 "keeps the
+// selector gradient").
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace sas {
+
+namespace {
+
+// ------------------------------------------------------------------ forward ---
+
+// One warp per (b, kv head, t) row, all G heads of the group at once. Lane
+// `l` scores keys l and l + 32 of each kept block and owns D/32 output dims.
+template <typename T, int D, int GMAX, int BS>
+__global__ void __launch_bounds__(128)
+fwd_simt_kernel(Shape sh, const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                const int32_t* __restrict__ idx, const float* __restrict__ gl,
+                const int32_t* __restrict__ nsel, T* __restrict__ o, float* __restrict__ attn_lse) {
+    constexpr int W = 4;
+    constexpr int KPL = BS / 32;
+    constexpr int DPL = D / 32;
+    constexpr int V16 = vec16<T>();
+    __shared__ float s_q[W][GMAX][D];
+    __shared__ float s_p[W][BS][GMAX];
+
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * W + w;
+    if (row >= sh.rows()) return;
+    const int G = sh.G;
+    const int64_t bg = row / sh.T;
+    const int t = (int)(row % sh.T);
+    const int b = (int)(bg / sh.Hkv), g = (int)(bg % sh.Hkv);
+    const int C = t / BS;
+    const int n = nsel[row];
+    const float qscale = sh.scale * kLog2e;   // logits in log2 units
+
+#pragma unroll
+    for (int h = 0; h < GMAX; ++h) {
+        if (h < G) {
+            const T* qh = q + (((int64_t)b * sh.Hq + g * G + h) * sh.T + t) * D;
+            for (int d = lane; d < D; d += 32) s_q[w][h][d] = Elem<T>::to_f(qh[d]) * qscale;
+        }
+    }
+    __syncwarp();
+
+    float m[GMAX], l[GMAX], acc[GMAX][DPL];
+#pragma unroll
+    for (int h = 0; h < GMAX; ++h) {
+        m[h] = -INFINITY; l[h] = 0.f;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
+    }
+    const T* kb = k + bg * (int64_t)sh.T * D;
+    const T* vb = v + bg * (int64_t)sh.T * D;
+
+    for (int jj = 0; jj <= n; ++jj) {
+        const bool hist = jj < n;
+        const int j = hist ? idx[row * sh.K + jj] : C;
+        const float lg = hist ? gl[row * sh.K + jj] * kLog2e : 0.f;
+        const int ntok = hist ? BS : (t - C * BS + 1);
+        if ((unsigned)j > (unsigned)C) continue;   // not a valid selection: skipped, never read
+
+        float sc[KPL][GMAX];
+#pragma unroll
+        for (int kk = 0; kk < KPL; ++kk) {
+            const int key = lane + 32 * kk;
+#pragma unroll
+            for (int h = 0; h < GMAX; ++h) sc[kk][h] = 0.f;
+            if (key < ntok) {
+                const T* kr = kb + ((int64_t)j * BS + key) * D;
+#pragma unroll 4
+                for (int c = 0; c < D / V16; ++c) {
+                    float kv[V16];
+                    load_vec<T, V16>(kr + c * V16, kv);
+#pragma unroll
+                    for (int h = 0; h < GMAX; ++h) {
+                        if (h < G) {
+#pragma unroll
+                            for (int e = 0; e < V16; ++e) sc[kk][h] = fmaf(s_q[w][h][c * V16 + e], kv[e], sc[kk][h]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int h = 0; h < GMAX; ++h) sc[kk][h] += lg;
+            } else {
+#pragma unroll
+                for (int h = 0; h < GMAX; ++h) sc[kk][h] = -INFINITY;
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < GMAX; ++h) {
+            if (h >= G) continue;
+            float mx = sc[0][h];
+#pragma unroll
+            for (int kk = 1; kk < KPL; ++kk) mx = fmaxf(mx, sc[kk][h]);
+            mx = warp_max(mx);
+            const float mn = fmaxf(m[h], mx);
+            const float corr = (m[h] == -INFINITY) ? 0.f : exp2f(m[h] - mn);
+            float ps = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < KPL; ++kk) {
+                const float pk = (mn == -INFINITY) ? 0.f : exp2f(sc[kk][h] - mn);
+                s_p[w][lane + 32 * kk][h] = pk;
+                ps += pk;
+            }
+            ps = warp_sum(ps);
+            l[h] = l[h] * corr + ps;
+            m[h] = mn;
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) acc[h][e] *= corr;
+        }
+        __syncwarp();
+        for (int key = 0; key < ntok; ++key) {
+            float vv[DPL];
+            load_vec<T, DPL>(vb + ((int64_t)j * BS + key) * D + lane * DPL, vv);
+#pragma unroll
+            for (int h = 0; h < GMAX; ++h) {
+                if (h < G) {
+                    const float pk = s_p[w][key][h];
+#pragma unroll
+                    for (int e = 0; e < DPL; ++e) acc[h][e] = fmaf(pk, vv[e], acc[h][e]);
+                }
+            }
+        }
+        __syncwarp();
+    }
+#pragma unroll
+    for (int h = 0; h < GMAX; ++h) {
+        if (h >= G) continue;
+        const int64_t orow = ((int64_t)b * sh.Hq + g * G + h) * sh.T + t;
+        const float inv = 1.f / l[h];
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) o[orow * D + lane * DPL + e] = Elem<T>::from_f(acc[h][e] * inv);
+        if (lane == 0) attn_lse[orow] = (m[h] + log2f(l[h])) * kLn2;
+    }
+}
+
+// ---------------------------------------------------------- D = rowsum(dO*O) ---
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+rowdot_kernel(int64_t rows, const T* __restrict__ o, const T* __restrict__ dO, float* __restrict__ Dd) {
+    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    constexpr int DPL = D / 32;
+    float a[DPL], b[DPL];
+    load_vec<T, DPL>(o + row * D + lane * DPL, a);
+    load_vec<T, DPL>(dO + row * D + lane * DPL, b);
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) s = fmaf(a[e], b[e], s);
+    s = warp_sum(s);
+    if (lane == 0) Dd[row] = s;
+}
+
+// ----------------------------------------------------------------- backward ---
+
+// One CTA per (b, kv head, key block j), 4 threads per key. It visits every
+// query that attends block j: all of tile j (the block is their current block,
+// causal) and, from the column bitmap, each later query that kept j. dK_j and
+// dV_j accumulate in registers; dQ goes to an fp32 buffer by atomic add; the
+// per-(row, slot) log-gate gradient Gsum is summed over the G heads here.
+template <typename T, int D, int GMAX, int BS>
+__global__ void __launch_bounds__(BS * 4)
+bwd_simt_kernel(Shape sh, const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                const T* __restrict__ dO, const float* __restrict__ attn_lse, const float* __restrict__ Dd,
+                const int32_t* __restrict__ idx, const float* __restrict__ gl, const int32_t* __restrict__ nsel,
+                const uint64_t* __restrict__ maskT, float* __restrict__ dq_acc, T* __restrict__ dk,
+                T* __restrict__ dv, float* __restrict__ gsum) {
+    constexpr int NT = BS * 4;
+    constexpr int DS = D + 4;          // padded row stride: conflict-free for (kk, qd) threads
+    constexpr int DQ = D / 4;
+    extern __shared__ float smem[];
+    float* Ks = smem;                  // [BS][DS]
+    float* Vs = Ks + BS * DS;          // [BS][DS]
+    float* qs = Vs + BS * DS;          // [GMAX][D]
+    float* dOs = qs + GMAX * D;        // [GMAX][D]
+    float* dSs = dOs + GMAX * D;       // [GMAX][BS]
+    float* st = dSs + GMAX * BS;       // [2][GMAX]: lse, D
+    float* red = st + 2 * GMAX;        // [NT/32]
+
+    const int G = sh.G;
+    const int j = blockIdx.x % sh.nT;
+    const int64_t bg = blockIdx.x / sh.nT;
+    const int b = (int)(bg / sh.Hkv), g = (int)(bg % sh.Hkv);
+    const int tid = threadIdx.x;
+    const int kk = tid >> 2, qd = tid & 3;
+    const float scale = sh.scale;
+
+    const T* kb = k + (bg * sh.T + (int64_t)j * BS) * D;
+    const T* vb = v + (bg * sh.T + (int64_t)j * BS) * D;
+    for (int e = tid; e < BS * D; e += NT) {
+        Ks[(e / D) * DS + e % D] = Elem<T>::to_f(kb[e]);
+        Vs[(e / D) * DS + e % D] = Elem<T>::to_f(vb[e]);
+    }
+    float dk_r[DQ], dv_r[DQ];
+#pragma unroll
+    for (int i = 0; i < DQ; ++i) { dk_r[i] = 0.f; dv_r[i] = 0.f; }
+    __syncthreads();
+
+    const uint64_t* col = maskT + (bg * sh.NB + j) * (int64_t)sh.nT;
+
+    // Token stream: tile j fully (diagonal), then set bits of later tiles.
+    int tau = j;
+    uint64_t word = (BS == 64) ? ~0ull : ((1ull << BS) - 1ull);
+    while (true) {
+        if (word == 0ull) {
+            if (++tau >= sh.nT) break;
+            word = col[tau];
+            continue;
+        }
+        const int r = __ffsll((long long)word) - 1;
+        word &= word - 1ull;
+        const bool diag = tau == j;
+        const int t = tau * BS + r;
+        const int64_t row = bg * sh.T + t;
+        int slot = -1;
+        float lg = 0.f;
+        if (!diag) {
+            // position of j in the row's ascending kept list
+            const int32_t* ir = idx + row * sh.K;
+            int lo = 0, hi = nsel[row] - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (ir[mid] < j) lo = mid + 1; else hi = mid;
+            }
+            slot = lo;
+            lg = gl[row * sh.K + slot];
+        }
+        const int kmax = diag ? r : BS - 1;   // causal limit inside the current block
+
+        for (int e = tid; e < G * D; e += NT) {
+            const int h = e / D, d = e % D;
+            const int64_t qrow = ((int64_t)b * sh.Hq + g * G + h) * sh.T + t;
+            qs[h * D + d] = Elem<T>::to_f(q[qrow * D + d]);
+            dOs[h * D + d] = Elem<T>::to_f(dO[qrow * D + d]);
+        }
+        if (tid < G) {
+            const int64_t qrow = ((int64_t)b * sh.Hq + g * G + tid) * sh.T + t;
+            st[tid] = attn_lse[qrow];
+            st[GMAX + tid] = Dd[qrow];
+        }
+        __syncthreads();
+
+#pragma unroll
+        for (int h = 0; h < GMAX; ++h) {
+            if (h >= G) continue;
+            float sd = 0.f, pd = 0.f;
+#pragma unroll
+            for (int i = 0; i < DQ; ++i) {
+                sd = fmaf(qs[h * D + qd + 4 * i], Ks[kk * DS + qd + 4 * i], sd);
+                pd = fmaf(dOs[h * D + qd + 4 * i], Vs[kk * DS + qd + 4 * i], pd);
+            }
+            sd += __shfl_xor_sync(0xffffffffu, sd, 1);
+            sd += __shfl_xor_sync(0xffffffffu, sd, 2);
+            pd += __shfl_xor_sync(0xffffffffu, pd, 1);
+            pd += __shfl_xor_sync(0xffffffffu, pd, 2);
+            const float P = (kk <= kmax) ? expf(scale * sd + lg - st[h]) : 0.f;
+            const float dS = P * (pd - st[GMAX + h]);
+#pragma unroll
+            for (int i = 0; i < DQ; ++i) {
+                dv_r[i] = fmaf(P, dOs[h * D + qd + 4 * i], dv_r[i]);
+                dk_r[i] = fmaf(scale * dS, qs[h * D + qd + 4 * i], dk_r[i]);
+            }
+            if (qd == 0) dSs[h * BS + kk] = dS;
+        }
+        __syncthreads();
+
+        for (int e = tid; e < G * D; e += NT) {
+            const int h = e / D, d = e % D;
+            float a = 0.f;
+#pragma unroll 8
+            for (int x = 0; x < BS; ++x) a = fmaf(dSs[h * BS + x], Ks[x * DS + d], a);
+            const int64_t qrow = ((int64_t)b * sh.Hq + g * G + h) * sh.T + t;
+            atomicAdd(&dq_acc[qrow * D + d], scale * a);
+        }
+        if (!diag) {
+            float a = 0.f;
+            for (int e = tid; e < G * BS; e += NT) a += dSs[e];
+            a = warp_sum(a);
+            if ((tid & 31) == 0) red[tid >> 5] = a;
+        }
+        __syncthreads();
+        if (!diag && tid == 0) {
+            float a = 0.f;
+            for (int w = 0; w < NT / 32; ++w) a += red[w];
+            gsum[row * sh.K + slot] = a;
+        }
+    }
+
+    T* dkb = dk + (bg * sh.T + (int64_t)j * BS) * D;
+    T* dvb = dv + (bg * sh.T + (int64_t)j * BS) * D;
+#pragma unroll
+    for (int i = 0; i < DQ; ++i) {
+        dkb[kk * D + qd + 4 * i] = Elem<T>::from_f(dk_r[i]);
+        dvb[kk * D + qd + 4 * i] = Elem<T>::from_f(dv_r[i]);
+    }
+}
+
+template <typename T>
+__global__ void cast_kernel(int64_t n, const float* __restrict__ src, T* __restrict__ dst) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        dst[i] = Elem<T>::from_f(src[i]);
+}
+
+// ------------------------------------------------------- score gradient (K5) ---
+
+// ds_i = [i kept] Gsum_i - g_i sum_{k kept} Gsum_k for i < C, 0 otherwise,
+// with g_i = exp(s_i - score_lse) (arXiv text 4: d log g_i / d s_k = [i=k] - g_k).
+// One warp per (b, kv head, t) row; every column of the row is written.
+__global__ void __launch_bounds__(256)
+dscore_kernel(Shape sh, const float* __restrict__ scores, const float* __restrict__ slse,
+              const int32_t* __restrict__ idx, const int32_t* __restrict__ nsel,
+              const float* __restrict__ gsum, float* __restrict__ ds) {
+    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= sh.rows()) return;
+    const int t = (int)(row % sh.T);
+    const int C = (int)(((int64_t)sh.q_offset + t) / sh.bs);
+    const int n = nsel[row];
+    const bool on = sh.gate == SAS_GATE_SOFTMAX;
+    int si[2];
+    float sg[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int slot = lane + 32 * r;
+        si[r] = slot < n ? idx[row * sh.K + slot] : -1;
+        sg[r] = slot < n ? gsum[row * sh.K + slot] : 0.f;
+    }
+    const float tot = warp_sum(sg[0] + sg[1]);
+    const float lse = slse[row];
+    const float* sr = scores + row * sh.NB;
+    float* dr = ds + row * sh.NB;
+    int base = 0;
+    for (int c0 = 0; c0 < sh.NB; c0 += 32) {
+        uint32_t bits = 0;
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+            if (si[r] >= c0 && si[r] < c0 + 32) bits |= 1u << (si[r] - c0);
+        const uint32_t mask = __reduce_or_sync(0xffffffffu, bits);
+        const int slot = base + __popc(mask & ((1u << lane) - 1u));
+        const float g0 = __shfl_sync(0xffffffffu, sg[0], slot & 31);
+        const float g1 = __shfl_sync(0xffffffffu, sg[1], slot & 31);
+        const int i = c0 + lane;
+        float val = 0.f;
+        if (on && i < C) {
+            val = -expf(sr[i] - lse) * tot;
+            if ((mask >> lane) & 1u) val += slot < 32 ? g0 : g1;
+        }
+        if (i < sh.NB) dr[i] = val;
+        base += __popc(mask);
+    }
+}
+
+template <typename T, int D, int GMAX, int BS>
+cudaError_t run_fwd(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
+                    const float* gl, const int32_t* nsel, void* o, float* lse, cudaStream_t st) {
+    const int64_t grid = (s.rows() + 3) / 4;
+    fwd_simt_kernel<T, D, GMAX, BS><<<(unsigned)grid, 128, 0, st>>>(
+        s, (const T*)q, (const T*)k, (const T*)v, idx, gl, nsel, (T*)o, lse);
+    return cudaGetLastError();
+}
+
+template <typename T, int D, int GMAX, int BS>
+cudaError_t run_bwd(const Shape& s, const void* q, const void* k, const void* v, const void* dO,
+                    const float* lse, const float* Dd, const int32_t* idx, const float* gl,
+                    const int32_t* nsel, const uint64_t* maskT, float* dq_acc, void* dk, void* dv,
+                    float* gsum, cudaStream_t st) {
+    constexpr int NT = BS * 4;
+    const size_t smem = sizeof(float) * (2 * BS * (D + 4) + 2 * GMAX * D + GMAX * BS + 2 * GMAX + NT / 32);
+    auto kern = bwd_simt_kernel<T, D, GMAX, BS>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = (int64_t)s.B * s.Hkv * s.nT;
+    kern<<<(unsigned)grid, NT, smem, st>>>(s, (const T*)q, (const T*)k, (const T*)v, (const T*)dO, lse, Dd, idx,
+                                           gl, nsel, maskT, dq_acc, (T*)dk, (T*)dv, gsum);
+    return cudaGetLastError();
+}
+
+template <typename T, int D, int BS>
+cudaError_t fwd_g(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
+                  const float* gl, const int32_t* nsel, void* o, float* lse, cudaStream_t st) {
+    if (s.G <= 4) return run_fwd<T, D, 4, BS>(s, q, k, v, idx, gl, nsel, o, lse, st);
+    return run_fwd<T, D, 8, BS>(s, q, k, v, idx, gl, nsel, o, lse, st);
+}
+template <typename T, int D>
+cudaError_t fwd_b(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
+                  const float* gl, const int32_t* nsel, void* o, float* lse, cudaStream_t st) {
+    if (s.bs == 32) return fwd_g<T, D, 32>(s, q, k, v, idx, gl, nsel, o, lse, st);
+    return fwd_g<T, D, 64>(s, q, k, v, idx, gl, nsel, o, lse, st);
+}
+template <typename T>
+cudaError_t fwd_d(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
+                  const float* gl, const int32_t* nsel, void* o, float* lse, cudaStream_t st) {
+    if (s.D == 64) return fwd_b<T, 64>(s, q, k, v, idx, gl, nsel, o, lse, st);
+    return fwd_b<T, 128>(s, q, k, v, idx, gl, nsel, o, lse, st);
+}
+
+template <typename T, int D, int BS>
+cudaError_t bwd_g(const Shape& s, const void* q, const void* k, const void* v, const void* dO,
+                  const float* lse, const float* Dd, const int32_t* idx, const float* gl,
+                  const int32_t* nsel, const uint64_t* maskT, float* dq_acc, void* dk, void* dv,
+                  float* gsum, cudaStream_t st) {
+    if (s.G <= 4) return run_bwd<T, D, 4, BS>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, gsum, st);
+    return run_bwd<T, D, 8, BS>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, gsum, st);
+}
+template <typename T, int D>
+cudaError_t bwd_b(const Shape& s, const void* q, const void* k, const void* v, const void* dO,
+                  const float* lse, const float* Dd, const int32_t* idx, const float* gl,
+                  const int32_t* nsel, const uint64_t* maskT, float* dq_acc, void* dk, void* dv,
+                  float* gsum, cudaStream_t st) {
+    if (s.bs == 32) return bwd_g<T, D, 32>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, gsum, st);
+    return bwd_g<T, D, 64>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, gsum, st);
+}
+template <typename T>
+cudaError_t bwd_d(const Shape& s, const void* q, const void* k, const void* v, const void* dO,
+                  const float* lse, const float* Dd, const int32_t* idx, const float* gl,
+                  const int32_t* nsel, const uint64_t* maskT, float* dq_acc, void* dk, void* dv,
+                  float* gsum, cudaStream_t st) {
+    if (s.D == 64) return bwd_b<T, 64>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, gsum, st);
+    return bwd_b<T, 128>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, gsum, st);
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_simt(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
+                            const float* gl, const int32_t* nsel, void* o, float* lse, cudaStream_t st) {
+    if (s.dtype == SAS_DT_FP32) return fwd_d<float>(s, q, k, v, idx, gl, nsel, o, lse, st);
+    return fwd_d<__nv_bfloat16>(s, q, k, v, idx, gl, nsel, o, lse, st);
+}
+
+cudaError_t launch_bwd_rowdot(const Shape& s, const void* o, const void* dO, float* Dd, cudaStream_t st) {
+    const int64_t rows = (int64_t)s.B * s.Hq * s.T;
+    const unsigned grid = (unsigned)((rows + 7) / 8);
+    if (s.dtype == SAS_DT_FP32) {
+        if (s.D == 64) rowdot_kernel<float, 64><<<grid, 256, 0, st>>>(rows, (const float*)o, (const float*)dO, Dd);
+        else rowdot_kernel<float, 128><<<grid, 256, 0, st>>>(rows, (const float*)o, (const float*)dO, Dd);
+    } else {
+        using B16 = __nv_bfloat16;
+        if (s.D == 64) rowdot_kernel<B16, 64><<<grid, 256, 0, st>>>(rows, (const B16*)o, (const B16*)dO, Dd);
+        else rowdot_kernel<B16, 128><<<grid, 256, 0, st>>>(rows, (const B16*)o, (const B16*)dO, Dd);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_simt(const Shape& s, const void* q, const void* k, const void* v, const void* dO,
+                            const float* lse, const float* Dd, const int32_t* idx, const float* gl,
+                            const int32_t* nsel, const uint64_t* maskT, float* dq_acc, void* dk, void* dv,
+                            float* gsum, cudaStream_t st) {
+    if (s.dtype == SAS_DT_FP32)
+        return bwd_d<float>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, gsum, st);
+    return bwd_d<__nv_bfloat16>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, gsum, st);
+}
+
+cudaError_t launch_cast_dq(const Shape& s, const float* dq_acc, void* dq, cudaStream_t st) {
+    const int64_t n = (int64_t)s.B * s.Hq * s.T * s.D;
+    const unsigned grid = (unsigned)std::min<int64_t>((n + 255) / 256, 148 * 16);
+    if (s.dtype == SAS_DT_FP32) cast_kernel<float><<<grid, 256, 0, st>>>(n, dq_acc, (float*)dq);
+    else cast_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(n, dq_acc, (__nv_bfloat16*)dq);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dscore(const Shape& s, const float* scores, const float* slse, const int32_t* idx,
+                          const int32_t* nsel, const float* gsum, float* ds, cudaStream_t st) {
+    const unsigned grid = (unsigned)((s.rows() + 7) / 8);
+    dscore_kernel<<<grid, 256, 0, st>>>(s, scores, slse, idx, nsel, gsum, ds);
+    return cudaGetLastError();
+}
+
+}  // namespace sas

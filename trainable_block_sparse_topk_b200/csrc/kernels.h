@@ -1,0 +1,57 @@
+// kernels.h -- internal launchers of libsas (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace sas {
+
+// Problem shape, validated and derived from sas_desc by the entry points.
+struct Shape {
+    int B, T, q_offset, Hq, Hkv, G, D, bs, K;
+    int NB;        // ceil((q_offset + T) / bs): score columns per row
+    int nT;        // T / bs (training only): query tiles per (b, kv head)
+    float scale;   // softmax scale on q.k
+    int dtype;     // sas_dtype
+    int gate;      // sas_gate
+    __host__ __device__ int64_t rows() const { return (int64_t)B * Hkv * T; }
+};
+
+// K1: gate normaliser + hard top-K for every (b, kv head, t) row.
+cudaError_t launch_block_topk(const Shape& s, const float* scores, int32_t* idx, float* gate_logit,
+                              float* score_lse, int32_t* n_sel, cudaStream_t st);
+bool topk_row_supported(int64_t max_candidates);
+
+// K1b: column-major selection bitmap maskT[b, g, j, tau] (bit r: query
+// tau*bs + r kept block j). Requires training shapes (q_offset 0, T % bs 0).
+cudaError_t launch_sel_bitmap_T(const Shape& s, const int32_t* idx, const int32_t* n_sel,
+                                uint64_t* maskT, cudaStream_t st);
+
+// Query-centric CUDA-core forward (fp32 and bf16).
+cudaError_t launch_fwd_simt(const Shape& s, const void* q, const void* k, const void* v,
+                            const int32_t* idx, const float* gate_logit, const int32_t* n_sel,
+                            void* o, float* attn_lse, cudaStream_t st);
+
+// Backward pieces.
+cudaError_t launch_bwd_rowdot(const Shape& s, const void* o, const void* dO, float* Dd, cudaStream_t st);
+cudaError_t launch_bwd_simt(const Shape& s, const void* q, const void* k, const void* v, const void* dO,
+                            const float* attn_lse, const float* Dd, const int32_t* idx,
+                            const float* gate_logit, const int32_t* n_sel, const uint64_t* maskT,
+                            float* dq_acc, void* dk, void* dv, float* gsum, cudaStream_t st);
+cudaError_t launch_cast_dq(const Shape& s, const float* dq_acc, void* dq, cudaStream_t st);
+cudaError_t launch_dscore(const Shape& s, const float* scores, const float* score_lse,
+                          const int32_t* idx, const int32_t* n_sel, const float* gsum, float* dscores,
+                          cudaStream_t st);
+
+// Decode.
+struct DecodePlan {
+    int bpc;      // blocks per CTA
+    int splits;   // CTAs per (b, kv head)
+};
+DecodePlan decode_plan(const Shape& s, bool dense);
+size_t decode_ws_bytes(const Shape& s);
+cudaError_t launch_decode(const Shape& s, const void* q, const void* kc, const void* vc, int64_t stride,
+                          const int32_t* idx, const float* gate_logit, const int32_t* n_sel, void* o,
+                          float* part, cudaStream_t st);
+
+}  // namespace sas

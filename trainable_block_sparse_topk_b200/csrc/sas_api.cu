@@ -1,0 +1,215 @@
+// sas_api.cu -- the C ABI of libsas (declared in include/sas.h).
+//
+// Every entry point validates its arguments completely before it launches
+// anything, carves its workspace from the caller's buffer, and enqueues its
+// kernels on the caller's stream. Nothing here allocates, frees or
+// synchronises the host.
+#include <cmath>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace sas {
+
+// Reader for the decode translation unit's wait-timeout counter.
+cudaError_t read_decode_timeouts(unsigned int* out);
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+enum class Kind { kTopk, kTrain, kDecode };
+
+sas_status make_shape(const sas_desc* d, Kind kind, Shape* s) {
+    if (!d || !s) return SAS_ERR_INVALID_ARG;
+    if (d->batch < 1 || d->seq_len < 1 || d->q_offset < 0 || d->n_q_heads < 1 || d->n_kv_heads < 1 ||
+        d->head_dim < 1 || d->block_size < 1 || d->top_k < 1)
+        return SAS_ERR_INVALID_ARG;
+    if (d->n_q_heads % d->n_kv_heads != 0) return SAS_ERR_INVALID_ARG;
+    if (d->dtype != SAS_DT_BF16 && d->dtype != SAS_DT_FP32) return SAS_ERR_INVALID_ARG;
+    if (d->gate != SAS_GATE_SOFTMAX && d->gate != SAS_GATE_NONE) return SAS_ERR_INVALID_ARG;
+    if (!(d->softmax_scale <= 0.f) && !std::isfinite(d->softmax_scale)) return SAS_ERR_INVALID_ARG;
+    if (std::isnan(d->softmax_scale)) return SAS_ERR_INVALID_ARG;
+    const int G = d->n_q_heads / d->n_kv_heads;
+    if (G > 8) return SAS_ERR_UNSUPPORTED;
+    if (d->head_dim != 64 && d->head_dim != 128) return SAS_ERR_UNSUPPORTED;
+    if (d->block_size != 32 && d->block_size != 64) return SAS_ERR_UNSUPPORTED;
+    if (d->top_k > 64) return SAS_ERR_UNSUPPORTED;
+    const int64_t len = (int64_t)d->q_offset + d->seq_len;
+    if (len > (int64_t)1 << 30) return SAS_ERR_UNSUPPORTED;
+    if (!topk_row_supported((len - 1) / d->block_size)) return SAS_ERR_UNSUPPORTED;
+    if (kind == Kind::kTrain) {
+        if (d->q_offset != 0 || d->seq_len % d->block_size != 0) return SAS_ERR_UNSUPPORTED;
+    }
+    if (kind == Kind::kDecode && d->seq_len != 1) return SAS_ERR_INVALID_ARG;
+    s->B = d->batch;
+    s->T = d->seq_len;
+    s->q_offset = d->q_offset;
+    s->Hq = d->n_q_heads;
+    s->Hkv = d->n_kv_heads;
+    s->G = G;
+    s->D = d->head_dim;
+    s->bs = d->block_size;
+    s->K = d->top_k;
+    s->NB = (int)((len + d->block_size - 1) / d->block_size);
+    s->nT = d->seq_len / d->block_size;
+    s->scale = d->softmax_scale > 0.f ? d->softmax_scale : 1.f / std::sqrt((float)d->head_dim);
+    s->dtype = d->dtype;
+    s->gate = d->gate;
+    if ((int64_t)s->B * s->Hkv * s->T > ((int64_t)1 << 31) / 64) return SAS_ERR_UNSUPPORTED;
+    return SAS_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Training workspace layout (each piece 256-byte aligned).
+struct TrainWs {
+    size_t maskT, Dd, gsum, dq_acc, total;
+};
+
+TrainWs bwd_layout(const Shape& s) {
+    TrainWs w{};
+    size_t off = 0;
+    w.maskT = off; off += align256(sizeof(uint64_t) * (size_t)s.B * s.Hkv * s.NB * s.nT);
+    w.Dd = off;    off += align256(sizeof(float) * (size_t)s.B * s.Hq * s.T);
+    w.gsum = off;  off += align256(sizeof(float) * (size_t)s.B * s.Hkv * s.T * s.K);
+    w.dq_acc = off;
+    if (s.dtype != SAS_DT_FP32) off += align256(sizeof(float) * (size_t)s.B * s.Hq * s.T * s.D);
+    w.total = off;
+    return w;
+}
+
+size_t ws_bytes(int op, const Shape& s) {
+    switch (op) {
+        case SAS_OP_TOPK: return 0;
+        case SAS_OP_FWD: return 0;
+        case SAS_OP_BWD: return bwd_layout(s).total;
+        case SAS_OP_DECODE: return align256(decode_ws_bytes(s));
+        default: return 0;
+    }
+}
+
+sas_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SAS_OK : SAS_ERR_CUDA; }
+
+template <typename... P>
+bool any_null(P... p) { return ((p == nullptr) || ...); }
+template <typename... P>
+bool any_misaligned(P... p) { return (!aligned16(p) || ...); }
+
+}  // namespace
+}  // namespace sas
+
+using namespace sas;
+
+extern "C" {
+
+const char* sas_status_string(sas_status st) {
+    switch (st) {
+        case SAS_OK: return "ok";
+        case SAS_ERR_INVALID_ARG: return "invalid argument";
+        case SAS_ERR_UNSUPPORTED: return "unsupported shape or option";
+        case SAS_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case SAS_ERR_WORKSPACE: return "workspace missing or too small";
+        case SAS_ERR_CUDA: return "CUDA launch or runtime error";
+        default: return "unknown status";
+    }
+}
+
+sas_status sas_workspace_size(int32_t op, const sas_desc* desc, size_t* bytes) {
+    if (!bytes) return SAS_ERR_INVALID_ARG;
+    if (op < SAS_OP_TOPK || op > SAS_OP_DECODE) return SAS_ERR_INVALID_ARG;
+    const Kind kind = op == SAS_OP_TOPK ? Kind::kTopk : (op == SAS_OP_DECODE ? Kind::kDecode : Kind::kTrain);
+    Shape s;
+    sas_status st = make_shape(desc, kind, &s);
+    if (st != SAS_OK) return st;
+    *bytes = ws_bytes(op, s);
+    return SAS_OK;
+}
+
+sas_status sas_block_topk(const sas_desc* desc, const float* scores, int32_t* idx, float* gate_logit,
+                          float* score_lse, int32_t* n_sel, void* stream) {
+    Shape s;
+    sas_status st = make_shape(desc, Kind::kTopk, &s);
+    if (st != SAS_OK) return st;
+    if (any_null(scores, idx, gate_logit, score_lse, n_sel)) return SAS_ERR_INVALID_ARG;
+    if (any_misaligned(scores, idx, gate_logit, score_lse, n_sel)) return SAS_ERR_MISALIGNED;
+    return cuda_status(launch_block_topk(s, scores, idx, gate_logit, score_lse, n_sel, (cudaStream_t)stream));
+}
+
+sas_status sas_gated_attn_fwd(const sas_desc* desc, const void* q, const void* k, const void* v,
+                              const int32_t* idx, const float* gate_logit, const int32_t* n_sel, void* o,
+                              float* attn_lse, void* ws, size_t ws_bytes_, void* stream) {
+    Shape s;
+    sas_status st = make_shape(desc, Kind::kTrain, &s);
+    if (st != SAS_OK) return st;
+    if (any_null(q, k, v, idx, gate_logit, n_sel, o, attn_lse)) return SAS_ERR_INVALID_ARG;
+    if (any_misaligned(q, k, v, idx, gate_logit, n_sel, o, attn_lse)) return SAS_ERR_MISALIGNED;
+    const size_t need = ws_bytes(SAS_OP_FWD, s);
+    if (need > 0 && (ws == nullptr || ws_bytes_ < need)) return SAS_ERR_WORKSPACE;
+    if (ws && !aligned16(ws)) return SAS_ERR_MISALIGNED;
+    cudaStream_t cs = (cudaStream_t)stream;
+    return cuda_status(launch_fwd_simt(s, q, k, v, idx, gate_logit, n_sel, o, attn_lse, cs));
+}
+
+sas_status sas_gated_attn_bwd(const sas_desc* desc, const void* q, const void* k, const void* v, const void* o,
+                              const void* dO, const float* attn_lse, const float* scores, const float* score_lse,
+                              const int32_t* idx, const float* gate_logit, const int32_t* n_sel, void* dq,
+                              void* dk, void* dv, float* dscores, void* ws, size_t ws_bytes_, void* stream) {
+    Shape s;
+    sas_status st = make_shape(desc, Kind::kTrain, &s);
+    if (st != SAS_OK) return st;
+    if (any_null(q, k, v, o, dO, attn_lse, scores, score_lse, idx, gate_logit, n_sel, dq, dk, dv, dscores))
+        return SAS_ERR_INVALID_ARG;
+    if (any_misaligned(q, k, v, o, dO, attn_lse, scores, score_lse, idx, gate_logit, n_sel, dq, dk, dv, dscores))
+        return SAS_ERR_MISALIGNED;
+    const TrainWs L = bwd_layout(s);
+    if (ws == nullptr || ws_bytes_ < L.total) return SAS_ERR_WORKSPACE;
+    if (!aligned16(ws)) return SAS_ERR_MISALIGNED;
+    cudaStream_t cs = (cudaStream_t)stream;
+    unsigned char* w = static_cast<unsigned char*>(ws);
+    uint64_t* maskT = reinterpret_cast<uint64_t*>(w + L.maskT);
+    float* Dd = reinterpret_cast<float*>(w + L.Dd);
+    float* gsum = reinterpret_cast<float*>(w + L.gsum);
+    float* dq_acc = s.dtype == SAS_DT_FP32 ? static_cast<float*>(dq) : reinterpret_cast<float*>(w + L.dq_acc);
+
+    cudaError_t e = cudaMemsetAsync(dq_acc, 0, sizeof(float) * (size_t)s.B * s.Hq * s.T * s.D, cs);
+    if (e == cudaSuccess) e = launch_sel_bitmap_T(s, idx, n_sel, maskT, cs);
+    if (e == cudaSuccess) e = launch_bwd_rowdot(s, o, dO, Dd, cs);
+    if (e == cudaSuccess)
+        e = launch_bwd_simt(s, q, k, v, dO, attn_lse, Dd, idx, gate_logit, n_sel, maskT, dq_acc, dk, dv, gsum, cs);
+    if (e == cudaSuccess && s.dtype != SAS_DT_FP32) e = launch_cast_dq(s, dq_acc, dq, cs);
+    if (e == cudaSuccess) e = launch_dscore(s, scores, score_lse, idx, n_sel, gsum, dscores, cs);
+    return cuda_status(e);
+}
+
+sas_status sas_sparse_decode(const sas_desc* desc, const void* q, const void* k_cache, const void* v_cache,
+                             int64_t cache_stride_tokens, const int32_t* idx, const float* gate_logit,
+                             const int32_t* n_sel, void* o, void* ws, size_t ws_bytes_, void* stream) {
+    Shape s;
+    sas_status st = make_shape(desc, Kind::kDecode, &s);
+    if (st != SAS_OK) return st;
+    if (any_null(q, k_cache, v_cache, o)) return SAS_ERR_INVALID_ARG;
+    if (idx != nullptr && any_null(gate_logit, n_sel)) return SAS_ERR_INVALID_ARG;
+    if (cache_stride_tokens < (int64_t)s.q_offset + 1) return SAS_ERR_INVALID_ARG;
+    if (any_misaligned(q, k_cache, v_cache, o)) return SAS_ERR_MISALIGNED;
+    if (idx != nullptr && any_misaligned(idx, gate_logit, n_sel)) return SAS_ERR_MISALIGNED;
+    const size_t need = ws_bytes(SAS_OP_DECODE, s);
+    if (ws == nullptr || ws_bytes_ < need) return SAS_ERR_WORKSPACE;
+    if (!aligned16(ws)) return SAS_ERR_MISALIGNED;
+    return cuda_status(launch_decode(s, q, k_cache, v_cache, cache_stride_tokens, idx, gate_logit, n_sel, o,
+                                     static_cast<float*>(ws), (cudaStream_t)stream));
+}
+
+// Diagnostics: number of bounded device-side waits that gave up since the
+// library was loaded (0 in normal operation). Synchronises the device.
+sas_status sas_device_timeouts(uint32_t* count) {
+    if (!count) return SAS_ERR_INVALID_ARG;
+    unsigned int c = 0;
+    cudaError_t e = read_decode_timeouts(&c);
+    if (e != cudaSuccess) return SAS_ERR_CUDA;
+    *count = c;
+    return SAS_OK;
+}
+
+}  // extern "C"
