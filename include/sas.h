@@ -156,6 +156,11 @@ sas_status sas_sparse_decode(const sas_desc* desc, const void* q, const void* k_
  * its output instead of hanging. Synchronises the current device. */
 sas_status sas_device_timeouts(uint32_t* count);
 
+/* Diagnostics (no counterpart on the pages): number of CUDA kernels this
+ * library has launched since it was loaded, counted on the host after each
+ * successful launch. Memsets issued through the runtime are not counted. */
+uint64_t sas_kernel_launches(void);
+
 /* Static, NUL-terminated description of a status code (never NULL). */
 const char* sas_status_string(sas_status status);
 

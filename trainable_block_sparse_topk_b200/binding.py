@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
         L.sas_status_string.argtypes = [ctypes.c_int]
         L.sas_status_string.restype = ctypes.c_char_p
         L.sas_device_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+        L.sas_kernel_launches.argtypes = []
+        L.sas_kernel_launches.restype = ctypes.c_uint64
         for f in ("sas_workspace_size", "sas_block_topk", "sas_gated_attn_fwd", "sas_gated_attn_bwd",
                   "sas_sparse_decode", "sas_device_timeouts"):
             getattr(L, f).restype = ctypes.c_int
@@ -156,3 +158,7 @@ def sas_device_timeouts() -> int:
     c = ctypes.c_uint32(0)
     _check("sas_device_timeouts", lib().sas_device_timeouts(ctypes.byref(c)))
     return int(c.value)
+
+
+def sas_kernel_launches() -> int:
+    return int(lib().sas_kernel_launches())

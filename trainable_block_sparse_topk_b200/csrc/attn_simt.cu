@@ -373,7 +373,9 @@ cudaError_t run_fwd(const Shape& s, const void* q, const void* k, const void* v,
     const int64_t grid = (s.rows() + 3) / 4;
     fwd_simt_kernel<T, D, GMAX, BS><<<(unsigned)grid, 128, 0, st>>>(
         s, (const T*)q, (const T*)k, (const T*)v, idx, gl, nsel, (T*)o, lse);
-    return cudaGetLastError();
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) count_launches(1);
+    return e;
 }
 
 template <typename T, int D, int GMAX, int BS>
@@ -389,7 +391,9 @@ cudaError_t run_bwd(const Shape& s, const void* q, const void* k, const void* v,
     const int64_t grid = (int64_t)s.B * s.Hkv * s.nT;
     kern<<<(unsigned)grid, NT, smem, st>>>(s, (const T*)q, (const T*)k, (const T*)v, (const T*)dO, lse, Dd, idx,
                                            gl, nsel, maskT, dq_acc, (T*)dk, (T*)dv, gsum);
-    return cudaGetLastError();
+    e = cudaGetLastError();
+    if (e == cudaSuccess) count_launches(1);
+    return e;
 }
 
 template <typename T, int D, int BS>
@@ -455,7 +459,9 @@ cudaError_t launch_bwd_rowdot(const Shape& s, const void* o, const void* dO, flo
         if (s.D == 64) rowdot_kernel<B16, 64><<<grid, 256, 0, st>>>(rows, (const B16*)o, (const B16*)dO, Dd);
         else rowdot_kernel<B16, 128><<<grid, 256, 0, st>>>(rows, (const B16*)o, (const B16*)dO, Dd);
     }
-    return cudaGetLastError();
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) count_launches(1);
+    return e;
 }
 
 cudaError_t launch_bwd_simt(const Shape& s, const void* q, const void* k, const void* v, const void* dO,
@@ -472,14 +478,18 @@ cudaError_t launch_cast_dq(const Shape& s, const float* dq_acc, void* dq, cudaSt
     const unsigned grid = (unsigned)std::min<int64_t>((n + 255) / 256, 148 * 16);
     if (s.dtype == SAS_DT_FP32) cast_kernel<float><<<grid, 256, 0, st>>>(n, dq_acc, (float*)dq);
     else cast_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(n, dq_acc, (__nv_bfloat16*)dq);
-    return cudaGetLastError();
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) count_launches(1);
+    return e;
 }
 
 cudaError_t launch_dscore(const Shape& s, const float* scores, const float* slse, const int32_t* idx,
                           const int32_t* nsel, const float* gsum, float* ds, cudaStream_t st) {
     const unsigned grid = (unsigned)((s.rows() + 7) / 8);
     dscore_kernel<<<grid, 256, 0, st>>>(s, scores, slse, idx, nsel, gsum, ds);
-    return cudaGetLastError();
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) count_launches(1);
+    return e;
 }
 
 }  // namespace sas

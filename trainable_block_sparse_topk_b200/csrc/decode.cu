@@ -304,9 +304,12 @@ cudaError_t run_decode(const DecArgs& a, cudaStream_t st) {
     kern<<<(unsigned)grid, kDecThreads, smem, st>>>(a);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    count_launches(1);
     decode_combine_kernel<T, D><<<(unsigned)(a.sh.B * a.sh.Hkv), 256, 0, st>>>(a.sh, a.part, a.splits,
                                                                                 static_cast<T*>(a.o));
-    return cudaGetLastError();
+    e = cudaGetLastError();
+    if (e == cudaSuccess) count_launches(1);
+    return e;
 }
 
 template <typename T, int D, int BS>

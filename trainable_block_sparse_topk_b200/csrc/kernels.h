@@ -6,6 +6,9 @@
 
 namespace sas {
 
+// Host-side count of kernels this library has launched (sas_kernel_launches).
+void count_launches(unsigned n);
+
 // Problem shape, validated and derived from sas_desc by the entry points.
 struct Shape {
     int B, T, q_offset, Hq, Hkv, G, D, bs, K;

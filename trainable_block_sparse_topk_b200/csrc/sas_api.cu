@@ -4,6 +4,7 @@
 // anything, carves its workspace from the caller's buffer, and enqueues its
 // kernels on the caller's stream. Nothing here allocates, frees or
 // synchronises the host.
+#include <atomic>
 #include <cmath>
 #include <cstring>
 
@@ -14,6 +15,9 @@ namespace sas {
 
 // Reader for the decode translation unit's wait-timeout counter.
 cudaError_t read_decode_timeouts(unsigned int* out);
+
+static std::atomic<unsigned long long> g_launches{0};
+void count_launches(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
 namespace {
 
@@ -200,6 +204,10 @@ sas_status sas_sparse_decode(const sas_desc* desc, const void* q, const void* k_
     return cuda_status(launch_decode(s, q, k_cache, v_cache, cache_stride_tokens, idx, gate_logit, n_sel, o,
                                      static_cast<float*>(ws), (cudaStream_t)stream));
 }
+
+// Diagnostics: kernels launched by this library since it was loaded (host
+// count, incremented after each successful launch).
+uint64_t sas_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 // Diagnostics: number of bounded device-side waits that gave up since the
 // library was loaded (0 in normal operation). Synchronises the device.

@@ -251,7 +251,9 @@ cudaError_t run_topk(const Shape& s, const float* scores, int32_t* idx, float* g
     const int rpc = NT == 32 ? 8 : 1;
     const int64_t grid = (rows + rpc - 1) / rpc;
     block_topk_kernel<NT, SLOTS><<<(unsigned)grid, NT == 32 ? 256 : NT, 0, st>>>(s, scores, idx, gl, lse, nsel);
-    return cudaGetLastError();
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) count_launches(1);
+    return e;
 }
 
 // ------------------------------------------------------------ K1b: bitmap ---
@@ -305,7 +307,9 @@ cudaError_t launch_sel_bitmap_T(const Shape& s, const int32_t* idx, const int32_
     }
     const int64_t grid = (int64_t)s.B * s.Hkv * s.nT;
     sel_bitmap_T_kernel<<<(unsigned)grid, 256, smem, st>>>(s, idx, nsel, maskT);
-    return cudaGetLastError();
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) count_launches(1);
+    return e;
 }
 
 }  // namespace sas
