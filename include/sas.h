@@ -150,6 +150,33 @@ sas_status sas_sparse_decode(const sas_desc* desc, const void* q, const void* k_
                              const float* gate_logit, const int32_t* n_sel, void* o, void* ws,
                              size_t ws_bytes, void* stream);
 
+/* Sparse decode that allocates nothing (the paper has no counterpart: this is
+ * an interface convenience, not part of the method).
+ *
+ * For callers that cannot call cudaMalloc: a serving loop with a fixed device
+ * memory budget set aside at start-up, a plug-in whose host framework owns all
+ * device allocations, or a path where an allocation and its implicit
+ * synchronisation are not allowed. Same arguments, results and checks as
+ * sas_sparse_decode, minus the workspace: the split partials live in a static
+ * device array of SAS_NOALLOC_SCRATCH_BYTES inside libsas, which every GPU
+ * that loads the library holds until the process exits.
+ *  - Returns SAS_ERR_WORKSPACE, launching nothing, when the shape needs more
+ *    than SAS_NOALLOC_SCRATCH_BYTES of partials (4 * B * Hkv * splits * G *
+ *    (d + 2) bytes; splits = K + 1 for sparse decode).
+ *  - The first call on each device looks up the array's device address (a
+ *    runtime call that allocates nothing); make that first call before any
+ *    stream capture.
+ *  - All calls share the one array and it keeps the last call's contents.
+ *    Each call writes every partial it reads, so nothing needs clearing, but
+ *    calls that overlap on the GPU (different streams, or different host
+ *    threads on one device, with no ordering between them) race on it.
+ *  - No cudaMalloc, cudaFree or allocating library routine is called. */
+#define SAS_NOALLOC_SCRATCH_BYTES (8u << 20)
+sas_status sas_sparse_decode_noalloc(const sas_desc* desc, const void* q, const void* k_cache,
+                                     const void* v_cache, int64_t cache_stride_tokens,
+                                     const int32_t* idx, const float* gate_logit,
+                                     const int32_t* n_sel, void* o, void* stream);
+
 /* Diagnostics (no counterpart on the pages): number of device-side waits for
  * an asynchronous copy that gave up after their ~1 s bound since the library
  * was loaded; 0 in normal operation. A kernel whose wait gave up leaves NaN in

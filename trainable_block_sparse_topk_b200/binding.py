@@ -71,13 +71,14 @@ def lib() -> ctypes.CDLL:
         L.sas_gated_attn_fwd.argtypes = [D, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.sas_gated_attn_bwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.sas_sparse_decode.argtypes = [D, P, P, P, ctypes.c_int64, P, P, P, P, P, ctypes.c_size_t, P]
+        L.sas_sparse_decode_noalloc.argtypes = [D, P, P, P, ctypes.c_int64, P, P, P, P, P]
         L.sas_status_string.argtypes = [ctypes.c_int]
         L.sas_status_string.restype = ctypes.c_char_p
         L.sas_device_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
         L.sas_kernel_launches.argtypes = []
         L.sas_kernel_launches.restype = ctypes.c_uint64
         for f in ("sas_workspace_size", "sas_block_topk", "sas_gated_attn_fwd", "sas_gated_attn_bwd",
-                  "sas_sparse_decode", "sas_device_timeouts"):
+                  "sas_sparse_decode", "sas_sparse_decode_noalloc", "sas_device_timeouts"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -152,6 +153,17 @@ def sas_sparse_decode(desc, q, k_cache, v_cache, cache_stride_tokens, idx, gate_
         ctypes.byref(desc), _dev(q, "q", dt), _dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
         int(cache_stride_tokens), _dev(idx, "idx", i32), _dev(gate_logit, "gate_logit", f32),
         _dev(n_sel, "n_sel", i32), _dev(o, "o", dt), _dev(ws, "ws"), nbytes, _stream(stream)))
+
+
+def sas_sparse_decode_noalloc(desc, q, k_cache, v_cache, cache_stride_tokens, idx, gate_logit, n_sel, o,
+                              stream=None) -> None:
+    """sas_sparse_decode without a workspace: the library's static scratch
+    array holds the split partials (see include/sas.h)."""
+    dt, f32, i32 = desc.torch_dtype, torch.float32, torch.int32
+    _check("sas_sparse_decode_noalloc", lib().sas_sparse_decode_noalloc(
+        ctypes.byref(desc), _dev(q, "q", dt), _dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
+        int(cache_stride_tokens), _dev(idx, "idx", i32), _dev(gate_logit, "gate_logit", f32),
+        _dev(n_sel, "n_sel", i32), _dev(o, "o", dt), _stream(stream)))
 
 
 def sas_device_timeouts() -> int:

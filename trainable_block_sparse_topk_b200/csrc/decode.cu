@@ -12,6 +12,7 @@
 // with a single instruction. The CTA writes an unnormalised partial (m, l, o)
 // for the G heads, and a second kernel merges the partials by log-sum-exp.
 #include <algorithm>
+#include <mutex>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -368,3 +369,63 @@ size_t decode_ws_bytes(const Shape& s) {
 }
 
 }  // namespace sas
+
+// ------------------------------------------------- decode without allocation ---
+//
+// Some callers of decode cannot call cudaMalloc at all: code that runs with a
+// fixed memory budget carved out up front, plug-ins whose host framework owns
+// every device allocation, or paths where an allocation (or its implicit
+// synchronisation) is not allowed. For them, sas_sparse_decode_noalloc keeps the
+// split partials in this file-scope device array instead of a caller workspace.
+// Every GPU that loads the library holds it until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SAS_NOALLOC_SCRATCH_BYTES];
+
+namespace sas {
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device. In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device (with that device current) and cached.
+cudaError_t noalloc_scratch(float** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (g_scratch_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = static_cast<float*>(g_scratch_ptr[dev]);
+    return cudaSuccess;
+}
+
+}  // namespace
+
+}  // namespace sas
+
+extern "C" sas_status sas_sparse_decode_noalloc(const sas_desc* desc, const void* q, const void* k_cache,
+                                                const void* v_cache, int64_t cache_stride_tokens,
+                                                const int32_t* idx, const float* gate_logit,
+                                                const int32_t* n_sel, void* o, void* stream) {
+    using namespace sas;
+    Shape s;
+    sas_status st = check_decode_args(desc, q, k_cache, v_cache, cache_stride_tokens, idx, gate_logit, n_sel, o, &s);
+    if (st != SAS_OK) return st;
+    const DecodePlan p = decode_plan(s, idx == nullptr);
+    const size_t need = sizeof(float) * (size_t)s.B * s.Hkv * p.splits * s.G * (s.D + 2);
+    if (need > (size_t)SAS_NOALLOC_SCRATCH_BYTES) return SAS_ERR_WORKSPACE;
+    float* part = nullptr;
+    if (noalloc_scratch(&part) != cudaSuccess) return SAS_ERR_CUDA;
+    // Every split record is written before the merge reads it, so nothing in
+    // the shared array has to start at zero.
+    const cudaError_t e = launch_decode(s, q, k_cache, v_cache, cache_stride_tokens, idx, gate_logit, n_sel, o,
+                                        part, (cudaStream_t)stream);
+    return e == cudaSuccess ? SAS_OK : SAS_ERR_CUDA;
+}

@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "../../include/sas.h"
+
 namespace sas {
 
 // Host-side count of kernels this library has launched (sas_kernel_launches).
@@ -45,6 +47,11 @@ cudaError_t launch_cast_dq(const Shape& s, const float* dq_acc, void* dq, cudaSt
 cudaError_t launch_dscore(const Shape& s, const float* scores, const float* score_lse,
                           const int32_t* idx, const int32_t* n_sel, const float* gsum, float* dscores,
                           cudaStream_t st);
+
+// Decode argument checks shared by the decode entry points (sas_api.cu).
+sas_status check_decode_args(const sas_desc* desc, const void* q, const void* k_cache, const void* v_cache,
+                             int64_t cache_stride_tokens, const int32_t* idx, const float* gate_logit,
+                             const int32_t* n_sel, const void* o, Shape* s);
 
 // Decode.
 struct DecodePlan {

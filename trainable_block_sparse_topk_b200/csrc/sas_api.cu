@@ -102,6 +102,20 @@ template <typename... P>
 bool any_misaligned(P... p) { return (!aligned16(p) || ...); }
 
 }  // namespace
+
+sas_status check_decode_args(const sas_desc* desc, const void* q, const void* k_cache, const void* v_cache,
+                             int64_t cache_stride_tokens, const int32_t* idx, const float* gate_logit,
+                             const int32_t* n_sel, const void* o, Shape* s) {
+    sas_status st = make_shape(desc, Kind::kDecode, s);
+    if (st != SAS_OK) return st;
+    if (any_null(q, k_cache, v_cache, o)) return SAS_ERR_INVALID_ARG;
+    if (idx != nullptr && any_null(gate_logit, n_sel)) return SAS_ERR_INVALID_ARG;
+    if (cache_stride_tokens < (int64_t)s->q_offset + 1) return SAS_ERR_INVALID_ARG;
+    if (any_misaligned(q, k_cache, v_cache, o)) return SAS_ERR_MISALIGNED;
+    if (idx != nullptr && any_misaligned(idx, gate_logit, n_sel)) return SAS_ERR_MISALIGNED;
+    return SAS_OK;
+}
+
 }  // namespace sas
 
 using namespace sas;
@@ -191,13 +205,8 @@ sas_status sas_sparse_decode(const sas_desc* desc, const void* q, const void* k_
                              int64_t cache_stride_tokens, const int32_t* idx, const float* gate_logit,
                              const int32_t* n_sel, void* o, void* ws, size_t ws_bytes_, void* stream) {
     Shape s;
-    sas_status st = make_shape(desc, Kind::kDecode, &s);
+    sas_status st = check_decode_args(desc, q, k_cache, v_cache, cache_stride_tokens, idx, gate_logit, n_sel, o, &s);
     if (st != SAS_OK) return st;
-    if (any_null(q, k_cache, v_cache, o)) return SAS_ERR_INVALID_ARG;
-    if (idx != nullptr && any_null(gate_logit, n_sel)) return SAS_ERR_INVALID_ARG;
-    if (cache_stride_tokens < (int64_t)s.q_offset + 1) return SAS_ERR_INVALID_ARG;
-    if (any_misaligned(q, k_cache, v_cache, o)) return SAS_ERR_MISALIGNED;
-    if (idx != nullptr && any_misaligned(idx, gate_logit, n_sel)) return SAS_ERR_MISALIGNED;
     const size_t need = ws_bytes(SAS_OP_DECODE, s);
     if (ws == nullptr || ws_bytes_ < need) return SAS_ERR_WORKSPACE;
     if (!aligned16(ws)) return SAS_ERR_MISALIGNED;
