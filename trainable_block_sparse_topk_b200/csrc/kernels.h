@@ -37,6 +37,11 @@ cudaError_t launch_fwd_simt(const Shape& s, const void* q, const void* k, const 
                             const int32_t* idx, const float* gate_logit, const int32_t* n_sel,
                             void* o, float* attn_lse, cudaStream_t st);
 
+// Tensor-core forward (tcgen05 + TMA): bf16, d = 128, block 64.
+bool fwd_tc_supported(const Shape& s);
+cudaError_t launch_fwd_tc(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
+                          const float* gate_logit, const int32_t* n_sel, void* o, float* attn_lse, cudaStream_t st);
+
 // Backward pieces.
 cudaError_t launch_bwd_rowdot(const Shape& s, const void* o, const void* dO, float* Dd, cudaStream_t st);
 cudaError_t launch_bwd_simt(const Shape& s, const void* q, const void* k, const void* v, const void* dO,

@@ -6,6 +6,7 @@
 // synchronises the host.
 #include <atomic>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 
 #include "common.cuh"
@@ -13,8 +14,16 @@
 
 namespace sas {
 
-// Reader for the decode translation unit's wait-timeout counter.
+// Readers for the wait-timeout counters of the translation units that wait.
 cudaError_t read_decode_timeouts(unsigned int* out);
+cudaError_t read_fwd_tc_timeouts(unsigned int* out);
+
+// SAS_FORCE_SIMT=1 routes bf16 training calls to the CUDA-core kernels (a
+// second GPU implementation, used to cross-check the tensor-core path).
+static bool force_simt() {
+    const char* e = std::getenv("SAS_FORCE_SIMT");
+    return e != nullptr && e[0] == '1';
+}
 
 static std::atomic<unsigned long long> g_launches{0};
 void count_launches(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
@@ -167,6 +176,8 @@ sas_status sas_gated_attn_fwd(const sas_desc* desc, const void* q, const void* k
     if (need > 0 && (ws == nullptr || ws_bytes_ < need)) return SAS_ERR_WORKSPACE;
     if (ws && !aligned16(ws)) return SAS_ERR_MISALIGNED;
     cudaStream_t cs = (cudaStream_t)stream;
+    if (fwd_tc_supported(s) && !force_simt())
+        return cuda_status(launch_fwd_tc(s, q, k, v, idx, gate_logit, n_sel, o, attn_lse, cs));
     return cuda_status(launch_fwd_simt(s, q, k, v, idx, gate_logit, n_sel, o, attn_lse, cs));
 }
 
@@ -222,10 +233,11 @@ uint64_t sas_kernel_launches(void) { return g_launches.load(std::memory_order_re
 // library was loaded (0 in normal operation). Synchronises the device.
 sas_status sas_device_timeouts(uint32_t* count) {
     if (!count) return SAS_ERR_INVALID_ARG;
-    unsigned int c = 0;
-    cudaError_t e = read_decode_timeouts(&c);
+    unsigned int c0 = 0, c1 = 0;
+    cudaError_t e = read_decode_timeouts(&c0);
+    if (e == cudaSuccess) e = read_fwd_tc_timeouts(&c1);
     if (e != cudaSuccess) return SAS_ERR_CUDA;
-    *count = c;
+    *count = c0 + c1;
     return SAS_OK;
 }
 
