@@ -1,0 +1,462 @@
+// attn_bwd_tc.cu -- gated block-sparse backward on the sm_100a tensor cores.
+//
+// Gradients of o = softmax(a) V with a_j = scale q.k_j + log g_blk(j) (SAS
+// study note 2-2, 3-6 "keeps the selector gradient"; arXiv text 4):
+//   P = exp(a - lse), dP = dO V^T, dS = P (dP - D) with D = rowsum(dO o),
+//   dV += P^T dO, dK += scale dS^T q, dQ = scale dS K,
+//   Gsum[row, slot] = sum of dS over the block's tokens and the group's heads
+// (the gradient of the row's log-gate of that block; the score gradient is
+// formed from it by the epilogue kernel).
+//
+// Tiling: key-block-centric. One CTA owns key block j of one (batch, KV
+// group). It streams the (token, head) rows whose attention includes j -- the
+// block's own 64 tokens (causally) and every later token whose selection kept
+// j, read from the column bitmap -- in chunks of 128 gathered rows (128/G
+// tokens x G heads), so every MMA row is a kept row. Per chunk:
+//   S = Q K_j^T and dP = dO V_j^T  (M=128 rows, N=64 keys, K=d)   -> TMEM
+//   P, dS in the compute warps (thread = row = TMEM lane), Gsum per token
+//   dV^T += dO^T P, dK^T += Q^T dS (M=d, N=64, K=128 rows)        -> TMEM
+//   dQ = dS K_j (M=128 rows, N=d, K=64)                            -> TMEM
+//   dQ rows are added into the fp32 accumulator with vector atomics.
+// TMEM: S|dP double buffer [0,256), dQ [256,384), dV^T [384,448),
+// dK^T [448,512). S/dP of chunk c+1 are computed while the compute warps
+// build P/dS of chunk c and read back dQ of chunk c-1.
+//
+// Roles (256 threads): warps 0 and 3 gather chunk rows (even / odd chunks)
+// with 16-byte cp.async into the two 128-byte-swizzled Q/dO stages (warp 0
+// also loads K_j, V_j by TMA), warp 1 lane 0 issues the MMAs, warp 2 owns the
+// TMEM allocation, warps 4-7 compute. No TMA multicast is used.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace sas {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kBS = 64;
+constexpr int kRows = 128;
+constexpr int kD = 128;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColDQ = 256, kColDV = 384, kColDK = 448;
+
+struct BwdTcArgs {
+    Shape sh;
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* dO;
+    const float* lse;
+    const float* Dd;
+    const int32_t* idx;
+    const float* gl;
+    const int32_t* nsel;
+    const uint64_t* maskT;
+    float* dq_acc;
+    __nv_bfloat16* dk;
+    __nv_bfloat16* dv;
+    float* gsum;
+    int tpc;   // tokens per chunk = 128 / G
+};
+
+struct BwdSmem {
+    static constexpr uint32_t kK = 0;                          // K_j: 2 halves x [64 x 128 B]
+    static constexpr uint32_t kV = 16384;                      // V_j
+    static constexpr uint32_t kStage = 32768;                  // 2 x (Q [2 x 128 x 128 B] | dO [same])
+    static constexpr uint32_t kStageBytes = 65536;
+    static constexpr uint32_t kP = kStage + 2 * kStageBytes;   // P  [128 x 128 B]
+    static constexpr uint32_t kDS = kP + 16384;                // dS [128 x 128 B]
+    static constexpr uint32_t kMeta = kDS + 16384;             // 2 x per-chunk metadata
+    static constexpr uint32_t kMetaBytes = 5 * 512 + 16;       // tok_t, tok_slot, tok_lg, row_lse, row_D, ntok
+    static constexpr uint32_t kGs = kMeta + 2 * kMetaBytes;    // per-token Gsum [2][128] f32
+    static constexpr uint32_t kBar = kGs + 1024;
+    static constexpr int kNumBars = 13;
+    static constexpr uint32_t kMisc = kBar + 8 * kNumBars;     // tmem base, chunk count, abort
+    static constexpr uint32_t kTotal = kMisc + 16;
+};
+
+struct Meta {
+    int* tok_t;
+    int* tok_slot;
+    float* tok_lg;
+    float* row_lse;
+    float* row_D;
+    int* ntok;
+    __device__ explicit Meta(unsigned char* p)
+        : tok_t(reinterpret_cast<int*>(p)),
+          tok_slot(reinterpret_cast<int*>(p + 512)),
+          tok_lg(reinterpret_cast<float*>(p + 1024)),
+          row_lse(reinterpret_cast<float*>(p + 1536)),
+          row_D(reinterpret_cast<float*>(p + 2048)),
+          ntok(reinterpret_cast<int*>(p + 2560)) {}
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, BwdTcArgs a) {
+    using L = BwdSmem;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
+    uint64_t* kv_full = bars + 0;
+    uint64_t* st_full = bars + 1;     // [2], 32 arrivals (the loader warp)
+    uint64_t* st_empty = bars + 3;    // [2]
+    uint64_t* s_full = bars + 5;      // [2]
+    uint64_t* p_full = bars + 7;      // 4 arrivals (compute warps)
+    uint64_t* p_empty = bars + 8;
+    uint64_t* dq_full = bars + 9;
+    uint64_t* dq_empty = bars + 10;   // 4 arrivals
+    uint64_t* done = bars + 11;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMisc);
+    int* nc_slot = reinterpret_cast<int*>(sm + L::kMisc + 4);
+    volatile int* abort = reinterpret_cast<volatile int*>(sm + L::kMisc + 8);
+    float* tok_gs = reinterpret_cast<float*>(sm + L::kGs);
+
+    const Shape& sh = a.sh;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int G = sh.G, K = sh.K, T = sh.T;
+    const int ngroups = sh.B * sh.Hkv;
+    const int j = (int)(blockIdx.x / ngroups);
+    const int bg = (int)(blockIdx.x % ngroups);
+    const int b = bg / sh.Hkv, g = bg % sh.Hkv;
+    const int tpc = a.tpc;
+    const uint64_t* col = a.maskT + ((int64_t)bg * sh.NB + j) * sh.nT;
+
+    if (tid == 0) {
+        for (int i = 0; i < L::kNumBars; ++i) {
+            uint64_t* bar = &bars[i];
+            uint32_t cnt = 1;
+            if (bar == &st_full[0] || bar == &st_full[1]) cnt = 32;
+            if (bar == p_full || bar == dq_empty) cnt = 4;
+            mbar_init(bar, cnt);
+        }
+        *nc_slot = kBS;   // the block's own tokens; later tiles are added below
+        *abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 2) {
+        tc::tmem_alloc(tmem_slot, kTmemCols);
+        tc::tmem_relinquish();
+    }
+    for (int i = tid; i < 2 * kRows; i += kThreads) tok_gs[i] = 0.f;
+    __syncthreads();
+    {
+        int cnt = 0;
+        for (int tau = j + 1 + tid; tau < sh.nT; tau += kThreads) cnt += __popcll(col[tau]);
+        cnt = __reduce_add_sync(0xffffffffu, cnt);
+        if (lane == 0 && cnt) atomicAdd(nc_slot, cnt);
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+    const int ntok_total = *nc_slot;
+    const int nc = (ntok_total + tpc - 1) / tpc;
+    const uint32_t sbase = smem_u32(sm);
+
+    if (warp == 0 || warp == 3) {
+        // ---------------------------------------------------------- loaders ---
+        const int L0 = warp == 0 ? 0 : 1;           // this warp fills chunks c = L0, L0 + 2, ...
+        unsigned char* stq = sm + L::kStage + L0 * L::kStageBytes;
+        unsigned char* stdo = stq + 32768;
+        Meta meta(sm + L::kMeta + L0 * L::kMetaBytes);
+        if (warp == 0 && lane == 0) {
+            tc::prefetch_tmap(&tm_k);
+            tc::prefetch_tmap(&tm_v);
+            mbar_arrive_expect_tx(kv_full, 32768);
+            const int kr = (int)((int64_t)bg * T + (int64_t)j * kBS);
+            for (int h = 0; h < 2; ++h) {
+                tc::tma_load_2d(sm + L::kK + h * 8192, &tm_k, h * 64, kr, kv_full);
+                tc::tma_load_2d(sm + L::kV + h * 8192, &tm_v, h * 64, kr, kv_full);
+            }
+        }
+        // token stream cursor (lane 0 only): the block's own tile, then the bitmap
+        int cur_tau = j;
+        uint64_t cur_w = ~0ull;
+        auto next_token = [&]() -> int {
+            while (cur_w == 0ull) {
+                if (++cur_tau >= sh.nT) return -1;
+                cur_w = col[cur_tau];
+            }
+            const int bit = __ffsll((long long)cur_w) - 1;
+            cur_w &= cur_w - 1ull;
+            return cur_tau * kBS + bit;
+        };
+        if (L0 == 1 && lane == 0) for (int i = 0; i < tpc; ++i) next_token();   // skip chunk 0
+        for (int c = L0; c < nc; c += 2) {
+            if (c >= 2 && !tc::warp_wait_bar(&st_empty[L0], (uint32_t)(((c >> 1) - 1) & 1), abort)) break;
+            if (lane == 0) {
+                int n = 0;
+                for (; n < tpc; ++n) {
+                    const int t = next_token();
+                    if (t < 0) break;
+                    meta.tok_t[n] = t;
+                }
+                *meta.ntok = n;
+                for (int i = 0; i < tpc; ++i) next_token();   // skip the other loader's chunk
+            }
+            __syncwarp();
+            const int n = *meta.ntok;
+            for (int i = lane; i < n; i += 32) {
+                const int t = meta.tok_t[i];
+                int slot = -1;
+                float lg = 0.f;
+                if ((t >> 6) != j) {
+                    const int64_t row = (int64_t)bg * T + t;
+                    const int32_t* ir = a.idx + row * K;
+                    int lo = 0, hi = a.nsel[row] - 1;
+                    while (lo < hi) {
+                        const int mid = (lo + hi) >> 1;
+                        if (ir[mid] < j) lo = mid + 1; else hi = mid;
+                    }
+                    slot = lo;
+                    lg = a.gl[row * K + lo];
+                }
+                meta.tok_slot[i] = slot;
+                meta.tok_lg[i] = lg;
+            }
+            for (int i = lane; i < kRows; i += 32) {
+                const int ti = i / G, h = i - ti * G;
+                float lse = 0.f, Dv = 0.f;
+                if (ti < n) {
+                    const int64_t qrow = ((int64_t)b * sh.Hq + g * G + h) * T + meta.tok_t[ti];
+                    lse = a.lse[qrow];
+                    Dv = a.Dd[qrow];
+                }
+                meta.row_lse[i] = lse;
+                meta.row_D[i] = Dv;
+            }
+            // rows: one row per step, lanes 0-15 copy q, lanes 16-31 copy dO (16 x 16 B each)
+            const int cc = lane & 15;
+            unsigned char* dstb = (lane < 16 ? stq : stdo) + (cc >> 3) * 16384;
+            const __nv_bfloat16* srcb = lane < 16 ? a.q : a.dO;
+            for (int i = 0; i < kRows; ++i) {
+                const int ti = i / G, h = i - ti * G;
+                unsigned char* dst = dstb + tc::sw128_offset(i, (cc & 7) * 8);
+                if (ti < n) {
+                    const int64_t qrow = ((int64_t)b * sh.Hq + g * G + h) * T + meta.tok_t[ti];
+                    tc::cp_async16(dst, srcb + qrow * kD + cc * 8);
+                } else {
+                    *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+                }
+            }
+            tc::cp_async_wait_all();
+            tc::fence_async_shared();
+            __syncwarp();
+            tc::mbar_arrive(&st_full[L0]);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------- MMA issuer ---
+        if (lane == 0) {
+            constexpr uint32_t id_sp = tc::idesc_bf16_f32(128, kBS, false, false);   // S, dP
+            constexpr uint32_t id_kv = tc::idesc_bf16_f32(128, kBS, true, true);     // dV^T, dK^T
+            constexpr uint32_t id_dq = tc::idesc_bf16_f32(128, kD, false, true);     // dQ
+            const uint32_t ka = sbase + L::kK, va = sbase + L::kV;
+            const uint32_t pa = sbase + L::kP, dsa = sbase + L::kDS;
+            auto issue_sdp = [&](int c) {
+                const uint32_t qa = sbase + L::kStage + (c & 1) * L::kStageBytes, doa = qa + 32768;
+                const uint32_t dsp = tmem + (uint32_t)((c & 1) * 128);
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+                    const uint32_t offk = (kk >> 2) * 8192 + (kk & 3) * 32;
+                    tc::mma_ss(dsp, tc::smem_desc_sw128(qa + off, 16, 1024), tc::smem_desc_sw128(ka + offk, 16, 1024),
+                               id_sp, kk > 0);
+                    tc::mma_ss(dsp + 64, tc::smem_desc_sw128(doa + off, 16, 1024),
+                               tc::smem_desc_sw128(va + offk, 16, 1024), id_sp, kk > 0);
+                }
+                tc::mma_commit(&s_full[c & 1]);
+            };
+            bool ok = tc::wait_bar(kv_full, 0u, abort) && tc::wait_bar(&st_full[0], 0u, abort);
+            tc::fence_after_sync();
+            if (ok) issue_sdp(0);
+            for (int c = 0; ok && c < nc; ++c) {
+                if (c + 1 < nc) {
+                    if (!tc::wait_bar(&st_full[(c + 1) & 1], (uint32_t)(((c + 1) >> 1) & 1), abort)) break;
+                    tc::fence_after_sync();
+                    issue_sdp(c + 1);
+                }
+                if (!tc::wait_bar(p_full, (uint32_t)(c & 1), abort)) break;
+                tc::fence_after_sync();
+                const uint32_t qa = sbase + L::kStage + (c & 1) * L::kStageBytes, doa = qa + 32768;
+#pragma unroll
+                for (int kk = 0; kk < kRows / 16; ++kk) {
+                    const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
+                    tc::mma_ss(tmem + kColDV, tc::smem_desc_sw128(doa + kk * 2048, 16384, 1024),
+                               tc::smem_desc_sw128(pa + kk * 2048, 16384, 1024), id_kv, acc);
+                    tc::mma_ss(tmem + kColDK, tc::smem_desc_sw128(qa + kk * 2048, 16384, 1024),
+                               tc::smem_desc_sw128(dsa + kk * 2048, 16384, 1024), id_kv, acc);
+                }
+                if (c >= 1 && !tc::wait_bar(dq_empty, (uint32_t)((c - 1) & 1), abort)) break;
+                tc::fence_after_sync();
+#pragma unroll
+                for (int kk = 0; kk < kBS / 16; ++kk)
+                    tc::mma_ss(tmem + kColDQ, tc::smem_desc_sw128(dsa + kk * 32, 16, 1024),
+                               tc::smem_desc_sw128(ka + kk * 2048, 8192, 1024), id_dq, kk > 0);
+                tc::mma_commit(dq_full);
+                tc::mma_commit(&st_empty[c & 1]);
+                tc::mma_commit(p_empty);
+            }
+            tc::mma_commit(done);
+        }
+    } else if (warp >= 4) {
+        // ----------------------------------------------------- compute warps ---
+        const int r = (warp - 4) * 32 + lane;      // chunk row == TMEM lane
+        const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const float qk = sh.scale * kLog2e;
+        const float dscale = sh.scale;
+        bool ok = true;
+        int64_t prev_dq_row = -1;                  // dq accumulator row of this thread in chunk c-1
+        auto dq_epilogue = [&](int c) -> bool {    // read dQ of chunk c back and add it to the fp32 accumulator
+            if (!tc::warp_wait_bar(dq_full, (uint32_t)(c & 1), abort)) return false;
+            tc::fence_after_sync();
+#pragma unroll 1
+            for (int cb = 0; cb < kD / 16; ++cb) {
+                uint32_t v[16];
+                tc::tmem_ld16(lane_base + kColDQ + cb * 16, v);
+                tc::tmem_wait_ld();
+                if (prev_dq_row >= 0) {
+                    float* dst = a.dq_acc + prev_dq_row * kD + cb * 16;
+#pragma unroll
+                    for (int e = 0; e < 16; e += 4)
+                        tc::red_add_v4(dst + e, __uint_as_float(v[e]) * dscale, __uint_as_float(v[e + 1]) * dscale,
+                                       __uint_as_float(v[e + 2]) * dscale, __uint_as_float(v[e + 3]) * dscale);
+                }
+            }
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(dq_empty);
+            return true;
+        };
+        for (int c = 0; c < nc; ++c) {
+            const int st = c & 1;
+            if (!tc::warp_wait_bar(&st_full[st], (uint32_t)((c >> 1) & 1), abort)) { ok = false; break; }
+            Meta meta(sm + L::kMeta + st * L::kMetaBytes);
+            const int n = *meta.ntok;
+            const int ti = r / G, h = r - ti * G;
+            const bool valid = ti < n;
+            int t = 0, kmax = -1;
+            float lgl = 0.f, lse2 = 0.f, Dv = 0.f;
+            bool diag = false;
+            if (valid) {
+                t = meta.tok_t[ti];
+                diag = (t >> 6) == j;
+                kmax = diag ? (t & 63) : kBS - 1;
+                lgl = meta.tok_lg[ti];
+                lse2 = meta.row_lse[r];
+                Dv = meta.row_D[r];
+            }
+            const float bias = (lgl - lse2) * kLog2e;
+            const int64_t dq_row = valid ? ((int64_t)b * sh.Hq + g * G + h) * T + t : -1;
+            if (!tc::warp_wait_bar(&s_full[st], (uint32_t)((c >> 1) & 1), abort)) { ok = false; break; }
+            tc::fence_after_sync();
+            uint32_t sv[kBS], pv[kBS];
+#pragma unroll
+            for (int cb = 0; cb < kBS / 16; ++cb) {
+                tc::tmem_ld16(lane_base + (uint32_t)(st * 128 + cb * 16), sv + cb * 16);
+                tc::tmem_ld16(lane_base + (uint32_t)(st * 128 + 64 + cb * 16), pv + cb * 16);
+            }
+            tc::tmem_wait_ld();
+            uint32_t pk[kBS / 2], dk2[kBS / 2];
+            float rowsum = 0.f;
+#pragma unroll
+            for (int k = 0; k < kBS; k += 2) {
+                const float p0 = (k <= kmax) ? exp2f(fmaf(__uint_as_float(sv[k]), qk, bias)) : 0.f;
+                const float p1 = (k + 1 <= kmax) ? exp2f(fmaf(__uint_as_float(sv[k + 1]), qk, bias)) : 0.f;
+                const float d0 = p0 * (__uint_as_float(pv[k]) - Dv);
+                const float d1 = p1 * (__uint_as_float(pv[k + 1]) - Dv);
+                rowsum += d0 + d1;
+                __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);
+                __nv_bfloat162 hd = __floats2bfloat162_rn(d0, d1);
+                pk[k / 2] = *reinterpret_cast<uint32_t*>(&hp);
+                dk2[k / 2] = *reinterpret_cast<uint32_t*>(&hd);
+            }
+            // Gsum of the token: its G rows are in this chunk
+            float* gs = tok_gs + st * kRows;
+            if (valid && !diag) atomicAdd(&gs[ti], rowsum);
+            tc::named_bar(1, 128);
+            if (r < n) {
+                const int slot = meta.tok_slot[r];
+                if (slot >= 0) a.gsum[((int64_t)bg * T + meta.tok_t[r]) * K + slot] = gs[r];
+                gs[r] = 0.f;
+            }
+            // P and dS of chunk c-1 must have been consumed by its MMAs
+            if (c >= 1 && !tc::warp_wait_bar(p_empty, (uint32_t)((c - 1) & 1), abort)) { ok = false; break; }
+#pragma unroll
+            for (int cb = 0; cb < kBS / 8; ++cb) {
+                const uint32_t off = tc::sw128_offset(r, cb * 8);
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sbase + L::kP + off), "r"(pk[cb * 4]),
+                             "r"(pk[cb * 4 + 1]), "r"(pk[cb * 4 + 2]), "r"(pk[cb * 4 + 3])
+                             : "memory");
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sbase + L::kDS + off), "r"(dk2[cb * 4]),
+                             "r"(dk2[cb * 4 + 1]), "r"(dk2[cb * 4 + 2]), "r"(dk2[cb * 4 + 3])
+                             : "memory");
+            }
+            tc::fence_async_shared();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(p_full);
+            if (c >= 1 && !dq_epilogue(c - 1)) { ok = false; break; }
+            prev_dq_row = dq_row;
+        }
+        if (ok && nc > 0) ok = dq_epilogue(nc - 1);
+        // dV^T and dK^T: TMEM lane r holds column r of d for the block's 64 keys
+        if (ok && tc::warp_wait_bar(done, 0u, abort)) {
+            tc::fence_after_sync();
+            __nv_bfloat16* dvb = a.dv + ((int64_t)bg * T + (int64_t)j * kBS) * kD;
+            __nv_bfloat16* dkb = a.dk + ((int64_t)bg * T + (int64_t)j * kBS) * kD;
+#pragma unroll 1
+            for (int cb = 0; cb < kBS / 16; ++cb) {
+                uint32_t vv[16], kv[16];
+                tc::tmem_ld16(lane_base + kColDV + cb * 16, vv);
+                tc::tmem_ld16(lane_base + kColDK + cb * 16, kv);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int key = cb * 16 + e;
+                    dvb[(int64_t)key * kD + r] = __float2bfloat16_rn(__uint_as_float(vv[e]));
+                    dkb[(int64_t)key * kD + r] = __float2bfloat16_rn(__uint_as_float(kv[e]) * dscale);
+                }
+            }
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 2) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace
+
+bool bwd_tc_supported(const Shape& s) {
+    return s.dtype == SAS_DT_BF16 && s.D == kD && s.bs == kBS && s.K <= 64 && s.G <= 8 && s.q_offset == 0 &&
+           s.T % kBS == 0 && (int64_t)s.B * s.Hq * s.T < ((int64_t)1 << 31);
+}
+
+cudaError_t launch_bwd_tc(const Shape& s, const void* q, const void* k, const void* v, const void* dO,
+                          const float* lse, const float* Dd, const int32_t* idx, const float* gl,
+                          const int32_t* nsel, const uint64_t* maskT, float* dq_acc, void* dk, void* dv,
+                          float* gsum, cudaStream_t st) {
+    CUtensorMap mk, mv;
+    if (!encode_bf16_2d(&mk, k, (uint64_t)s.B * s.Hkv * s.T, kD, kBS) ||
+        !encode_bf16_2d(&mv, v, (uint64_t)s.B * s.Hkv * s.T, kD, kBS))
+        return cudaErrorInvalidValue;
+    const size_t smem = BwdSmem::kTotal + 1024;
+    cudaError_t e = cudaFuncSetAttribute(bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    BwdTcArgs a{s, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dO), lse, Dd, idx, gl, nsel,
+                maskT, dq_acc, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), gsum, kRows / s.G};
+    const int64_t grid = (int64_t)s.B * s.Hkv * s.nT;
+    bwd_tc_kernel<<<(unsigned)grid, kThreads, smem, st>>>(mk, mv, a);
+    e = cudaGetLastError();
+    if (e == cudaSuccess) count_launches(1);
+    return e;
+}
+
+cudaError_t read_bwd_tc_timeouts(unsigned int* out) {
+    return cudaMemcpyFromSymbol(out, g_sas_wait_timeouts, sizeof(unsigned int));
+}
+
+}  // namespace sas

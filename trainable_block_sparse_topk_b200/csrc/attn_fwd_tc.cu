@@ -76,37 +76,6 @@ struct FwdSmem {
     static constexpr uint32_t kTotal = kMisc + 16;
 };
 
-// Bounded wait shared by all roles: gives up after ~1 s or when another role
-// has already given up, raising the CTA's abort flag.
-__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = global_ns();
-    while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (*abort) return false;
-        if (global_ns() - t0 > 1000000000ull) {
-            *abort = 1;
-            atomicAdd(&g_sas_wait_timeouts, 1u);
-            return false;
-        }
-    }
-}
-
-// Bounded wait that ignores the abort flag: used to let copies already in
-// flight land before an aborting CTA exits.
-__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-    const uint64_t t0 = global_ns();
-    while (!mbar_try_wait(bar, parity))
-        if (global_ns() - t0 > 1000000000ull) return;
-}
-
-// Warp-uniform variant: lane 0 waits, the result is broadcast.
-__device__ __forceinline__ bool warp_wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort) {
-    int ok = 0;
-    if ((threadIdx.x & 31) == 0) ok = wait_bar(bar, parity, abort) ? 1 : 0;
-    return __shfl_sync(0xffffffffu, ok, 0) != 0;
-}
-
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -216,7 +185,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             int issued = 0;
             for (int j = 0; j < n; ++j) {
                 const int s = j % kStages;
-                if (j >= kStages && !wait_bar(&kv_empty[s], (uint32_t)((j / kStages - 1) & 1), abort)) break;
+                if (j >= kStages && !tc::wait_bar(&kv_empty[s], (uint32_t)((j / kStages - 1) & 1), abort)) break;
                 const int blk = ulist[j];
                 const int kr = (int)((int64_t)bg * sh.T + (int64_t)blk * kBS);
                 unsigned char* st = sKV + s * L::kStageBytes;
@@ -231,7 +200,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             if (*abort) {
                 // let the loads this thread started land before the CTA exits
                 for (int j = issued - kStages; j < issued; ++j)
-                    if (j >= 0) drain_wait(&kv_full[j % kStages], (uint32_t)((j / kStages) & 1));
+                    if (j >= 0) tc::drain_wait(&kv_full[j % kStages], (uint32_t)((j / kStages) & 1));
             }
         }
     } else if (warp == 1) {
@@ -240,12 +209,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             constexpr uint32_t idesc_s = tc::idesc_bf16_f32(128, kBS, false, false);
             constexpr uint32_t idesc_pv = tc::idesc_bf16_f32(128, D, false, true);
             const uint32_t qa = smem_u32(sQ), kva = smem_u32(sKV), pa = smem_u32(sP);
-            bool ok = wait_bar(q_full, 0u, abort);
+            bool ok = tc::wait_bar(q_full, 0u, abort);
             tc::fence_after_sync();
             for (int j = 0; ok && j <= n; ++j) {
                 if (j < n) {
                     const int s = j % kStages;
-                    if (!wait_bar(&kv_full[s], (uint32_t)((j / kStages) & 1), abort)) break;
+                    if (!tc::wait_bar(&kv_full[s], (uint32_t)((j / kStages) & 1), abort)) break;
                     tc::fence_after_sync();
                     const uint32_t kaddr = kva + s * L::kStageBytes;
                     const uint32_t d_s = tmem + (uint32_t)((j & 1) * kBS);
@@ -260,7 +229,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
                 if (j >= 1) {
                     const int jp = j - 1;
-                    if (!wait_bar(&p_full[jp & 1], (uint32_t)((jp >> 1) & 1), abort)) break;
+                    if (!tc::wait_bar(&p_full[jp & 1], (uint32_t)((jp >> 1) & 1), abort)) break;
                     tc::fence_after_sync();
                     const int sp = jp % kStages;
                     const uint32_t vaddr = kva + sp * L::kStageBytes + L::DH * L::kKHalf;
@@ -291,7 +260,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         bool ok = true;
         for (int j = 0; j < n; ++j) {
             const int blk = ulist[j];
-            if (!warp_wait_bar(&s_full[j & 1], (uint32_t)((j >> 1) & 1), abort)) { ok = false; break; }
+            if (!tc::warp_wait_bar(&s_full[j & 1], (uint32_t)((j >> 1) & 1), abort)) { ok = false; break; }
             tc::fence_after_sync();
             uint32_t sr[kBS];
 #pragma unroll
@@ -330,7 +299,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             if (__any_sync(0xffffffffu, resc)) {
                 // the previous P V must be complete before O is rescaled in place
-                if (!warp_wait_bar(&p_empty[(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1), abort)) { ok = false; break; }
+                if (!tc::warp_wait_bar(&p_empty[(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1), abort)) { ok = false; break; }
                 tc::fence_after_sync();
 #pragma unroll 1
                 for (int c = 0; c < D / 16; ++c) {
@@ -356,7 +325,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             l += psum;
             // P buffer j&1 was last read by P V of block j-2
-            if (j >= 2 && !warp_wait_bar(&p_empty[j & 1], (uint32_t)(((j - 2) >> 1) & 1), abort)) { ok = false; break; }
+            if (j >= 2 && !tc::warp_wait_bar(&p_empty[j & 1], (uint32_t)(((j - 2) >> 1) & 1), abort)) { ok = false; break; }
             unsigned char* prow = sP + (j & 1) * L::kPBytes;
 #pragma unroll
             for (int c = 0; c < kBS / 8; ++c) {
@@ -370,7 +339,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&p_full[j & 1]);
         }
-        if (ok && warp_wait_bar(o_done, 0u, abort)) {
+        if (ok && tc::warp_wait_bar(o_done, 0u, abort)) {
             tc::fence_after_sync();
             const int head = (r < kTok) ? h0 : h1;
             const bool write = r < kTok || h1_valid;
@@ -413,25 +382,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     }
 }
 
-bool encode_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
-    const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {cols * 2};
-    const cuuint32_t box[2] = {64, box_rows};
-    const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = cuTensorMapEncodeTiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
-                                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 template <int D>
 cudaError_t run_fwd_tc(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
                        const float* gl, const int32_t* nsel, void* o, float* lse, cudaStream_t st) {
     CUtensorMap mq, mk, mv;
-    if (!encode_2d(&mq, q, (uint64_t)s.B * s.Hq * s.T, D, 64) ||
-        !encode_2d(&mk, k, (uint64_t)s.B * s.Hkv * s.T, D, kBS) ||
-        !encode_2d(&mv, v, (uint64_t)s.B * s.Hkv * s.T, D, kBS))
+    if (!encode_bf16_2d(&mq, q, (uint64_t)s.B * s.Hq * s.T, D, 64) ||
+        !encode_bf16_2d(&mk, k, (uint64_t)s.B * s.Hkv * s.T, D, kBS) ||
+        !encode_bf16_2d(&mv, v, (uint64_t)s.B * s.Hkv * s.T, D, kBS))
         return cudaErrorInvalidValue;
     const size_t smem = FwdSmem<D>::kTotal + 1024;
     auto kern = fwd_tc_kernel<D>;
@@ -446,6 +403,18 @@ cudaError_t run_fwd_tc(const Shape& s, const void* q, const void* k, const void*
 }
 
 }  // namespace
+
+bool encode_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {cols * 2};
+    const cuuint32_t box[2] = {64, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = cuTensorMapEncodeTiled(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                                              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
 
 bool fwd_tc_supported(const Shape& s) {
     return s.dtype == SAS_DT_BF16 && s.D == 128 && s.bs == kBS && s.NB <= kMaxNB && s.K <= 64 && s.G <= 8 &&

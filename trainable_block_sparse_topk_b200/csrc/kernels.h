@@ -6,6 +6,8 @@
 
 #include "../../include/sas.h"
 
+struct CUtensorMap_st;   // cuda.h: CUtensorMap
+
 namespace sas {
 
 // Host-side count of kernels this library has launched (sas_kernel_launches).
@@ -36,6 +38,16 @@ cudaError_t launch_sel_bitmap_T(const Shape& s, const int32_t* idx, const int32_
 cudaError_t launch_fwd_simt(const Shape& s, const void* q, const void* k, const void* v,
                             const int32_t* idx, const float* gate_logit, const int32_t* n_sel,
                             void* o, float* attn_lse, cudaStream_t st);
+
+// 2D bf16 tensor map [rows x cols] with 64 x box_rows boxes, 128-byte swizzle.
+bool encode_bf16_2d(::CUtensorMap_st* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
+
+// Tensor-core backward (tcgen05 + TMA + cp.async gathers): bf16, d = 128, block 64.
+bool bwd_tc_supported(const Shape& s);
+cudaError_t launch_bwd_tc(const Shape& s, const void* q, const void* k, const void* v, const void* dO,
+                          const float* attn_lse, const float* Dd, const int32_t* idx, const float* gate_logit,
+                          const int32_t* n_sel, const uint64_t* maskT, float* dq_acc, void* dk, void* dv,
+                          float* gsum, cudaStream_t st);
 
 // Tensor-core forward (tcgen05 + TMA): bf16, d = 128, block 64.
 bool fwd_tc_supported(const Shape& s);

@@ -17,6 +17,7 @@ namespace sas {
 // Readers for the wait-timeout counters of the translation units that wait.
 cudaError_t read_decode_timeouts(unsigned int* out);
 cudaError_t read_fwd_tc_timeouts(unsigned int* out);
+cudaError_t read_bwd_tc_timeouts(unsigned int* out);
 
 // SAS_FORCE_SIMT=1 routes bf16 training calls to the CUDA-core kernels (a
 // second GPU implementation, used to cross-check the tensor-core path).
@@ -205,8 +206,13 @@ sas_status sas_gated_attn_bwd(const sas_desc* desc, const void* q, const void* k
     cudaError_t e = cudaMemsetAsync(dq_acc, 0, sizeof(float) * (size_t)s.B * s.Hq * s.T * s.D, cs);
     if (e == cudaSuccess) e = launch_sel_bitmap_T(s, idx, n_sel, maskT, cs);
     if (e == cudaSuccess) e = launch_bwd_rowdot(s, o, dO, Dd, cs);
-    if (e == cudaSuccess)
-        e = launch_bwd_simt(s, q, k, v, dO, attn_lse, Dd, idx, gate_logit, n_sel, maskT, dq_acc, dk, dv, gsum, cs);
+    if (e == cudaSuccess) {
+        if (bwd_tc_supported(s) && !force_simt())
+            e = launch_bwd_tc(s, q, k, v, dO, attn_lse, Dd, idx, gate_logit, n_sel, maskT, dq_acc, dk, dv, gsum, cs);
+        else
+            e = launch_bwd_simt(s, q, k, v, dO, attn_lse, Dd, idx, gate_logit, n_sel, maskT, dq_acc, dk, dv, gsum,
+                                cs);
+    }
     if (e == cudaSuccess && s.dtype != SAS_DT_FP32) e = launch_cast_dq(s, dq_acc, dq, cs);
     if (e == cudaSuccess) e = launch_dscore(s, scores, score_lse, idx, n_sel, gsum, dscores, cs);
     return cuda_status(e);
@@ -233,11 +239,12 @@ uint64_t sas_kernel_launches(void) { return g_launches.load(std::memory_order_re
 // library was loaded (0 in normal operation). Synchronises the device.
 sas_status sas_device_timeouts(uint32_t* count) {
     if (!count) return SAS_ERR_INVALID_ARG;
-    unsigned int c0 = 0, c1 = 0;
+    unsigned int c0 = 0, c1 = 0, c2 = 0;
     cudaError_t e = read_decode_timeouts(&c0);
     if (e == cudaSuccess) e = read_fwd_tc_timeouts(&c1);
+    if (e == cudaSuccess) e = read_bwd_tc_timeouts(&c2);
     if (e != cudaSuccess) return SAS_ERR_CUDA;
-    *count = c0 + c1;
+    *count = c0 + c1 + c2;
     return SAS_OK;
 }
 
