@@ -70,7 +70,10 @@ struct BwdSmem {
     static constexpr uint32_t kMeta = kDS + 16384;             // 2 x per-chunk metadata
     static constexpr uint32_t kMetaBytes = 5 * 512 + 16;       // tok_t, tok_slot, tok_lg, row_lse, row_D, ntok
     static constexpr uint32_t kGs = kMeta + 2 * kMetaBytes;    // per-token Gsum [2][128] f32
-    static constexpr uint32_t kBar = kGs + 1024;
+    static constexpr uint32_t kColW = kGs + 1024;              // u64 [kMaxNT]: the block's bitmap column
+    static constexpr uint32_t kPre = kColW + 8 * 1024;         // i32 [kMaxNT]: stream index of tile tau's first token
+    static constexpr uint32_t kQoff = kPre + 4 * 1024;         // i32 [2][128]: q/dO row of each chunk row (-1: pad)
+    static constexpr uint32_t kBar = kQoff + 2 * 4 * kRows;
     static constexpr int kNumBars = 13;
     static constexpr uint32_t kMisc = kBar + 8 * kNumBars;     // tmem base, chunk count, abort
     static constexpr uint32_t kTotal = kMisc + 16;
@@ -138,13 +141,31 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         tc::tmem_alloc(tmem_slot, kTmemCols);
         tc::tmem_relinquish();
     }
+    // The token stream of block j: its own 64 tokens, then the tokens of later
+    // tiles that kept j, in order. colw holds the bitmap column, pre[tau] the
+    // stream index of tile tau's first token (valid for tau > j).
+    unsigned long long* colw = reinterpret_cast<unsigned long long*>(sm + L::kColW);
+    int* pre = reinterpret_cast<int*>(sm + L::kPre);
     for (int i = tid; i < 2 * kRows; i += kThreads) tok_gs[i] = 0.f;
+    for (int tau = tid; tau < sh.nT; tau += kThreads) colw[tau] = tau > j ? col[tau] : 0ull;
     __syncthreads();
-    {
-        int cnt = 0;
-        for (int tau = j + 1 + tid; tau < sh.nT; tau += kThreads) cnt += __popcll(col[tau]);
-        cnt = __reduce_add_sync(0xffffffffu, cnt);
-        if (lane == 0 && cnt) atomicAdd(nc_slot, cnt);
+    if (warp == 0) {
+        const int per = (sh.nT + 31) / 32;       // consecutive tiles per lane
+        const int t0 = lane * per, t1 = min(t0 + per, sh.nT);
+        int sum = 0;
+        for (int tau = t0; tau < t1; ++tau) sum += __popcll(colw[tau]);
+        int inc = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (lane >= o) inc += y;
+        }
+        int run = kBS + inc - sum;
+        for (int tau = t0; tau < t1; ++tau) {
+            pre[tau] = run;
+            run += __popcll(colw[tau]);
+        }
+        if (lane == 31) *nc_slot = kBS + inc;
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -170,35 +191,26 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 tc::tma_load_2d(sm + L::kV + h * 8192, &tm_v, h * 64, kr, kv_full);
             }
         }
-        // token stream cursor (lane 0 only): the block's own tile, then the bitmap
-        int cur_tau = j;
-        uint64_t cur_w = ~0ull;
-        auto next_token = [&]() -> int {
-            while (cur_w == 0ull) {
-                if (++cur_tau >= sh.nT) return -1;
-                cur_w = col[cur_tau];
+        // token of stream index s: the block's own tile first, then the bitmap
+        auto token_at = [&](int s) -> int {
+            if (s < kBS) return j * kBS + s;
+            int lo = j + 1, hi = sh.nT - 1;      // last tile with pre[tile] <= s
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (pre[mid] <= s) lo = mid; else hi = mid - 1;
             }
-            const int bit = __ffsll((long long)cur_w) - 1;
-            cur_w &= cur_w - 1ull;
-            return cur_tau * kBS + bit;
+            uint64_t w = colw[lo];
+            for (int r = s - pre[lo]; r > 0; --r) w &= w - 1ull;
+            return lo * kBS + __ffsll((long long)w) - 1;
         };
-        if (L0 == 1 && lane == 0) for (int i = 0; i < tpc; ++i) next_token();   // skip chunk 0
+        int* qoff = reinterpret_cast<int*>(sm + L::kQoff) + L0 * kRows;
         for (int c = L0; c < nc; c += 2) {
             if (c >= 2 && !tc::warp_wait_bar(&st_empty[L0], (uint32_t)(((c >> 1) - 1) & 1), abort)) break;
-            if (lane == 0) {
-                int n = 0;
-                for (; n < tpc; ++n) {
-                    const int t = next_token();
-                    if (t < 0) break;
-                    meta.tok_t[n] = t;
-                }
-                *meta.ntok = n;
-                for (int i = 0; i < tpc; ++i) next_token();   // skip the other loader's chunk
-            }
-            __syncwarp();
-            const int n = *meta.ntok;
+            const int n = min(tpc, ntok_total - c * tpc);
+            if (lane == 0) *meta.ntok = n;
             for (int i = lane; i < n; i += 32) {
-                const int t = meta.tok_t[i];
+                const int t = token_at(c * tpc + i);
+                meta.tok_t[i] = t;
                 int slot = -1;
                 float lg = 0.f;
                 if ((t >> 6) != j) {
@@ -215,30 +227,31 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 meta.tok_slot[i] = slot;
                 meta.tok_lg[i] = lg;
             }
+            __syncwarp();
             for (int i = lane; i < kRows; i += 32) {
                 const int ti = i / G, h = i - ti * G;
                 float lse = 0.f, Dv = 0.f;
+                int qrow = -1;
                 if (ti < n) {
-                    const int64_t qrow = ((int64_t)b * sh.Hq + g * G + h) * T + meta.tok_t[ti];
+                    qrow = (int)(((int64_t)b * sh.Hq + g * G + h) * T + meta.tok_t[ti]);
                     lse = a.lse[qrow];
                     Dv = a.Dd[qrow];
                 }
                 meta.row_lse[i] = lse;
                 meta.row_D[i] = Dv;
+                qoff[i] = qrow;
             }
+            __syncwarp();
             // rows: one row per step, lanes 0-15 copy q, lanes 16-31 copy dO (16 x 16 B each)
             const int cc = lane & 15;
             unsigned char* dstb = (lane < 16 ? stq : stdo) + (cc >> 3) * 16384;
-            const __nv_bfloat16* srcb = lane < 16 ? a.q : a.dO;
+            const __nv_bfloat16* srcb = (lane < 16 ? a.q : a.dO) + cc * 8;
+#pragma unroll 4
             for (int i = 0; i < kRows; ++i) {
-                const int ti = i / G, h = i - ti * G;
+                const int qrow = qoff[i];
                 unsigned char* dst = dstb + tc::sw128_offset(i, (cc & 7) * 8);
-                if (ti < n) {
-                    const int64_t qrow = ((int64_t)b * sh.Hq + g * G + h) * T + meta.tok_t[ti];
-                    tc::cp_async16(dst, srcb + qrow * kD + cc * 8);
-                } else {
-                    *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-                }
+                if (qrow >= 0) tc::cp_async16(dst, srcb + (int64_t)qrow * kD);
+                else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
             }
             tc::cp_async_wait_all();
             tc::fence_async_shared();
@@ -432,7 +445,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
 
 bool bwd_tc_supported(const Shape& s) {
     return s.dtype == SAS_DT_BF16 && s.D == kD && s.bs == kBS && s.K <= 64 && s.G <= 8 && s.q_offset == 0 &&
-           s.T % kBS == 0 && (int64_t)s.B * s.Hq * s.T < ((int64_t)1 << 31);
+           s.T % kBS == 0 && s.nT <= 1024 && (int64_t)s.B * s.Hq * s.T < ((int64_t)1 << 31);
 }
 
 cudaError_t launch_bwd_tc(const Shape& s, const void* q, const void* k, const void* v, const void* dO,

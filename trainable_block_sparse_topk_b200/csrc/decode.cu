@@ -272,26 +272,46 @@ decode_partial_kernel(DecArgs a) {
     }
 }
 
-// Merge the splits of each (b, kv head): o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
+// Merge the splits of one (b, kv head, query head):
+//   o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s.
+// The split weights are formed once in shared memory; each thread then reads
+// its output column of every split with independent loads.
+constexpr int kMaxSplits = 1024;
+
 template <typename T, int D>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(128)
 decode_combine_kernel(Shape sh, const float* __restrict__ part, int splits, T* __restrict__ o) {
-    const int64_t bg = blockIdx.x;
+    __shared__ float w[kMaxSplits];
+    __shared__ float red[4];
     const int G = sh.G;
+    const int h = blockIdx.x % G;
+    const int64_t bg = blockIdx.x / G;
     const int b = (int)(bg / sh.Hkv), g = (int)(bg % sh.Hkv);
-    const float* base = part + bg * (int64_t)splits * G * (D + 2);
-    for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
-        const int h = e / D, d = e % D;
-        float M = -INFINITY;
-        for (int s = 0; s < splits; ++s) M = fmaxf(M, base[((int64_t)s * G + h) * (D + 2) + D]);
-        float L = 0.f, O = 0.f;
-        for (int s = 0; s < splits; ++s) {
-            const float* r = base + ((int64_t)s * G + h) * (D + 2);
-            const float w = r[D] == -INFINITY ? 0.f : exp2f(r[D] - M);
-            L = fmaf(w, r[D + 1], L);
-            O = fmaf(w, r[d], O);
-        }
-        o[((int64_t)b * sh.Hq + (int64_t)g * G + h) * D + d] = Elem<T>::from_f(O / L);
+    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+    auto rec = [&](int s) { return part + ((bg * splits + s) * G + h) * (int64_t)(D + 2); };
+    float m = -INFINITY;
+    for (int s = tid; s < splits; s += 128) m = fmaxf(m, rec(s)[D]);
+    m = warp_max(m);
+    if (lane == 0) red[wp] = m;
+    __syncthreads();
+    const float M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    __syncthreads();
+    float l = 0.f;
+    for (int s = tid; s < splits; s += 128) {
+        const float* r = rec(s);
+        const float ws = r[D] == -INFINITY ? 0.f : exp2f(r[D] - M);
+        w[s] = ws;
+        l = fmaf(ws, r[D + 1], l);
+    }
+    l = warp_sum(l);
+    if (lane == 0) red[wp] = l;
+    __syncthreads();
+    const float L = red[0] + red[1] + red[2] + red[3];
+    for (int d = tid; d < D; d += 128) {
+        float acc = 0.f;
+#pragma unroll 8
+        for (int s = 0; s < splits; ++s) acc = fmaf(w[s], rec(s)[d], acc);
+        o[((int64_t)b * sh.Hq + (int64_t)g * G + h) * D + d] = Elem<T>::from_f(acc / L);
     }
 }
 
@@ -306,8 +326,8 @@ cudaError_t run_decode(const DecArgs& a, cudaStream_t st) {
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launches(1);
-    decode_combine_kernel<T, D><<<(unsigned)(a.sh.B * a.sh.Hkv), 256, 0, st>>>(a.sh, a.part, a.splits,
-                                                                                static_cast<T*>(a.o));
+    decode_combine_kernel<T, D><<<(unsigned)(a.sh.B * a.sh.Hkv * a.sh.G), 128, 0, st>>>(a.sh, a.part, a.splits,
+                                                                                       static_cast<T*>(a.o));
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
     return e;
@@ -343,6 +363,7 @@ DecodePlan decode_plan(const Shape& s, bool dense) {
     const int64_t groups = (int64_t)s.B * s.Hkv;
     const int64_t target = 148 * 4;   // CTAs: a few per SM
     int64_t bpc = (groups * nblk + target - 1) / target;
+    bpc = std::max<int64_t>(bpc, (nblk + kMaxSplits - 1) / kMaxSplits);   // the merge takes <= kMaxSplits
     bpc = std::max<int64_t>(1, bpc);
     p.bpc = (int)bpc;
     p.splits = (int)((nblk + bpc - 1) / bpc);
