@@ -56,7 +56,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     with cf.ThreadPoolExecutor(max_workers=max(1, os.cpu_count() or 1)) as ex:
         objs = list(ex.map(lambda s: _compile(s, verbose), _sources()))
     tmp = LIB + f".tmp{os.getpid()}"
-    subprocess.check_call([NVCC, *ARCH, "-shared", "-o", tmp, *objs, "-lcuda"])
+    subprocess.check_call([NVCC, *ARCH, "-shared", "-o", tmp, *objs])
     os.replace(tmp, LIB)
     return LIB
 

@@ -129,7 +129,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         for (int i = 0; i < L::kNumBars; ++i) {
             uint64_t* bar = &bars[i];
             uint32_t cnt = 1;
-            if (bar == &st_full[0] || bar == &st_full[1]) cnt = 32;
+            if (bar == &st_full[0] || bar == &st_full[1]) cnt = 64;
             if (bar == p_full || bar == dq_empty) cnt = 4;
             mbar_init(bar, cnt);
         }
@@ -214,15 +214,15 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 int slot = -1;
                 float lg = 0.f;
                 if ((t >> 6) != j) {
+                    // slot of j in the row's ascending kept list = number of kept blocks below j
                     const int64_t row = (int64_t)bg * T + t;
                     const int32_t* ir = a.idx + row * K;
-                    int lo = 0, hi = a.nsel[row] - 1;
-                    while (lo < hi) {
-                        const int mid = (lo + hi) >> 1;
-                        if (ir[mid] < j) lo = mid + 1; else hi = mid;
-                    }
-                    slot = lo;
-                    lg = a.gl[row * K + lo];
+                    const int ns = a.nsel[row];
+                    int below = 0;
+#pragma unroll 8
+                    for (int s = 0; s < K; ++s) below += (s < ns && ir[s] < j) ? 1 : 0;
+                    slot = min(below, K - 1);
+                    lg = a.gl[row * K + slot];
                 }
                 meta.tok_slot[i] = slot;
                 meta.tok_lg[i] = lg;
@@ -253,9 +253,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 if (qrow >= 0) tc::cp_async16(dst, srcb + (int64_t)qrow * kD);
                 else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
             }
-            tc::cp_async_wait_all();
-            tc::fence_async_shared();
-            __syncwarp();
+            // st_full completes after 64 arrivals: each lane arrives once for its
+            // plain shared-memory stores now and once when its copies have landed.
+            tc::cp_async_mbar_arrive_noinc(&st_full[L0]);
             tc::mbar_arrive(&st_full[L0]);
         }
     } else if (warp == 1) {
@@ -281,11 +281,13 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 tc::mma_commit(&s_full[c & 1]);
             };
             bool ok = tc::wait_bar(kv_full, 0u, abort) && tc::wait_bar(&st_full[0], 0u, abort);
+            tc::fence_async_shared();   // rows written by cp.async / plain stores -> MMA operand reads
             tc::fence_after_sync();
             if (ok) issue_sdp(0);
             for (int c = 0; ok && c < nc; ++c) {
                 if (c + 1 < nc) {
                     if (!tc::wait_bar(&st_full[(c + 1) & 1], (uint32_t)(((c + 1) >> 1) & 1), abort)) break;
+                    tc::fence_async_shared();
                     tc::fence_after_sync();
                     issue_sdp(c + 1);
                 }
