@@ -23,8 +23,8 @@
 // build P/dS of chunk c and read back dQ of chunk c-1.
 //
 // Roles (256 threads): warps 0 and 3 gather chunk rows (even / odd chunks)
-// with 16-byte cp.async into the two 128-byte-swizzled Q/dO stages (warp 0
-// also loads K_j, V_j by TMA), warp 1 lane 0 issues the MMAs, warp 2 owns the
+// with TMA tile::gather4 loads into the two 128-byte-swizzled Q/dO stages
+// (warp 0 also loads K_j, V_j by TMA), warp 1 lane 0 issues the MMAs, warp 2 owns the
 // TMEM allocation, warps 4-7 compute. No TMA multicast is used.
 #include <cuda.h>
 
@@ -44,6 +44,8 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColDQ = 256, kColDV = 384, kColDK = 448;
 
 struct BwdTcArgs {
+    CUtensorMap tm_q;    // q  [B*Hq*T, d], one-row boxes of 64 columns, 128-byte swizzle (gather4)
+    CUtensorMap tm_do;   // dO, same
     Shape sh;
     const __nv_bfloat16* q;
     const __nv_bfloat16* dO;
@@ -96,13 +98,14 @@ struct Meta {
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
-bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, BwdTcArgs a) {
+bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+              const __grid_constant__ BwdTcArgs a) {
     using L = BwdSmem;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
     uint64_t* kv_full = bars + 0;
-    uint64_t* st_full = bars + 1;     // [2], 32 arrivals (the loader warp)
+    uint64_t* st_full = bars + 1;     // [2], the loader's arrive + the gather bytes
     uint64_t* st_empty = bars + 3;    // [2]
     uint64_t* s_full = bars + 5;      // [2]
     uint64_t* p_full = bars + 7;      // 4 arrivals (compute warps)
@@ -129,7 +132,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         for (int i = 0; i < L::kNumBars; ++i) {
             uint64_t* bar = &bars[i];
             uint32_t cnt = 1;
-            if (bar == &st_full[0] || bar == &st_full[1]) cnt = 64;
+            if (bar == &st_full[0] || bar == &st_full[1]) cnt = 1;   // the loader's arrive.expect_tx
             if (bar == p_full || bar == dq_empty) cnt = 4;
             mbar_init(bar, cnt);
         }
@@ -242,21 +245,25 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 qoff[i] = qrow;
             }
             __syncwarp();
-            // rows: one row per step, lanes 0-15 copy q, lanes 16-31 copy dO (16 x 16 B each)
-            const int cc = lane & 15;
-            unsigned char* dstb = (lane < 16 ? stq : stdo) + (cc >> 3) * 16384;
-            const __nv_bfloat16* srcb = (lane < 16 ? a.q : a.dO) + cc * 8;
-#pragma unroll 4
-            for (int i = 0; i < kRows; ++i) {
-                const int qrow = qoff[i];
-                unsigned char* dst = dstb + tc::sw128_offset(i, (cc & 7) * 8);
-                if (qrow >= 0) tc::cp_async16(dst, srcb + (int64_t)qrow * kD);
-                else *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+            // rows: TMA gather of 4 rows x 64 columns per instruction; lane l
+            // fetches rows 4l..4l+3 of both d halves of q and dO. Padding rows
+            // re-read the chunk's first row (their P and dS are zero).
+            if (lane == 0) mbar_arrive_expect_tx(&st_full[L0], 65536u);
+            __syncwarp();
+            {
+                int rr[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int qrow = qoff[4 * lane + e];
+                    rr[e] = qrow >= 0 ? qrow : qoff[0];
+                }
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const uint32_t off = hh * 16384 + 4 * lane * 128;
+                    tc::tma_gather4(stq + off, &a.tm_q, hh * 64, rr, &st_full[L0]);
+                    tc::tma_gather4(stdo + off, &a.tm_do, hh * 64, rr, &st_full[L0]);
+                }
             }
-            // st_full completes after 64 arrivals: each lane arrives once for its
-            // plain shared-memory stores now and once when its copies have landed.
-            tc::cp_async_mbar_arrive_noinc(&st_full[L0]);
-            tc::mbar_arrive(&st_full[L0]);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------- MMA issuer ---
@@ -454,14 +461,16 @@ cudaError_t launch_bwd_tc(const Shape& s, const void* q, const void* k, const vo
                           const float* lse, const float* Dd, const int32_t* idx, const float* gl,
                           const int32_t* nsel, const uint64_t* maskT, float* dq_acc, void* dk, void* dv,
                           float* gsum, cudaStream_t st) {
-    CUtensorMap mk, mv;
+    CUtensorMap mk, mv, mq, mdo;
     if (!encode_bf16_2d(&mk, k, (uint64_t)s.B * s.Hkv * s.T, kD, kBS) ||
-        !encode_bf16_2d(&mv, v, (uint64_t)s.B * s.Hkv * s.T, kD, kBS))
+        !encode_bf16_2d(&mv, v, (uint64_t)s.B * s.Hkv * s.T, kD, kBS) ||
+        !encode_bf16_2d(&mq, q, (uint64_t)s.B * s.Hq * s.T, kD, 1) ||
+        !encode_bf16_2d(&mdo, dO, (uint64_t)s.B * s.Hq * s.T, kD, 1))
         return cudaErrorInvalidValue;
     const size_t smem = BwdSmem::kTotal + 1024;
     cudaError_t e = cudaFuncSetAttribute(bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    BwdTcArgs a{s, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dO), lse, Dd, idx, gl, nsel,
+    BwdTcArgs a{mq, mdo, s, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dO), lse, Dd, idx, gl, nsel,
                 maskT, dq_acc, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), gsum, kRows / s.G};
     const int64_t grid = (int64_t)s.B * s.Hkv * s.nT;
     bwd_tc_kernel<<<(unsigned)grid, kThreads, smem, st>>>(mk, mv, a);
