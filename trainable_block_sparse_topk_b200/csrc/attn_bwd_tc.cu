@@ -69,13 +69,12 @@ struct BwdSmem {
     static constexpr uint32_t kStageBytes = 65536;
     static constexpr uint32_t kP = kStage + 2 * kStageBytes;   // P  [128 x 128 B]
     static constexpr uint32_t kDS = kP + 16384;                // dS [128 x 128 B]
-    static constexpr uint32_t kMeta = kDS + 16384;             // 2 x per-chunk metadata
-    static constexpr uint32_t kMetaBytes = 5 * 512 + 16;       // tok_t, tok_slot, tok_lg, row_lse, row_D, ntok
-    static constexpr uint32_t kGs = kMeta + 2 * kMetaBytes;    // per-token Gsum [2][128] f32
+    static constexpr uint32_t kMeta = kDS + 16384;             // 4 x per-chunk metadata (chunk c -> slot c & 3)
+    static constexpr uint32_t kMetaBytes = 6 * 512 + 16;       // tok_t, tok_slot, tok_lg, row_lse, row_D, qoff, ntok
+    static constexpr uint32_t kGs = kMeta + 4 * kMetaBytes;    // per-token Gsum [2][128] f32
     static constexpr uint32_t kColW = kGs + 1024;              // u64 [kMaxNT]: the block's bitmap column
     static constexpr uint32_t kPre = kColW + 8 * 1024;         // i32 [kMaxNT]: stream index of tile tau's first token
-    static constexpr uint32_t kQoff = kPre + 4 * 1024;         // i32 [2][128]: q/dO row of each chunk row (-1: pad)
-    static constexpr uint32_t kBar = kQoff + 2 * 4 * kRows;
+    static constexpr uint32_t kBar = kPre + 4 * 1024;
     static constexpr int kNumBars = 13;
     static constexpr uint32_t kMisc = kBar + 8 * kNumBars;     // tmem base, chunk count, abort
     static constexpr uint32_t kTotal = kMisc + 16;
@@ -87,6 +86,7 @@ struct Meta {
     float* tok_lg;
     float* row_lse;
     float* row_D;
+    int* qoff;     // q/dO row of each chunk row, -1 for padding
     int* ntok;
     __device__ explicit Meta(unsigned char* p)
         : tok_t(reinterpret_cast<int*>(p)),
@@ -94,7 +94,8 @@ struct Meta {
           tok_lg(reinterpret_cast<float*>(p + 1024)),
           row_lse(reinterpret_cast<float*>(p + 1536)),
           row_D(reinterpret_cast<float*>(p + 2048)),
-          ntok(reinterpret_cast<int*>(p + 2560)) {}
+          qoff(reinterpret_cast<int*>(p + 2560)),
+          ntok(reinterpret_cast<int*>(p + 3072)) {}
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -183,7 +184,6 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         const int L0 = warp == 0 ? 0 : 1;           // this warp fills chunks c = L0, L0 + 2, ...
         unsigned char* stq = sm + L::kStage + L0 * L::kStageBytes;
         unsigned char* stdo = stq + 32768;
-        Meta meta(sm + L::kMeta + L0 * L::kMetaBytes);
         if (warp == 0 && lane == 0) {
             tc::prefetch_tmap(&tm_k);
             tc::prefetch_tmap(&tm_v);
@@ -206,9 +206,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             for (int r = s - pre[lo]; r > 0; --r) w &= w - 1ull;
             return lo * kBS + __ffsll((long long)w) - 1;
         };
-        int* qoff = reinterpret_cast<int*>(sm + L::kQoff) + L0 * kRows;
-        for (int c = L0; c < nc; c += 2) {
-            if (c >= 2 && !tc::warp_wait_bar(&st_empty[L0], (uint32_t)(((c >> 1) - 1) & 1), abort)) break;
+        // metadata of chunk c into ring slot c & 3 (global loads only; no stage needed)
+        auto prep = [&](int c) {
+            Meta meta(sm + L::kMeta + (c & 3) * L::kMetaBytes);
             const int n = min(tpc, ntok_total - c * tpc);
             if (lane == 0) *meta.ntok = n;
             for (int i = lane; i < n; i += 32) {
@@ -242,12 +242,17 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 }
                 meta.row_lse[i] = lse;
                 meta.row_D[i] = Dv;
-                qoff[i] = qrow;
+                meta.qoff[i] = qrow;
             }
             __syncwarp();
+        };
+        if (L0 < nc) prep(L0);
+        for (int c = L0; c < nc; c += 2) {
+            if (c >= 2 && !tc::warp_wait_bar(&st_empty[L0], (uint32_t)(((c >> 1) - 1) & 1), abort)) break;
             // rows: TMA gather of 4 rows x 64 columns per instruction; lane l
             // fetches rows 4l..4l+3 of both d halves of q and dO. Padding rows
             // re-read the chunk's first row (their P and dS are zero).
+            const int* qoff = Meta(sm + L::kMeta + (c & 3) * L::kMetaBytes).qoff;
             if (lane == 0) mbar_arrive_expect_tx(&st_full[L0], 65536u);
             __syncwarp();
             {
@@ -264,6 +269,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                     tc::tma_gather4(stdo + off, &a.tm_do, hh * 64, rr, &st_full[L0]);
                 }
             }
+            if (c + 2 < nc) prep(c + 2);   // overlaps the wait for this stage's next release
         }
     } else if (warp == 1) {
         // ------------------------------------------------------- MMA issuer ---
@@ -288,36 +294,60 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 tc::mma_commit(&s_full[c & 1]);
             };
             bool ok = tc::wait_bar(kv_full, 0u, abort) && tc::wait_bar(&st_full[0], 0u, abort);
-            tc::fence_async_shared();   // rows written by cp.async / plain stores -> MMA operand reads
             tc::fence_after_sync();
             if (ok) issue_sdp(0);
-            for (int c = 0; ok && c < nc; ++c) {
-                if (c + 1 < nc) {
-                    if (!tc::wait_bar(&st_full[(c + 1) & 1], (uint32_t)(((c + 1) >> 1) & 1), abort)) break;
-                    tc::fence_async_shared();
+            // Issue whichever step is ready: S/dP of the next chunk (TMEM double
+            // buffer: at most one chunk ahead), dV/dK of the current chunk once
+            // its P/dS are in shared memory, then its dQ once the previous dQ
+            // has been read back.
+            int sdp_next = 1, c = 0;
+            bool kv_issued = false;
+            uint64_t t0 = global_ns();
+            while (ok && c < nc) {
+                bool progressed = false;
+                if (sdp_next < nc && sdp_next <= c + 1 &&
+                    mbar_test_wait(&st_full[sdp_next & 1], (uint32_t)((sdp_next >> 1) & 1))) {
                     tc::fence_after_sync();
-                    issue_sdp(c + 1);
+                    issue_sdp(sdp_next);
+                    ++sdp_next;
+                    progressed = true;
                 }
-                if (!tc::wait_bar(p_full, (uint32_t)(c & 1), abort)) break;
-                tc::fence_after_sync();
-                const uint32_t qa = sbase + L::kStage + (c & 1) * L::kStageBytes, doa = qa + 32768;
+                if (!kv_issued && mbar_test_wait(p_full, (uint32_t)(c & 1))) {
+                    tc::fence_after_sync();
+                    const uint32_t qa = sbase + L::kStage + (c & 1) * L::kStageBytes, doa = qa + 32768;
 #pragma unroll
-                for (int kk = 0; kk < kRows / 16; ++kk) {
-                    const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
-                    tc::mma_ss(tmem + kColDV, tc::smem_desc_sw128(doa + kk * 2048, 16384, 1024),
-                               tc::smem_desc_sw128(pa + kk * 2048, 16384, 1024), id_kv, acc);
-                    tc::mma_ss(tmem + kColDK, tc::smem_desc_sw128(qa + kk * 2048, 16384, 1024),
-                               tc::smem_desc_sw128(dsa + kk * 2048, 16384, 1024), id_kv, acc);
+                    for (int kk = 0; kk < kRows / 16; ++kk) {
+                        const uint32_t acc = (c > 0 || kk > 0) ? 1u : 0u;
+                        tc::mma_ss(tmem + kColDV, tc::smem_desc_sw128(doa + kk * 2048, 16384, 1024),
+                                   tc::smem_desc_sw128(pa + kk * 2048, 16384, 1024), id_kv, acc);
+                        tc::mma_ss(tmem + kColDK, tc::smem_desc_sw128(qa + kk * 2048, 16384, 1024),
+                                   tc::smem_desc_sw128(dsa + kk * 2048, 16384, 1024), id_kv, acc);
+                    }
+                    tc::mma_commit(&st_empty[c & 1]);   // the stage's Q and dO are no longer needed
+                    kv_issued = true;
+                    progressed = true;
                 }
-                if (c >= 1 && !tc::wait_bar(dq_empty, (uint32_t)((c - 1) & 1), abort)) break;
-                tc::fence_after_sync();
+                if (kv_issued && (c == 0 || mbar_test_wait(dq_empty, (uint32_t)((c - 1) & 1)))) {
+                    tc::fence_after_sync();
 #pragma unroll
-                for (int kk = 0; kk < kBS / 16; ++kk)
-                    tc::mma_ss(tmem + kColDQ, tc::smem_desc_sw128(dsa + kk * 32, 16, 1024),
-                               tc::smem_desc_sw128(ka + kk * 2048, 8192, 1024), id_dq, kk > 0);
-                tc::mma_commit(dq_full);
-                tc::mma_commit(&st_empty[c & 1]);
-                tc::mma_commit(p_empty);
+                    for (int kk = 0; kk < kBS / 16; ++kk)
+                        tc::mma_ss(tmem + kColDQ, tc::smem_desc_sw128(dsa + kk * 32, 16, 1024),
+                                   tc::smem_desc_sw128(ka + kk * 2048, 8192, 1024), id_dq, kk > 0);
+                    tc::mma_commit(dq_full);
+                    tc::mma_commit(p_empty);
+                    ++c;
+                    kv_issued = false;
+                    progressed = true;
+                }
+                if (progressed) {
+                    t0 = global_ns();
+                } else if (*abort) {
+                    ok = false;
+                } else if (global_ns() - t0 > 1000000000ull) {
+                    *abort = 1;
+                    atomicAdd(&g_sas_wait_timeouts, 1u);
+                    ok = false;
+                }
             }
             tc::mma_commit(done);
         }
@@ -353,7 +383,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         for (int c = 0; c < nc; ++c) {
             const int st = c & 1;
             if (!tc::warp_wait_bar(&st_full[st], (uint32_t)((c >> 1) & 1), abort)) { ok = false; break; }
-            Meta meta(sm + L::kMeta + st * L::kMetaBytes);
+            Meta meta(sm + L::kMeta + (c & 3) * L::kMetaBytes);
             const int n = *meta.ntok;
             const int ti = r / G, h = r - ti * G;
             const bool valid = ti < n;
