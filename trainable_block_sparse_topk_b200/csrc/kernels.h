@@ -49,7 +49,14 @@ cudaError_t launch_bwd_tc(const Shape& s, const void* q, const void* k, const vo
                           const int32_t* n_sel, const uint64_t* maskT, float* dq_acc, void* dk, void* dv,
                           float* gsum, cudaStream_t st);
 
-// Tensor-core forward (tcgen05 + TMA): bf16, d = 128, block 64.
+// Tensor-core forward over gathered rows (two passes + finalize): bf16, d = 128, block 64.
+bool fwd_rows_supported(const Shape& s);
+size_t fwd_rows_ws_bytes(const Shape& s);
+cudaError_t launch_fwd_rows(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
+                            const float* gate_logit, const int32_t* n_sel, const uint64_t* maskT, void* ws, void* o,
+                            float* attn_lse, cudaStream_t st);
+
+// Tensor-core forward over query tiles (union of the tile's selections): bf16, d = 128, block 64.
 bool fwd_tc_supported(const Shape& s);
 cudaError_t launch_fwd_tc(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
                           const float* gate_logit, const int32_t* n_sel, void* o, float* attn_lse, cudaStream_t st);

@@ -18,11 +18,19 @@ namespace sas {
 cudaError_t read_decode_timeouts(unsigned int* out);
 cudaError_t read_fwd_tc_timeouts(unsigned int* out);
 cudaError_t read_bwd_tc_timeouts(unsigned int* out);
+cudaError_t read_fwd_rows_timeouts(unsigned int* out);
 
 // SAS_FORCE_SIMT=1 routes bf16 training calls to the CUDA-core kernels (a
 // second GPU implementation, used to cross-check the tensor-core path).
 static bool force_simt() {
     const char* e = std::getenv("SAS_FORCE_SIMT");
+    return e != nullptr && e[0] == '1';
+}
+
+// SAS_FWD_UNION=1 routes the bf16 forward to the query-tile kernel instead of
+// the gathered-row kernels (the two compute the same result; used to cross-check).
+static bool fwd_union() {
+    const char* e = std::getenv("SAS_FWD_UNION");
     return e != nullptr && e[0] == '1';
 }
 
@@ -94,10 +102,17 @@ TrainWs bwd_layout(const Shape& s) {
     return w;
 }
 
+// Forward workspace: column bitmap, then the gathered-row kernels' row
+// statistics and fp32 output accumulator.
+size_t fwd_ws_bytes(const Shape& s) {
+    if (!fwd_rows_supported(s)) return 0;
+    return align256(sizeof(uint64_t) * (size_t)s.B * s.Hkv * s.NB * s.nT) + align256(fwd_rows_ws_bytes(s));
+}
+
 size_t ws_bytes(int op, const Shape& s) {
     switch (op) {
         case SAS_OP_TOPK: return 0;
-        case SAS_OP_FWD: return 0;
+        case SAS_OP_FWD: return fwd_ws_bytes(s);
         case SAS_OP_BWD: return bwd_layout(s).total;
         case SAS_OP_DECODE: return align256(decode_ws_bytes(s));
         default: return 0;
@@ -177,6 +192,14 @@ sas_status sas_gated_attn_fwd(const sas_desc* desc, const void* q, const void* k
     if (need > 0 && (ws == nullptr || ws_bytes_ < need)) return SAS_ERR_WORKSPACE;
     if (ws && !aligned16(ws)) return SAS_ERR_MISALIGNED;
     cudaStream_t cs = (cudaStream_t)stream;
+    if (fwd_rows_supported(s) && !force_simt() && !fwd_union()) {
+        unsigned char* w = static_cast<unsigned char*>(ws);
+        uint64_t* maskT = reinterpret_cast<uint64_t*>(w);
+        void* rows_ws = w + align256(sizeof(uint64_t) * (size_t)s.B * s.Hkv * s.NB * s.nT);
+        cudaError_t e = launch_sel_bitmap_T(s, idx, n_sel, maskT, cs);
+        if (e == cudaSuccess) e = launch_fwd_rows(s, q, k, v, idx, gate_logit, n_sel, maskT, rows_ws, o, attn_lse, cs);
+        return cuda_status(e);
+    }
     if (fwd_tc_supported(s) && !force_simt())
         return cuda_status(launch_fwd_tc(s, q, k, v, idx, gate_logit, n_sel, o, attn_lse, cs));
     return cuda_status(launch_fwd_simt(s, q, k, v, idx, gate_logit, n_sel, o, attn_lse, cs));
@@ -239,12 +262,13 @@ uint64_t sas_kernel_launches(void) { return g_launches.load(std::memory_order_re
 // library was loaded (0 in normal operation). Synchronises the device.
 sas_status sas_device_timeouts(uint32_t* count) {
     if (!count) return SAS_ERR_INVALID_ARG;
-    unsigned int c0 = 0, c1 = 0, c2 = 0;
+    unsigned int c0 = 0, c1 = 0, c2 = 0, c3 = 0;
     cudaError_t e = read_decode_timeouts(&c0);
     if (e == cudaSuccess) e = read_fwd_tc_timeouts(&c1);
     if (e == cudaSuccess) e = read_bwd_tc_timeouts(&c2);
+    if (e == cudaSuccess) e = read_fwd_rows_timeouts(&c3);
     if (e != cudaSuccess) return SAS_ERR_CUDA;
-    *count = c0 + c1 + c2;
+    *count = c0 + c1 + c2 + c3;
     return SAS_OK;
 }
 
