@@ -98,7 +98,7 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
     uint64_t* kv_full = bars + 0;
     uint64_t* st_full = bars + 1;     // [2]: the loader's arrive + the gather bytes
-    uint64_t* st_empty = bars + 3;    // [2]
+    uint64_t* st_empty = bars + 3;    // [2] MMA commit + 4 compute-warp arrivals
     uint64_t* s_full = bars + 5;      // [2]
     uint64_t* s_empty = bars + 7;     // [2] pass A: 4 arrivals (compute warps)
     uint64_t* p_full = bars + 9;      // pass B: 4 arrivals
@@ -127,6 +127,10 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             uint32_t cnt = 1;
             if (bar == &s_empty[0] || bar == &s_empty[1] || bar == p_full || bar == &o_empty[0] || bar == &o_empty[1])
                 cnt = 4;
+            // a stage is refilled only after the MMA has read its rows and the
+            // compute warps have waited for it: its phases then cannot run two
+            // ahead of any waiter
+            if (bar == &st_empty[0] || bar == &st_empty[1]) cnt = 5;
             mbar_init(bar, cnt);
         }
         *abort = 0;
@@ -354,6 +358,8 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 m = meta.row_m[r];
                 qrow = meta.qoff[r];
             }
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&st_empty[st]);
             if (!tc::warp_wait_bar(&s_full[st], (uint32_t)((c >> 1) & 1), abort)) { ok = false; break; }
             tc::fence_after_sync();
             uint32_t sv[kBS];
