@@ -269,20 +269,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                     tc::tma_gather4(stdo + off, &a.tm_do, hh * 64, rr, &st_full[L0]);
                 }
             }
-            if (c + 2 < nc) {
-                // metadata of this warp's next chunk, and an L2 prefetch of its rows so
-                // that its gather, one stage cycle later, reads from L2
-                prep(c + 2);
-                const int* q2 = Meta(sm + L::kMeta + ((c + 2) & 3) * L::kMetaBytes).qoff;
-                int rr[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) rr[e] = q2[4 * lane + e] >= 0 ? q2[4 * lane + e] : q2[0];
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    tc::tma_prefetch_gather4(&a.tm_q, hh * 64, rr);
-                    tc::tma_prefetch_gather4(&a.tm_do, hh * 64, rr);
-                }
-            }   // overlaps the wait for this stage's next release
+            if (c + 2 < nc) prep(c + 2);   // overlaps the wait for this stage's next release
         }
     } else if (warp == 1) {
         // ------------------------------------------------------- MMA issuer ---

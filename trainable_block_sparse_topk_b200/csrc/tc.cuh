@@ -38,14 +38,6 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, i
         : "memory");
 }
 
-// L2 prefetch of the four rows a tma_gather4 with the same arguments would read.
-__device__ __forceinline__ void tma_prefetch_gather4(const CUtensorMap* map, int x, const int* y) {
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile::gather4 [%0, {%1, %2, %3, %4, %5}];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(x), "r"(y[0]), "r"(y[1]), "r"(y[2]), "r"(y[3])
-                 : "memory");
-}
-
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
