@@ -112,10 +112,9 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const Shape& sh = a.sh;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = sh.G, K = sh.K, T = sh.T;
-    // group-major order: resident CTAs share one (batch, KV group), whose q/dO
-    // rows then stay in L2 while its key blocks gather them; heavy blocks first
-    const int j = (int)(blockIdx.x % sh.nT);
-    const int bg = (int)(blockIdx.x / sh.nT);
+    const int ngroups = sh.B * sh.Hkv;
+    const int j = (int)(blockIdx.x / ngroups);
+    const int bg = (int)(blockIdx.x % ngroups);
     const int b = bg / sh.Hkv, g = bg % sh.Hkv;
     const int tpc = a.tpc;
     const uint64_t* col = a.maskT + ((int64_t)bg * sh.NB + j) * sh.nT;
