@@ -36,7 +36,7 @@ namespace sas {
 
 namespace {
 
-constexpr int kThreads = 384;   // 4 service warps + 8 compute warps
+constexpr int kThreads = 256;
 constexpr int kBS = 64;
 constexpr int kRows = 128;
 constexpr int kD = 128;
@@ -109,10 +109,10 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     uint64_t* st_full = bars + 1;     // [2], the loader's arrive + the gather bytes
     uint64_t* st_empty = bars + 3;    // [2]
     uint64_t* s_full = bars + 5;      // [2]
-    uint64_t* p_full = bars + 7;      // 8 arrivals (compute warps)
+    uint64_t* p_full = bars + 7;      // 4 arrivals (compute warps)
     uint64_t* p_empty = bars + 8;
     uint64_t* dq_full = bars + 9;
-    uint64_t* dq_empty = bars + 10;   // 8 arrivals
+    uint64_t* dq_empty = bars + 10;   // 4 arrivals
     uint64_t* done = bars + 11;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMisc);
     int* nc_slot = reinterpret_cast<int*>(sm + L::kMisc + 4);
@@ -134,7 +134,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             uint64_t* bar = &bars[i];
             uint32_t cnt = 1;
             if (bar == &st_full[0] || bar == &st_full[1]) cnt = 1;   // the loader's arrive.expect_tx
-            if (bar == p_full || bar == dq_empty) cnt = 8;
+            if (bar == p_full || bar == dq_empty) cnt = 4;
             mbar_init(bar, cnt);
         }
         *nc_slot = kBS;   // the block's own tokens; later tiles are added below
@@ -353,10 +353,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         }
     } else if (warp >= 4) {
         // ----------------------------------------------------- compute warps ---
-        // warp w covers TMEM lanes 32 (w % 4) .. + 31 (rows) and half (w - 4) / 4
-        // of the block's 64 keys and of dQ's d columns
-        const int r = (warp & 3) * 32 + lane;      // chunk row == TMEM lane
-        const int half = (warp - 4) >> 2;
+        const int r = (warp - 4) * 32 + lane;      // chunk row == TMEM lane
         const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const float qk = sh.scale * kLog2e;
         const float dscale = sh.scale;
@@ -366,7 +363,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             if (!tc::warp_wait_bar(dq_full, (uint32_t)(c & 1), abort)) return false;
             tc::fence_after_sync();
 #pragma unroll 1
-            for (int cb = half * (kD / 32); cb < (half + 1) * (kD / 32); ++cb) {
+            for (int cb = 0; cb < kD / 16; ++cb) {
                 uint32_t v[16];
                 tc::tmem_ld16(lane_base + kColDQ + cb * 16, v);
                 tc::tmem_wait_ld();
@@ -405,21 +402,19 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             const int64_t dq_row = valid ? ((int64_t)b * sh.Hq + g * G + h) * T + t : -1;
             if (!tc::warp_wait_bar(&s_full[st], (uint32_t)((c >> 1) & 1), abort)) { ok = false; break; }
             tc::fence_after_sync();
-            constexpr int kH = kBS / 2;            // keys per half
-            const int k0 = half * kH;
-            uint32_t sv[kH], pv[kH];
+            uint32_t sv[kBS], pv[kBS];
 #pragma unroll
-            for (int cb = 0; cb < kH / 16; ++cb) {
-                tc::tmem_ld16(lane_base + (uint32_t)(st * 128 + k0 + cb * 16), sv + cb * 16);
-                tc::tmem_ld16(lane_base + (uint32_t)(st * 128 + 64 + k0 + cb * 16), pv + cb * 16);
+            for (int cb = 0; cb < kBS / 16; ++cb) {
+                tc::tmem_ld16(lane_base + (uint32_t)(st * 128 + cb * 16), sv + cb * 16);
+                tc::tmem_ld16(lane_base + (uint32_t)(st * 128 + 64 + cb * 16), pv + cb * 16);
             }
             tc::tmem_wait_ld();
-            uint32_t pk[kH / 2], dk2[kH / 2];
+            uint32_t pk[kBS / 2], dk2[kBS / 2];
             float rowsum = 0.f;
 #pragma unroll
-            for (int k = 0; k < kH; k += 2) {
-                const float p0 = (k0 + k <= kmax) ? exp2f(fmaf(__uint_as_float(sv[k]), qk, bias)) : 0.f;
-                const float p1 = (k0 + k + 1 <= kmax) ? exp2f(fmaf(__uint_as_float(sv[k + 1]), qk, bias)) : 0.f;
+            for (int k = 0; k < kBS; k += 2) {
+                const float p0 = (k <= kmax) ? exp2f(fmaf(__uint_as_float(sv[k]), qk, bias)) : 0.f;
+                const float p1 = (k + 1 <= kmax) ? exp2f(fmaf(__uint_as_float(sv[k + 1]), qk, bias)) : 0.f;
                 const float d0 = p0 * (__uint_as_float(pv[k]) - Dv);
                 const float d1 = p1 * (__uint_as_float(pv[k + 1]) - Dv);
                 rowsum += d0 + d1;
@@ -431,8 +426,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             // Gsum of the token: its G rows are in this chunk
             float* gs = tok_gs + st * kRows;
             if (valid && !diag) atomicAdd(&gs[ti], rowsum);
-            tc::named_bar(1, 256);
-            if (half == 0 && r < n) {
+            tc::named_bar(1, 128);
+            if (r < n) {
                 const int slot = meta.tok_slot[r];
                 if (slot >= 0) a.gsum[((int64_t)bg * T + meta.tok_t[r]) * K + slot] = gs[r];
                 gs[r] = 0.f;
@@ -440,8 +435,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             // P and dS of chunk c-1 must have been consumed by its MMAs
             if (c >= 1 && !tc::warp_wait_bar(p_empty, (uint32_t)((c - 1) & 1), abort)) { ok = false; break; }
 #pragma unroll
-            for (int cb = 0; cb < kH / 8; ++cb) {
-                const uint32_t off = tc::sw128_offset(r, k0 + cb * 8);
+            for (int cb = 0; cb < kBS / 8; ++cb) {
+                const uint32_t off = tc::sw128_offset(r, cb * 8);
                 asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sbase + L::kP + off), "r"(pk[cb * 4]),
                              "r"(pk[cb * 4 + 1]), "r"(pk[cb * 4 + 2]), "r"(pk[cb * 4 + 3])
                              : "memory");
@@ -463,7 +458,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             __nv_bfloat16* dvb = a.dv + ((int64_t)bg * T + (int64_t)j * kBS) * kD;
             __nv_bfloat16* dkb = a.dk + ((int64_t)bg * T + (int64_t)j * kBS) * kD;
 #pragma unroll 1
-            for (int cb = half * (kBS / 32); cb < (half + 1) * (kBS / 32); ++cb) {
+            for (int cb = 0; cb < kBS / 16; ++cb) {
                 uint32_t vv[16], kv[16];
                 tc::tmem_ld16(lane_base + kColDV + cb * 16, vv);
                 tc::tmem_ld16(lane_base + kColDK + cb * 16, kv);

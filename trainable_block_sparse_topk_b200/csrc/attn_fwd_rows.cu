@@ -34,7 +34,7 @@ namespace sas {
 
 namespace {
 
-constexpr int kThreads = 384;   // 4 service warps + 8 compute warps
+constexpr int kThreads = 256;
 constexpr int kBS = 64;
 constexpr int kRows = 128;
 constexpr int kD = 128;
@@ -98,13 +98,13 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
     uint64_t* kv_full = bars + 0;
     uint64_t* st_full = bars + 1;     // [2]: the loader's arrive + the gather bytes
-    uint64_t* st_empty = bars + 3;    // [2] MMA commit + 8 compute-warp arrivals
+    uint64_t* st_empty = bars + 3;    // [2] MMA commit + 4 compute-warp arrivals
     uint64_t* s_full = bars + 5;      // [2]
-    uint64_t* s_empty = bars + 7;     // [2] pass A: 8 arrivals (compute warps)
-    uint64_t* p_full = bars + 9;      // pass B: 8 arrivals
+    uint64_t* s_empty = bars + 7;     // [2] pass A: 4 arrivals (compute warps)
+    uint64_t* p_full = bars + 9;      // pass B: 4 arrivals
     uint64_t* p_empty = bars + 10;
     uint64_t* o_full = bars + 11;     // [2]
-    uint64_t* o_empty = bars + 13;    // [2] 8 arrivals
+    uint64_t* o_empty = bars + 13;    // [2] 4 arrivals
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMisc);
     int* ntok_slot = reinterpret_cast<int*>(sm + L::kMisc + 4);
     volatile int* abort = reinterpret_cast<volatile int*>(sm + L::kMisc + 8);
@@ -126,11 +126,11 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             uint64_t* bar = &bars[i];
             uint32_t cnt = 1;
             if (bar == &s_empty[0] || bar == &s_empty[1] || bar == p_full || bar == &o_empty[0] || bar == &o_empty[1])
-                cnt = 8;
+                cnt = 4;
             // a stage is refilled only after the MMA has read its rows and the
             // compute warps have waited for it: its phases then cannot run two
             // ahead of any waiter
-            if (bar == &st_empty[0] || bar == &st_empty[1]) cnt = 9;
+            if (bar == &st_empty[0] || bar == &st_empty[1]) cnt = 5;
             mbar_init(bar, cnt);
         }
         *abort = 0;
@@ -314,12 +314,7 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         }
     } else if (warp >= 4) {
         // ----------------------------------------------------- compute warps ---
-        // warp w covers TMEM lanes 32 (w % 4) .. + 31 (rows) and half (w - 4) / 4
-        // of the block's 64 keys and of O's d columns
-        const int r = (warp & 3) * 32 + lane;      // chunk row == TMEM lane
-        const int half = (warp - 4) >> 2;
-        constexpr int kH = kBS / 2;
-        const int k0 = half * kH;
+        const int r = (warp - 4) * 32 + lane;      // chunk row == TMEM lane
         const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const float qk = sh.scale * kLog2e;
         bool ok = true;
@@ -329,7 +324,7 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             tc::fence_after_sync();
             const uint32_t col0 = 128 + (uint32_t)((c & 1) * kD);
 #pragma unroll 1
-            for (int cb = half * (kD / 32); cb < (half + 1) * (kD / 32); ++cb) {
+            for (int cb = 0; cb < kD / 16; ++cb) {
                 uint32_t v[16];
                 tc::tmem_ld16(lane_base + col0 + cb * 16, v);
                 tc::tmem_wait_ld();
@@ -367,28 +362,27 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             if (lane == 0) tc::mbar_arrive(&st_empty[st]);
             if (!tc::warp_wait_bar(&s_full[st], (uint32_t)((c >> 1) & 1), abort)) { ok = false; break; }
             tc::fence_after_sync();
-            uint32_t sv[kH];
+            uint32_t sv[kBS];
 #pragma unroll
-            for (int cb = 0; cb < kH / 16; ++cb)
-                tc::tmem_ld16(lane_base + (uint32_t)(st * kBS + k0 + cb * 16), sv + cb * 16);
+            for (int cb = 0; cb < kBS / 16; ++cb) tc::tmem_ld16(lane_base + (uint32_t)(st * kBS + cb * 16), sv + cb * 16);
             tc::tmem_wait_ld();
             if (!kOut) {
                 float mx = -INFINITY;
 #pragma unroll
-                for (int k = 0; k < kH; ++k)
-                    if (k0 + k <= kmax) mx = fmaxf(mx, fmaf(__uint_as_float(sv[k]), qk, lg2));
+                for (int k = 0; k < kBS; ++k)
+                    if (k <= kmax) mx = fmaxf(mx, fmaf(__uint_as_float(sv[k]), qk, lg2));
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(&s_empty[st]);
                 if (valid && mx > -INFINITY) atomicMax(a.rowmax + qrow, float_key(mx));
             } else {
-                uint32_t pk[kH / 2];
+                uint32_t pk[kBS / 2];
                 float rs = 0.f;
                 const float bias = lg2 - m;
 #pragma unroll
-                for (int k = 0; k < kH; k += 2) {
-                    const float p0 = (k0 + k <= kmax) ? exp2f(fmaf(__uint_as_float(sv[k]), qk, bias)) : 0.f;
-                    const float p1 = (k0 + k + 1 <= kmax) ? exp2f(fmaf(__uint_as_float(sv[k + 1]), qk, bias)) : 0.f;
+                for (int k = 0; k < kBS; k += 2) {
+                    const float p0 = (k <= kmax) ? exp2f(fmaf(__uint_as_float(sv[k]), qk, bias)) : 0.f;
+                    const float p1 = (k + 1 <= kmax) ? exp2f(fmaf(__uint_as_float(sv[k + 1]), qk, bias)) : 0.f;
                     rs += p0 + p1;
                     __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);
                     pk[k / 2] = *reinterpret_cast<uint32_t*>(&hp);
@@ -396,8 +390,8 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 if (valid) atomicAdd(a.l_acc + qrow, rs);
                 if (c >= 1 && !tc::warp_wait_bar(p_empty, (uint32_t)((c - 1) & 1), abort)) { ok = false; break; }
 #pragma unroll
-                for (int cb = 0; cb < kH / 8; ++cb) {
-                    const uint32_t off = tc::sw128_offset(r, k0 + cb * 8);
+                for (int cb = 0; cb < kBS / 8; ++cb) {
+                    const uint32_t off = tc::sw128_offset(r, cb * 8);
                     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sbase + L::kP + off),
                                  "r"(pk[cb * 4]), "r"(pk[cb * 4 + 1]), "r"(pk[cb * 4 + 2]), "r"(pk[cb * 4 + 3])
                                  : "memory");
