@@ -309,7 +309,7 @@ def run_ours(args, rank, world, local_rank):
     # roofline of the dominant call
     dom = max(("fwd", "bwd", "topk", "decode"), key=lambda p: mean[p])
     # the bench workload (bf16, d 128, block 64) runs the tensor-core kernels
-    kernel_file = {"fwd": "attn_fwd_tc.cu", "bwd": "attn_bwd_tc.cu", "topk": "topk.cu", "decode": "decode.cu"}[dom]
+    kernel_file = {"fwd": "attn_fwd_rows.cu", "bwd": "attn_bwd_tc.cu", "topk": "topk.cu", "decode": "decode.cu"}[dom]
     if dom in ("fwd", "bwd"):
         fl = f_fwd if dom == "fwd" else f_bwd
         ach = fl / (mean[dom] * 1e-3) / 1e12
