@@ -14,8 +14,8 @@
 //     keys -> M (log2 units);
 //   pass B (kOut = true):  S again, P = 2^(a log2 e - M) (<= 1), the row sums
 //     l += sum P (fp32 atomics) and O += P V_j (M=128 rows, N=d, K=64 keys)
-//     read back from TMEM and added into an fp32 accumulator with vector
-//     atomics.
+//     read back from TMEM, staged per row in shared memory and added into an
+//     fp32 accumulator by bulk-copy reductions (whole lines at L2).
 // A finalize kernel writes o = O / l and the row log-sum-exp M ln2 + ln l.
 // Executed MMA work is 6 d FLOP per kept (query head, key) pair (the S
 // product twice) with no masked rows, against 4 d in the definition.
@@ -59,7 +59,9 @@ struct RowsSmem {
     static constexpr uint32_t kStage = kOut ? 32768 : 16384;       // 2 x Q [2 x 128 x 128 B]
     static constexpr uint32_t kStageBytes = 32768;
     static constexpr uint32_t kP = kStage + 2 * kStageBytes;       // P [128 x 128 B] (pass B)
-    static constexpr uint32_t kMeta = kP + (kOut ? 16384 : 0);     // 4 x per-chunk metadata
+    static constexpr uint32_t kOst = kP + (kOut ? 16384 : 0);      // O rows, fp32, kOstRow apart (pass B)
+    static constexpr uint32_t kOstRow = kD * 4 + 16;               // padded: conflict-free 16-byte stores
+    static constexpr uint32_t kMeta = kOst + (kOut ? kRows * kOstRow : 0);  // 4 x per-chunk metadata
     static constexpr uint32_t kMetaBytes = 4 * 512 + 16;           // tok_t, tok_lg, row_m, qoff, ntok
     static constexpr uint32_t kBar = kMeta + 4 * kMetaBytes;
     static constexpr int kNumBars = 16;
@@ -319,26 +321,33 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         const float qk = sh.scale * kLog2e;
         bool ok = true;
         int prev_row = -1;
-        auto o_epilogue = [&](int c) -> bool {     // O of chunk c: TMEM -> fp32 accumulator
+        // O of chunk c: TMEM -> this thread's padded shared-memory row -> one
+        // 512-byte bulk add into the fp32 accumulator row. The row is reused
+        // only after the previous bulk add of this thread has read it.
+        const uint32_t orow = sbase + L::kOst + (uint32_t)r * L::kOstRow;
+        auto o_epilogue = [&](int c) -> bool {
             if (!tc::warp_wait_bar(&o_full[c & 1], (uint32_t)((c >> 1) & 1), abort)) return false;
             tc::fence_after_sync();
             const uint32_t col0 = 128 + (uint32_t)((c & 1) * kD);
+            tc::bulk_wait_read0();
 #pragma unroll 1
             for (int cb = 0; cb < kD / 16; ++cb) {
                 uint32_t v[16];
                 tc::tmem_ld16(lane_base + col0 + cb * 16, v);
                 tc::tmem_wait_ld();
-                if (prev_row >= 0) {
-                    float* dst = a.o_acc + (int64_t)prev_row * kD + cb * 16;
 #pragma unroll
-                    for (int e = 0; e < 16; e += 4)
-                        tc::red_add_v4(dst + e, __uint_as_float(v[e]), __uint_as_float(v[e + 1]),
-                                       __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
-                }
+                for (int e = 0; e < 16; e += 4)
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(orow + (cb * 16 + e) * 4),
+                                 "r"(v[e]), "r"(v[e + 1]), "r"(v[e + 2]), "r"(v[e + 3]) : "memory");
             }
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&o_empty[c & 1]);
+            if (prev_row >= 0) {
+                tc::fence_async_shared();
+                tc::bulk_reduce_add_f32(a.o_acc + (int64_t)prev_row * kD, orow, kD * 4);
+                tc::bulk_commit();
+            }
             return true;
         };
         for (int c = 0; c < nc; ++c) {
@@ -405,6 +414,7 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             }
         }
         if (kOut && ok && nc > 0) o_epilogue(nc - 1);
+        if (kOut) tc::bulk_wait0();
     }
     tc::fence_before_sync();
     __syncthreads();

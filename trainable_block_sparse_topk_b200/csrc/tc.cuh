@@ -100,6 +100,19 @@ __device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c
                  : "memory");
 }
 
+// dst[0 .. bytes/4) += src (fp32) by the bulk-copy engine: whole 128-byte
+// lines reach L2 instead of per-thread vector atomics. Both addresses 16-byte
+// aligned, bytes a multiple of 16. Tracked in this thread's bulk group.
+__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, uint32_t src_smem, uint32_t bytes) {
+    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;"
+                 ::"l"(dst), "r"(src_smem), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until this thread's committed bulk operations have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Wait until this thread's committed bulk operations have completed.
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Named barrier over `count` threads (id 1..15).
 __device__ __forceinline__ void named_bar(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
