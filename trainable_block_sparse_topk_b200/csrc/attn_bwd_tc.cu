@@ -17,7 +17,8 @@
 //   P, dS in the compute warps (thread = row = TMEM lane), Gsum per token
 //   dV^T += dO^T P, dK^T += Q^T dS (M=d, N=64, K=128 rows)        -> TMEM
 //   dQ = dS K_j (M=128 rows, N=d, K=64)                            -> TMEM
-//   dQ rows are added into the fp32 accumulator with vector atomics.
+//   dQ rows are added into the fp32 accumulator with vector atomics, lanes
+//   regrouped so that each warp-wide reduction covers whole L2 sectors.
 // TMEM: S|dP double buffer [0,256), dQ [256,384), dV^T [384,448),
 // dK^T [448,512). S/dP of chunk c+1 are computed while the compute warps
 // build P/dS of chunk c and read back dQ of chunk c-1.
@@ -362,18 +363,45 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         auto dq_epilogue = [&](int c) -> bool {    // read dQ of chunk c back and add it to the fp32 accumulator
             if (!tc::warp_wait_bar(dq_full, (uint32_t)(c & 1), abort)) return false;
             tc::fence_after_sync();
+            // Lanes 4i..4i+3 trade 16-byte pieces (a 4x4 transpose) so that each
+            // vector reduction of the warp covers 64 contiguous bytes of 8 rows:
+            // whole 32-byte sectors reach L2 instead of halves.
+            const int qd = lane & 3;
+            int64_t rows4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int src = (lane & ~3) + e;
+                rows4[e] = (int64_t)__shfl_sync(0xffffffffu, (long long)prev_dq_row, src);
+            }
 #pragma unroll 1
             for (int cb = 0; cb < kD / 16; ++cb) {
                 uint32_t v[16];
                 tc::tmem_ld16(lane_base + kColDQ + cb * 16, v);
                 tc::tmem_wait_ld();
-                if (prev_dq_row >= 0) {
-                    float* dst = a.dq_acc + prev_dq_row * kD + cb * 16;
+                float x[16];
 #pragma unroll
-                    for (int e = 0; e < 16; e += 4)
-                        tc::red_add_v4(dst + e, __uint_as_float(v[e]) * dscale, __uint_as_float(v[e + 1]) * dscale,
-                                       __uint_as_float(v[e + 2]) * dscale, __uint_as_float(v[e + 3]) * dscale);
+                for (int e = 0; e < 16; ++e) x[e] = __uint_as_float(v[e]) * dscale;
+#pragma unroll
+                for (int m = 1; m <= 2; m <<= 1) {
+#pragma unroll
+                    for (int k0 = 0; k0 < 4; ++k0) {
+                        if (k0 & m) continue;
+                        const int k1 = k0 | m;
+                        const bool hi = (qd & m) != 0;
+#pragma unroll
+                        for (int f = 0; f < 4; ++f) {
+                            const float snd = hi ? x[k0 * 4 + f] : x[k1 * 4 + f];
+                            const float rcv = __shfl_xor_sync(0xffffffffu, snd, m);
+                            if (hi) x[k0 * 4 + f] = rcv; else x[k1 * 4 + f] = rcv;
+                        }
+                    }
                 }
+                // x[4e .. 4e+3] = columns cb*16 + 4 qd .. +3 of row (lane & ~3) + e
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (rows4[e] >= 0)
+                        tc::red_add_v4(a.dq_acc + rows4[e] * kD + cb * 16 + qd * 4, x[4 * e], x[4 * e + 1],
+                                       x[4 * e + 2], x[4 * e + 3]);
             }
             tc::fence_before_sync();
             __syncwarp();
