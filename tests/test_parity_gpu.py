@@ -364,3 +364,32 @@ def test_every_training_path_matches_oracle(path, monkeypatch):
                    "dv": out["dv"][b:b + 1, g:g + 1].float().numpy(), "ds": out["ds"][b, g].numpy()}
             for key, val in got.items():
                 assert U.normwise(val, r[key]) <= TOL_BF16_GRAD, (path, key)
+
+
+def test_rows_beyond_the_softmax_shift_are_recomputed():
+    """The gathered-row forward shifts each row's softmax by the row's own
+    logit. Rows planted so that a neighbour key's logit exceeds the own one by
+    about 650 (log2 units) overflow that shift; they must come out of the exact
+    recompute, elementwise equal to the oracle, and the backward must follow."""
+    w = synth.Workload("far", "train", 1, 512, 4, 1, 128, 64, 3, "bf16", 33, 0.5, score_kind="gauss")
+    x = synth.train_inputs(w)
+    gen = torch.Generator().manual_seed(5)
+    u = torch.where(torch.rand(w.head_dim, generator=gen) < 0.5, -1.0, 1.0)
+    for t in (130, 301, 302, 450):                 # the key t-1 shares t's block
+        x["q"][0, :, t] = 20.0 * u
+        x["k"][0, 0, t] = -u
+        x["k"][0, 0, t - 1] = u
+    x["scores"] = synth.train_scores(w, x["q"], x["k"])
+    x, out = U.run_train(w, inputs=x)
+    d = U.group_desc(w)
+    a = U.group_arrays(x, w, 0, 0)
+    o, lse = oracle.fwd(d, a["q"], a["k"], a["v"], a["s"])
+    go = out["o"][0].float().numpy().transpose(1, 0, 2)
+    assert np.isfinite(go).all()
+    assert np.abs(go - o).max() <= TOL_BF16_O
+    np.testing.assert_allclose(out["lse"][0].numpy().T, lse, atol=1e-4 * np.abs(lse).max(), rtol=0)
+    r = oracle.bwd(d, a["q"], a["k"], a["v"], a["s"], a["dO"])
+    got = {"dq": out["dq"][0].float().numpy().transpose(1, 0, 2), "dk": out["dk"].float().numpy(),
+           "dv": out["dv"].float().numpy(), "ds": out["ds"][0, 0].numpy()}
+    for key, val in got.items():
+        assert U.normwise(val, r[key]) <= TOL_BF16_GRAD, key

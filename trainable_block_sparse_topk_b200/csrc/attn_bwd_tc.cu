@@ -20,13 +20,16 @@
 //   dQ rows are added into the fp32 accumulator with vector atomics, lanes
 //   regrouped so that each warp-wide reduction covers whole L2 sectors.
 // TMEM: S|dP double buffer [0,256), dQ [256,384), dV^T [384,448),
-// dK^T [448,512). S/dP of chunk c+1 are computed while the compute warps
-// build P/dS of chunk c and read back dQ of chunk c-1.
+// dK^T [448,512). S/dP of chunk c+1 are computed while warps 4-7 build P/dS
+// of chunk c and warps 0-3 read back and add dQ of chunk c-1.
 //
-// Roles (256 threads): warps 0 and 3 gather chunk rows (even / odd chunks)
-// with TMA tile::gather4 loads into the two 128-byte-swizzled Q/dO stages
-// (warp 0 also loads K_j, V_j by TMA), warp 1 lane 0 issues the MMAs, warp 2 owns the
-// TMEM allocation, warps 4-7 compute. No TMA multicast is used.
+// Roles (384 threads): warps 0-3 epilogue (dQ reductions, final dK/dV),
+// warps 4-7 P/dS and Gsum (thread = row = TMEM lane in both groups), warps 8
+// and 11 gather chunk rows (even / odd chunks) with coalesced 16-byte cp.async
+// copies into the two 128-byte-swizzled Q/dO stages (TMA tile::gather4 moves
+// random rows at a fraction of that rate; warp 8 also loads K_j, V_j by TMA),
+// warp 9 lane 0 issues the MMAs, warp 10 owns the TMEM allocation. No TMA
+// multicast is used.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -37,7 +40,7 @@ namespace sas {
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;   // epilogue warps 0-3, P/dS warps 4-7, loaders 8 and 11, MMA 9, TMEM 10
 constexpr int kBS = 64;
 constexpr int kRows = 128;
 constexpr int kD = 128;
@@ -45,8 +48,6 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColDQ = 256, kColDV = 384, kColDK = 448;
 
 struct BwdTcArgs {
-    CUtensorMap tm_q;    // q  [B*Hq*T, d], one-row boxes of 64 columns, 128-byte swizzle (gather4)
-    CUtensorMap tm_do;   // dO, same
     Shape sh;
     const __nv_bfloat16* q;
     const __nv_bfloat16* dO;
@@ -73,10 +74,11 @@ struct BwdSmem {
     static constexpr uint32_t kMeta = kDS + 16384;             // 4 x per-chunk metadata (chunk c -> slot c & 3)
     static constexpr uint32_t kMetaBytes = 6 * 512 + 16;       // tok_t, tok_slot, tok_lg, row_lse, row_D, qoff, ntok
     static constexpr uint32_t kGs = kMeta + 4 * kMetaBytes;    // per-token Gsum [2][128] f32
-    static constexpr uint32_t kColW = kGs + 1024;              // u64 [kMaxNT]: the block's bitmap column
+    static constexpr uint32_t kIds = kGs + 1024;               // i32 [2][128]: dQ accumulator row per chunk row
+    static constexpr uint32_t kColW = kIds + 1024;             // u64 [kMaxNT]: the block's bitmap column
     static constexpr uint32_t kPre = kColW + 8 * 1024;         // i32 [kMaxNT]: stream index of tile tau's first token
     static constexpr uint32_t kBar = kPre + 4 * 1024;
-    static constexpr int kNumBars = 13;
+    static constexpr int kNumBars = 14;
     static constexpr uint32_t kMisc = kBar + 8 * kNumBars;     // tmem base, chunk count, abort
     static constexpr uint32_t kTotal = kMisc + 16;
 };
@@ -107,7 +109,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     unsigned char* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
     uint64_t* kv_full = bars + 0;
-    uint64_t* st_full = bars + 1;     // [2], the loader's arrive + the gather bytes
+    uint64_t* st_full = bars + 1;     // [2], the loader's arrive once its copies have landed
     uint64_t* st_empty = bars + 3;    // [2]
     uint64_t* s_full = bars + 5;      // [2]
     uint64_t* p_full = bars + 7;      // 4 arrivals (compute warps)
@@ -115,10 +117,12 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     uint64_t* dq_full = bars + 9;
     uint64_t* dq_empty = bars + 10;   // 4 arrivals
     uint64_t* done = bars + 11;
+    uint64_t* ids_full = bars + 12;   // [2] 4 arrivals: the chunk's dQ row ids are in ids[]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMisc);
     int* nc_slot = reinterpret_cast<int*>(sm + L::kMisc + 4);
     volatile int* abort = reinterpret_cast<volatile int*>(sm + L::kMisc + 8);
     float* tok_gs = reinterpret_cast<float*>(sm + L::kGs);
+    int* ids = reinterpret_cast<int*>(sm + L::kIds);
 
     const Shape& sh = a.sh;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -134,15 +138,15 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         for (int i = 0; i < L::kNumBars; ++i) {
             uint64_t* bar = &bars[i];
             uint32_t cnt = 1;
-            if (bar == &st_full[0] || bar == &st_full[1]) cnt = 1;   // the loader's arrive.expect_tx
-            if (bar == p_full || bar == dq_empty) cnt = 4;
+            if (bar == p_full || bar == dq_empty || bar == &ids_full[0] || bar == &ids_full[1]) cnt = 4;
+            if (bar == &st_full[0] || bar == &st_full[1]) cnt = 33;   // 32 cp.async arrivals + the loader's
             mbar_init(bar, cnt);
         }
         *nc_slot = kBS;   // the block's own tokens; later tiles are added below
         *abort = 0;
         fence_mbar_init();
     }
-    if (warp == 2) {
+    if (warp == 10) {
         tc::tmem_alloc(tmem_slot, kTmemCols);
         tc::tmem_relinquish();
     }
@@ -180,12 +184,12 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     const int nc = (ntok_total + tpc - 1) / tpc;
     const uint32_t sbase = smem_u32(sm);
 
-    if (warp == 0 || warp == 3) {
+    if (warp == 8 || warp == 11) {
         // ---------------------------------------------------------- loaders ---
-        const int L0 = warp == 0 ? 0 : 1;           // this warp fills chunks c = L0, L0 + 2, ...
+        const int L0 = warp == 8 ? 0 : 1;           // this warp fills chunks c = L0, L0 + 2, ...
         unsigned char* stq = sm + L::kStage + L0 * L::kStageBytes;
         unsigned char* stdo = stq + 32768;
-        if (warp == 0 && lane == 0) {
+        if (warp == 8 && lane == 0) {
             tc::prefetch_tmap(&tm_k);
             tc::prefetch_tmap(&tm_v);
             mbar_arrive_expect_tx(kv_full, 32768);
@@ -244,6 +248,12 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 meta.row_lse[i] = lse;
                 meta.row_D[i] = Dv;
                 meta.qoff[i] = qrow;
+                if (qrow >= 0) {              // the rows are copied about two chunks later
+                    tc::prefetch_l2(a.q + (int64_t)qrow * kD);
+                    tc::prefetch_l2(a.q + (int64_t)qrow * kD + 64);
+                    tc::prefetch_l2(a.dO + (int64_t)qrow * kD);
+                    tc::prefetch_l2(a.dO + (int64_t)qrow * kD + 64);
+                }
             }
             __syncwarp();
         };
@@ -254,25 +264,32 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             // fetches rows 4l..4l+3 of both d halves of q and dO. Padding rows
             // re-read the chunk's first row (their P and dS are zero).
             const int* qoff = Meta(sm + L::kMeta + (c & 3) * L::kMetaBytes).qoff;
-            if (lane == 0) mbar_arrive_expect_tx(&st_full[L0], 65536u);
-            __syncwarp();
             {
-                int rr[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int qrow = qoff[4 * lane + e];
-                    rr[e] = qrow >= 0 ? qrow : qoff[0];
-                }
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const uint32_t off = hh * 16384 + 4 * lane * 128;
-                    tc::tma_gather4(stq + off, &a.tm_q, hh * 64, rr, &st_full[L0]);
-                    tc::tma_gather4(stdo + off, &a.tm_do, hh * 64, rr, &st_full[L0]);
+                // 16 lanes copy one 256-byte row (16-byte pieces, coalesced), two
+                // rows per instruction, into the swizzled tile; row i's piece p
+                // lands in d-half p / 8 at 16-byte chunk p % 8.
+                const int p = lane & 15, hh = p >> 3, col = (p & 7) * 8;
+                const int q0 = qoff[0];
+#pragma unroll 4
+                for (int i = 0; i < kRows / 2; ++i) {
+                    const int row = 2 * i + (lane >> 4);
+                    int qrow = qoff[row];
+                    if (qrow < 0) qrow = q0;
+                    const uint32_t off = hh * 16384 + tc::sw128_offset(row, col);
+                    tc::cp_async16(stq + off, a.q + (int64_t)qrow * kD + p * 8);
+                    tc::cp_async16(stdo + off, a.dO + (int64_t)qrow * kD + p * 8);
                 }
             }
-            if (c + 2 < nc) prep(c + 2);   // overlaps the wait for this stage's next release
+            // st_full completes once every lane's copies have landed (32 async
+            // arrivals) and lane 0 has published the chunk's metadata; the MMA
+            // thread fences the async proxy after its wait
+            tc::cp_async_mbar_arrive_noinc(&st_full[L0]);
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&st_full[L0]);
+            if (c + 2 < nc) prep(c + 2);   // overlaps the copies in flight
         }
-    } else if (warp == 1) {
+        tc::cp_async_wait_all();
+    } else if (warp == 9) {
         // ------------------------------------------------------- MMA issuer ---
         if (lane == 0) {
             constexpr uint32_t id_sp = tc::idesc_bf16_f32(128, kBS, false, false);   // S, dP
@@ -295,6 +312,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 tc::mma_commit(&s_full[c & 1]);
             };
             bool ok = tc::wait_bar(kv_full, 0u, abort) && tc::wait_bar(&st_full[0], 0u, abort);
+            tc::fence_async_shared();   // the stage was written by cp.async (generic proxy)
             tc::fence_after_sync();
             if (ok) issue_sdp(0);
             // Issue whichever step is ready: S/dP of the next chunk (TMEM double
@@ -308,6 +326,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 bool progressed = false;
                 if (sdp_next < nc && sdp_next <= c + 1 &&
                     mbar_test_wait(&st_full[sdp_next & 1], (uint32_t)((sdp_next >> 1) & 1))) {
+                    tc::fence_async_shared();
                     tc::fence_after_sync();
                     issue_sdp(sdp_next);
                     ++sdp_next;
@@ -352,65 +371,14 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             }
             tc::mma_commit(done);
         }
-    } else if (warp >= 4) {
-        // ----------------------------------------------------- compute warps ---
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------- P / dS warps (4 - 7) ---
         const int r = (warp - 4) * 32 + lane;      // chunk row == TMEM lane
         const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const float qk = sh.scale * kLog2e;
-        const float dscale = sh.scale;
-        bool ok = true;
-        int64_t prev_dq_row = -1;                  // dq accumulator row of this thread in chunk c-1
-        auto dq_epilogue = [&](int c) -> bool {    // read dQ of chunk c back and add it to the fp32 accumulator
-            if (!tc::warp_wait_bar(dq_full, (uint32_t)(c & 1), abort)) return false;
-            tc::fence_after_sync();
-            // Lanes 4i..4i+3 trade 16-byte pieces (a 4x4 transpose) so that each
-            // vector reduction of the warp covers 64 contiguous bytes of 8 rows:
-            // whole 32-byte sectors reach L2 instead of halves.
-            const int qd = lane & 3;
-            int64_t rows4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int src = (lane & ~3) + e;
-                rows4[e] = (int64_t)__shfl_sync(0xffffffffu, (long long)prev_dq_row, src);
-            }
-#pragma unroll 1
-            for (int cb = 0; cb < kD / 16; ++cb) {
-                uint32_t v[16];
-                tc::tmem_ld16(lane_base + kColDQ + cb * 16, v);
-                tc::tmem_wait_ld();
-                float x[16];
-#pragma unroll
-                for (int e = 0; e < 16; ++e) x[e] = __uint_as_float(v[e]) * dscale;
-#pragma unroll
-                for (int m = 1; m <= 2; m <<= 1) {
-#pragma unroll
-                    for (int k0 = 0; k0 < 4; ++k0) {
-                        if (k0 & m) continue;
-                        const int k1 = k0 | m;
-                        const bool hi = (qd & m) != 0;
-#pragma unroll
-                        for (int f = 0; f < 4; ++f) {
-                            const float snd = hi ? x[k0 * 4 + f] : x[k1 * 4 + f];
-                            const float rcv = __shfl_xor_sync(0xffffffffu, snd, m);
-                            if (hi) x[k0 * 4 + f] = rcv; else x[k1 * 4 + f] = rcv;
-                        }
-                    }
-                }
-                // x[4e .. 4e+3] = columns cb*16 + 4 qd .. +3 of row (lane & ~3) + e
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    if (rows4[e] >= 0)
-                        tc::red_add_v4(a.dq_acc + rows4[e] * kD + cb * 16 + qd * 4, x[4 * e], x[4 * e + 1],
-                                       x[4 * e + 2], x[4 * e + 3]);
-            }
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(dq_empty);
-            return true;
-        };
         for (int c = 0; c < nc; ++c) {
             const int st = c & 1;
-            if (!tc::warp_wait_bar(&st_full[st], (uint32_t)((c >> 1) & 1), abort)) { ok = false; break; }
+            if (!tc::warp_wait_bar(&st_full[st], (uint32_t)((c >> 1) & 1), abort)) break;
             Meta meta(sm + L::kMeta + (c & 3) * L::kMetaBytes);
             const int n = *meta.ntok;
             const int ti = r / G, h = r - ti * G;
@@ -427,59 +395,129 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 Dv = meta.row_D[r];
             }
             const float bias = (lgl - lse2) * kLog2e;
-            const int64_t dq_row = valid ? ((int64_t)b * sh.Hq + g * G + h) * T + t : -1;
-            if (!tc::warp_wait_bar(&s_full[st], (uint32_t)((c >> 1) & 1), abort)) { ok = false; break; }
+            const int dq_row = valid ? (int)(((int64_t)b * sh.Hq + g * G + h) * T + t) : -1;
+            // token r of the chunk, for its Gsum (read now: the metadata slot is
+            // refilled once the chunk's last MMAs are issued)
+            const int gs_slot = r < n ? meta.tok_slot[r] : -1;
+            const int gs_tok = r < n ? meta.tok_t[r] : 0;
+            if (!tc::warp_wait_bar(&s_full[st], (uint32_t)((c >> 1) & 1), abort)) break;
+            // P and dS of chunk c-1 must have been consumed by its MMAs; that also
+            // means the epilogue warps are done with chunk c-2, whose row-id slot
+            // is reused here
+            if (c >= 1 && !tc::warp_wait_bar(p_empty, (uint32_t)((c - 1) & 1), abort)) break;
+            ids[st * kRows + r] = dq_row;
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&ids_full[st]);
             tc::fence_after_sync();
-            uint32_t sv[kBS], pv[kBS];
-#pragma unroll
-            for (int cb = 0; cb < kBS / 16; ++cb) {
-                tc::tmem_ld16(lane_base + (uint32_t)(st * 128 + cb * 16), sv + cb * 16);
-                tc::tmem_ld16(lane_base + (uint32_t)(st * 128 + 64 + cb * 16), pv + cb * 16);
-            }
-            tc::tmem_wait_ld();
-            uint32_t pk[kBS / 2], dk2[kBS / 2];
             float rowsum = 0.f;
 #pragma unroll
-            for (int k = 0; k < kBS; k += 2) {
-                const float p0 = (k <= kmax) ? exp2f(fmaf(__uint_as_float(sv[k]), qk, bias)) : 0.f;
-                const float p1 = (k + 1 <= kmax) ? exp2f(fmaf(__uint_as_float(sv[k + 1]), qk, bias)) : 0.f;
-                const float d0 = p0 * (__uint_as_float(pv[k]) - Dv);
-                const float d1 = p1 * (__uint_as_float(pv[k + 1]) - Dv);
-                rowsum += d0 + d1;
-                __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);
-                __nv_bfloat162 hd = __floats2bfloat162_rn(d0, d1);
-                pk[k / 2] = *reinterpret_cast<uint32_t*>(&hp);
-                dk2[k / 2] = *reinterpret_cast<uint32_t*>(&hd);
-            }
-            // Gsum of the token: its G rows are in this chunk
-            float* gs = tok_gs + st * kRows;
-            if (valid && !diag) atomicAdd(&gs[ti], rowsum);
-            tc::named_bar(1, 128);
-            if (r < n) {
-                const int slot = meta.tok_slot[r];
-                if (slot >= 0) a.gsum[((int64_t)bg * T + meta.tok_t[r]) * K + slot] = gs[r];
-                gs[r] = 0.f;
-            }
-            // P and dS of chunk c-1 must have been consumed by its MMAs
-            if (c >= 1 && !tc::warp_wait_bar(p_empty, (uint32_t)((c - 1) & 1), abort)) { ok = false; break; }
+            for (int hf = 0; hf < 2; ++hf) {           // 32 keys at a time
+                uint32_t sv[32], pv[32];
 #pragma unroll
-            for (int cb = 0; cb < kBS / 8; ++cb) {
-                const uint32_t off = tc::sw128_offset(r, cb * 8);
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sbase + L::kP + off), "r"(pk[cb * 4]),
-                             "r"(pk[cb * 4 + 1]), "r"(pk[cb * 4 + 2]), "r"(pk[cb * 4 + 3])
-                             : "memory");
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sbase + L::kDS + off), "r"(dk2[cb * 4]),
-                             "r"(dk2[cb * 4 + 1]), "r"(dk2[cb * 4 + 2]), "r"(dk2[cb * 4 + 3])
-                             : "memory");
+                for (int cb = 0; cb < 2; ++cb) {
+                    tc::tmem_ld16(lane_base + (uint32_t)(st * 128 + hf * 32 + cb * 16), sv + cb * 16);
+                    tc::tmem_ld16(lane_base + (uint32_t)(st * 128 + 64 + hf * 32 + cb * 16), pv + cb * 16);
+                }
+                tc::tmem_wait_ld();
+                uint32_t pk[16], dk2[16];
+#pragma unroll
+                for (int k = 0; k < 32; k += 2) {
+                    const int kk = hf * 32 + k;
+                    const float p0 = (kk <= kmax) ? exp2f(fmaf(__uint_as_float(sv[k]), qk, bias)) : 0.f;
+                    const float p1 = (kk + 1 <= kmax) ? exp2f(fmaf(__uint_as_float(sv[k + 1]), qk, bias)) : 0.f;
+                    const float d0 = p0 * (__uint_as_float(pv[k]) - Dv);
+                    const float d1 = p1 * (__uint_as_float(pv[k + 1]) - Dv);
+                    rowsum += d0 + d1;
+                    __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);
+                    __nv_bfloat162 hd = __floats2bfloat162_rn(d0, d1);
+                    pk[k / 2] = *reinterpret_cast<uint32_t*>(&hp);
+                    dk2[k / 2] = *reinterpret_cast<uint32_t*>(&hd);
+                }
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb) {
+                    const uint32_t off = tc::sw128_offset(r, hf * 32 + cb * 8);
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sbase + L::kP + off), "r"(pk[cb * 4]),
+                                 "r"(pk[cb * 4 + 1]), "r"(pk[cb * 4 + 2]), "r"(pk[cb * 4 + 3])
+                                 : "memory");
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(sbase + L::kDS + off),
+                                 "r"(dk2[cb * 4]), "r"(dk2[cb * 4 + 1]), "r"(dk2[cb * 4 + 2]), "r"(dk2[cb * 4 + 3])
+                                 : "memory");
+                }
             }
             tc::fence_async_shared();
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(p_full);
-            if (c >= 1 && !dq_epilogue(c - 1)) { ok = false; break; }
-            prev_dq_row = dq_row;
+            // Gsum of the token: its G rows are in this chunk
+            float* gs = tok_gs + st * kRows;
+            if (valid && !diag) atomicAdd(&gs[ti], rowsum);
+            tc::named_bar(1, 128);
+            if (r < n) {
+                if (gs_slot >= 0) a.gsum[((int64_t)bg * T + gs_tok) * K + gs_slot] = gs[r];
+                gs[r] = 0.f;
+            }
         }
-        if (ok && nc > 0) ok = dq_epilogue(nc - 1);
+    } else if (warp < 4) {
+        // ------------------------------------------- epilogue warps (0 - 3) ---
+        const int r = warp * 32 + lane;            // chunk row == TMEM lane
+        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        const float dscale = sh.scale;
+        const int qd = lane & 3;
+        bool ok = true;
+        for (int c = 0; c < nc; ++c) {
+            const int st = c & 1;
+            if (!tc::warp_wait_bar(&ids_full[st], (uint32_t)((c >> 1) & 1), abort)) { ok = false; break; }
+            const int dq_row = ids[st * kRows + r];
+            // Lanes 4i..4i+3 trade 16-byte pieces (a 4x4 transpose) so that each
+            // vector reduction of the warp covers 64 contiguous bytes of 8 rows:
+            // whole 32-byte sectors reach L2 instead of halves.
+            int rows4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) rows4[e] = __shfl_sync(0xffffffffu, dq_row, (lane & ~3) + e);
+            if (!tc::warp_wait_bar(dq_full, (uint32_t)(c & 1), abort)) { ok = false; break; }
+            tc::fence_after_sync();
+#pragma unroll 1
+            for (int hb = 0; hb < 2; ++hb) {           // 64 columns at a time
+                uint32_t v[64];
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb) tc::tmem_ld16(lane_base + kColDQ + hb * 64 + cb * 16, v + cb * 16);
+                tc::tmem_wait_ld();
+                if (hb == 1) {                          // dQ of this chunk is out of TMEM
+                    tc::fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(dq_empty);
+                }
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb) {
+                    float x[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) x[e] = __uint_as_float(v[cb * 16 + e]) * dscale;
+#pragma unroll
+                    for (int m = 1; m <= 2; m <<= 1) {
+#pragma unroll
+                        for (int k0 = 0; k0 < 4; ++k0) {
+                            if (k0 & m) continue;
+                            const int k1 = k0 | m;
+                            const bool hi = (qd & m) != 0;
+#pragma unroll
+                            for (int f = 0; f < 4; ++f) {
+                                const float snd = hi ? x[k0 * 4 + f] : x[k1 * 4 + f];
+                                const float rcv = __shfl_xor_sync(0xffffffffu, snd, m);
+                                if (hi) x[k0 * 4 + f] = rcv; else x[k1 * 4 + f] = rcv;
+                            }
+                        }
+                    }
+                    // x[4e .. 4e+3] = columns 4 qd .. 4 qd + 3 of this 16-column
+                    // slice, row (lane & ~3) + e
+                    const int col = hb * 64 + cb * 16 + qd * 4;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        if (rows4[e] >= 0)
+                            tc::red_add_v4(a.dq_acc + (int64_t)rows4[e] * kD + col, x[4 * e], x[4 * e + 1],
+                                           x[4 * e + 2], x[4 * e + 3]);
+                }
+            }
+        }
         // dV^T and dK^T: TMEM lane r holds column r of d for the block's 64 keys
         if (ok && tc::warp_wait_bar(done, 0u, abort)) {
             tc::fence_after_sync();
@@ -502,7 +540,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     }
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 2) {
+    if (warp == 10) {
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, kTmemCols);
     }
@@ -519,16 +557,14 @@ cudaError_t launch_bwd_tc(const Shape& s, const void* q, const void* k, const vo
                           const float* lse, const float* Dd, const int32_t* idx, const float* gl,
                           const int32_t* nsel, const uint64_t* maskT, float* dq_acc, void* dk, void* dv,
                           float* gsum, cudaStream_t st) {
-    CUtensorMap mk, mv, mq, mdo;
+    CUtensorMap mk, mv;
     if (!encode_bf16_2d(&mk, k, (uint64_t)s.B * s.Hkv * s.T, kD, kBS) ||
-        !encode_bf16_2d(&mv, v, (uint64_t)s.B * s.Hkv * s.T, kD, kBS) ||
-        !encode_bf16_2d(&mq, q, (uint64_t)s.B * s.Hq * s.T, kD, 1) ||
-        !encode_bf16_2d(&mdo, dO, (uint64_t)s.B * s.Hq * s.T, kD, 1))
+        !encode_bf16_2d(&mv, v, (uint64_t)s.B * s.Hkv * s.T, kD, kBS))
         return cudaErrorInvalidValue;
     const size_t smem = BwdSmem::kTotal + 1024;
     cudaError_t e = cudaFuncSetAttribute(bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    BwdTcArgs a{mq, mdo, s, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dO), lse, Dd, idx, gl, nsel,
+    BwdTcArgs a{s, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dO), lse, Dd, idx, gl, nsel,
                 maskT, dq_acc, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), gsum, kRows / s.G};
     const int64_t grid = (int64_t)s.B * s.Hkv * s.nT;
     bwd_tc_kernel<<<(unsigned)grid, kThreads, smem, st>>>(mk, mv, a);

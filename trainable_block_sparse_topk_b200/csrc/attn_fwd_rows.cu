@@ -8,22 +8,27 @@
 // every key block j instead gathers exactly the (token, head) rows that attend
 // it (its own tile causally, and the later tokens whose selection kept j, from
 // the column bitmap), in chunks of 128 rows, so every MMA row is a kept row.
-// Two passes over the same row streams:
-//   pass A (kOut = false): S = Q K_j^T, per row the maximum of a over the
-//     block, combined across blocks with an atomic max on order-preserving
-//     keys -> M (log2 units);
-//   pass B (kOut = true):  S again, P = 2^(a log2 e - M) (<= 1), the row sums
-//     l += sum P (fp32 atomics) and O += P V_j (M=128 rows, N=d, K=64 keys)
-//     read back from TMEM, staged per row in shared memory and added into an
-//     fp32 accumulator by bulk-copy reductions (whole lines at L2).
-// A finalize kernel writes o = O / l and the row log-sum-exp M ln2 + ln l.
-// Executed MMA work is 6 d FLOP per kept (query head, key) pair (the S
-// product twice) with no masked rows, against 4 d in the definition.
 //
-// Roles (256 threads): warps 0 and 3 gather rows (even / odd chunks) with TMA
-// tile::gather4 into two 128-byte-swizzled Q stages; warp 0 also loads K_j
-// (and V_j) by TMA; warp 1 lane 0 issues the MMAs; warp 2 owns TMEM; warps 4-7
-// compute (thread = row = TMEM lane). No TMA multicast is used.
+// One pass: softmax is unchanged by any per-row shift M, so instead of the row
+// maximum the shift is the row's own logit a_t = scale q_t.k_t (its key is
+// always attended, with gate weight 1), computed by a small kernel first. Per
+// chunk: S = Q K_j^T, P = 2^(a log2 e - M), the row sums l += sum P (fp32
+// atomics) and O += P V_j (M=128 rows, N=d, K=64 keys), read back from TMEM,
+// staged per row in shared memory and added into an fp32 accumulator by
+// bulk-copy reductions (whole lines at L2). A finalize kernel writes o = O / l
+// and the row log-sum-exp (M + log2 l) ln 2. Since P_t = 1, l >= 1: nothing
+// underflows. A row whose largest logit exceeds a_t by more than ~80 (log2
+// units) could overflow, so the finalize flags any row with l > 2^80 or a
+// non-finite output and a CUDA-core kernel recomputes the flagged rows
+// exactly (with the running maximum).
+// Executed MMA work is the definition's 4 d FLOP per kept (query head, key)
+// pair, with no masked rows.
+//
+// Roles (256 threads): warps 0 and 3 gather rows (even / odd chunks) with
+// coalesced 16-byte cp.async copies into two 128-byte-swizzled Q stages (TMA
+// tile::gather4 moves random rows at a fraction of that rate); warp 0 also
+// loads K_j and V_j by TMA; warp 1 lane 0 issues the MMAs; warp 2 owns TMEM;
+// warps 4-7 compute (thread = row = TMEM lane). No TMA multicast is used.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -40,34 +45,33 @@ constexpr int kRows = 128;
 constexpr int kD = 128;
 
 struct FwdRowsArgs {
-    CUtensorMap tm_q;     // q [B*Hq*T, d], one-row boxes of 64 columns, 128-byte swizzle (gather4)
     Shape sh;
+    const __nv_bfloat16* q;   // [B*Hq*T, d]
     const int32_t* idx;
     const float* gl;
     const int32_t* nsel;
     const uint64_t* maskT;
-    uint32_t* rowmax;     // [B*Hq*T] order-preserving key of the row maximum of a (log2 units)
+    const float* shift;   // [B*Hq*T] the row's softmax shift M (log2 units)
     float* l_acc;         // [B*Hq*T]
     float* o_acc;         // [B*Hq*T, d]
     int tpc;              // tokens per chunk = 128 / G
 };
 
-template <bool kOut>
 struct RowsSmem {
     static constexpr uint32_t kK = 0;                              // K_j: 2 halves x [64 x 128 B]
-    static constexpr uint32_t kV = 16384;                          // V_j (pass B)
-    static constexpr uint32_t kStage = kOut ? 32768 : 16384;       // 2 x Q [2 x 128 x 128 B]
+    static constexpr uint32_t kV = 16384;                          // V_j
+    static constexpr uint32_t kStage = 32768;                      // 2 x Q [2 x 128 x 128 B]
     static constexpr uint32_t kStageBytes = 32768;
-    static constexpr uint32_t kP = kStage + 2 * kStageBytes;       // P [128 x 128 B] (pass B)
-    static constexpr uint32_t kOst = kP + (kOut ? 16384 : 0);      // O rows, fp32, kOstRow apart (pass B)
+    static constexpr uint32_t kP = kStage + 2 * kStageBytes;       // P [128 x 128 B]
+    static constexpr uint32_t kOst = kP + 16384;                   // O rows, fp32, kOstRow apart
     static constexpr uint32_t kOstRow = kD * 4 + 16;               // padded: conflict-free 16-byte stores
-    static constexpr uint32_t kMeta = kOst + (kOut ? kRows * kOstRow : 0);  // 4 x per-chunk metadata
+    static constexpr uint32_t kMeta = kOst + kRows * kOstRow;      // 4 x per-chunk metadata
     static constexpr uint32_t kMetaBytes = 4 * 512 + 16;           // tok_t, tok_lg, row_m, qoff, ntok
     static constexpr uint32_t kBar = kMeta + 4 * kMetaBytes;
-    static constexpr int kNumBars = 16;
+    static constexpr int kNumBars = 14;
     static constexpr uint32_t kMisc = kBar + 8 * kNumBars;         // tmem base, token count, abort
     static constexpr uint32_t kColW = kMisc + 16;                  // u64 [nT] bitmap column, then i32 [nT] prefix
-    static constexpr uint32_t kTmemCols = kOut ? 512 : 128;
+    static constexpr uint32_t kTmemCols = 512;                     // S double [0,128), O double [128,384)
     static uint32_t total(int nT) { return kColW + 12 * (uint32_t)nT + 16; }
 };
 
@@ -85,28 +89,21 @@ struct RowMeta {
           ntok(reinterpret_cast<int*>(p + 2048)) {}
 };
 
-__device__ __forceinline__ float key_to_float(uint32_t k) {
-    const uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
-    return __uint_as_float(u);
-}
-
-template <bool kOut>
-__global__ void __launch_bounds__(kThreads, kOut ? 1 : 2)
+__global__ void __launch_bounds__(kThreads, 1)
 fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const __grid_constant__ FwdRowsArgs a) {
-    using L = RowsSmem<kOut>;
+    using L = RowsSmem;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
     uint64_t* kv_full = bars + 0;
-    uint64_t* st_full = bars + 1;     // [2]: the loader's arrive + the gather bytes
+    uint64_t* st_full = bars + 1;     // [2]: the loader's arrive once its copies have landed
     uint64_t* st_empty = bars + 3;    // [2] MMA commit + 4 compute-warp arrivals
     uint64_t* s_full = bars + 5;      // [2]
-    uint64_t* s_empty = bars + 7;     // [2] pass A: 4 arrivals (compute warps)
-    uint64_t* p_full = bars + 9;      // pass B: 4 arrivals
-    uint64_t* p_empty = bars + 10;
-    uint64_t* o_full = bars + 11;     // [2]
-    uint64_t* o_empty = bars + 13;    // [2] 4 arrivals
+    uint64_t* p_full = bars + 7;      // 4 arrivals
+    uint64_t* p_empty = bars + 8;
+    uint64_t* o_full = bars + 9;      // [2]
+    uint64_t* o_empty = bars + 11;    // [2] 4 arrivals
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMisc);
     int* ntok_slot = reinterpret_cast<int*>(sm + L::kMisc + 4);
     volatile int* abort = reinterpret_cast<volatile int*>(sm + L::kMisc + 8);
@@ -127,12 +124,12 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         for (int i = 0; i < L::kNumBars; ++i) {
             uint64_t* bar = &bars[i];
             uint32_t cnt = 1;
-            if (bar == &s_empty[0] || bar == &s_empty[1] || bar == p_full || bar == &o_empty[0] || bar == &o_empty[1])
-                cnt = 4;
+            if (bar == p_full || bar == &o_empty[0] || bar == &o_empty[1]) cnt = 4;
             // a stage is refilled only after the MMA has read its rows and the
             // compute warps have waited for it: its phases then cannot run two
             // ahead of any waiter
             if (bar == &st_empty[0] || bar == &st_empty[1]) cnt = 5;
+            if (bar == &st_full[0] || bar == &st_full[1]) cnt = 33;   // 32 cp.async arrivals + the loader's
             mbar_init(bar, cnt);
         }
         *abort = 0;
@@ -177,12 +174,12 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         unsigned char* stq = sm + L::kStage + L0 * L::kStageBytes;
         if (warp == 0 && lane == 0) {
             tc::prefetch_tmap(&tm_k);
-            if (kOut) tc::prefetch_tmap(&tm_v);
-            mbar_arrive_expect_tx(kv_full, kOut ? 32768u : 16384u);
+            tc::prefetch_tmap(&tm_v);
+            mbar_arrive_expect_tx(kv_full, 32768u);
             const int kr = (int)((int64_t)bg * T + (int64_t)j * kBS);
             for (int h = 0; h < 2; ++h) {
                 tc::tma_load_2d(sm + L::kK + h * 8192, &tm_k, h * 64, kr, kv_full);
-                if (kOut) tc::tma_load_2d(sm + L::kV + h * 8192, &tm_v, h * 64, kr, kv_full);
+                tc::tma_load_2d(sm + L::kV + h * 8192, &tm_v, h * 64, kr, kv_full);
             }
         }
         auto token_at = [&](int s) -> int {
@@ -223,10 +220,14 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 float m = 0.f;
                 if (ti < n) {
                     qrow = (int)(((int64_t)b * sh.Hq + g * G + h) * T + meta.tok_t[ti]);
-                    if (kOut) m = key_to_float(a.rowmax[qrow]);
+                    m = a.shift[qrow];
                 }
                 meta.row_m[i] = m;
                 meta.qoff[i] = qrow;
+                if (qrow >= 0) {              // the row is copied about two chunks later
+                    tc::prefetch_l2(a.q + (int64_t)qrow * kD);
+                    tc::prefetch_l2(a.q + (int64_t)qrow * kD + 64);
+                }
             }
             __syncwarp();
         };
@@ -234,19 +235,29 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         for (int c = L0; c < nc; c += 2) {
             if (c >= 2 && !tc::warp_wait_bar(&st_empty[L0], (uint32_t)(((c >> 1) - 1) & 1), abort)) break;
             const int* qoff = RowMeta(sm + L::kMeta + (c & 3) * L::kMetaBytes).qoff;
-            if (lane == 0) mbar_arrive_expect_tx(&st_full[L0], 32768u);
-            __syncwarp();
-            int rr[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int qrow = qoff[4 * lane + e];
-                rr[e] = qrow >= 0 ? qrow : qoff[0];    // padding rows re-read a valid row; they are masked
+            {
+                // 16 lanes copy one 256-byte q row (16-byte pieces, coalesced), two
+                // rows per instruction; piece p lands in d-half p / 8 at 16-byte
+                // chunk p % 8 of the swizzled row. Padding rows re-read a valid row.
+                const int p = lane & 15, hh = p >> 3, col = (p & 7) * 8;
+                const int q0 = qoff[0];
+#pragma unroll 4
+                for (int i = 0; i < kRows / 2; ++i) {
+                    const int row = 2 * i + (lane >> 4);
+                    int qrow = qoff[row];
+                    if (qrow < 0) qrow = q0;
+                    tc::cp_async16(stq + hh * 16384 + tc::sw128_offset(row, col), a.q + (int64_t)qrow * kD + p * 8);
+                }
             }
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh)
-                tc::tma_gather4(stq + hh * 16384 + 4 * lane * 128, &a.tm_q, hh * 64, rr, &st_full[L0]);
-            if (c + 2 < nc) prep(c + 2);
+            // st_full completes once every lane's copies have landed (32 async
+            // arrivals) and lane 0 has published the chunk's metadata; the MMA
+            // thread fences the async proxy after its wait
+            tc::cp_async_mbar_arrive_noinc(&st_full[L0]);
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&st_full[L0]);
+            if (c + 2 < nc) prep(c + 2);   // overlaps the copies in flight
         }
+        tc::cp_async_wait_all();
     } else if (warp == 1) {
         // ------------------------------------------------------- MMA issuer ---
         if (lane == 0) {
@@ -267,14 +278,7 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 tc::mma_commit(&st_empty[c & 1]);     // Q of the stage is read only by S
             };
             bool ok = tc::wait_bar(kv_full, 0u, abort);
-            if (!kOut) {
-                for (int c = 0; ok && c < nc; ++c) {
-                    if (!tc::wait_bar(&st_full[c & 1], (uint32_t)((c >> 1) & 1), abort)) break;
-                    if (c >= 2 && !tc::wait_bar(&s_empty[c & 1], (uint32_t)(((c >> 1) - 1) & 1), abort)) break;
-                    tc::fence_after_sync();
-                    issue_s(c);
-                }
-            } else {
+            {
                 // S of the next chunk (TMEM double buffer, at most one chunk ahead),
                 // then O of the current chunk once P is in shared memory and its
                 // O buffer has been read back.
@@ -284,6 +288,7 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     bool progressed = false;
                     if (s_next < nc && s_next <= c + 1 &&
                         mbar_test_wait(&st_full[s_next & 1], (uint32_t)((s_next >> 1) & 1))) {
+                        tc::fence_async_shared();
                         tc::fence_after_sync();
                         issue_s(s_next);
                         ++s_next;
@@ -375,16 +380,7 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 #pragma unroll
             for (int cb = 0; cb < kBS / 16; ++cb) tc::tmem_ld16(lane_base + (uint32_t)(st * kBS + cb * 16), sv + cb * 16);
             tc::tmem_wait_ld();
-            if (!kOut) {
-                float mx = -INFINITY;
-#pragma unroll
-                for (int k = 0; k < kBS; ++k)
-                    if (k <= kmax) mx = fmaxf(mx, fmaf(__uint_as_float(sv[k]), qk, lg2));
-                tc::fence_before_sync();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&s_empty[st]);
-                if (valid && mx > -INFINITY) atomicMax(a.rowmax + qrow, float_key(mx));
-            } else {
+            {
                 uint32_t pk[kBS / 2];
                 float rs = 0.f;
                 const float bias = lg2 - m;
@@ -413,8 +409,8 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 prev_row = qrow;
             }
         }
-        if (kOut && ok && nc > 0) o_epilogue(nc - 1);
-        if (kOut) tc::bulk_wait0();
+        if (ok && nc > 0) o_epilogue(nc - 1);
+        tc::bulk_wait0();
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -424,35 +420,80 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     }
 }
 
-// o = O / l (bf16) and attn_lse = M ln 2 + ln l, one warp per row.
+// M = scale log2e q_t.k_t for each of the G query heads of a (b, kv head, t)
+// row, one warp per row (lane l holds dims 4l .. 4l+3).
 __global__ void __launch_bounds__(256)
-fwd_rows_finalize_kernel(int64_t rows, const uint32_t* __restrict__ rowmax, const float* __restrict__ l_acc,
-                         const float* __restrict__ o_acc, __nv_bfloat16* __restrict__ o, float* __restrict__ lse) {
+fwd_rows_shift_kernel(Shape sh, const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                      float* __restrict__ shift) {
+    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);   // (b * Hkv + g) * T + t
+    const int lane = threadIdx.x & 31;
+    if (row >= sh.rows()) return;
+    const int64_t bg = row / sh.T;
+    const int t = (int)(row % sh.T);
+    const int b = (int)(bg / sh.Hkv), g = (int)(bg % sh.Hkv);
+    float kv[4];
+    load_vec<__nv_bfloat16, 4>(k + row * kD + lane * 4, kv);
+    const float qk = sh.scale * kLog2e;
+    for (int h = 0; h < sh.G; ++h) {
+        const int64_t qrow = ((int64_t)b * sh.Hq + g * sh.G + h) * sh.T + t;
+        float qv[4];
+        load_vec<__nv_bfloat16, 4>(q + qrow * kD + lane * 4, qv);
+        float d = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) d = fmaf(qv[e], kv[e], d);
+        d = warp_sum(d);
+        if (lane == 0) shift[qrow] = d * qk;
+    }
+}
+
+// o = O / l (bf16) and attn_lse = (M + log2 l) ln 2, one warp per query-head
+// row. Rows whose sum or output left the safe range are listed (as their
+// (b, kv head, t) row) for the exact recompute instead.
+__global__ void __launch_bounds__(256)
+fwd_rows_finalize_kernel(Shape sh, const float* __restrict__ shift, const float* __restrict__ l_acc,
+                         const float* __restrict__ o_acc, __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
+                         int32_t* __restrict__ list, int32_t* __restrict__ list_n) {
+    const int64_t rows = (int64_t)sh.B * sh.Hq * sh.T;
     const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= rows) return;
     const float l = l_acc[row];
-    const float inv = 1.f / l;
     const float4 v = reinterpret_cast<const float4*>(o_acc + row * kD)[lane];
+    const bool fin = isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
+    const bool bad = __any_sync(0xffffffffu, !fin) || !(l >= 0.5f && l <= 0x1p80f);
+    if (bad) {
+        if (lane == 0) {
+            const int64_t bh = row / sh.T;
+            const int t = (int)(row % sh.T);
+            const int b = (int)(bh / sh.Hq), h = (int)(bh % sh.Hq);
+            list[atomicAdd(list_n, 1)] = (int32_t)(((int64_t)b * sh.Hkv + h / sh.G) * sh.T + t);
+        }
+        return;
+    }
+    const float inv = 1.f / l;
     __nv_bfloat162 lo = __floats2bfloat162_rn(v.x * inv, v.y * inv);
     __nv_bfloat162 hi = __floats2bfloat162_rn(v.z * inv, v.w * inv);
     uint2 packed = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
     reinterpret_cast<uint2*>(o + row * kD)[lane] = packed;
-    if (lane == 0) lse[row] = (key_to_float(rowmax[row]) + log2f(l)) * kLn2;
+    if (lane == 0) lse[row] = (shift[row] + log2f(l)) * kLn2;
 }
 
-template <bool kOut>
-cudaError_t launch_pass(const CUtensorMap& mk, const CUtensorMap& mv, const FwdRowsArgs& a, cudaStream_t st) {
-    const size_t smem = RowsSmem<kOut>::total(a.sh.nT) + 1024;
-    auto kern = fwd_rows_kernel<kOut>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    const int64_t grid = (int64_t)a.sh.B * a.sh.Hkv * a.sh.nT;
-    kern<<<(unsigned)grid, kThreads, smem, st>>>(mk, mv, a);
-    e = cudaGetLastError();
-    if (e == cudaSuccess) count_launches(1);
-    return e;
-}
+// Workspace: shift [rows] f32 | list [rows] i32 | l [rows] f32 | O [rows, d] f32 | list count
+struct RowsWs {
+    float* shift;
+    int32_t* list;
+    float* l_acc;
+    float* o_acc;
+    int32_t* list_n;
+    size_t zero_bytes;   // l, O and the count are contiguous and start at zero
+    RowsWs(void* ws, int64_t rows)
+        : shift(static_cast<float*>(ws)),
+          list(reinterpret_cast<int32_t*>(shift + rows)),
+          l_acc(reinterpret_cast<float*>(list + rows)),
+          o_acc(l_acc + rows),
+          list_n(reinterpret_cast<int32_t*>(o_acc + rows * kD)),
+          zero_bytes(4 * (size_t)rows + 4 * (size_t)rows * kD + 16) {}
+};
 
 }  // namespace
 
@@ -463,40 +504,50 @@ bool fwd_rows_supported(const Shape& s) {
 
 size_t fwd_rows_ws_bytes(const Shape& s) {
     const size_t rows = (size_t)s.B * s.Hq * s.T;
-    return 4 * rows + 4 * rows + 4 * rows * kD;
+    return 12 * rows + 4 * rows * kD + 16;
 }
 
 cudaError_t launch_fwd_rows(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
                             const float* gl, const int32_t* nsel, const uint64_t* maskT, void* ws, void* o,
                             float* lse, cudaStream_t st) {
     const int64_t rows = (int64_t)s.B * s.Hq * s.T;
-    uint32_t* rowmax = static_cast<uint32_t*>(ws);
-    float* l_acc = reinterpret_cast<float*>(rowmax + rows);
-    float* o_acc = l_acc + rows;
+    const RowsWs w(ws, rows);
     CUtensorMap mk, mv;
     FwdRowsArgs a{};
     if (!encode_bf16_2d(&mk, k, (uint64_t)s.B * s.Hkv * s.T, kD, kBS) ||
-        !encode_bf16_2d(&mv, v, (uint64_t)s.B * s.Hkv * s.T, kD, kBS) ||
-        !encode_bf16_2d(&a.tm_q, q, (uint64_t)rows, kD, 1))
+        !encode_bf16_2d(&mv, v, (uint64_t)s.B * s.Hkv * s.T, kD, kBS))
         return cudaErrorInvalidValue;
     a.sh = s;
+    a.q = static_cast<const __nv_bfloat16*>(q);
     a.idx = idx;
     a.gl = gl;
     a.nsel = nsel;
     a.maskT = maskT;
-    a.rowmax = rowmax;
-    a.l_acc = l_acc;
-    a.o_acc = o_acc;
+    a.shift = w.shift;
+    a.l_acc = w.l_acc;
+    a.o_acc = w.o_acc;
     a.tpc = kRows / s.G;
-    cudaError_t e = cudaMemsetAsync(ws, 0, fwd_rows_ws_bytes(s), st);
-    if (e == cudaSuccess) e = launch_pass<false>(mk, mv, a, st);
-    if (e == cudaSuccess) e = launch_pass<true>(mk, mv, a, st);
+    cudaError_t e = cudaMemsetAsync(w.l_acc, 0, w.zero_bytes, st);
     if (e != cudaSuccess) return e;
-    fwd_rows_finalize_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(rows, rowmax, l_acc, o_acc,
-                                                                          static_cast<__nv_bfloat16*>(o), lse);
+    fwd_rows_shift_kernel<<<(unsigned)((s.rows() + 7) / 8), 256, 0, st>>>(s, a.q, static_cast<const __nv_bfloat16*>(k),
+                                                                           w.shift);
     e = cudaGetLastError();
-    if (e == cudaSuccess) count_launches(1);
-    return e;
+    if (e != cudaSuccess) return e;
+    count_launches(1);
+    const size_t smem = RowsSmem::total(s.nT) + 1024;
+    e = cudaFuncSetAttribute(fwd_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    fwd_rows_kernel<<<(unsigned)((int64_t)s.B * s.Hkv * s.nT), kThreads, smem, st>>>(mk, mv, a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    count_launches(1);
+    fwd_rows_finalize_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(s, w.shift, w.l_acc, w.o_acc,
+                                                                         static_cast<__nv_bfloat16*>(o), lse, w.list,
+                                                                         w.list_n);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    count_launches(1);
+    return launch_fwd_simt_rows(s, q, k, v, idx, gl, nsel, w.list, w.list_n, o, lse, st);
 }
 
 cudaError_t read_fwd_rows_timeouts(unsigned int* out) {

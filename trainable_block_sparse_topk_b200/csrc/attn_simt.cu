@@ -23,23 +23,48 @@ namespace {
 
 // ------------------------------------------------------------------ forward ---
 
+template <typename T, int D, int GMAX, int BS>
+__device__ __forceinline__ void fwd_simt_row(const Shape& sh, const T* __restrict__ q, const T* __restrict__ k,
+                                             const T* __restrict__ v, const int32_t* __restrict__ idx,
+                                             const float* __restrict__ gl, const int32_t* __restrict__ nsel,
+                                             T* __restrict__ o, float* __restrict__ attn_lse, int64_t row,
+                                             float (*s_qw)[D], float (*s_pw)[GMAX], int lane);
+
 // One warp per (b, kv head, t) row, all G heads of the group at once. Lane
 // `l` scores keys l and l + 32 of each kept block and owns D/32 output dims.
+// With `list` set, the warps instead stride over the rows list[0 .. *list_n)
+// (recomputing rows another kernel flagged); otherwise warp w of block x takes
+// row 4 x + w.
 template <typename T, int D, int GMAX, int BS>
 __global__ void __launch_bounds__(128)
 fwd_simt_kernel(Shape sh, const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                 const int32_t* __restrict__ idx, const float* __restrict__ gl,
-                const int32_t* __restrict__ nsel, T* __restrict__ o, float* __restrict__ attn_lse) {
+                const int32_t* __restrict__ nsel, T* __restrict__ o, float* __restrict__ attn_lse,
+                const int32_t* __restrict__ list, const int32_t* __restrict__ list_n) {
     constexpr int W = 4;
+    __shared__ float s_q[W][GMAX][D];
+    __shared__ float s_p[W][BS][GMAX];
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (list != nullptr) {
+        const int n = *list_n;
+        for (int i = (int)blockIdx.x * W + w; i < n; i += (int)gridDim.x * W)
+            fwd_simt_row<T, D, GMAX, BS>(sh, q, k, v, idx, gl, nsel, o, attn_lse, list[i], s_q[w], s_p[w], lane);
+        return;
+    }
+    const int64_t row = (int64_t)blockIdx.x * W + w;
+    if (row >= sh.rows()) return;
+    fwd_simt_row<T, D, GMAX, BS>(sh, q, k, v, idx, gl, nsel, o, attn_lse, row, s_q[w], s_p[w], lane);
+}
+
+template <typename T, int D, int GMAX, int BS>
+__device__ __forceinline__ void fwd_simt_row(const Shape& sh, const T* __restrict__ q, const T* __restrict__ k,
+                                             const T* __restrict__ v, const int32_t* __restrict__ idx,
+                                             const float* __restrict__ gl, const int32_t* __restrict__ nsel,
+                                             T* __restrict__ o, float* __restrict__ attn_lse, int64_t row,
+                                             float (*s_qw)[D], float (*s_pw)[GMAX], int lane) {
     constexpr int KPL = BS / 32;
     constexpr int DPL = D / 32;
     constexpr int V16 = vec16<T>();
-    __shared__ float s_q[W][GMAX][D];
-    __shared__ float s_p[W][BS][GMAX];
-
-    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t row = (int64_t)blockIdx.x * W + w;
-    if (row >= sh.rows()) return;
     const int G = sh.G;
     const int64_t bg = row / sh.T;
     const int t = (int)(row % sh.T);
@@ -52,7 +77,7 @@ fwd_simt_kernel(Shape sh, const T* __restrict__ q, const T* __restrict__ k, cons
     for (int h = 0; h < GMAX; ++h) {
         if (h < G) {
             const T* qh = q + (((int64_t)b * sh.Hq + g * G + h) * sh.T + t) * D;
-            for (int d = lane; d < D; d += 32) s_q[w][h][d] = Elem<T>::to_f(qh[d]) * qscale;
+            for (int d = lane; d < D; d += 32) s_qw[h][d] = Elem<T>::to_f(qh[d]) * qscale;
         }
     }
     __syncwarp();
@@ -90,7 +115,7 @@ fwd_simt_kernel(Shape sh, const T* __restrict__ q, const T* __restrict__ k, cons
                     for (int h = 0; h < GMAX; ++h) {
                         if (h < G) {
 #pragma unroll
-                            for (int e = 0; e < V16; ++e) sc[kk][h] = fmaf(s_q[w][h][c * V16 + e], kv[e], sc[kk][h]);
+                            for (int e = 0; e < V16; ++e) sc[kk][h] = fmaf(s_qw[h][c * V16 + e], kv[e], sc[kk][h]);
                         }
                     }
                 }
@@ -114,7 +139,7 @@ fwd_simt_kernel(Shape sh, const T* __restrict__ q, const T* __restrict__ k, cons
 #pragma unroll
             for (int kk = 0; kk < KPL; ++kk) {
                 const float pk = (mn == -INFINITY) ? 0.f : exp2f(sc[kk][h] - mn);
-                s_p[w][lane + 32 * kk][h] = pk;
+                s_pw[lane + 32 * kk][h] = pk;
                 ps += pk;
             }
             ps = warp_sum(ps);
@@ -130,7 +155,7 @@ fwd_simt_kernel(Shape sh, const T* __restrict__ q, const T* __restrict__ k, cons
 #pragma unroll
             for (int h = 0; h < GMAX; ++h) {
                 if (h < G) {
-                    const float pk = s_p[w][key][h];
+                    const float pk = s_pw[key][h];
 #pragma unroll
                     for (int e = 0; e < DPL; ++e) acc[h][e] = fmaf(pk, vv[e], acc[h][e]);
                 }
@@ -372,7 +397,7 @@ cudaError_t run_fwd(const Shape& s, const void* q, const void* k, const void* v,
                     const float* gl, const int32_t* nsel, void* o, float* lse, cudaStream_t st) {
     const int64_t grid = (s.rows() + 3) / 4;
     fwd_simt_kernel<T, D, GMAX, BS><<<(unsigned)grid, 128, 0, st>>>(
-        s, (const T*)q, (const T*)k, (const T*)v, idx, gl, nsel, (T*)o, lse);
+        s, (const T*)q, (const T*)k, (const T*)v, idx, gl, nsel, (T*)o, lse, nullptr, nullptr);
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
     return e;
@@ -446,6 +471,23 @@ cudaError_t launch_fwd_simt(const Shape& s, const void* q, const void* k, const 
                             const float* gl, const int32_t* nsel, void* o, float* lse, cudaStream_t st) {
     if (s.dtype == SAS_DT_FP32) return fwd_d<float>(s, q, k, v, idx, gl, nsel, o, lse, st);
     return fwd_d<__nv_bfloat16>(s, q, k, v, idx, gl, nsel, o, lse, st);
+}
+
+cudaError_t launch_fwd_simt_rows(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
+                                 const float* gl, const int32_t* nsel, const int32_t* list, const int32_t* list_n,
+                                 void* o, float* lse, cudaStream_t st) {
+    if (s.dtype != SAS_DT_BF16 || s.D != 128 || s.bs != 64) return cudaErrorInvalidValue;
+    using B16 = __nv_bfloat16;
+    const unsigned grid = 148;   // a few warps per SM; the rows to redo are normally none
+    if (s.G <= 4)
+        fwd_simt_kernel<B16, 128, 4, 64><<<grid, 128, 0, st>>>(s, (const B16*)q, (const B16*)k, (const B16*)v, idx, gl,
+                                                               nsel, (B16*)o, lse, list, list_n);
+    else
+        fwd_simt_kernel<B16, 128, 8, 64><<<grid, 128, 0, st>>>(s, (const B16*)q, (const B16*)k, (const B16*)v, idx, gl,
+                                                               nsel, (B16*)o, lse, list, list_n);
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) count_launches(1);
+    return e;
 }
 
 cudaError_t launch_bwd_rowdot(const Shape& s, const void* o, const void* dO, float* Dd, cudaStream_t st) {

@@ -38,6 +38,11 @@ cudaError_t launch_sel_bitmap_T(const Shape& s, const int32_t* idx, const int32_
 cudaError_t launch_fwd_simt(const Shape& s, const void* q, const void* k, const void* v,
                             const int32_t* idx, const float* gate_logit, const int32_t* n_sel,
                             void* o, float* attn_lse, cudaStream_t st);
+// The CUDA-core forward over the (b, kv head, t) rows list[0 .. *list_n)
+// (device count); bf16, d 128, block 64.
+cudaError_t launch_fwd_simt_rows(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
+                                 const float* gl, const int32_t* nsel, const int32_t* list, const int32_t* list_n,
+                                 void* o, float* lse, cudaStream_t st);
 
 // 2D bf16 tensor map [rows x cols] with 64 x box_rows boxes, 128-byte swizzle.
 bool encode_bf16_2d(::CUtensorMap_st* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
