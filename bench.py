@@ -92,6 +92,18 @@ def traffic_record(kernel_file):
     return None
 
 
+def max_over_ranks(x, world, device):
+    """Max of a per-rank float (a device-timed duration) over all ranks of the
+    process group; the value itself at N = 1."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ------------------------------------------------------------------- clocks ---
 
 class ClockSampler:
@@ -294,11 +306,7 @@ def run_ours(args, rank, world, local_rank):
 
     part_ms = {p: [ev[i].elapsed_time(ev[i + 1]) for ev in evs] for i, p in enumerate(parts)}
     step_ms = [ev[0].elapsed_time(ev[5]) for ev in evs]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
 
     f_fwd, f_bwd, per_head_pairs = train_flops(tw)
     flops = f_fwd + f_bwd
@@ -431,12 +439,7 @@ def run_e2e(args, tw, dw, x, q1c, s1c, dc, vc, dev, dt, flops, world):
         step()
     e1.record(stream)
     torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     return {"value": flops * world * args.steps / (ms * 1e-3) / 1e12, "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms / args.steps}
 
