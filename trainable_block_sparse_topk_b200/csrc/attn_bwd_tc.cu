@@ -23,8 +23,9 @@
 // dK^T [448,512). S/dP of chunk c+1 are computed while warps 4-7 build P/dS
 // of chunk c and warps 0-3 read back and add dQ of chunk c-1.
 //
-// Roles (384 threads): warps 0-3 epilogue (dQ reductions, final dK/dV),
-// warps 4-7 P/dS and Gsum (thread = row = TMEM lane in both groups), warps 8
+// Roles (512 threads): warps 0-3 epilogue (dQ reductions, final dK/dV),
+// warps 4-7 and 12-15 P/dS and Gsum for keys 0-31 and 32-63 of the block
+// (thread = row = TMEM lane in every group), warps 8
 // and 11 gather chunk rows (even / odd chunks) with coalesced 16-byte cp.async
 // copies into the two 128-byte-swizzled Q/dO stages (TMA tile::gather4 moves
 // random rows at a fraction of that rate; warp 8 also loads K_j, V_j by TMA),
@@ -40,7 +41,7 @@ namespace sas {
 
 namespace {
 
-constexpr int kThreads = 384;   // epilogue warps 0-3, P/dS warps 4-7, loaders 8 and 11, MMA 9, TMEM 10
+constexpr int kThreads = 512;   // epilogue warps 0-3, P/dS warps 4-7 and 12-15, loaders 8 and 11, MMA 9, TMEM 10
 constexpr int kBS = 64;
 constexpr int kRows = 128;
 constexpr int kD = 128;
@@ -112,7 +113,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     uint64_t* st_full = bars + 1;     // [2], the loader's arrive once its copies have landed
     uint64_t* st_empty = bars + 3;    // [2]
     uint64_t* s_full = bars + 5;      // [2]
-    uint64_t* p_full = bars + 7;      // 4 arrivals (compute warps)
+    uint64_t* p_full = bars + 7;      // 8 arrivals (P/dS warps)
     uint64_t* p_empty = bars + 8;
     uint64_t* dq_full = bars + 9;
     uint64_t* dq_empty = bars + 10;   // 4 arrivals
@@ -138,7 +139,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         for (int i = 0; i < L::kNumBars; ++i) {
             uint64_t* bar = &bars[i];
             uint32_t cnt = 1;
-            if (bar == p_full || bar == dq_empty || bar == &ids_full[0] || bar == &ids_full[1]) cnt = 4;
+            if (bar == dq_empty || bar == &ids_full[0] || bar == &ids_full[1]) cnt = 4;
+            if (bar == p_full) cnt = 8;
             if (bar == &st_full[0] || bar == &st_full[1]) cnt = 33;   // 32 cp.async arrivals + the loader's
             mbar_init(bar, cnt);
         }
@@ -211,14 +213,31 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             for (int r = s - pre[lo]; r > 0; --r) w &= w - 1ull;
             return lo * kBS + __ffsll((long long)w) - 1;
         };
-        // metadata of chunk c into ring slot c & 3 (global loads only; no stage needed)
+        // metadata of chunk c into ring slot c & 3 (global loads only; no stage
+        // needed). Independent loads go out together -- every row's lse and D
+        // with every token's kept list -- then the log-gates of block j.
         auto prep = [&](int c) {
             Meta meta(sm + L::kMeta + (c & 3) * L::kMetaBytes);
             const int n = min(tpc, ntok_total - c * tpc);
             if (lane == 0) *meta.ntok = n;
+            for (int i = lane; i < n; i += 32) meta.tok_t[i] = token_at(c * tpc + i);
+            __syncwarp();
+            float lse[kRows / 32], Dv[kRows / 32];
+            int qrow[kRows / 32];
+#pragma unroll
+            for (int u = 0; u < kRows / 32; ++u) {
+                const int i = lane + 32 * u, ti = i / G, h = i - ti * G;
+                qrow[u] = -1;
+                lse[u] = 0.f;
+                Dv[u] = 0.f;
+                if (ti < n) {
+                    qrow[u] = (int)(((int64_t)b * sh.Hq + g * G + h) * T + meta.tok_t[ti]);
+                    lse[u] = a.lse[qrow[u]];
+                    Dv[u] = a.Dd[qrow[u]];
+                }
+            }
             for (int i = lane; i < n; i += 32) {
-                const int t = token_at(c * tpc + i);
-                meta.tok_t[i] = t;
+                const int t = meta.tok_t[i];
                 int slot = -1;
                 float lg = 0.f;
                 if ((t >> 6) != j) {
@@ -227,32 +246,28 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                     const int32_t* ir = a.idx + row * K;
                     const int ns = a.nsel[row];
                     int below = 0;
-#pragma unroll 8
-                    for (int s = 0; s < K; ++s) below += (s < ns && ir[s] < j) ? 1 : 0;
+#pragma unroll 16
+                    for (int s = 0; s < K; ++s) {
+                        const int v = ir[s];
+                        below += (s < ns) & (v < j);
+                    }
                     slot = min(below, K - 1);
                     lg = a.gl[row * K + slot];
                 }
                 meta.tok_slot[i] = slot;
                 meta.tok_lg[i] = lg;
             }
-            __syncwarp();
-            for (int i = lane; i < kRows; i += 32) {
-                const int ti = i / G, h = i - ti * G;
-                float lse = 0.f, Dv = 0.f;
-                int qrow = -1;
-                if (ti < n) {
-                    qrow = (int)(((int64_t)b * sh.Hq + g * G + h) * T + meta.tok_t[ti]);
-                    lse = a.lse[qrow];
-                    Dv = a.Dd[qrow];
-                }
-                meta.row_lse[i] = lse;
-                meta.row_D[i] = Dv;
-                meta.qoff[i] = qrow;
-                if (qrow >= 0) {              // the rows are copied about two chunks later
-                    tc::prefetch_l2(a.q + (int64_t)qrow * kD);
-                    tc::prefetch_l2(a.q + (int64_t)qrow * kD + 64);
-                    tc::prefetch_l2(a.dO + (int64_t)qrow * kD);
-                    tc::prefetch_l2(a.dO + (int64_t)qrow * kD + 64);
+#pragma unroll
+            for (int u = 0; u < kRows / 32; ++u) {
+                const int i = lane + 32 * u;
+                meta.row_lse[i] = lse[u];
+                meta.row_D[i] = Dv[u];
+                meta.qoff[i] = qrow[u];
+                if (qrow[u] >= 0) {           // the rows are copied about two chunks later
+                    tc::prefetch_l2(a.q + (int64_t)qrow[u] * kD);
+                    tc::prefetch_l2(a.q + (int64_t)qrow[u] * kD + 64);
+                    tc::prefetch_l2(a.dO + (int64_t)qrow[u] * kD);
+                    tc::prefetch_l2(a.dO + (int64_t)qrow[u] * kD + 64);
                 }
             }
             __syncwarp();
@@ -367,13 +382,16 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                     *abort = 1;
                     atomicAdd(&g_sas_wait_timeouts, 1u);
                     ok = false;
+                } else {
+                    __nanosleep(40);   // back off: leave issue slots to the other warps of this SMSP
                 }
             }
             tc::mma_commit(done);
         }
-    } else if (warp >= 4 && warp < 8) {
-        // ------------------------------------------- P / dS warps (4 - 7) ---
-        const int r = (warp - 4) * 32 + lane;      // chunk row == TMEM lane
+    } else if ((warp >= 4 && warp < 8) || warp >= 12) {
+        // ------------------------------ P / dS warps (4 - 7: keys 0-31, 12 - 15: keys 32-63) ---
+        const int r = (warp & 3) * 32 + lane;      // chunk row == TMEM lane
+        const int hf = warp >= 12 ? 1 : 0;         // which 32 keys of the block
         const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const float qk = sh.scale * kLog2e;
         for (int c = 0; c < nc; ++c) {
@@ -405,13 +423,14 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             // means the epilogue warps are done with chunk c-2, whose row-id slot
             // is reused here
             if (c >= 1 && !tc::warp_wait_bar(p_empty, (uint32_t)((c - 1) & 1), abort)) break;
-            ids[st * kRows + r] = dq_row;
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&ids_full[st]);
+            if (hf == 0) {
+                ids[st * kRows + r] = dq_row;
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&ids_full[st]);
+            }
             tc::fence_after_sync();
             float rowsum = 0.f;
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {           // 32 keys at a time
+            {
                 uint32_t sv[32], pv[32];
 #pragma unroll
                 for (int cb = 0; cb < 2; ++cb) {
@@ -451,8 +470,8 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             // Gsum of the token: its G rows are in this chunk
             float* gs = tok_gs + st * kRows;
             if (valid && !diag) atomicAdd(&gs[ti], rowsum);
-            tc::named_bar(1, 128);
-            if (r < n) {
+            tc::named_bar(1, 256);
+            if (hf == 0 && r < n) {
                 if (gs_slot >= 0) a.gsum[((int64_t)bg * T + gs_tok) * K + gs_slot] = gs[r];
                 gs[r] = 0.f;
             }
@@ -477,45 +496,41 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             if (!tc::warp_wait_bar(dq_full, (uint32_t)(c & 1), abort)) { ok = false; break; }
             tc::fence_after_sync();
 #pragma unroll 1
-            for (int hb = 0; hb < 2; ++hb) {           // 64 columns at a time
-                uint32_t v[64];
-#pragma unroll
-                for (int cb = 0; cb < 4; ++cb) tc::tmem_ld16(lane_base + kColDQ + hb * 64 + cb * 16, v + cb * 16);
+            for (int cb = 0; cb < kD / 16; ++cb) {      // 16 columns at a time
+                uint32_t v[16];
+                tc::tmem_ld16(lane_base + kColDQ + cb * 16, v);
                 tc::tmem_wait_ld();
-                if (hb == 1) {                          // dQ of this chunk is out of TMEM
+                if (cb == kD / 16 - 1) {                 // dQ of this chunk is out of TMEM
                     tc::fence_before_sync();
                     __syncwarp();
                     if (lane == 0) tc::mbar_arrive(dq_empty);
                 }
+                float x[16];
 #pragma unroll
-                for (int cb = 0; cb < 4; ++cb) {
-                    float x[16];
+                for (int e = 0; e < 16; ++e) x[e] = __uint_as_float(v[e]) * dscale;
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) x[e] = __uint_as_float(v[cb * 16 + e]) * dscale;
+                for (int m = 1; m <= 2; m <<= 1) {
 #pragma unroll
-                    for (int m = 1; m <= 2; m <<= 1) {
+                    for (int k0 = 0; k0 < 4; ++k0) {
+                        if (k0 & m) continue;
+                        const int k1 = k0 | m;
+                        const bool hi = (qd & m) != 0;
 #pragma unroll
-                        for (int k0 = 0; k0 < 4; ++k0) {
-                            if (k0 & m) continue;
-                            const int k1 = k0 | m;
-                            const bool hi = (qd & m) != 0;
-#pragma unroll
-                            for (int f = 0; f < 4; ++f) {
-                                const float snd = hi ? x[k0 * 4 + f] : x[k1 * 4 + f];
-                                const float rcv = __shfl_xor_sync(0xffffffffu, snd, m);
-                                if (hi) x[k0 * 4 + f] = rcv; else x[k1 * 4 + f] = rcv;
-                            }
+                        for (int f = 0; f < 4; ++f) {
+                            const float snd = hi ? x[k0 * 4 + f] : x[k1 * 4 + f];
+                            const float rcv = __shfl_xor_sync(0xffffffffu, snd, m);
+                            if (hi) x[k0 * 4 + f] = rcv; else x[k1 * 4 + f] = rcv;
                         }
                     }
-                    // x[4e .. 4e+3] = columns 4 qd .. 4 qd + 3 of this 16-column
-                    // slice, row (lane & ~3) + e
-                    const int col = hb * 64 + cb * 16 + qd * 4;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        if (rows4[e] >= 0)
-                            tc::red_add_v4(a.dq_acc + (int64_t)rows4[e] * kD + col, x[4 * e], x[4 * e + 1],
-                                           x[4 * e + 2], x[4 * e + 3]);
                 }
+                // x[4e .. 4e+3] = columns 4 qd .. 4 qd + 3 of this 16-column
+                // slice, row (lane & ~3) + e
+                const int col = cb * 16 + qd * 4;
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (rows4[e] >= 0)
+                        tc::red_add_v4(a.dq_acc + (int64_t)rows4[e] * kD + col, x[4 * e], x[4 * e + 1],
+                                       x[4 * e + 2], x[4 * e + 3]);
             }
         }
         // dV^T and dK^T: TMEM lane r holds column r of d for the block's 64 keys

@@ -193,13 +193,29 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             for (int r = s - pre[lo]; r > 0; --r) w &= w - 1ull;
             return lo * kBS + __ffsll((long long)w) - 1;
         };
+        // metadata of chunk c into ring slot c & 3. Independent loads go out
+        // together -- every row's shift with every token's kept list -- then
+        // the log-gates of block j.
         auto prep = [&](int c) {
             RowMeta meta(sm + L::kMeta + (c & 3) * L::kMetaBytes);
             const int n = min(tpc, ntok_total - c * tpc);
             if (lane == 0) *meta.ntok = n;
+            for (int i = lane; i < n; i += 32) meta.tok_t[i] = token_at(c * tpc + i);
+            __syncwarp();
+            float m[kRows / 32];
+            int qrow[kRows / 32];
+#pragma unroll
+            for (int u = 0; u < kRows / 32; ++u) {
+                const int i = lane + 32 * u, ti = i / G, h = i - ti * G;
+                qrow[u] = -1;
+                m[u] = 0.f;
+                if (ti < n) {
+                    qrow[u] = (int)(((int64_t)b * sh.Hq + g * G + h) * T + meta.tok_t[ti]);
+                    m[u] = a.shift[qrow[u]];
+                }
+            }
             for (int i = lane; i < n; i += 32) {
-                const int t = token_at(c * tpc + i);
-                meta.tok_t[i] = t;
+                const int t = meta.tok_t[i];
                 float lg = 0.f;
                 if ((t >> 6) != j) {
                     // log-gate of block j in the token's ascending kept list
@@ -207,26 +223,23 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     const int32_t* ir = a.idx + row * K;
                     const int ns = a.nsel[row];
                     int below = 0;
-#pragma unroll 8
-                    for (int s = 0; s < K; ++s) below += (s < ns && ir[s] < j) ? 1 : 0;
+#pragma unroll 16
+                    for (int s = 0; s < K; ++s) {
+                        const int v = ir[s];
+                        below += (s < ns) & (v < j);
+                    }
                     lg = a.gl[row * K + min(below, K - 1)];
                 }
                 meta.tok_lg[i] = lg;
             }
-            __syncwarp();
-            for (int i = lane; i < kRows; i += 32) {
-                const int ti = i / G, h = i - ti * G;
-                int qrow = -1;
-                float m = 0.f;
-                if (ti < n) {
-                    qrow = (int)(((int64_t)b * sh.Hq + g * G + h) * T + meta.tok_t[ti]);
-                    m = a.shift[qrow];
-                }
-                meta.row_m[i] = m;
-                meta.qoff[i] = qrow;
-                if (qrow >= 0) {              // the row is copied about two chunks later
-                    tc::prefetch_l2(a.q + (int64_t)qrow * kD);
-                    tc::prefetch_l2(a.q + (int64_t)qrow * kD + 64);
+#pragma unroll
+            for (int u = 0; u < kRows / 32; ++u) {
+                const int i = lane + 32 * u;
+                meta.row_m[i] = m[u];
+                meta.qoff[i] = qrow[u];
+                if (qrow[u] >= 0) {           // the row is copied about two chunks later
+                    tc::prefetch_l2(a.q + (int64_t)qrow[u] * kD);
+                    tc::prefetch_l2(a.q + (int64_t)qrow[u] * kD + 64);
                 }
             }
             __syncwarp();
@@ -315,6 +328,8 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         *abort = 1;
                         atomicAdd(&g_sas_wait_timeouts, 1u);
                         ok = false;
+                    } else {
+                        __nanosleep(40);   // back off: leave issue slots to the other warps of this SMSP
                     }
                 }
             }
