@@ -47,11 +47,7 @@ constexpr int kD = 128;
 struct FwdRowsArgs {
     Shape sh;
     const __nv_bfloat16* q;   // [B*Hq*T, d]
-    const int32_t* idx;
-    const float* gl;
-    const int32_t* nsel;
-    const uint64_t* maskT;
-    const float* shift;   // [B*Hq*T] the row's softmax shift M (log2 units)
+    SelStream ss;         // per-block token streams: {t, log-gate}, the shift M of each head
     float* l_acc;         // [B*Hq*T]
     float* o_acc;         // [B*Hq*T, d]
     int tpc;              // tokens per chunk = 128 / G
@@ -65,28 +61,22 @@ struct RowsSmem {
     static constexpr uint32_t kP = kStage + 2 * kStageBytes;       // P [128 x 128 B]
     static constexpr uint32_t kOst = kP + 16384;                   // O rows, fp32, kOstRow apart
     static constexpr uint32_t kOstRow = kD * 4 + 16;               // padded: conflict-free 16-byte stores
-    static constexpr uint32_t kMeta = kOst + kRows * kOstRow;      // 4 x per-chunk metadata
-    static constexpr uint32_t kMetaBytes = 4 * 512 + 16;           // tok_t, tok_lg, row_m, qoff, ntok
+    static constexpr uint32_t kMeta = kOst + kRows * kOstRow;      // 4 x chunk stream entries (chunk c -> slot c & 3)
+    static constexpr uint32_t kMetaBytes = 4096;                   // int4 ent[<=128], then f32 rv[<= 512]
     static constexpr uint32_t kBar = kMeta + 4 * kMetaBytes;
-    static constexpr int kNumBars = 14;
-    static constexpr uint32_t kMisc = kBar + 8 * kNumBars;         // tmem base, token count, abort
-    static constexpr uint32_t kColW = kMisc + 16;                  // u64 [nT] bitmap column, then i32 [nT] prefix
+    static constexpr int kNumBars = 18;
+    static constexpr uint32_t kMisc = kBar + 8 * kNumBars;         // tmem base, stream length, first entry, abort
     static constexpr uint32_t kTmemCols = 512;                     // S double [0,128), O double [128,384)
-    static uint32_t total(int nT) { return kColW + 12 * (uint32_t)nT + 16; }
+    static constexpr uint32_t kTotal = kMisc + 16;
 };
 
+// One ring slot: the chunk's stream entries (token, log-gate) and each entry's
+// per-head shift, copied in by the bulk-copy engine.
 struct RowMeta {
-    int* tok_t;
-    float* tok_lg;
-    float* row_m;
-    int* qoff;
-    int* ntok;
-    __device__ explicit RowMeta(unsigned char* p)
-        : tok_t(reinterpret_cast<int*>(p)),
-          tok_lg(reinterpret_cast<float*>(p + 512)),
-          row_m(reinterpret_cast<float*>(p + 1024)),
-          qoff(reinterpret_cast<int*>(p + 1536)),
-          ntok(reinterpret_cast<int*>(p + 2048)) {}
+    const int4* ent;
+    const float* rv;
+    __device__ explicit RowMeta(const unsigned char* p)
+        : ent(reinterpret_cast<const int4*>(p)), rv(reinterpret_cast<const float*>(p + 2048)) {}
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -104,21 +94,20 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     uint64_t* p_empty = bars + 8;
     uint64_t* o_full = bars + 9;      // [2]
     uint64_t* o_empty = bars + 11;    // [2] 4 arrivals
+    uint64_t* meta_full = bars + 13;  // [4] ring slot c & 3 holds chunk c's stream entries (tx bytes)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMisc);
-    int* ntok_slot = reinterpret_cast<int*>(sm + L::kMisc + 4);
-    volatile int* abort = reinterpret_cast<volatile int*>(sm + L::kMisc + 8);
+    int* ntok_slot = reinterpret_cast<int*>(sm + L::kMisc + 4);      // [2]: stream length, first entry
+    volatile int* abort = reinterpret_cast<volatile int*>(sm + L::kMisc + 12);
 
     const Shape& sh = a.sh;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int G = sh.G, K = sh.K, T = sh.T;
+    const int G = sh.G, T = sh.T;
     const int ngroups = sh.B * sh.Hkv;
     const int j = (int)(blockIdx.x / ngroups);
     const int bg = (int)(blockIdx.x % ngroups);
     const int b = bg / sh.Hkv, g = bg % sh.Hkv;
     const int tpc = a.tpc;
-    const uint64_t* col = a.maskT + ((int64_t)bg * sh.NB + j) * sh.nT;
-    unsigned long long* colw = reinterpret_cast<unsigned long long*>(sm + L::kColW);
-    int* pre = reinterpret_cast<int*>(sm + L::kColW + 8 * sh.nT);
+    const int rvs = a.ss.rvs;
 
     if (tid == 0) {
         for (int i = 0; i < L::kNumBars; ++i) {
@@ -132,6 +121,8 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             if (bar == &st_full[0] || bar == &st_full[1]) cnt = 33;   // 32 cp.async arrivals + the loader's
             mbar_init(bar, cnt);
         }
+        ntok_slot[0] = a.ss.count[(int64_t)bg * sh.NB + j];   // tokens in block j's stream
+        ntok_slot[1] = a.ss.base[(int64_t)bg * sh.NB + j];    // its first entry
         *abort = 0;
         fence_mbar_init();
     }
@@ -139,32 +130,12 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         tc::tmem_alloc(tmem_slot, L::kTmemCols);
         tc::tmem_relinquish();
     }
-    // token stream of block j: its own 64 tokens, then later tokens that kept j
-    for (int tau = tid; tau < sh.nT; tau += kThreads) colw[tau] = tau > j ? col[tau] : 0ull;
-    __syncthreads();
-    if (warp == 0) {
-        const int per = (sh.nT + 31) / 32;
-        const int t0 = lane * per, t1 = min(t0 + per, sh.nT);
-        int sum = 0;
-        for (int tau = t0; tau < t1; ++tau) sum += __popcll(colw[tau]);
-        int inc = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, inc, o);
-            if (lane >= o) inc += y;
-        }
-        int run = kBS + inc - sum;
-        for (int tau = t0; tau < t1; ++tau) {
-            pre[tau] = run;
-            run += __popcll(colw[tau]);
-        }
-        if (lane == 31) *ntok_slot = kBS + inc;
-    }
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const int ntok_total = *ntok_slot;
+    const int ntok_total = ntok_slot[0];
+    const int64_t ebase = ntok_slot[1];
     const int nc = (ntok_total + tpc - 1) / tpc;
     const uint32_t sbase = smem_u32(sm);
 
@@ -182,83 +153,37 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 tc::tma_load_2d(sm + L::kV + h * 8192, &tm_v, h * 64, kr, kv_full);
             }
         }
-        auto token_at = [&](int s) -> int {
-            if (s < kBS) return j * kBS + s;
-            int lo = j + 1, hi = sh.nT - 1;      // last tile with pre[tile] <= s
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (pre[mid] <= s) lo = mid; else hi = mid - 1;
+        // chunk c's stream entries -> ring slot c & 3 (bulk copies, completion on meta_full)
+        auto request = [&](int c) {
+            if (lane == 0) {
+                const int n = min(tpc, ntok_total - c * tpc);
+                const int64_t e0 = ebase + (int64_t)c * tpc;
+                unsigned char* slot = sm + L::kMeta + (c & 3) * L::kMetaBytes;
+                const uint32_t be = 16u * (uint32_t)n, br = 4u * (uint32_t)(n * rvs);
+                mbar_arrive_expect_tx(&meta_full[c & 3], be + br);
+                bulk_g2s(slot, a.ss.ent + e0, be, &meta_full[c & 3]);
+                bulk_g2s(slot + 2048, a.ss.rv + e0 * rvs, br, &meta_full[c & 3]);
             }
-            uint64_t w = colw[lo];
-            for (int r = s - pre[lo]; r > 0; --r) w &= w - 1ull;
-            return lo * kBS + __ffsll((long long)w) - 1;
         };
-        // metadata of chunk c into ring slot c & 3. Independent loads go out
-        // together -- every row's shift with every token's kept list -- then
-        // the log-gates of block j.
-        auto prep = [&](int c) {
-            RowMeta meta(sm + L::kMeta + (c & 3) * L::kMetaBytes);
-            const int n = min(tpc, ntok_total - c * tpc);
-            if (lane == 0) *meta.ntok = n;
-            for (int i = lane; i < n; i += 32) meta.tok_t[i] = token_at(c * tpc + i);
-            __syncwarp();
-            float m[kRows / 32];
-            int qrow[kRows / 32];
-#pragma unroll
-            for (int u = 0; u < kRows / 32; ++u) {
-                const int i = lane + 32 * u, ti = i / G, h = i - ti * G;
-                qrow[u] = -1;
-                m[u] = 0.f;
-                if (ti < n) {
-                    qrow[u] = (int)(((int64_t)b * sh.Hq + g * G + h) * T + meta.tok_t[ti]);
-                    m[u] = a.shift[qrow[u]];
-                }
-            }
-            for (int i = lane; i < n; i += 32) {
-                const int t = meta.tok_t[i];
-                float lg = 0.f;
-                if ((t >> 6) != j) {
-                    // log-gate of block j in the token's ascending kept list
-                    const int64_t row = (int64_t)bg * T + t;
-                    const int32_t* ir = a.idx + row * K;
-                    const int ns = a.nsel[row];
-                    int below = 0;
-#pragma unroll 16
-                    for (int s = 0; s < K; ++s) {
-                        const int v = ir[s];
-                        below += (s < ns) & (v < j);
-                    }
-                    lg = a.gl[row * K + min(below, K - 1)];
-                }
-                meta.tok_lg[i] = lg;
-            }
-#pragma unroll
-            for (int u = 0; u < kRows / 32; ++u) {
-                const int i = lane + 32 * u;
-                meta.row_m[i] = m[u];
-                meta.qoff[i] = qrow[u];
-                if (qrow[u] >= 0) {           // the row is copied about two chunks later
-                    tc::prefetch_l2(a.q + (int64_t)qrow[u] * kD);
-                    tc::prefetch_l2(a.q + (int64_t)qrow[u] * kD + 64);
-                }
-            }
-            __syncwarp();
-        };
-        if (L0 < nc) prep(L0);
+        if (L0 < nc) request(L0);
         for (int c = L0; c < nc; c += 2) {
             if (c >= 2 && !tc::warp_wait_bar(&st_empty[L0], (uint32_t)(((c >> 1) - 1) & 1), abort)) break;
-            const int* qoff = RowMeta(sm + L::kMeta + (c & 3) * L::kMetaBytes).qoff;
+            // slot (c + 2) & 3 held chunk c - 2, whose readers are done with it once its stage is released
+            if (c + 2 < nc) request(c + 2);
+            if (!tc::warp_wait_bar(&meta_full[c & 3], (uint32_t)((c >> 2) & 1), abort)) break;
+            const int4* ent = RowMeta(sm + L::kMeta + (c & 3) * L::kMetaBytes).ent;
+            const int n = min(tpc, ntok_total - c * tpc);
             {
                 // 16 lanes copy one 256-byte q row (16-byte pieces, coalesced), two
                 // rows per instruction; piece p lands in d-half p / 8 at 16-byte
                 // chunk p % 8 of the swizzled row. Padding rows re-read a valid row.
                 const int p = lane & 15, hh = p >> 3, col = (p & 7) * 8;
-                const int q0 = qoff[0];
 #pragma unroll 4
                 for (int i = 0; i < kRows / 2; ++i) {
                     const int row = 2 * i + (lane >> 4);
-                    int qrow = qoff[row];
-                    if (qrow < 0) qrow = q0;
+                    int ti = row / G, h = row - ti * G;
+                    if (ti >= n) ti = 0, h = 0;
+                    const int qrow = (int)(((int64_t)b * sh.Hq + g * G + h) * T + ent[ti].x);
                     tc::cp_async16(stq + hh * 16384 + tc::sw128_offset(row, col), a.q + (int64_t)qrow * kD + p * 8);
                 }
             }
@@ -268,7 +193,6 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             tc::cp_async_mbar_arrive_noinc(&st_full[L0]);
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&st_full[L0]);
-            if (c + 2 < nc) prep(c + 2);   // overlaps the copies in flight
         }
         tc::cp_async_wait_all();
     } else if (warp == 1) {
@@ -373,19 +297,20 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         for (int c = 0; c < nc; ++c) {
             const int st = c & 1;
             if (!tc::warp_wait_bar(&st_full[st], (uint32_t)((c >> 1) & 1), abort)) { ok = false; break; }
-            RowMeta meta(sm + L::kMeta + (c & 3) * L::kMetaBytes);
-            const int n = *meta.ntok;
-            const int ti = r / G;
+            const RowMeta meta(sm + L::kMeta + (c & 3) * L::kMetaBytes);
+            const int n = min(tpc, ntok_total - c * tpc);
+            const int ti = r / G, h = r - ti * G;
             const bool valid = ti < n;
             int kmax = -1;
             float lg2 = 0.f, m = 0.f;
             int qrow = -1;
             if (valid) {
-                const int t = meta.tok_t[ti];
+                const int4 e = meta.ent[ti];
+                const int t = e.x;
                 kmax = ((t >> 6) == j) ? (t & 63) : kBS - 1;
-                lg2 = meta.tok_lg[ti] * kLog2e;
-                m = meta.row_m[r];
-                qrow = meta.qoff[r];
+                lg2 = __int_as_float(e.y) * kLog2e;
+                m = meta.rv[ti * rvs + h];
+                qrow = (int)(((int64_t)b * sh.Hq + g * G + h) * T + t);
             }
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&st_empty[st]);
@@ -493,7 +418,8 @@ fwd_rows_finalize_kernel(Shape sh, const float* __restrict__ shift, const float*
     if (lane == 0) lse[row] = (shift[row] + log2f(l)) * kLn2;
 }
 
-// Workspace: shift [rows] f32 | list [rows] i32 | l [rows] f32 | O [rows, d] f32 | list count
+// Workspace: shift [rows] f32 | list [rows] i32 | l [rows] f32 | O [rows, d] f32 | list count |
+// (256-aligned) the token streams
 struct RowsWs {
     float* shift;
     int32_t* list;
@@ -508,6 +434,7 @@ struct RowsWs {
           o_acc(l_acc + rows),
           list_n(reinterpret_cast<int32_t*>(o_acc + rows * kD)),
           zero_bytes(4 * (size_t)rows + 4 * (size_t)rows * kD + 16) {}
+    static size_t head_bytes(int64_t rows) { return (12 * (size_t)rows + 4 * (size_t)rows * kD + 16 + 255) & ~(size_t)255; }
 };
 
 }  // namespace
@@ -518,8 +445,7 @@ bool fwd_rows_supported(const Shape& s) {
 }
 
 size_t fwd_rows_ws_bytes(const Shape& s) {
-    const size_t rows = (size_t)s.B * s.Hq * s.T;
-    return 12 * rows + 4 * rows * kD + 16;
+    return RowsWs::head_bytes((int64_t)s.B * s.Hq * s.T) + sel_stream_bytes(s, 1);
 }
 
 cudaError_t launch_fwd_rows(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
@@ -534,11 +460,7 @@ cudaError_t launch_fwd_rows(const Shape& s, const void* q, const void* k, const 
         return cudaErrorInvalidValue;
     a.sh = s;
     a.q = static_cast<const __nv_bfloat16*>(q);
-    a.idx = idx;
-    a.gl = gl;
-    a.nsel = nsel;
-    a.maskT = maskT;
-    a.shift = w.shift;
+    a.ss = sel_stream_at(static_cast<unsigned char*>(ws) + RowsWs::head_bytes(rows), s, 1);
     a.l_acc = w.l_acc;
     a.o_acc = w.o_acc;
     a.tpc = kRows / s.G;
@@ -549,7 +471,9 @@ cudaError_t launch_fwd_rows(const Shape& s, const void* q, const void* k, const 
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launches(1);
-    const size_t smem = RowsSmem::total(s.nT) + 1024;
+    e = launch_sel_stream(s, maskT, idx, gl, nsel, w.shift, nullptr, 1, a.ss, st);
+    if (e != cudaSuccess) return e;
+    const size_t smem = RowsSmem::kTotal + 1024;
     e = cudaFuncSetAttribute(fwd_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     fwd_rows_kernel<<<(unsigned)((int64_t)s.B * s.Hkv * s.nT), kThreads, smem, st>>>(mk, mv, a);

@@ -34,6 +34,27 @@ bool topk_row_supported(int64_t max_candidates);
 cudaError_t launch_sel_bitmap_T(const Shape& s, const int32_t* idx, const int32_t* n_sel,
                                 uint64_t* maskT, cudaStream_t st);
 
+// Per-key-block token streams of the gathered-row kernels (stream.cu). For
+// block (b, g, j): entries base[(b*Hkv+g)*NB+j] .. + count[...], each
+// ent = {t, bits of the log-gate of j for t, slot of j in t's kept list, 0}
+// and rv[e*rvs + h*vals + v] = row value v (v0, v1) of query head h of token t.
+struct SelStream {
+    int4* ent;
+    float* rv;
+    int* base;
+    int* count;
+    int* pre;       // [blocks, nT]: entries before query tile tau in block j's run (tau > j)
+    int* counter;   // allocation counter, zeroed by launch_sel_stream
+    int rvs;        // floats per entry in rv (G * vals rounded up to 4)
+};
+int sel_stream_rvs(const Shape& s, int vals);
+int64_t sel_stream_capacity(const Shape& s);
+size_t sel_stream_bytes(const Shape& s, int vals);
+SelStream sel_stream_at(void* ws, const Shape& s, int vals);
+cudaError_t launch_sel_stream(const Shape& s, const uint64_t* maskT, const int32_t* idx, const float* gl,
+                              const int32_t* nsel, const float* v0, const float* v1, int vals, const SelStream& st,
+                              cudaStream_t stream);
+
 // Query-centric CUDA-core forward (fp32 and bf16).
 cudaError_t launch_fwd_simt(const Shape& s, const void* q, const void* k, const void* v,
                             const int32_t* idx, const float* gate_logit, const int32_t* n_sel,
