@@ -188,6 +188,23 @@ sas_status sas_device_timeouts(uint32_t* count);
  * successful launch. Memsets issued through the runtime are not counted. */
 uint64_t sas_kernel_launches(void);
 
+/* Diagnostics (no counterpart on the pages): per-kernel device time.
+ * sas_kernel_timing(names) clears earlier records and makes every later
+ * entry-point call record a pair of CUDA events on its stream around each
+ * kernel it launches whose name is in `names`, a comma-separated list of
+ * kernel names ("bwd_tc", "fwd_rows", "block_topk", "decode_partial", ... --
+ * the kernel names without the "_kernel" suffix), or around every kernel when
+ * `names` is "*". sas_kernel_timing(NULL) stops recording and keeps the
+ * records. Each recorded pair costs a few microseconds of device time between
+ * kernels, so time only what is needed. Not for use while a stream is being
+ * captured into a CUDA graph.
+ * sas_kernel_time(name, &ms, &n) waits for the recorded events of that kernel
+ * and returns their summed duration (ms) and count (n; 0 and 0.0 if none).
+ * Returns SAS_ERR_INVALID_ARG for a NULL argument, SAS_ERR_CUDA if an event
+ * could not be created, recorded or read. Records are process-wide. */
+sas_status sas_kernel_timing(const char* names);
+sas_status sas_kernel_time(const char* kernel, double* total_ms, uint32_t* launches);
+
 /* Static, NUL-terminated description of a status code (never NULL). */
 const char* sas_status_string(sas_status status);
 

@@ -177,3 +177,12 @@ def test_binding_refuses_host_tensors(L):
     s = torch.zeros(1, 2, 256, 4)
     with pytest.raises(ValueError):
         B.sas_block_topk(d, s, s, s, s, s)
+
+
+def test_kernel_timing_records_nothing_without_launches(L):
+    assert B.sas_kernel_timing("*") is None
+    assert B.sas_kernel_time("bwd_tc") == (0.0, 0)
+    assert B.sas_kernel_timing(None) is None
+    ms, n = ctypes.c_double(1.0), ctypes.c_uint32(7)
+    assert L.sas_kernel_time(None, ctypes.byref(ms), ctypes.byref(n)) == B.SAS_ERR_INVALID_ARG
+    assert L.sas_kernel_time(b"fwd_rows", None, ctypes.byref(n)) == B.SAS_ERR_INVALID_ARG

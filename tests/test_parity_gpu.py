@@ -393,3 +393,28 @@ def test_rows_beyond_the_softmax_shift_are_recomputed():
            "dv": out["dv"].float().numpy(), "ds": out["ds"][0, 0].numpy()}
     for key, val in got.items():
         assert U.normwise(val, r[key]) <= TOL_BF16_GRAD, key
+
+
+def test_kernel_timing_hook_times_each_launch():
+    """sas_kernel_timing / sas_kernel_time: one forward call on the tiny fp32
+    workload records one CUDA-core forward launch with a positive duration;
+    nothing is recorded once timing is off."""
+    w = synth.workload("tiny")
+    B.sas_kernel_timing("fwd_simt,block_topk")
+    U.run_train(w, with_bwd=False)
+    B.sas_kernel_timing(None)
+    ms, n = B.sas_kernel_time("fwd_simt")
+    assert n == 1 and ms > 0.0
+    assert B.sas_kernel_time("block_topk")[1] == 1
+    U.run_train(w, with_bwd=False)
+    assert B.sas_kernel_time("fwd_simt")[1] == 1
+
+
+def test_kernel_timing_filter():
+    """Only the kernels named in the filter are recorded."""
+    w = synth.workload("tiny")
+    B.sas_kernel_timing("block_topk")
+    U.run_train(w, with_bwd=False)
+    B.sas_kernel_timing(None)
+    assert B.sas_kernel_time("block_topk")[1] == 1
+    assert B.sas_kernel_time("fwd_simt") == (0.0, 0)

@@ -77,8 +77,11 @@ def lib() -> ctypes.CDLL:
         L.sas_device_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
         L.sas_kernel_launches.argtypes = []
         L.sas_kernel_launches.restype = ctypes.c_uint64
+        L.sas_kernel_timing.argtypes = [ctypes.c_char_p]
+        L.sas_kernel_time.argtypes = [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint32)]
         for f in ("sas_workspace_size", "sas_block_topk", "sas_gated_attn_fwd", "sas_gated_attn_bwd",
-                  "sas_sparse_decode", "sas_sparse_decode_noalloc", "sas_device_timeouts"):
+                  "sas_sparse_decode", "sas_sparse_decode_noalloc", "sas_device_timeouts", "sas_kernel_timing",
+                  "sas_kernel_time"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -174,3 +177,17 @@ def sas_device_timeouts() -> int:
 
 def sas_kernel_launches() -> int:
     return int(lib().sas_kernel_launches())
+
+
+def sas_kernel_timing(names: str | None) -> None:
+    """Record per-kernel CUDA events for the comma-separated kernel names
+    ("*" for every kernel); None stops recording."""
+    _check("sas_kernel_timing", lib().sas_kernel_timing(None if names is None else names.encode()))
+
+
+def sas_kernel_time(kernel: str) -> tuple[float, int]:
+    """(summed device ms, launches) recorded for `kernel` while timing was on."""
+    ms = ctypes.c_double(0.0)
+    n = ctypes.c_uint32(0)
+    _check("sas_kernel_time", lib().sas_kernel_time(kernel.encode(), ctypes.byref(ms), ctypes.byref(n)))
+    return float(ms.value), int(n.value)

@@ -582,7 +582,10 @@ cudaError_t launch_bwd_tc(const Shape& s, const void* q, const void* k, const vo
     BwdTcArgs a{s, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dO), lse, Dd, idx, gl, nsel,
                 maskT, dq_acc, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), gsum, kRows / s.G};
     const int64_t grid = (int64_t)s.B * s.Hkv * s.nT;
-    bwd_tc_kernel<<<(unsigned)grid, kThreads, smem, st>>>(mk, mv, a);
+    {
+        KernelTimer kt("bwd_tc", st);
+        bwd_tc_kernel<<<(unsigned)grid, kThreads, smem, st>>>(mk, mv, a);
+    }
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
     return e;

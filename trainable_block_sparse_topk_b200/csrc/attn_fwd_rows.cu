@@ -466,8 +466,11 @@ cudaError_t launch_fwd_rows(const Shape& s, const void* q, const void* k, const 
     a.tpc = kRows / s.G;
     cudaError_t e = cudaMemsetAsync(w.l_acc, 0, w.zero_bytes, st);
     if (e != cudaSuccess) return e;
-    fwd_rows_shift_kernel<<<(unsigned)((s.rows() + 7) / 8), 256, 0, st>>>(s, a.q, static_cast<const __nv_bfloat16*>(k),
-                                                                           w.shift);
+    {
+        KernelTimer kt("fwd_rows_shift", st);
+        fwd_rows_shift_kernel<<<(unsigned)((s.rows() + 7) / 8), 256, 0, st>>>(s, a.q, static_cast<const __nv_bfloat16*>(k),
+                                                                               w.shift);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launches(1);
@@ -476,13 +479,19 @@ cudaError_t launch_fwd_rows(const Shape& s, const void* q, const void* k, const 
     const size_t smem = RowsSmem::kTotal + 1024;
     e = cudaFuncSetAttribute(fwd_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    fwd_rows_kernel<<<(unsigned)((int64_t)s.B * s.Hkv * s.nT), kThreads, smem, st>>>(mk, mv, a);
+    {
+        KernelTimer kt("fwd_rows", st);
+        fwd_rows_kernel<<<(unsigned)((int64_t)s.B * s.Hkv * s.nT), kThreads, smem, st>>>(mk, mv, a);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launches(1);
-    fwd_rows_finalize_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(s, w.shift, w.l_acc, w.o_acc,
-                                                                         static_cast<__nv_bfloat16*>(o), lse, w.list,
-                                                                         w.list_n);
+    {
+        KernelTimer kt("fwd_rows_finalize", st);
+        fwd_rows_finalize_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(s, w.shift, w.l_acc, w.o_acc,
+                                                                             static_cast<__nv_bfloat16*>(o), lse, w.list,
+                                                                             w.list_n);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launches(1);

@@ -396,7 +396,10 @@ cudaError_t run_fwd_tc(const Shape& s, const void* q, const void* k, const void*
     if (e != cudaSuccess) return e;
     FwdTcArgs a{s, idx, gl, nsel, static_cast<__nv_bfloat16*>(o), lse, (s.G + 1) / 2};
     const int64_t grid = (int64_t)s.B * s.Hkv * s.nT * a.hp;
-    kern<<<(unsigned)grid, kThreads, smem, st>>>(mq, mk, mv, a);
+    {
+        KernelTimer kt("fwd_tc", st);
+        kern<<<(unsigned)grid, kThreads, smem, st>>>(mq, mk, mv, a);
+    }
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
     return e;

@@ -396,6 +396,7 @@ template <typename T, int D, int GMAX, int BS>
 cudaError_t run_fwd(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
                     const float* gl, const int32_t* nsel, void* o, float* lse, cudaStream_t st) {
     const int64_t grid = (s.rows() + 3) / 4;
+    KernelTimer kt("fwd_simt", st);
     fwd_simt_kernel<T, D, GMAX, BS><<<(unsigned)grid, 128, 0, st>>>(
         s, (const T*)q, (const T*)k, (const T*)v, idx, gl, nsel, (T*)o, lse, nullptr, nullptr);
     const cudaError_t e = cudaGetLastError();
@@ -414,8 +415,11 @@ cudaError_t run_bwd(const Shape& s, const void* q, const void* k, const void* v,
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int64_t grid = (int64_t)s.B * s.Hkv * s.nT;
-    kern<<<(unsigned)grid, NT, smem, st>>>(s, (const T*)q, (const T*)k, (const T*)v, (const T*)dO, lse, Dd, idx,
-                                           gl, nsel, maskT, dq_acc, (T*)dk, (T*)dv, gsum);
+    {
+        KernelTimer kt("bwd_simt", st);
+        kern<<<(unsigned)grid, NT, smem, st>>>(s, (const T*)q, (const T*)k, (const T*)v, (const T*)dO, lse, Dd, idx,
+                                               gl, nsel, maskT, dq_acc, (T*)dk, (T*)dv, gsum);
+    }
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
     return e;
@@ -479,6 +483,7 @@ cudaError_t launch_fwd_simt_rows(const Shape& s, const void* q, const void* k, c
     if (s.dtype != SAS_DT_BF16 || s.D != 128 || s.bs != 64) return cudaErrorInvalidValue;
     using B16 = __nv_bfloat16;
     const unsigned grid = 148;   // a few warps per SM; the rows to redo are normally none
+    KernelTimer kt("fwd_rows_fixup", st);
     if (s.G <= 4)
         fwd_simt_kernel<B16, 128, 4, 64><<<grid, 128, 0, st>>>(s, (const B16*)q, (const B16*)k, (const B16*)v, idx, gl,
                                                                nsel, (B16*)o, lse, list, list_n);
@@ -493,6 +498,7 @@ cudaError_t launch_fwd_simt_rows(const Shape& s, const void* q, const void* k, c
 cudaError_t launch_bwd_rowdot(const Shape& s, const void* o, const void* dO, float* Dd, cudaStream_t st) {
     const int64_t rows = (int64_t)s.B * s.Hq * s.T;
     const unsigned grid = (unsigned)((rows + 7) / 8);
+    KernelTimer kt("rowdot", st);
     if (s.dtype == SAS_DT_FP32) {
         if (s.D == 64) rowdot_kernel<float, 64><<<grid, 256, 0, st>>>(rows, (const float*)o, (const float*)dO, Dd);
         else rowdot_kernel<float, 128><<<grid, 256, 0, st>>>(rows, (const float*)o, (const float*)dO, Dd);
@@ -518,6 +524,7 @@ cudaError_t launch_bwd_simt(const Shape& s, const void* q, const void* k, const 
 cudaError_t launch_cast_dq(const Shape& s, const float* dq_acc, void* dq, cudaStream_t st) {
     const int64_t n = (int64_t)s.B * s.Hq * s.T * s.D;
     const unsigned grid = (unsigned)std::min<int64_t>((n + 255) / 256, 148 * 16);
+    KernelTimer kt("cast_dq", st);
     if (s.dtype == SAS_DT_FP32) cast_kernel<float><<<grid, 256, 0, st>>>(n, dq_acc, (float*)dq);
     else cast_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(n, dq_acc, (__nv_bfloat16*)dq);
     const cudaError_t e = cudaGetLastError();
@@ -528,6 +535,7 @@ cudaError_t launch_cast_dq(const Shape& s, const float* dq_acc, void* dq, cudaSt
 cudaError_t launch_dscore(const Shape& s, const float* scores, const float* slse, const int32_t* idx,
                           const int32_t* nsel, const float* gsum, float* ds, cudaStream_t st) {
     const unsigned grid = (unsigned)((s.rows() + 7) / 8);
+    KernelTimer kt("dscore", st);
     dscore_kernel<<<grid, 256, 0, st>>>(s, scores, slse, idx, nsel, gsum, ds);
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);

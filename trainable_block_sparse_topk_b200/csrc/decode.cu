@@ -322,12 +322,18 @@ cudaError_t run_decode(const DecArgs& a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int64_t grid = (int64_t)a.sh.B * a.sh.Hkv * a.splits;
-    kern<<<(unsigned)grid, kDecThreads, smem, st>>>(a);
+    {
+        KernelTimer kt("decode_partial", st);
+        kern<<<(unsigned)grid, kDecThreads, smem, st>>>(a);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launches(1);
-    decode_combine_kernel<T, D><<<(unsigned)(a.sh.B * a.sh.Hkv * a.sh.G), 128, 0, st>>>(a.sh, a.part, a.splits,
-                                                                                       static_cast<T*>(a.o));
+    {
+        KernelTimer kt("decode_combine", st);
+        decode_combine_kernel<T, D><<<(unsigned)(a.sh.B * a.sh.Hkv * a.sh.G), 128, 0, st>>>(a.sh, a.part, a.splits,
+                                                                                           static_cast<T*>(a.o));
+    }
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
     return e;

@@ -13,6 +13,21 @@ namespace sas {
 // Host-side count of kernels this library has launched (sas_kernel_launches).
 void count_launches(unsigned n);
 
+// While per-kernel timing is on (sas_kernel_timing), records a CUDA event on
+// `st` at construction and another at destruction under `name`.
+class KernelTimer {
+public:
+    KernelTimer(const char* name, cudaStream_t st);
+    ~KernelTimer();
+    KernelTimer(const KernelTimer&) = delete;
+    KernelTimer& operator=(const KernelTimer&) = delete;
+
+private:
+    const char* name_;
+    cudaStream_t st_;
+    void* start_;
+};
+
 // Problem shape, validated and derived from sas_desc by the entry points.
 struct Shape {
     int B, T, q_offset, Hq, Hkv, G, D, bs, K;

@@ -8,6 +8,9 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -36,6 +39,63 @@ static bool fwd_union() {
 
 static std::atomic<unsigned long long> g_launches{0};
 void count_launches(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+// ------------------------------------------------------- per-kernel timing ---
+namespace {
+struct TimingRec {
+    const char* name;
+    cudaEvent_t a, b;
+};
+std::mutex g_tmu;
+std::atomic<bool> g_timing{false};
+std::atomic<bool> g_timing_err{false};
+std::vector<TimingRec> g_recs;
+std::vector<cudaEvent_t> g_pool;
+std::string g_filter;   // ",a,b," or "*"
+
+bool timed(const char* name) {   // g_tmu held
+    if (g_filter == "*") return true;
+    return g_filter.find("," + std::string(name) + ",") != std::string::npos;
+}
+
+cudaEvent_t take_event() {   // g_tmu held
+    if (!g_pool.empty()) {
+        cudaEvent_t e = g_pool.back();
+        g_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+}  // namespace
+
+KernelTimer::KernelTimer(const char* name, cudaStream_t st) : name_(name), st_(st), start_(nullptr) {
+    if (!g_timing.load(std::memory_order_relaxed)) return;
+    std::lock_guard<std::mutex> lk(g_tmu);
+    if (!timed(name)) return;
+    cudaEvent_t e = take_event();
+    if (e == nullptr || cudaEventRecord(e, st_) != cudaSuccess) {
+        g_timing_err = true;
+        if (e) g_pool.push_back(e);
+        return;
+    }
+    start_ = e;
+}
+
+KernelTimer::~KernelTimer() {
+    if (start_ == nullptr) return;
+    std::lock_guard<std::mutex> lk(g_tmu);
+    cudaEvent_t a = static_cast<cudaEvent_t>(start_);
+    cudaEvent_t b = take_event();
+    if (b == nullptr || cudaEventRecord(b, st_) != cudaSuccess) {
+        g_timing_err = true;
+        g_pool.push_back(a);
+        if (b) g_pool.push_back(b);
+        return;
+    }
+    g_recs.push_back({name_, a, b});
+}
 
 namespace {
 
@@ -257,6 +317,40 @@ sas_status sas_sparse_decode(const sas_desc* desc, const void* q, const void* k_
 // Diagnostics: kernels launched by this library since it was loaded (host
 // count, incremented after each successful launch).
 uint64_t sas_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+sas_status sas_kernel_timing(const char* names) {
+    std::lock_guard<std::mutex> lk(g_tmu);
+    if (names != nullptr) {
+        for (const TimingRec& r : g_recs) {
+            g_pool.push_back(r.a);
+            g_pool.push_back(r.b);
+        }
+        g_recs.clear();
+        g_timing_err = false;
+        g_filter = std::strcmp(names, "*") == 0 ? std::string("*") : "," + std::string(names) + ",";
+    }
+    g_timing = names != nullptr;
+    return SAS_OK;
+}
+
+sas_status sas_kernel_time(const char* kernel, double* total_ms, uint32_t* launches) {
+    if (!kernel || !total_ms || !launches) return SAS_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lk(g_tmu);
+    if (g_timing_err) return SAS_ERR_CUDA;
+    double sum = 0.0;
+    uint32_t n = 0;
+    for (const TimingRec& r : g_recs) {
+        if (std::strcmp(r.name, kernel) != 0) continue;
+        float ms = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess)
+            return SAS_ERR_CUDA;
+        sum += ms;
+        ++n;
+    }
+    *total_ms = sum;
+    *launches = n;
+    return SAS_OK;
+}
 
 // Diagnostics: number of bounded device-side waits that gave up since the
 // library was loaded (0 in normal operation). Synchronises the device.

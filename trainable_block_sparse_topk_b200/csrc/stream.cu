@@ -175,13 +175,19 @@ cudaError_t launch_sel_stream(const Shape& s, const uint64_t* maskT, const int32
     cudaError_t e = cudaMemsetAsync(st.counter, 0, sizeof(int), stream);
     if (e != cudaSuccess) return e;
     const int64_t grid = (int64_t)s.B * s.Hkv * s.NB;
-    sel_stream_index_kernel<<<(unsigned)grid, kThreads, 0, stream>>>(s, maskT, v0, v1, vals, st);
+    {
+        KernelTimer kt("sel_stream_index", stream);
+        sel_stream_index_kernel<<<(unsigned)grid, kThreads, 0, stream>>>(s, maskT, v0, v1, vals, st);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launches(1);
     const int64_t rpb = kThreads / 32;
-    sel_stream_fill_kernel<<<(unsigned)((s.rows() + rpb - 1) / rpb), kThreads, 0, stream>>>(s, maskT, idx, gl, nsel,
-                                                                                            v0, v1, vals, st);
+    {
+        KernelTimer kt("sel_stream_fill", stream);
+        sel_stream_fill_kernel<<<(unsigned)((s.rows() + rpb - 1) / rpb), kThreads, 0, stream>>>(s, maskT, idx, gl, nsel,
+                                                                                                v0, v1, vals, st);
+    }
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
     return e;

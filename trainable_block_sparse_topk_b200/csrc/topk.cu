@@ -250,6 +250,7 @@ cudaError_t run_topk(const Shape& s, const float* scores, int32_t* idx, float* g
     const int64_t rows = s.rows();
     const int rpc = NT == 32 ? 8 : 1;
     const int64_t grid = (rows + rpc - 1) / rpc;
+    KernelTimer kt("block_topk", st);
     block_topk_kernel<NT, SLOTS><<<(unsigned)grid, NT == 32 ? 256 : NT, 0, st>>>(s, scores, idx, gl, lse, nsel);
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
@@ -306,6 +307,7 @@ cudaError_t launch_sel_bitmap_T(const Shape& s, const int32_t* idx, const int32_
         if (e != cudaSuccess) return e;
     }
     const int64_t grid = (int64_t)s.B * s.Hkv * s.nT;
+    KernelTimer kt("sel_bitmap_T", st);
     sel_bitmap_T_kernel<<<(unsigned)grid, 256, smem, st>>>(s, idx, nsel, maskT);
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
