@@ -31,6 +31,8 @@
 // warps 4-7 compute (thread = row = TMEM lane). No TMA multicast is used.
 #include <cuda.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tc.cuh"
@@ -387,35 +389,52 @@ fwd_rows_shift_kernel(Shape sh, const __nv_bfloat16* __restrict__ q, const __nv_
 }
 
 // o = O / l (bf16) and attn_lse = (M + log2 l) ln 2, one warp per query-head
-// row. Rows whose sum or output left the safe range are listed (as their
+// row; each warp takes kRowsU rows per pass and issues all their loads before
+// using any. Rows whose sum or output left the safe range are listed (as their
 // (b, kv head, t) row) for the exact recompute instead.
+constexpr int kRowsU = 4;
+
 __global__ void __launch_bounds__(256)
 fwd_rows_finalize_kernel(Shape sh, const float* __restrict__ shift, const float* __restrict__ l_acc,
                          const float* __restrict__ o_acc, __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
                          int32_t* __restrict__ list, int32_t* __restrict__ list_n) {
     const int64_t rows = (int64_t)sh.B * sh.Hq * sh.T;
-    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    if (row >= rows) return;
-    const float l = l_acc[row];
-    const float4 v = reinterpret_cast<const float4*>(o_acc + row * kD)[lane];
-    const bool fin = isfinite(v.x) && isfinite(v.y) && isfinite(v.z) && isfinite(v.w);
-    const bool bad = __any_sync(0xffffffffu, !fin) || !(l >= 0.5f && l <= 0x1p80f);
-    if (bad) {
-        if (lane == 0) {
-            const int64_t bh = row / sh.T;
-            const int t = (int)(row % sh.T);
-            const int b = (int)(bh / sh.Hq), h = (int)(bh % sh.Hq);
-            list[atomicAdd(list_n, 1)] = (int32_t)(((int64_t)b * sh.Hkv + h / sh.G) * sh.T + t);
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t r0 = warp * kRowsU; r0 < rows; r0 += nwarps * kRowsU) {
+        float4 v[kRowsU];
+        float l[kRowsU];
+#pragma unroll
+        for (int u = 0; u < kRowsU; ++u) {
+            const int64_t row = r0 + u;
+            if (row >= rows) continue;
+            v[u] = reinterpret_cast<const float4*>(o_acc + row * kD)[lane];
+            l[u] = l_acc[row];
         }
-        return;
+#pragma unroll
+        for (int u = 0; u < kRowsU; ++u) {
+            const int64_t row = r0 + u;
+            if (row >= rows) continue;                    // warp-uniform
+            const bool fin = isfinite(v[u].x) && isfinite(v[u].y) && isfinite(v[u].z) && isfinite(v[u].w);
+            const bool bad = __any_sync(0xffffffffu, !fin) || !(l[u] >= 0.5f && l[u] <= 0x1p80f);
+            if (bad) {
+                if (lane == 0) {
+                    const int64_t bh = row / sh.T;
+                    const int t = (int)(row % sh.T);
+                    const int b = (int)(bh / sh.Hq), h = (int)(bh % sh.Hq);
+                    list[atomicAdd(list_n, 1)] = (int32_t)(((int64_t)b * sh.Hkv + h / sh.G) * sh.T + t);
+                }
+                continue;
+            }
+            const float inv = 1.f / l[u];
+            __nv_bfloat162 lo = __floats2bfloat162_rn(v[u].x * inv, v[u].y * inv);
+            __nv_bfloat162 hi = __floats2bfloat162_rn(v[u].z * inv, v[u].w * inv);
+            uint2 packed = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+            reinterpret_cast<uint2*>(o + row * kD)[lane] = packed;
+            if (lane == 0) lse[row] = (shift[row] + log2f(l[u])) * kLn2;
+        }
     }
-    const float inv = 1.f / l;
-    __nv_bfloat162 lo = __floats2bfloat162_rn(v.x * inv, v.y * inv);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(v.z * inv, v.w * inv);
-    uint2 packed = make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
-    reinterpret_cast<uint2*>(o + row * kD)[lane] = packed;
-    if (lane == 0) lse[row] = (shift[row] + log2f(l)) * kLn2;
 }
 
 // Workspace: shift [rows] f32 | list [rows] i32 | l [rows] f32 | O [rows, d] f32 | list count |
@@ -488,7 +507,8 @@ cudaError_t launch_fwd_rows(const Shape& s, const void* q, const void* k, const 
     count_launches(1);
     {
         KernelTimer kt("fwd_rows_finalize", st);
-        fwd_rows_finalize_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(s, w.shift, w.l_acc, w.o_acc,
+        fwd_rows_finalize_kernel<<<(unsigned)std::min<int64_t>((rows + 8 * kRowsU - 1) / (8 * kRowsU), 148 * 16), 256, 0,
+                                   st>>>(s, w.shift, w.l_acc, w.o_acc,
                                                                              static_cast<__nv_bfloat16*>(o), lse, w.list,
                                                                              w.list_n);
     }

@@ -343,6 +343,32 @@ __global__ void cast_kernel(int64_t n, const float* __restrict__ src, T* __restr
         dst[i] = Elem<T>::from_f(src[i]);
 }
 
+// fp32 -> bf16, 8 values per thread and pass, two passes' loads in flight
+// (n8 = number of 8-value groups).
+__global__ void __launch_bounds__(256)
+cast_bf16x8_kernel(int64_t n8, const float4* __restrict__ src, uint4* __restrict__ dst) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += 2 * stride) {
+        float4 v[2][2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int64_t k = i + u * stride;
+            if (k < n8) {
+                v[u][0] = src[2 * k];
+                v[u][1] = src[2 * k + 1];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int64_t k = i + u * stride;
+            if (k >= n8) continue;
+            __nv_bfloat162 p[4] = {__floats2bfloat162_rn(v[u][0].x, v[u][0].y), __floats2bfloat162_rn(v[u][0].z, v[u][0].w),
+                                   __floats2bfloat162_rn(v[u][1].x, v[u][1].y), __floats2bfloat162_rn(v[u][1].z, v[u][1].w)};
+            dst[k] = *reinterpret_cast<const uint4*>(p);
+        }
+    }
+}
+
 // ------------------------------------------------------- score gradient (K5) ---
 
 // ds_i = [i kept] Gsum_i - g_i sum_{k kept} Gsum_k for i < C, 0 otherwise,
@@ -525,8 +551,13 @@ cudaError_t launch_cast_dq(const Shape& s, const float* dq_acc, void* dq, cudaSt
     const int64_t n = (int64_t)s.B * s.Hq * s.T * s.D;
     const unsigned grid = (unsigned)std::min<int64_t>((n + 255) / 256, 148 * 16);
     KernelTimer kt("cast_dq", st);
-    if (s.dtype == SAS_DT_FP32) cast_kernel<float><<<grid, 256, 0, st>>>(n, dq_acc, (float*)dq);
-    else cast_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(n, dq_acc, (__nv_bfloat16*)dq);
+    if (s.dtype == SAS_DT_FP32) {
+        cast_kernel<float><<<grid, 256, 0, st>>>(n, dq_acc, (float*)dq);
+    } else {   // n is a multiple of 8 (d is 64 or 128); both buffers are 16-byte aligned
+        const int64_t n8 = n / 8;
+        const unsigned g8 = (unsigned)std::min<int64_t>((n8 + 511) / 512, 148 * 8);
+        cast_bf16x8_kernel<<<g8, 256, 0, st>>>(n8, reinterpret_cast<const float4*>(dq_acc), static_cast<uint4*>(dq));
+    }
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
     return e;
