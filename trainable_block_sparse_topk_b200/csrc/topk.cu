@@ -7,9 +7,10 @@
 // normalised gate), and the kept blocks' log-gates are s_i minus it.
 //
 // Exactness: scores are compared through an order-preserving uint32 key, so the
-// K-th largest key is found exactly by an MSB-first radix select (4 passes of
-// 8 bits). The elements above it are kept, and the ones equal to it are kept
-// in index order until K are chosen. Each thread owns a contiguous run of
+// K-th largest key is found exactly: by a 32-step bitwise search with
+// warp-wide counts when one warp owns the row, by an MSB-first radix select
+// (4 passes of 8 bits) when a whole CTA does. The elements above it are kept,
+// and the ones equal to it are kept in index order until K are chosen. Each thread owns a contiguous run of
 // SLOTS candidates, so index order is (thread, slot) order and two prefix scans
 // (one for the ties, one for output positions) place everything.
 #include "common.cuh"
@@ -173,9 +174,29 @@ block_topk_kernel(Shape sh, const float* __restrict__ scores, int32_t* __restric
     lsum = G.sum_all(lsum);
     const float lse = (C > 0 && m != -INFINITY) ? m + logf(lsum) : -INFINITY;
 
-    // --- radix select the n-th largest key: 4 passes of 8 bits, MSB first ---
+    // --- the n-th largest key ---
     uint32_t prefix = 0, pmask = 0, need = (uint32_t)n;
-    if (n > 0) {
+    if (NT == 32 && n > 0) {
+        // One warp: bitwise search, MSB first. Bit b joins the answer when at
+        // least n keys are >= (answer | bit): the result is the largest v with
+        // #{keys >= v} >= n, i.e. the n-th largest key. Invalid slots hold key
+        // 0, which no candidate (>= 1) admits.
+        uint32_t thr = 0;
+#pragma unroll 1
+        for (int bit = 31; bit >= 0; --bit) {
+            const uint32_t cand = thr | (1u << bit);
+            uint32_t c = 0;
+#pragma unroll
+            for (int j = 0; j < SLOTS; ++j) c += key[j] >= cand ? 1u : 0u;
+            if (__reduce_add_sync(0xffffffffu, c) >= (uint32_t)n) thr = cand;
+        }
+        uint32_t gt = 0;
+#pragma unroll
+        for (int j = 0; j < SLOTS; ++j) gt += key[j] > thr ? 1u : 0u;
+        prefix = thr;
+        need = (uint32_t)n - __reduce_add_sync(0xffffffffu, gt);   // copies of thr to keep
+    } else if (n > 0) {
+        // radix select, 4 passes of 8 bits, MSB first
 #pragma unroll 1
         for (int pass = 0; pass < 4; ++pass) {
             const int shift = 24 - 8 * pass;
