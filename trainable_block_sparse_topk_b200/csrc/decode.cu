@@ -367,7 +367,7 @@ DecodePlan decode_plan(const Shape& s, bool dense) {
     }
     const int64_t nblk = C + 1;
     const int64_t groups = (int64_t)s.B * s.Hkv;
-    const int64_t target = 148 * 4;   // CTAs: a few per SM
+    const int64_t target = 148 * 3;   // CTAs: one wave (three ~67 KB, 256-thread CTAs fit per SM)
     int64_t bpc = (groups * nblk + target - 1) / target;
     bpc = std::max<int64_t>(bpc, (nblk + kMaxSplits - 1) / kMaxSplits);   // the merge takes <= kMaxSplits
     bpc = std::max<int64_t>(1, bpc);
