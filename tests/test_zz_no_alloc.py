@@ -59,10 +59,11 @@ def test_noalloc_matches_workspace_decode_twice():
 
 
 def test_noalloc_rejects_oversize():
-    """8 x 8 KV heads x 65 splits x 4 heads x 130 floats needs more than the
-    static array: refused before any launch, with the workspace status."""
+    """16 x 8 KV heads x 33 splits (two kept blocks per split) x 4 heads x 130
+    floats needs more than the static array: refused before any launch, with
+    the workspace status."""
     build()
-    w = synth.workload("decode", batch=8, seq=64 * 66)
+    w = synth.workload("decode", batch=16, seq=64 * 66)
     d = _desc(w, 64)
     kc = torch.zeros(w.batch, w.n_kv_heads, w.seq, w.head_dim, dtype=torch.bfloat16, device="cuda")
     q = torch.zeros(w.batch, w.n_q_heads, w.head_dim, dtype=torch.bfloat16, device="cuda")

@@ -14,8 +14,11 @@
 #include <algorithm>
 #include <mutex>
 
+#include <cuda.h>
+
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace sas {
 
@@ -272,6 +275,298 @@ decode_partial_kernel(DecArgs a) {
     }
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core variant (bf16, d = 128, block 64, G <= 8). Warp 0 moves blocks
+// into a 4-stage ring by TMA (K and V as two 64-column boxes each, 128-byte
+// swizzle); warps 1 and 2 each own every other stage and run the whole block
+// on mma.sync m16n8k16 with no CTA-wide barrier:
+//   S^T = K q^T   (M = 16 keys, N = 8 heads, K = 16 dims; 4 x 8 MMAs)
+//   online softmax per head in log2 units (scale applied in fp32 after the MMA)
+//   O^T += V^T P^T (M = 16 dims, N = 8 heads, K = 16 keys; 8 x 4 MMAs)
+// K rows come through ldmatrix, V rows through ldmatrix.trans, and the P tile
+// (keys x heads, accumulator layout) becomes the B operand by movmatrix.trans.
+// Rows of the current block at or after the new token may hold anything in the
+// cache: their scores are replaced by -inf and their V rows zeroed in shared
+// memory before the product. The two consumers merge their (m, l, O) at the
+// end and write one partial per CTA for the same merge kernel.
+constexpr int kMmaStages = 4;
+constexpr uint32_t kMmaStage = 32768;   // K box 0 | K box 1 | V box 0 | V box 1, 8 KiB each
+
+struct DecMmaArgs {
+    DecArgs d;
+};
+
+__device__ __forceinline__ uint32_t sw_addr(uint32_t box, int row, int chunk) {
+    return box + (uint32_t)row * 128u + (uint32_t)((chunk ^ (row & 7)) << 4);
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+__device__ __forceinline__ uint32_t movm_t(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+__device__ __forceinline__ void mma_bf16(float* c, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+                 "{%0, %1, %2, %3};"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__global__ void __launch_bounds__(96, 1)
+decode_mma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                  const __grid_constant__ DecMmaArgs args) {
+    constexpr int D = 128, BS = 64;
+    const DecArgs& a = args.d;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + kMmaStages * kMmaStage);
+    uint64_t* empty = full + kMmaStages;
+    float* xch = reinterpret_cast<float*>(empty + kMmaStages);   // consumer 1's m[8], l[8], O^T[128][8]
+
+    const Shape& sh = a.sh;
+    const int G = sh.G;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int split = blockIdx.x % a.splits;
+    const int64_t bg = blockIdx.x / a.splits;
+    const int b = (int)(bg / sh.Hkv), g = (int)(bg % sh.Hkv);
+    const int64_t N = (int64_t)sh.q_offset + 1;
+    const int C = (int)(sh.q_offset / BS);
+    const bool dense = a.idx == nullptr;
+    const int n = dense ? C : a.nsel[bg];
+    const int nblk = n + 1;
+    const int p0 = split * a.bpc;
+    const int cnt = max(min(p0 + a.bpc, nblk) - p0, 0);
+    auto block_of = [&](int pos) -> int {
+        if (dense) return pos;
+        if (pos >= n) return C;
+        const int j = a.idx[bg * sh.K + pos];
+        return ((unsigned)j < (unsigned)C) ? j : -1;
+    };
+    auto ntok_of = [&](int j) -> int { return j < 0 ? 0 : (j == C ? (int)(N - (int64_t)C * BS) : BS); };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kMmaStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == 0) {
+        // ---- producer ----
+        if (lane == 0) {
+            for (int i = 0; i < cnt; ++i) {
+                const int s = i % kMmaStages;
+                if (i >= kMmaStages && !mbar_wait_bounded(&empty[s], (uint32_t)(((i / kMmaStages) - 1) & 1))) break;
+                const int j = block_of(p0 + i);
+                if (j < 0) {
+                    tc::mbar_arrive(&full[s]);
+                    continue;
+                }
+                mbar_arrive_expect_tx(&full[s], kMmaStage);
+                const int row = (int)(bg * a.stride + (int64_t)j * BS);
+                unsigned char* st = sm + s * kMmaStage;
+                tc::tma_load_2d(st, &tm_k, 0, row, &full[s]);
+                tc::tma_load_2d(st + 8192, &tm_k, 64, row, &full[s]);
+                tc::tma_load_2d(st + 16384, &tm_v, 0, row, &full[s]);
+                tc::tma_load_2d(st + 24576, &tm_v, 64, row, &full[s]);
+            }
+        }
+        return;
+    }
+
+    // ---- consumers: warp 1 takes blocks 0, 2, ...; warp 2 blocks 1, 3, ... ----
+    const int cw = warp - 1;
+    const int gq = lane >> 2, tq = lane & 3;
+    const float qk = sh.scale * kLog2e;
+    // q^T as the B operand: b0 = q[head gq][16 ks + 2 tq, +1], b1 = the same + 8
+    uint32_t qb[8][2];
+    {
+        const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q) + ((int64_t)b * sh.Hq + (int64_t)g * G) * D;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            if (gq < G) {
+                qb[ks][0] = *reinterpret_cast<const uint32_t*>(qg + gq * D + 16 * ks + 2 * tq);
+                qb[ks][1] = *reinterpret_cast<const uint32_t*>(qg + gq * D + 16 * ks + 2 * tq + 8);
+            } else {
+                qb[ks][0] = qb[ks][1] = 0u;
+            }
+        }
+    }
+    float o[8][4];          // O^T: m-tile of 16 dims, (dim gq | gq+8) x (heads 2tq, 2tq+1)
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o[mt][e] = 0.f;
+    float mrun[2] = {-INFINITY, -INFINITY}, lrun[2] = {0.f, 0.f};   // heads 2tq, 2tq+1
+
+    const uint32_t sbase = smem_u32(sm);
+    bool ok = true;
+    for (int i = cw; i < cnt; i += 2) {
+        const int s = i % kMmaStages;
+        if (!mbar_wait_bounded(&full[s], (uint32_t)((i / kMmaStages) & 1))) { ok = false; break; }
+        const int j = block_of(p0 + i);
+        const int ntok = ntok_of(j);
+        if (ntok > 0) {
+            const uint32_t kb0 = sbase + s * kMmaStage, kb1 = kb0 + 8192, vb0 = kb0 + 16384, vb1 = kb0 + 24576;
+            if (ntok < BS) {   // the current block: clear V rows >= ntok (128 bytes per row and box)
+                unsigned char* v0p = sm + s * kMmaStage + 16384;
+                for (int e = ntok * 8 + lane; e < BS * 8; e += 32) {
+                    reinterpret_cast<uint4*>(v0p)[e] = make_uint4(0, 0, 0, 0);
+                    reinterpret_cast<uint4*>(v0p + 8192)[e] = make_uint4(0, 0, 0, 0);
+                }
+                __syncwarp();
+            }
+            const float lg = (!dense && p0 + i < n) ? a.gl[bg * sh.K + p0 + i] * kLog2e : 0.f;
+            // ---- S^T = K q^T ----
+            float sc[4][4];
+#pragma unroll
+            for (int mt = 0; mt < 4; ++mt) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sc[mt][e] = 0.f;
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    // matrices: (keys +0..7, dims +0..7), (keys +8..15, dims +0..7), (keys +0..7, dims +8..15), (keys +8.., dims +8..)
+                    const int key = 16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8;
+                    const int chunk = 2 * ks + (lane >> 4);
+                    const uint32_t addr = sw_addr(chunk < 8 ? kb0 : kb1, key, chunk & 7);
+                    uint32_t a0, a1, a2, a3;
+                    ldsm_x4(addr, a0, a1, a2, a3);
+                    mma_bf16(sc[mt], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+                }
+            }
+            // ---- online softmax (heads 2tq, 2tq+1; keys 16 mt + gq (+8)) ----
+            float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+            for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int key = 16 * mt + gq + (e >> 1) * 8;
+                    const float v = key < ntok ? fmaf(sc[mt][e], qk, lg) : -INFINITY;
+                    sc[mt][e] = v;
+                    mx[e & 1] = fmaxf(mx[e & 1], v);
+                }
+            float corr[2], psum[2] = {0.f, 0.f};
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 4));
+                mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 8));
+                mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 16));
+                const float mn = fmaxf(mrun[h], mx[h]);
+                corr[h] = mrun[h] == -INFINITY ? 0.f : exp2f(mrun[h] - mn);
+                mrun[h] = mn;
+            }
+            uint32_t pb[4][2];   // P^T as B operand per k-step (16 keys)
+#pragma unroll
+            for (int mt = 0; mt < 4; ++mt) {
+                float p[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float m = mrun[e & 1];
+                    p[e] = m == -INFINITY ? 0.f : exp2f(sc[mt][e] - m);
+                    psum[e & 1] += p[e];
+                }
+                pb[mt][0] = movm_t(pack_bf16(p[0], p[1]));   // keys 16 mt + 0..7
+                pb[mt][1] = movm_t(pack_bf16(p[2], p[3]));   // keys 16 mt + 8..15
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                psum[h] += __shfl_xor_sync(0xffffffffu, psum[h], 4);
+                psum[h] += __shfl_xor_sync(0xffffffffu, psum[h], 8);
+                psum[h] += __shfl_xor_sync(0xffffffffu, psum[h], 16);
+                lrun[h] = lrun[h] * corr[h] + psum[h];
+            }
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                o[mt][0] *= corr[0];
+                o[mt][1] *= corr[1];
+                o[mt][2] *= corr[0];
+                o[mt][3] *= corr[1];
+            }
+            // ---- O^T += V^T P^T ----
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {        // dims 16 mt .. + 15
+#pragma unroll
+                for (int kst = 0; kst < 4; ++kst) { // keys 16 kst .. + 15
+                    // matrices (transposed on load): (keys +0..7, dims +0..7), (keys +0..7, dims +8..15),
+                    // (keys +8..15, dims +0..7), (keys +8..15, dims +8..15)
+                    const int key = 16 * kst + (lane & 7) + (lane >> 4) * 8;
+                    const int chunk = 2 * mt + ((lane >> 3) & 1);
+                    const uint32_t addr = sw_addr(chunk < 8 ? vb0 : vb1, key, chunk & 7);
+                    uint32_t a0, a1, a2, a3;
+                    ldsm_x4_t(addr, a0, a1, a2, a3);
+                    mma_bf16(o[mt], a0, a1, a2, a3, pb[kst][0], pb[kst][1]);
+                }
+            }
+        }
+        tc::fence_async_shared();   // the zeroed rows are rewritten by TMA next
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&empty[s]);
+    }
+
+    // ---- merge the two consumers; consumer 0 writes the CTA's partial ----
+    float* rec = a.part + (bg * a.splits + split) * (int64_t)G * (D + 2);
+    if (cw == 1) {
+        if (gq == 0) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) { xch[2 * tq + h] = mrun[h]; xch[8 + 2 * tq + h] = lrun[h]; }
+        }
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int dim = 16 * mt + gq + (e >> 1) * 8, h = 2 * tq + (e & 1);
+                xch[16 + dim * 8 + h] = o[mt][e];
+            }
+    }
+    asm volatile("bar.sync 1, 64;" ::: "memory");
+    if (cw == 0) {
+        float m2[2], l2[2], w1[2], w2[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            m2[h] = xch[2 * tq + h];
+            l2[h] = xch[8 + 2 * tq + h];
+            const float M = fmaxf(mrun[h], m2[h]);
+            w1[h] = mrun[h] == -INFINITY ? 0.f : exp2f(mrun[h] - M);
+            w2[h] = m2[h] == -INFINITY ? 0.f : exp2f(m2[h] - M);
+            mrun[h] = M;
+            lrun[h] = lrun[h] * w1[h] + l2[h] * w2[h];
+        }
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int dim = 16 * mt + gq + (e >> 1) * 8, h = 2 * tq + (e & 1);
+                const float v = o[mt][e] * w1[e & 1] + xch[16 + dim * 8 + h] * w2[e & 1];
+                if (h < G) rec[h * (D + 2) + dim] = ok ? v : __int_as_float(0x7fc00000);
+            }
+        if (gq == 0) {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int hh = 2 * tq + h;
+                if (hh < G) {
+                    rec[hh * (D + 2) + D] = mrun[h];
+                    rec[hh * (D + 2) + D + 1] = lrun[h];
+                }
+            }
+        }
+    }
+}
+
 // Merge the splits of one (b, kv head, query head):
 //   o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s.
 // The split weights are formed once in shared memory; each thread then reads
@@ -339,6 +634,32 @@ cudaError_t run_decode(const DecArgs& a, cudaStream_t st) {
     return e;
 }
 
+cudaError_t run_decode_mma(const DecArgs& a, cudaStream_t st) {
+    CUtensorMap mk, mv;
+    const uint64_t rows = (uint64_t)a.sh.B * a.sh.Hkv * (uint64_t)a.stride;
+    if (!encode_bf16_2d(&mk, a.kc, rows, 128, 64) || !encode_bf16_2d(&mv, a.vc, rows, 128, 64))
+        return cudaErrorInvalidValue;
+    const size_t smem = (size_t)kMmaStages * kMmaStage + 2 * kMmaStages * 8 + sizeof(float) * (16 + 128 * 8) + 1024;
+    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = (int64_t)a.sh.B * a.sh.Hkv * a.splits;
+    {
+        KernelTimer kt("decode_partial", st);
+        decode_mma_kernel<<<(unsigned)grid, 96, smem, st>>>(mk, mv, DecMmaArgs{a});
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    count_launches(1);
+    {
+        KernelTimer kt("decode_combine", st);
+        decode_combine_kernel<__nv_bfloat16, 128><<<(unsigned)(a.sh.B * a.sh.Hkv * a.sh.G), 128, 0, st>>>(
+            a.sh, a.part, a.splits, static_cast<__nv_bfloat16*>(a.o));
+    }
+    e = cudaGetLastError();
+    if (e == cudaSuccess) count_launches(1);
+    return e;
+}
+
 template <typename T, int D, int BS>
 cudaError_t decode_g(const DecArgs& a, cudaStream_t st) {
     if (a.sh.G <= 4) return run_decode<T, D, 4, BS>(a, st);
@@ -357,9 +678,25 @@ cudaError_t decode_d(const DecArgs& a, cudaStream_t st) {
 
 }  // namespace
 
+static bool decode_mma_supported(const Shape& s) {
+    return s.dtype == SAS_DT_BF16 && s.D == 128 && s.bs == 64 && s.G <= 8;
+}
+
 DecodePlan decode_plan(const Shape& s, bool dense) {
     DecodePlan p;
     const int64_t C = s.q_offset / s.bs;
+    if (decode_mma_supported(s)) {
+        // one CTA per SM (128 KiB of stages); two blocks per CTA for a
+        // selection, one wave of CTAs over every block for dense
+        const int64_t nblk = dense ? C + 1 : (int64_t)s.K + 1;
+        const int64_t groups = (int64_t)s.B * s.Hkv;
+        int64_t bpc = dense ? (groups * nblk + 147) / 148 : 2;
+        bpc = std::max<int64_t>(bpc, (nblk + kMaxSplits - 1) / kMaxSplits);
+        bpc = std::max<int64_t>(1, bpc);
+        p.bpc = (int)bpc;
+        p.splits = (int)((nblk + bpc - 1) / bpc);
+        return p;
+    }
     if (!dense) {
         p.bpc = 1;
         p.splits = s.K + 1;
@@ -381,6 +718,7 @@ cudaError_t launch_decode(const Shape& s, const void* q, const void* kc, const v
                           cudaStream_t st) {
     const DecodePlan p = decode_plan(s, idx == nullptr);
     DecArgs a{s, q, kc, vc, stride, idx, gl, nsel, part, o, p.bpc, p.splits};
+    if (decode_mma_supported(s)) return run_decode_mma(a, st);
     if (s.dtype == SAS_DT_FP32) return decode_d<float>(a, st);
     return decode_d<__nv_bfloat16>(a, st);
 }
