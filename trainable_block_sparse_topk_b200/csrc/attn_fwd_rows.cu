@@ -24,11 +24,13 @@
 // Executed MMA work is the definition's 4 d FLOP per kept (query head, key)
 // pair, with no masked rows.
 //
-// Roles (256 threads): warps 0 and 3 gather rows (even / odd chunks) with
+// Roles (384 threads): warps 8 and 11 gather rows (even / odd chunks) with
 // coalesced 16-byte cp.async copies into two 128-byte-swizzled Q stages (TMA
-// tile::gather4 moves random rows at a fraction of that rate); warp 0 also
-// loads K_j and V_j by TMA; warp 1 lane 0 issues the MMAs; warp 2 owns TMEM;
-// warps 4-7 compute (thread = row = TMEM lane). No TMA multicast is used.
+// tile::gather4 moves random rows at a fraction of that rate); warp 8 also
+// loads K_j and V_j by TMA; warp 9 lane 0 issues the MMAs; warp 10 owns TMEM;
+// warps 4-7 form P (thread = row = TMEM lane) and warps 0-3 read O back and
+// add it to the accumulator, so P of one chunk overlaps the output of the
+// previous one. No TMA multicast is used.
 #include <cuda.h>
 
 #include <algorithm>
@@ -41,7 +43,7 @@ namespace sas {
 
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;   // epilogue 0-3, P 4-7, loaders 8 and 11, MMA 9, TMEM 10
 constexpr int kBS = 64;
 constexpr int kRows = 128;
 constexpr int kD = 128;
@@ -65,8 +67,9 @@ struct RowsSmem {
     static constexpr uint32_t kOstRow = kD * 4 + 16;               // padded: conflict-free 16-byte stores
     static constexpr uint32_t kMeta = kOst + kRows * kOstRow;      // 4 x chunk stream entries (chunk c -> slot c & 3)
     static constexpr uint32_t kMetaBytes = 4096;                   // int4 ent[<=128], then f32 rv[<= 512]
-    static constexpr uint32_t kBar = kMeta + 4 * kMetaBytes;
-    static constexpr int kNumBars = 18;
+    static constexpr uint32_t kIds = kMeta + 4 * kMetaBytes;       // i32 [4][128]: O accumulator row per chunk row
+    static constexpr uint32_t kBar = kIds + 4 * kRows * 4;
+    static constexpr int kNumBars = 22;
     static constexpr uint32_t kMisc = kBar + 8 * kNumBars;         // tmem base, stream length, first entry, abort
     static constexpr uint32_t kTmemCols = 512;                     // S double [0,128), O double [128,384)
     static constexpr uint32_t kTotal = kMisc + 16;
@@ -97,6 +100,8 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     uint64_t* o_full = bars + 9;      // [2]
     uint64_t* o_empty = bars + 11;    // [2] 4 arrivals
     uint64_t* meta_full = bars + 13;  // [4] ring slot c & 3 holds chunk c's stream entries (tx bytes)
+    uint64_t* ids_full = bars + 17;   // [4] 4 arrivals: chunk c's O rows are in ids[c & 3]
+    int* ids = reinterpret_cast<int*>(sm + L::kIds);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMisc);
     int* ntok_slot = reinterpret_cast<int*>(sm + L::kMisc + 4);      // [2]: stream length, first entry
     volatile int* abort = reinterpret_cast<volatile int*>(sm + L::kMisc + 12);
@@ -116,6 +121,7 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             uint64_t* bar = &bars[i];
             uint32_t cnt = 1;
             if (bar == p_full || bar == &o_empty[0] || bar == &o_empty[1]) cnt = 4;
+            if (bar >= ids_full && bar < ids_full + 4) cnt = 4;
             // a stage is refilled only after the MMA has read its rows and the
             // compute warps have waited for it: its phases then cannot run two
             // ahead of any waiter
@@ -128,7 +134,7 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         *abort = 0;
         fence_mbar_init();
     }
-    if (warp == 2) {
+    if (warp == 10) {
         tc::tmem_alloc(tmem_slot, L::kTmemCols);
         tc::tmem_relinquish();
     }
@@ -141,11 +147,11 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int nc = (ntok_total + tpc - 1) / tpc;
     const uint32_t sbase = smem_u32(sm);
 
-    if (warp == 0 || warp == 3) {
+    if (warp == 8 || warp == 11) {
         // ---------------------------------------------------------- loaders ---
-        const int L0 = warp == 0 ? 0 : 1;
+        const int L0 = warp == 8 ? 0 : 1;
         unsigned char* stq = sm + L::kStage + L0 * L::kStageBytes;
-        if (warp == 0 && lane == 0) {
+        if (warp == 8 && lane == 0) {
             tc::prefetch_tmap(&tm_k);
             tc::prefetch_tmap(&tm_v);
             mbar_arrive_expect_tx(kv_full, 32768u);
@@ -197,7 +203,7 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             if (lane == 0) tc::mbar_arrive(&st_full[L0]);
         }
         tc::cp_async_wait_all();
-    } else if (warp == 1) {
+    } else if (warp == 9) {
         // ------------------------------------------------------- MMA issuer ---
         if (lane == 0) {
             constexpr uint32_t id_s = tc::idesc_bf16_f32(128, kBS, false, false);
@@ -260,45 +266,14 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 }
             }
         }
-    } else if (warp >= 4) {
-        // ----------------------------------------------------- compute warps ---
+    } else if (warp >= 4 && warp < 8) {
+        // --------------------------------------------------------- P warps ---
         const int r = (warp - 4) * 32 + lane;      // chunk row == TMEM lane
         const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const float qk = sh.scale * kLog2e;
-        bool ok = true;
-        int prev_row = -1;
-        // O of chunk c: TMEM -> this thread's padded shared-memory row -> one
-        // 512-byte bulk add into the fp32 accumulator row. The row is reused
-        // only after the previous bulk add of this thread has read it.
-        const uint32_t orow = sbase + L::kOst + (uint32_t)r * L::kOstRow;
-        auto o_epilogue = [&](int c) -> bool {
-            if (!tc::warp_wait_bar(&o_full[c & 1], (uint32_t)((c >> 1) & 1), abort)) return false;
-            tc::fence_after_sync();
-            const uint32_t col0 = 128 + (uint32_t)((c & 1) * kD);
-            tc::bulk_wait_read0();
-#pragma unroll 1
-            for (int cb = 0; cb < kD / 16; ++cb) {
-                uint32_t v[16];
-                tc::tmem_ld16(lane_base + col0 + cb * 16, v);
-                tc::tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 16; e += 4)
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(orow + (cb * 16 + e) * 4),
-                                 "r"(v[e]), "r"(v[e + 1]), "r"(v[e + 2]), "r"(v[e + 3]) : "memory");
-            }
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&o_empty[c & 1]);
-            if (prev_row >= 0) {
-                tc::fence_async_shared();
-                tc::bulk_reduce_add_f32(a.o_acc + (int64_t)prev_row * kD, orow, kD * 4);
-                tc::bulk_commit();
-            }
-            return true;
-        };
         for (int c = 0; c < nc; ++c) {
             const int st = c & 1;
-            if (!tc::warp_wait_bar(&st_full[st], (uint32_t)((c >> 1) & 1), abort)) { ok = false; break; }
+            if (!tc::warp_wait_bar(&st_full[st], (uint32_t)((c >> 1) & 1), abort)) break;
             const RowMeta meta(sm + L::kMeta + (c & 3) * L::kMetaBytes);
             const int n = min(tpc, ntok_total - c * tpc);
             const int ti = r / G, h = r - ti * G;
@@ -316,7 +291,7 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             }
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&st_empty[st]);
-            if (!tc::warp_wait_bar(&s_full[st], (uint32_t)((c >> 1) & 1), abort)) { ok = false; break; }
+            if (!tc::warp_wait_bar(&s_full[st], (uint32_t)((c >> 1) & 1), abort)) break;
             tc::fence_after_sync();
             uint32_t sv[kBS];
 #pragma unroll
@@ -335,7 +310,13 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     pk[k / 2] = *reinterpret_cast<uint32_t*>(&hp);
                 }
                 if (valid) atomicAdd(a.l_acc + qrow, rs);
-                if (c >= 1 && !tc::warp_wait_bar(p_empty, (uint32_t)((c - 1) & 1), abort)) { ok = false; break; }
+                // P of chunk c-1 has been consumed by its O product, which began only
+                // after the epilogue warps were done with chunk c-3 -- and so with
+                // the row ids of chunk c-4 that slot c & 3 held
+                if (c >= 1 && !tc::warp_wait_bar(p_empty, (uint32_t)((c - 1) & 1), abort)) break;
+                ids[(c & 3) * kRows + r] = qrow;
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(&ids_full[c & 3]);
 #pragma unroll
                 for (int cb = 0; cb < kBS / 8; ++cb) {
                     const uint32_t off = tc::sw128_offset(r, cb * 8);
@@ -347,16 +328,47 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(p_full);
-                if (c >= 1 && !o_epilogue(c - 1)) { ok = false; break; }
-                prev_row = qrow;
             }
         }
-        if (ok && nc > 0) o_epilogue(nc - 1);
+    } else if (warp < 4) {
+        // ------------------------------------------------------ epilogue warps ---
+        const int r = warp * 32 + lane;            // chunk row == TMEM lane
+        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        // O of chunk c: TMEM -> this thread's padded shared-memory row -> one
+        // 512-byte bulk add into the fp32 accumulator row. The row is reused
+        // only after the previous bulk add of this thread has read it.
+        const uint32_t orow = sbase + L::kOst + (uint32_t)r * L::kOstRow;
+        for (int c = 0; c < nc; ++c) {
+            if (!tc::warp_wait_bar(&ids_full[c & 3], (uint32_t)((c >> 2) & 1), abort)) break;
+            const int row_id = ids[(c & 3) * kRows + r];
+            if (!tc::warp_wait_bar(&o_full[c & 1], (uint32_t)((c >> 1) & 1), abort)) break;
+            tc::fence_after_sync();
+            const uint32_t col0 = 128 + (uint32_t)((c & 1) * kD);
+            tc::bulk_wait_read0();
+#pragma unroll 1
+            for (int cb = 0; cb < kD / 16; ++cb) {
+                uint32_t v[16];
+                tc::tmem_ld16(lane_base + col0 + cb * 16, v);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; e += 4)
+                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(orow + (cb * 16 + e) * 4),
+                                 "r"(v[e]), "r"(v[e + 1]), "r"(v[e + 2]), "r"(v[e + 3]) : "memory");
+            }
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&o_empty[c & 1]);
+            if (row_id >= 0) {
+                tc::fence_async_shared();
+                tc::bulk_reduce_add_f32(a.o_acc + (int64_t)row_id * kD, orow, kD * 4);
+                tc::bulk_commit();
+            }
+        }
         tc::bulk_wait0();
     }
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 2) {
+    if (warp == 10) {
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, L::kTmemCols);
     }
