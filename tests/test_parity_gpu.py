@@ -167,10 +167,14 @@ def test_tiny_variants_fp32(over):
     dict(batch=1, seq=384, n_q_heads=5, n_kv_heads=1, head_dim=128, block_size=64, top_k=2, dtype="bf16"),
     dict(batch=1, seq=320, n_q_heads=3, n_kv_heads=3, head_dim=128, block_size=32, top_k=5, dtype="fp32"),
     dict(batch=2, seq=192, n_q_heads=4, n_kv_heads=2, head_dim=64, block_size=64, top_k=1, dtype="fp32"),
+    dict(batch=1, seq=448, n_q_heads=2, n_kv_heads=2, head_dim=128, block_size=64, top_k=3, dtype="bf16"),
+    dict(batch=1, seq=512, n_q_heads=4, n_kv_heads=2, head_dim=128, block_size=64, top_k=4, dtype="bf16"),
 ])
 def test_small_shapes_elementwise(shape):
     """Ragged small problems over the supported ranges (G = 1..8, d 64/128,
-    block 32/64, both dtypes), every element against the oracle."""
+    block 32/64, both dtypes), every element against the oracle. The last two
+    run the gathered-row forward with two Q stages (G = 1) and with three at
+    the largest metadata slot that fits (G = 2)."""
     w = synth.Workload("small", "train", shape["batch"], shape["seq"], shape["n_q_heads"], shape["n_kv_heads"],
                        shape["head_dim"], shape["block_size"], shape["top_k"], shape["dtype"], 99, 0.5,
                        score_kind="gauss")

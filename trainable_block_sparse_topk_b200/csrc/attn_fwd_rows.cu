@@ -24,13 +24,14 @@
 // Executed MMA work is the definition's 4 d FLOP per kept (query head, key)
 // pair, with no masked rows.
 //
-// Roles (384 threads): warps 8 and 11 gather rows (even / odd chunks) with
-// coalesced 16-byte cp.async copies into two 128-byte-swizzled Q stages (TMA
-// tile::gather4 moves random rows at a fraction of that rate); warp 8 also
-// loads K_j and V_j by TMA; warp 9 lane 0 issues the MMAs; warp 10 owns TMEM;
-// warps 4-7 form P (thread = row = TMEM lane) and warps 0-3 read O back and
-// add it to the accumulator, so P of one chunk overlaps the output of the
-// previous one. No TMA multicast is used.
+// Roles (384 threads): warps 8, 11 and 10 gather rows (chunk c by loader
+// c mod 3) with coalesced 16-byte cp.async copies into three 128-byte-swizzled
+// Q stages (TMA tile::gather4 moves random rows at a fraction of that rate);
+// with G = 1 the chunk metadata needs more shared memory and two stages (warps
+// 8 and 11) are used. Warp 8 also loads K_j and V_j by TMA; warp 9 lane 0
+// issues the MMAs; warp 10 owns TMEM; warps 4-7 form P (thread = row = TMEM
+// lane) and warps 0-3 read O back and add it to the accumulator, so P of one
+// chunk overlaps the output of the previous one. No TMA multicast is used.
 #include <cuda.h>
 
 #include <algorithm>
@@ -47,6 +48,7 @@ constexpr int kThreads = 384;   // epilogue 0-3, P 4-7, loaders 8 and 11, MMA 9,
 constexpr int kBS = 64;
 constexpr int kRows = 128;
 constexpr int kD = 128;
+constexpr size_t kMaxSmemPerBlock = 232448;   // 227 KB of opt-in dynamic shared memory per CTA
 
 struct FwdRowsArgs {
     Shape sh;
@@ -55,52 +57,59 @@ struct FwdRowsArgs {
     float* l_acc;         // [B*Hq*T]
     float* o_acc;         // [B*Hq*T, d]
     int tpc;              // tokens per chunk = 128 / G
+    int meta_bytes;       // one metadata ring slot: tpc (16 + 4 rvs) bytes
 };
 
+// kSt Q stages (3 when shared memory allows, else 2); the metadata ring has
+// 2 kSt slots so each loader can request its next chunk's entries while it
+// gathers the current one.
+template <int kSt>
 struct RowsSmem {
     static constexpr uint32_t kK = 0;                              // K_j: 2 halves x [64 x 128 B]
     static constexpr uint32_t kV = 16384;                          // V_j
-    static constexpr uint32_t kStage = 32768;                      // 2 x Q [2 x 128 x 128 B]
+    static constexpr uint32_t kStage = 32768;                      // kSt x Q [2 x 128 x 128 B]
     static constexpr uint32_t kStageBytes = 32768;
-    static constexpr uint32_t kP = kStage + 2 * kStageBytes;       // P [128 x 128 B]
+    static constexpr uint32_t kP = kStage + kSt * kStageBytes;     // P [128 x 128 B]
     static constexpr uint32_t kOst = kP + 16384;                   // O rows, fp32, kOstRow apart
     static constexpr uint32_t kOstRow = kD * 4 + 16;               // padded: conflict-free 16-byte stores
-    static constexpr uint32_t kMeta = kOst + kRows * kOstRow;      // 4 x chunk stream entries (chunk c -> slot c & 3)
-    static constexpr uint32_t kMetaBytes = 4096;                   // int4 ent[<=128], then f32 rv[<= 512]
-    static constexpr uint32_t kIds = kMeta + 4 * kMetaBytes;       // i32 [4][128]: O accumulator row per chunk row
+    static constexpr uint32_t kIds = kOst + kRows * kOstRow;       // i32 [4][128]: O accumulator row per chunk row
     static constexpr uint32_t kBar = kIds + 4 * kRows * 4;
-    static constexpr int kNumBars = 22;
+    static constexpr int kMetaSlots = 2 * kSt;                     // chunk c -> slot c % kMetaSlots
+    static constexpr int kNumBars = 13 + 4 * kSt;
     static constexpr uint32_t kMisc = kBar + 8 * kNumBars;         // tmem base, stream length, first entry, abort
+    static constexpr uint32_t kMeta = (kMisc + 16 + 15) & ~15u;    // metadata ring, meta_bytes per slot
     static constexpr uint32_t kTmemCols = 512;                     // S double [0,128), O double [128,384)
-    static constexpr uint32_t kTotal = kMisc + 16;
+    static constexpr size_t total(int meta_bytes) { return kMeta + (size_t)kMetaSlots * meta_bytes; }
 };
 
-// One ring slot: the chunk's stream entries (token, log-gate) and each entry's
-// per-head shift, copied in by the bulk-copy engine.
+// One ring slot: the chunk's stream entries (token, log-gate) for tpc tokens,
+// then each entry's per-head shift, copied in by the bulk-copy engine.
 struct RowMeta {
     const int4* ent;
     const float* rv;
-    __device__ explicit RowMeta(const unsigned char* p)
-        : ent(reinterpret_cast<const int4*>(p)), rv(reinterpret_cast<const float*>(p + 2048)) {}
+    __device__ RowMeta(const unsigned char* p, int tpc)
+        : ent(reinterpret_cast<const int4*>(p)), rv(reinterpret_cast<const float*>(p + 16 * tpc)) {}
 };
 
+template <int kSt>
 __global__ void __launch_bounds__(kThreads, 1)
 fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const __grid_constant__ FwdRowsArgs a) {
-    using L = RowsSmem;
+    using L = RowsSmem<kSt>;
+    constexpr int kMS = L::kMetaSlots;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
     uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
     uint64_t* kv_full = bars + 0;
-    uint64_t* st_full = bars + 1;     // [2]: the loader's arrive once its copies have landed
-    uint64_t* st_empty = bars + 3;    // [2] MMA commit + 4 compute-warp arrivals
-    uint64_t* s_full = bars + 5;      // [2]
-    uint64_t* p_full = bars + 7;      // 4 arrivals
-    uint64_t* p_empty = bars + 8;
-    uint64_t* o_full = bars + 9;      // [2]
-    uint64_t* o_empty = bars + 11;    // [2] 4 arrivals
-    uint64_t* meta_full = bars + 13;  // [4] ring slot c & 3 holds chunk c's stream entries (tx bytes)
-    uint64_t* ids_full = bars + 17;   // [4] 4 arrivals: chunk c's O rows are in ids[c & 3]
+    uint64_t* st_full = bars + 1;             // [kSt]: the loader's arrive once its copies have landed
+    uint64_t* st_empty = st_full + kSt;       // [kSt] MMA commit + 4 compute-warp arrivals
+    uint64_t* s_full = st_empty + kSt;        // [2]
+    uint64_t* p_full = s_full + 2;            // 4 arrivals
+    uint64_t* p_empty = p_full + 1;
+    uint64_t* o_full = p_empty + 1;           // [2]
+    uint64_t* o_empty = o_full + 2;           // [2] 4 arrivals
+    uint64_t* meta_full = o_empty + 2;        // [kMS] ring slot c % kMS holds chunk c's stream entries (tx bytes)
+    uint64_t* ids_full = meta_full + kMS;     // [4] 4 arrivals: chunk c's O rows are in ids[c & 3]
     int* ids = reinterpret_cast<int*>(sm + L::kIds);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMisc);
     int* ntok_slot = reinterpret_cast<int*>(sm + L::kMisc + 4);      // [2]: stream length, first entry
@@ -125,8 +134,8 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             // a stage is refilled only after the MMA has read its rows and the
             // compute warps have waited for it: its phases then cannot run two
             // ahead of any waiter
-            if (bar == &st_empty[0] || bar == &st_empty[1]) cnt = 5;
-            if (bar == &st_full[0] || bar == &st_full[1]) cnt = 33;   // 32 cp.async arrivals + the loader's
+            if (bar >= st_empty && bar < st_empty + kSt) cnt = 5;
+            if (bar >= st_full && bar < st_full + kSt) cnt = 33;   // 32 cp.async arrivals + the loader's
             mbar_init(bar, cnt);
         }
         ntok_slot[0] = a.ss.count[(int64_t)bg * sh.NB + j];   // tokens in block j's stream
@@ -147,9 +156,11 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const int nc = (ntok_total + tpc - 1) / tpc;
     const uint32_t sbase = smem_u32(sm);
 
-    if (warp == 8 || warp == 11) {
+    if (warp == 8 || warp == 11 || (kSt == 3 && warp == 10)) {
         // ---------------------------------------------------------- loaders ---
-        const int L0 = warp == 8 ? 0 : 1;
+        // loader L0 fills stage L0 with chunks L0, L0 + kSt, ... (warp 10 joins
+        // once it has allocated TMEM)
+        const int L0 = warp == 8 ? 0 : warp == 11 ? 1 : 2;
         unsigned char* stq = sm + L::kStage + L0 * L::kStageBytes;
         if (warp == 8 && lane == 0) {
             tc::prefetch_tmap(&tm_k);
@@ -161,25 +172,26 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 tc::tma_load_2d(sm + L::kV + h * 8192, &tm_v, h * 64, kr, kv_full);
             }
         }
-        // chunk c's stream entries -> ring slot c & 3 (bulk copies, completion on meta_full)
+        // chunk c's stream entries -> ring slot c % kMS (bulk copies, completion on meta_full)
         auto request = [&](int c) {
             if (lane == 0) {
                 const int n = min(tpc, ntok_total - c * tpc);
                 const int64_t e0 = ebase + (int64_t)c * tpc;
-                unsigned char* slot = sm + L::kMeta + (c & 3) * L::kMetaBytes;
+                const int s = c % kMS;
+                unsigned char* slot = sm + L::kMeta + s * a.meta_bytes;
                 const uint32_t be = 16u * (uint32_t)n, br = 4u * (uint32_t)(n * rvs);
-                mbar_arrive_expect_tx(&meta_full[c & 3], be + br);
-                bulk_g2s(slot, a.ss.ent + e0, be, &meta_full[c & 3]);
-                bulk_g2s(slot + 2048, a.ss.rv + e0 * rvs, br, &meta_full[c & 3]);
+                mbar_arrive_expect_tx(&meta_full[s], be + br);
+                bulk_g2s(slot, a.ss.ent + e0, be, &meta_full[s]);
+                bulk_g2s(slot + 16 * tpc, a.ss.rv + e0 * rvs, br, &meta_full[s]);
             }
         };
         if (L0 < nc) request(L0);
-        for (int c = L0; c < nc; c += 2) {
-            if (c >= 2 && !tc::warp_wait_bar(&st_empty[L0], (uint32_t)(((c >> 1) - 1) & 1), abort)) break;
-            // slot (c + 2) & 3 held chunk c - 2, whose readers are done with it once its stage is released
-            if (c + 2 < nc) request(c + 2);
-            if (!tc::warp_wait_bar(&meta_full[c & 3], (uint32_t)((c >> 2) & 1), abort)) break;
-            const int4* ent = RowMeta(sm + L::kMeta + (c & 3) * L::kMetaBytes).ent;
+        for (int c = L0, k = 0; c < nc; c += kSt, ++k) {
+            if (k >= 1 && !tc::warp_wait_bar(&st_empty[L0], (uint32_t)((k - 1) & 1), abort)) break;
+            // slot (c + kSt) % kMS held chunk c - kSt, whose readers are done with it once its stage is released
+            if (c + kSt < nc) request(c + kSt);
+            if (!tc::warp_wait_bar(&meta_full[c % kMS], (uint32_t)((c / kMS) & 1), abort)) break;
+            const int4* ent = RowMeta(sm + L::kMeta + (c % kMS) * a.meta_bytes, tpc).ent;
             const int n = min(tpc, ntok_total - c * tpc);
             {
                 // 16 lanes copy one 256-byte q row (16-byte pieces, coalesced), two
@@ -210,7 +222,7 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             constexpr uint32_t id_o = tc::idesc_bf16_f32(128, kD, false, true);
             const uint32_t ka = sbase + L::kK, va = sbase + L::kV, pa = sbase + L::kP;
             auto issue_s = [&](int c) {
-                const uint32_t qa = sbase + L::kStage + (c & 1) * L::kStageBytes;
+                const uint32_t qa = sbase + L::kStage + (c % kSt) * L::kStageBytes;
                 const uint32_t ds = tmem + (uint32_t)((c & 1) * kBS);
 #pragma unroll
                 for (int kk = 0; kk < kD / 16; ++kk) {
@@ -220,7 +232,7 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                                id_s, kk > 0);
                 }
                 tc::mma_commit(&s_full[c & 1]);
-                tc::mma_commit(&st_empty[c & 1]);     // Q of the stage is read only by S
+                tc::mma_commit(&st_empty[c % kSt]);   // Q of the stage is read only by S
             };
             bool ok = tc::wait_bar(kv_full, 0u, abort);
             {
@@ -232,7 +244,7 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 while (ok && c < nc) {
                     bool progressed = false;
                     if (s_next < nc && s_next <= c + 1 &&
-                        mbar_test_wait(&st_full[s_next & 1], (uint32_t)((s_next >> 1) & 1))) {
+                        mbar_test_wait(&st_full[s_next % kSt], (uint32_t)((s_next / kSt) & 1))) {
                         tc::fence_async_shared();
                         tc::fence_after_sync();
                         issue_s(s_next);
@@ -272,9 +284,9 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         const uint32_t lane_base = tmem + ((uint32_t)((warp & 3) * 32) << 16);
         const float qk = sh.scale * kLog2e;
         for (int c = 0; c < nc; ++c) {
-            const int st = c & 1;
-            if (!tc::warp_wait_bar(&st_full[st], (uint32_t)((c >> 1) & 1), abort)) break;
-            const RowMeta meta(sm + L::kMeta + (c & 3) * L::kMetaBytes);
+            const int stg = c % kSt, st = c & 1;    // Q stage, S buffer
+            if (!tc::warp_wait_bar(&st_full[stg], (uint32_t)((c / kSt) & 1), abort)) break;
+            const RowMeta meta(sm + L::kMeta + (c % kMS) * a.meta_bytes, tpc);
             const int n = min(tpc, ntok_total - c * tpc);
             const int ti = r / G, h = r - ti * G;
             const bool valid = ti < n;
@@ -290,7 +302,7 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                 qrow = (int)(((int64_t)b * sh.Hq + g * G + h) * T + t);
             }
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&st_empty[st]);
+            if (lane == 0) tc::mbar_arrive(&st_empty[stg]);
             if (!tc::warp_wait_bar(&s_full[st], (uint32_t)((c >> 1) & 1), abort)) break;
             tc::fence_after_sync();
             uint32_t sv[kBS];
@@ -507,12 +519,17 @@ cudaError_t launch_fwd_rows(const Shape& s, const void* q, const void* k, const 
     count_launches(1);
     e = launch_sel_stream(s, maskT, idx, gl, nsel, w.shift, nullptr, 1, a.ss, st);
     if (e != cudaSuccess) return e;
-    const size_t smem = RowsSmem::kTotal + 1024;
-    e = cudaFuncSetAttribute(fwd_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    a.meta_bytes = a.tpc * (16 + 4 * a.ss.rvs);
+    // three Q stages when they fit in shared memory (G >= 2), else two
+    const size_t smem3 = RowsSmem<3>::total(a.meta_bytes) + 1024;
+    const bool three = smem3 <= kMaxSmemPerBlock;
+    const size_t smem = three ? smem3 : RowsSmem<2>::total(a.meta_bytes) + 1024;
+    auto kern = three ? fwd_rows_kernel<3> : fwd_rows_kernel<2>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     {
         KernelTimer kt("fwd_rows", st);
-        fwd_rows_kernel<<<(unsigned)((int64_t)s.B * s.Hkv * s.nT), kThreads, smem, st>>>(mk, mv, a);
+        kern<<<(unsigned)((int64_t)s.B * s.Hkv * s.nT), kThreads, smem, st>>>(mk, mv, a);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
