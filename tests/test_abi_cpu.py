@@ -62,21 +62,24 @@ def test_workspace_sizes(L):
     assert ws_size(B.SAS_OP_TOPK, d) == (0, 0)
     st, n = ws_size(B.SAS_OP_BWD, d)
     assert st == 0
-    # column bitmap + D + Gsum + fp32 dq accumulator, each 256-byte aligned
+    # per-block token streams: capacity B*Hkv*T*(K+1) entries of 16 bytes plus
+    # rvs per-head row values (rounded up to 16 bytes), per-block first entry
+    # and count, per-(block, query tile) running counts and the allocation
+    # counter; each piece 256-byte aligned
     NB, nT = 4, 4
+    cap = 1 * 2 * 256 * (3 + 1)
+    a = lambda p: (p + 255) // 256 * 256
+    stream = lambda rvs: a(16 * cap) + a(4 * cap * rvs) + 2 * a(4 * 2 * NB) + a(4 * 2 * NB * nT) + 256
+    # backward: column bitmap + D + Gsum + fp32 dq accumulator, then the
+    # streams with the lse and D of each of the G = 4 heads (rvs 8)
     parts = [8 * 1 * 2 * NB * nT, 4 * 8 * 256, 4 * 2 * 256 * 3, 4 * 8 * 256 * 128]
-    assert n == sum((p + 255) // 256 * 256 for p in parts)
+    assert n == sum(a(p) for p in parts) + a(stream(8))
     # forward (tensor-core shapes): column bitmap, then per query-head row the
     # shift, flagged-row list, l and the fp32 output accumulator plus the
-    # flagged-row count, then the per-block token streams: capacity
-    # B*Hkv*T*(K+1) entries of 16 bytes plus per-head shifts rounded up to 16
-    # bytes, per-block first entry and count, per-(block, query tile) running
-    # counts and the allocation counter; each piece 256-byte aligned
-    rows, cap, rvs = 8 * 256, 1 * 2 * 256 * (3 + 1), 4
-    a = lambda p: (p + 255) // 256 * 256
+    # flagged-row count, then the streams with the shift of each head (rvs 4)
+    rows = 8 * 256
     head = a(12 * rows + 4 * rows * 128 + 16)
-    stream = a(16 * cap) + a(4 * cap * rvs) + 2 * a(4 * 2 * NB) + a(4 * 2 * NB * nT) + 256
-    assert ws_size(B.SAS_OP_FWD, d) == (0, a(8 * 1 * 2 * NB * nT) + a(head + stream))
+    assert ws_size(B.SAS_OP_FWD, d) == (0, a(8 * 1 * 2 * NB * nT) + a(head + stream(4)))
     st, n32 = ws_size(B.SAS_OP_BWD, desc(dtype="fp32"))
     assert st == 0 and n32 < n            # fp32 accumulates dq in place
     dd = desc(seq_len=1, q_offset=4095)

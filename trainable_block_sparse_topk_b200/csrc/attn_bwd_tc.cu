@@ -11,8 +11,11 @@
 // Tiling: key-block-centric. One CTA owns key block j of one (batch, KV
 // group). It streams the (token, head) rows whose attention includes j -- the
 // block's own 64 tokens (causally) and every later token whose selection kept
-// j, read from the column bitmap -- in chunks of 128 gathered rows (128/G
-// tokens x G heads), so every MMA row is a kept row. Per chunk:
+// j -- in chunks of 128 gathered rows (128/G tokens x G heads), so every MMA
+// row is a kept row. The walk is laid out beforehand as a per-block token
+// stream (stream.cu) whose entries carry each token's log-gate and kept-list
+// slot and each row's lse and D; the CTA bulk-copies a chunk's entries into
+// a ring two chunks ahead. Per chunk:
 //   S = Q K_j^T and dP = dO V_j^T  (M=128 rows, N=64 keys, K=d)   -> TMEM
 //   P, dS in the compute warps (thread = row = TMEM lane), Gsum per token
 //   dV^T += dO^T P, dK^T += Q^T dS (M=d, N=64, K=128 rows)        -> TMEM
@@ -25,12 +28,12 @@
 //
 // Roles (512 threads): warps 0-3 epilogue (dQ reductions, final dK/dV),
 // warps 4-7 and 12-15 P/dS and Gsum for keys 0-31 and 32-63 of the block
-// (thread = row = TMEM lane in every group), warps 8
-// and 11 gather chunk rows (even / odd chunks) with coalesced 16-byte cp.async
-// copies into the two 128-byte-swizzled Q/dO stages (TMA tile::gather4 moves
-// random rows at a fraction of that rate; warp 8 also loads K_j, V_j by TMA),
-// warp 9 lane 0 issues the MMAs, warp 10 owns the TMEM allocation. No TMA
-// multicast is used.
+// (thread = row = TMEM lane in every group), warps 8 and 11 gather each
+// chunk's rows (rows 0-63 / 64-127) with coalesced 16-byte cp.async copies
+// into the two 128-byte-swizzled Q/dO stages (TMA tile::gather4 moves random
+// rows at a fraction of that rate; warp 8 also loads K_j, V_j by TMA), warp 9
+// lane 0 issues the MMAs, warp 10 owns the TMEM allocation. No TMA multicast
+// is used.
 #include <cuda.h>
 
 #include "common.cuh"
@@ -52,17 +55,13 @@ struct BwdTcArgs {
     Shape sh;
     const __nv_bfloat16* q;
     const __nv_bfloat16* dO;
-    const float* lse;
-    const float* Dd;
-    const int32_t* idx;
-    const float* gl;
-    const int32_t* nsel;
-    const uint64_t* maskT;
+    SelStream ss;        // per-block token streams: {t, log-gate, slot}, then lse and D of each head
     float* dq_acc;
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
     float* gsum;
-    int tpc;   // tokens per chunk = 128 / G
+    int tpc;             // tokens per chunk = 128 / G
+    int meta_bytes;      // one metadata ring slot: tpc (16 + 4 rvs) bytes
 };
 
 struct BwdSmem {
@@ -72,34 +71,23 @@ struct BwdSmem {
     static constexpr uint32_t kStageBytes = 65536;
     static constexpr uint32_t kP = kStage + 2 * kStageBytes;   // P  [128 x 128 B]
     static constexpr uint32_t kDS = kP + 16384;                // dS [128 x 128 B]
-    static constexpr uint32_t kMeta = kDS + 16384;             // 4 x per-chunk metadata (chunk c -> slot c & 3)
-    static constexpr uint32_t kMetaBytes = 6 * 512 + 16;       // tok_t, tok_slot, tok_lg, row_lse, row_D, qoff, ntok
-    static constexpr uint32_t kGs = kMeta + 4 * kMetaBytes;    // per-token Gsum [2][128] f32
+    static constexpr uint32_t kGs = kDS + 16384;               // per-token Gsum [2][128] f32
     static constexpr uint32_t kIds = kGs + 1024;               // i32 [2][128]: dQ accumulator row per chunk row
-    static constexpr uint32_t kColW = kIds + 1024;             // u64 [kMaxNT]: the block's bitmap column
-    static constexpr uint32_t kPre = kColW + 8 * 1024;         // i32 [kMaxNT]: stream index of tile tau's first token
-    static constexpr uint32_t kBar = kPre + 4 * 1024;
-    static constexpr int kNumBars = 14;
-    static constexpr uint32_t kMisc = kBar + 8 * kNumBars;     // tmem base, chunk count, abort
-    static constexpr uint32_t kTotal = kMisc + 16;
+    static constexpr uint32_t kBar = kIds + 1024;
+    static constexpr int kNumBars = 18;
+    static constexpr uint32_t kMisc = kBar + 8 * kNumBars;     // tmem base, stream length, first entry, abort
+    static constexpr uint32_t kMeta = (kMisc + 16 + 15) & ~15u;   // 4 x chunk stream entries (chunk c -> slot c & 3)
+    static constexpr size_t total(int meta_bytes) { return kMeta + 4 * (size_t)meta_bytes; }
 };
 
-struct Meta {
-    int* tok_t;
-    int* tok_slot;
-    float* tok_lg;
-    float* row_lse;
-    float* row_D;
-    int* qoff;     // q/dO row of each chunk row, -1 for padding
-    int* ntok;
-    __device__ explicit Meta(unsigned char* p)
-        : tok_t(reinterpret_cast<int*>(p)),
-          tok_slot(reinterpret_cast<int*>(p + 512)),
-          tok_lg(reinterpret_cast<float*>(p + 1024)),
-          row_lse(reinterpret_cast<float*>(p + 1536)),
-          row_D(reinterpret_cast<float*>(p + 2048)),
-          qoff(reinterpret_cast<int*>(p + 2560)),
-          ntok(reinterpret_cast<int*>(p + 3072)) {}
+// One metadata ring slot: the chunk's stream entries (token, log-gate, slot of
+// block j in the token's kept list) for tpc tokens, then per entry the lse and
+// D of each of its G query heads; copied in by the bulk-copy engine.
+struct ChunkMeta {
+    const int4* ent;
+    const float* rv;
+    __device__ ChunkMeta(const unsigned char* p, int tpc)
+        : ent(reinterpret_cast<const int4*>(p)), rv(reinterpret_cast<const float*>(p + 16 * tpc)) {}
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -119,9 +107,10 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     uint64_t* dq_empty = bars + 10;   // 4 arrivals
     uint64_t* done = bars + 11;
     uint64_t* ids_full = bars + 12;   // [2] 4 arrivals: the chunk's dQ row ids are in ids[]
+    uint64_t* meta_full = bars + 14;  // [4] ring slot c & 3 holds chunk c's stream entries (tx bytes)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMisc);
-    int* nc_slot = reinterpret_cast<int*>(sm + L::kMisc + 4);
-    volatile int* abort = reinterpret_cast<volatile int*>(sm + L::kMisc + 8);
+    int* ntok_slot = reinterpret_cast<int*>(sm + L::kMisc + 4);      // [2]: stream length, first entry
+    volatile int* abort = reinterpret_cast<volatile int*>(sm + L::kMisc + 12);
     float* tok_gs = reinterpret_cast<float*>(sm + L::kGs);
     int* ids = reinterpret_cast<int*>(sm + L::kIds);
 
@@ -133,7 +122,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     const int bg = (int)(blockIdx.x % ngroups);
     const int b = bg / sh.Hkv, g = bg % sh.Hkv;
     const int tpc = a.tpc;
-    const uint64_t* col = a.maskT + ((int64_t)bg * sh.NB + j) * sh.nT;
+    const int rvs = a.ss.rvs;
 
     if (tid == 0) {
         for (int i = 0; i < L::kNumBars; ++i) {
@@ -141,10 +130,12 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             uint32_t cnt = 1;
             if (bar == dq_empty || bar == &ids_full[0] || bar == &ids_full[1]) cnt = 4;
             if (bar == p_full) cnt = 8;
-            if (bar == &st_full[0] || bar == &st_full[1]) cnt = 33;   // 32 cp.async arrivals + the loader's
+            // both loaders fill every stage: 32 cp.async arrivals + one arrive each
+            if (bar == &st_full[0] || bar == &st_full[1]) cnt = 66;
             mbar_init(bar, cnt);
         }
-        *nc_slot = kBS;   // the block's own tokens; later tiles are added below
+        ntok_slot[0] = a.ss.count[(int64_t)bg * sh.NB + j];   // tokens in block j's stream
+        ntok_slot[1] = a.ss.base[(int64_t)bg * sh.NB + j];    // its first entry
         *abort = 0;
         fence_mbar_init();
     }
@@ -152,45 +143,21 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         tc::tmem_alloc(tmem_slot, kTmemCols);
         tc::tmem_relinquish();
     }
-    // The token stream of block j: its own 64 tokens, then the tokens of later
-    // tiles that kept j, in order. colw holds the bitmap column, pre[tau] the
-    // stream index of tile tau's first token (valid for tau > j).
-    unsigned long long* colw = reinterpret_cast<unsigned long long*>(sm + L::kColW);
-    int* pre = reinterpret_cast<int*>(sm + L::kPre);
     for (int i = tid; i < 2 * kRows; i += kThreads) tok_gs[i] = 0.f;
-    for (int tau = tid; tau < sh.nT; tau += kThreads) colw[tau] = tau > j ? col[tau] : 0ull;
-    __syncthreads();
-    if (warp == 0) {
-        const int per = (sh.nT + 31) / 32;       // consecutive tiles per lane
-        const int t0 = lane * per, t1 = min(t0 + per, sh.nT);
-        int sum = 0;
-        for (int tau = t0; tau < t1; ++tau) sum += __popcll(colw[tau]);
-        int inc = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, inc, o);
-            if (lane >= o) inc += y;
-        }
-        int run = kBS + inc - sum;
-        for (int tau = t0; tau < t1; ++tau) {
-            pre[tau] = run;
-            run += __popcll(colw[tau]);
-        }
-        if (lane == 31) *nc_slot = kBS + inc;
-    }
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const int ntok_total = *nc_slot;
+    const int ntok_total = ntok_slot[0];
+    const int64_t ebase = ntok_slot[1];
     const int nc = (ntok_total + tpc - 1) / tpc;
     const uint32_t sbase = smem_u32(sm);
 
     if (warp == 8 || warp == 11) {
         // ---------------------------------------------------------- loaders ---
-        const int L0 = warp == 8 ? 0 : 1;           // this warp fills chunks c = L0, L0 + 2, ...
-        unsigned char* stq = sm + L::kStage + L0 * L::kStageBytes;
-        unsigned char* stdo = stq + 32768;
+        // Both loaders gather every chunk (warp 8 rows 0-63, warp 11 rows
+        // 64-127); loader w requests the stream entries of chunks c = w mod 2.
+        const int w = warp == 8 ? 0 : 1;
         if (warp == 8 && lane == 0) {
             tc::prefetch_tmap(&tm_k);
             tc::prefetch_tmap(&tm_v);
@@ -201,107 +168,51 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 tc::tma_load_2d(sm + L::kV + h * 8192, &tm_v, h * 64, kr, kv_full);
             }
         }
-        // token of stream index s: the block's own tile first, then the bitmap
-        auto token_at = [&](int s) -> int {
-            if (s < kBS) return j * kBS + s;
-            int lo = j + 1, hi = sh.nT - 1;      // last tile with pre[tile] <= s
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (pre[mid] <= s) lo = mid; else hi = mid - 1;
+        // chunk c's stream entries -> ring slot c & 3 (bulk copies, completion on meta_full)
+        auto request = [&](int c) {
+            if (lane == 0) {
+                const int n = min(tpc, ntok_total - c * tpc);
+                const int64_t e0 = ebase + (int64_t)c * tpc;
+                unsigned char* slot = sm + L::kMeta + (c & 3) * a.meta_bytes;
+                const uint32_t be = 16u * (uint32_t)n, br = 4u * (uint32_t)(n * rvs);
+                mbar_arrive_expect_tx(&meta_full[c & 3], be + br);
+                bulk_g2s(slot, a.ss.ent + e0, be, &meta_full[c & 3]);
+                bulk_g2s(slot + 16 * tpc, a.ss.rv + e0 * rvs, br, &meta_full[c & 3]);
             }
-            uint64_t w = colw[lo];
-            for (int r = s - pre[lo]; r > 0; --r) w &= w - 1ull;
-            return lo * kBS + __ffsll((long long)w) - 1;
         };
-        // metadata of chunk c into ring slot c & 3 (global loads only; no stage
-        // needed). Independent loads go out together -- every row's lse and D
-        // with every token's kept list -- then the log-gates of block j.
-        auto prep = [&](int c) {
-            Meta meta(sm + L::kMeta + (c & 3) * L::kMetaBytes);
+        if (w < nc) request(w);
+        for (int c = 0; c < nc; ++c) {
+            if (c >= 2 && !tc::warp_wait_bar(&st_empty[c & 1], (uint32_t)(((c >> 1) - 1) & 1), abort)) break;
+            // slot (c + 2) & 3 held chunk c - 2, whose readers are done with it once its stage is released
+            if ((c & 1) == w && c + 2 < nc) request(c + 2);
+            if (!tc::warp_wait_bar(&meta_full[c & 3], (uint32_t)((c >> 2) & 1), abort)) break;
+            const int4* ent = ChunkMeta(sm + L::kMeta + (c & 3) * a.meta_bytes, tpc).ent;
             const int n = min(tpc, ntok_total - c * tpc);
-            if (lane == 0) *meta.ntok = n;
-            for (int i = lane; i < n; i += 32) meta.tok_t[i] = token_at(c * tpc + i);
-            __syncwarp();
-            float lse[kRows / 32], Dv[kRows / 32];
-            int qrow[kRows / 32];
-#pragma unroll
-            for (int u = 0; u < kRows / 32; ++u) {
-                const int i = lane + 32 * u, ti = i / G, h = i - ti * G;
-                qrow[u] = -1;
-                lse[u] = 0.f;
-                Dv[u] = 0.f;
-                if (ti < n) {
-                    qrow[u] = (int)(((int64_t)b * sh.Hq + g * G + h) * T + meta.tok_t[ti]);
-                    lse[u] = a.lse[qrow[u]];
-                    Dv[u] = a.Dd[qrow[u]];
-                }
-            }
-            for (int i = lane; i < n; i += 32) {
-                const int t = meta.tok_t[i];
-                int slot = -1;
-                float lg = 0.f;
-                if ((t >> 6) != j) {
-                    // slot of j in the row's ascending kept list = number of kept blocks below j
-                    const int64_t row = (int64_t)bg * T + t;
-                    const int32_t* ir = a.idx + row * K;
-                    const int ns = a.nsel[row];
-                    int below = 0;
-#pragma unroll 16
-                    for (int s = 0; s < K; ++s) {
-                        const int v = ir[s];
-                        below += (s < ns) & (v < j);
-                    }
-                    slot = min(below, K - 1);
-                    lg = a.gl[row * K + slot];
-                }
-                meta.tok_slot[i] = slot;
-                meta.tok_lg[i] = lg;
-            }
-#pragma unroll
-            for (int u = 0; u < kRows / 32; ++u) {
-                const int i = lane + 32 * u;
-                meta.row_lse[i] = lse[u];
-                meta.row_D[i] = Dv[u];
-                meta.qoff[i] = qrow[u];
-                if (qrow[u] >= 0) {           // the rows are copied about two chunks later
-                    tc::prefetch_l2(a.q + (int64_t)qrow[u] * kD);
-                    tc::prefetch_l2(a.q + (int64_t)qrow[u] * kD + 64);
-                    tc::prefetch_l2(a.dO + (int64_t)qrow[u] * kD);
-                    tc::prefetch_l2(a.dO + (int64_t)qrow[u] * kD + 64);
-                }
-            }
-            __syncwarp();
-        };
-        if (L0 < nc) prep(L0);
-        for (int c = L0; c < nc; c += 2) {
-            if (c >= 2 && !tc::warp_wait_bar(&st_empty[L0], (uint32_t)(((c >> 1) - 1) & 1), abort)) break;
-            // rows: TMA gather of 4 rows x 64 columns per instruction; lane l
-            // fetches rows 4l..4l+3 of both d halves of q and dO. Padding rows
-            // re-read the chunk's first row (their P and dS are zero).
-            const int* qoff = Meta(sm + L::kMeta + (c & 3) * L::kMetaBytes).qoff;
+            unsigned char* stq = sm + L::kStage + (c & 1) * L::kStageBytes;
+            unsigned char* stdo = stq + 32768;
             {
                 // 16 lanes copy one 256-byte row (16-byte pieces, coalesced), two
                 // rows per instruction, into the swizzled tile; row i's piece p
-                // lands in d-half p / 8 at 16-byte chunk p % 8.
+                // lands in d-half p / 8 at 16-byte chunk p % 8. Padding rows
+                // re-read the chunk's first row (their P and dS are zero).
                 const int p = lane & 15, hh = p >> 3, col = (p & 7) * 8;
-                const int q0 = qoff[0];
 #pragma unroll 4
-                for (int i = 0; i < kRows / 2; ++i) {
-                    const int row = 2 * i + (lane >> 4);
-                    int qrow = qoff[row];
-                    if (qrow < 0) qrow = q0;
+                for (int i = 0; i < kRows / 4; ++i) {
+                    const int row = w * (kRows / 2) + 2 * i + (lane >> 4);
+                    int ti = row / G, h = row - ti * G;
+                    if (ti >= n) ti = 0, h = 0;
+                    const int64_t qrow = ((int64_t)b * sh.Hq + g * G + h) * T + ent[ti].x;
                     const uint32_t off = hh * 16384 + tc::sw128_offset(row, col);
-                    tc::cp_async16(stq + off, a.q + (int64_t)qrow * kD + p * 8);
-                    tc::cp_async16(stdo + off, a.dO + (int64_t)qrow * kD + p * 8);
+                    tc::cp_async16(stq + off, a.q + qrow * kD + p * 8);
+                    tc::cp_async16(stdo + off, a.dO + qrow * kD + p * 8);
                 }
             }
-            // st_full completes once every lane's copies have landed (32 async
-            // arrivals) and lane 0 has published the chunk's metadata; the MMA
-            // thread fences the async proxy after its wait
-            tc::cp_async_mbar_arrive_noinc(&st_full[L0]);
+            // st_full completes once both loaders' copies have landed (32 async
+            // arrivals each) and each has arrived once; the MMA thread fences
+            // the async proxy after its wait
+            tc::cp_async_mbar_arrive_noinc(&st_full[c & 1]);
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&st_full[L0]);
-            if (c + 2 < nc) prep(c + 2);   // overlaps the copies in flight
+            if (lane == 0) tc::mbar_arrive(&st_full[c & 1]);
         }
         tc::cp_async_wait_all();
     } else if (warp == 9) {
@@ -397,27 +308,28 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         for (int c = 0; c < nc; ++c) {
             const int st = c & 1;
             if (!tc::warp_wait_bar(&st_full[st], (uint32_t)((c >> 1) & 1), abort)) break;
-            Meta meta(sm + L::kMeta + (c & 3) * L::kMetaBytes);
-            const int n = *meta.ntok;
+            const ChunkMeta meta(sm + L::kMeta + (c & 3) * a.meta_bytes, tpc);
+            const int n = min(tpc, ntok_total - c * tpc);
             const int ti = r / G, h = r - ti * G;
             const bool valid = ti < n;
             int t = 0, kmax = -1;
             float lgl = 0.f, lse2 = 0.f, Dv = 0.f;
             bool diag = false;
             if (valid) {
-                t = meta.tok_t[ti];
+                const int4 e = meta.ent[ti];
+                t = e.x;
                 diag = (t >> 6) == j;
                 kmax = diag ? (t & 63) : kBS - 1;
-                lgl = meta.tok_lg[ti];
-                lse2 = meta.row_lse[r];
-                Dv = meta.row_D[r];
+                lgl = __int_as_float(e.y);
+                lse2 = meta.rv[ti * rvs + 2 * h];
+                Dv = meta.rv[ti * rvs + 2 * h + 1];
             }
             const float bias = (lgl - lse2) * kLog2e;
             const int dq_row = valid ? (int)(((int64_t)b * sh.Hq + g * G + h) * T + t) : -1;
             // token r of the chunk, for its Gsum (read now: the metadata slot is
             // refilled once the chunk's last MMAs are issued)
-            const int gs_slot = r < n ? meta.tok_slot[r] : -1;
-            const int gs_tok = r < n ? meta.tok_t[r] : 0;
+            const int gs_slot = r < n ? meta.ent[r].z : -1;
+            const int gs_tok = r < n ? meta.ent[r].x : 0;
             if (!tc::warp_wait_bar(&s_full[st], (uint32_t)((c >> 1) & 1), abort)) break;
             // P and dS of chunk c-1 must have been consumed by its MMAs; that also
             // means the epilogue warps are done with chunk c-2, whose row-id slot
@@ -568,19 +480,33 @@ bool bwd_tc_supported(const Shape& s) {
            s.T % kBS == 0 && s.nT <= 1024 && (int64_t)s.B * s.Hq * s.T < ((int64_t)1 << 31);
 }
 
+size_t bwd_tc_ws_bytes(const Shape& s) { return sel_stream_bytes(s, 2); }
+
 cudaError_t launch_bwd_tc(const Shape& s, const void* q, const void* k, const void* v, const void* dO,
                           const float* lse, const float* Dd, const int32_t* idx, const float* gl,
-                          const int32_t* nsel, const uint64_t* maskT, float* dq_acc, void* dk, void* dv,
+                          const int32_t* nsel, const uint64_t* maskT, void* ws, float* dq_acc, void* dk, void* dv,
                           float* gsum, cudaStream_t st) {
     CUtensorMap mk, mv;
     if (!encode_bf16_2d(&mk, k, (uint64_t)s.B * s.Hkv * s.T, kD, kBS) ||
         !encode_bf16_2d(&mv, v, (uint64_t)s.B * s.Hkv * s.T, kD, kBS))
         return cudaErrorInvalidValue;
-    const size_t smem = BwdSmem::kTotal + 1024;
-    cudaError_t e = cudaFuncSetAttribute(bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    BwdTcArgs a{};
+    a.sh = s;
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.dO = static_cast<const __nv_bfloat16*>(dO);
+    a.ss = sel_stream_at(ws, s, 2);
+    a.dq_acc = dq_acc;
+    a.dk = static_cast<__nv_bfloat16*>(dk);
+    a.dv = static_cast<__nv_bfloat16*>(dv);
+    a.gsum = gsum;
+    a.tpc = kRows / s.G;
+    a.meta_bytes = a.tpc * (16 + 4 * a.ss.rvs);
+    // the streams carry each row's lse and D
+    cudaError_t e = launch_sel_stream(s, maskT, idx, gl, nsel, lse, Dd, 2, a.ss, st);
     if (e != cudaSuccess) return e;
-    BwdTcArgs a{s, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(dO), lse, Dd, idx, gl, nsel,
-                maskT, dq_acc, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv), gsum, kRows / s.G};
+    const size_t smem = BwdSmem::total(a.meta_bytes) + 1024;
+    e = cudaFuncSetAttribute(bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     const int64_t grid = (int64_t)s.B * s.Hkv * s.nT;
     {
         KernelTimer kt("bwd_tc", st);

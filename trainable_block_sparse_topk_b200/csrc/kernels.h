@@ -84,10 +84,12 @@ cudaError_t launch_fwd_simt_rows(const Shape& s, const void* q, const void* k, c
 bool encode_bf16_2d(::CUtensorMap_st* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows);
 
 // Tensor-core backward (tcgen05 + TMA + cp.async gathers): bf16, d = 128, block 64.
+// ws (bwd_tc_ws_bytes) holds the per-block token streams it builds first.
 bool bwd_tc_supported(const Shape& s);
+size_t bwd_tc_ws_bytes(const Shape& s);
 cudaError_t launch_bwd_tc(const Shape& s, const void* q, const void* k, const void* v, const void* dO,
                           const float* attn_lse, const float* Dd, const int32_t* idx, const float* gate_logit,
-                          const int32_t* n_sel, const uint64_t* maskT, float* dq_acc, void* dk, void* dv,
+                          const int32_t* n_sel, const uint64_t* maskT, void* ws, float* dq_acc, void* dk, void* dv,
                           float* gsum, cudaStream_t st);
 
 // Tensor-core forward over gathered rows (two passes + finalize): bf16, d = 128, block 64.

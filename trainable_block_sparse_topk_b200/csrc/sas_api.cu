@@ -147,7 +147,7 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // Training workspace layout (each piece 256-byte aligned).
 struct TrainWs {
-    size_t maskT, Dd, gsum, dq_acc, total;
+    size_t maskT, Dd, gsum, dq_acc, stream, total;
 };
 
 TrainWs bwd_layout(const Shape& s) {
@@ -158,6 +158,8 @@ TrainWs bwd_layout(const Shape& s) {
     w.gsum = off;  off += align256(sizeof(float) * (size_t)s.B * s.Hkv * s.T * s.K);
     w.dq_acc = off;
     if (s.dtype != SAS_DT_FP32) off += align256(sizeof(float) * (size_t)s.B * s.Hq * s.T * s.D);
+    w.stream = off;   // the tensor-core backward's per-block token streams
+    if (bwd_tc_supported(s)) off += align256(bwd_tc_ws_bytes(s));
     w.total = off;
     return w;
 }
@@ -291,7 +293,8 @@ sas_status sas_gated_attn_bwd(const sas_desc* desc, const void* q, const void* k
     if (e == cudaSuccess) e = launch_bwd_rowdot(s, o, dO, Dd, cs);
     if (e == cudaSuccess) {
         if (bwd_tc_supported(s) && !force_simt())
-            e = launch_bwd_tc(s, q, k, v, dO, attn_lse, Dd, idx, gate_logit, n_sel, maskT, dq_acc, dk, dv, gsum, cs);
+            e = launch_bwd_tc(s, q, k, v, dO, attn_lse, Dd, idx, gate_logit, n_sel, maskT, w + L.stream, dq_acc, dk,
+                              dv, gsum, cs);
         else
             e = launch_bwd_simt(s, q, k, v, dO, attn_lse, Dd, idx, gate_logit, n_sel, maskT, dq_acc, dk, dv, gsum,
                                 cs);
