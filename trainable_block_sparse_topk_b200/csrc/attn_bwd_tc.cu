@@ -331,15 +331,6 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             const int gs_slot = r < n ? meta.ent[r].z : -1;
             const int gs_tok = r < n ? meta.ent[r].x : 0;
             if (!tc::warp_wait_bar(&s_full[st], (uint32_t)((c >> 1) & 1), abort)) break;
-            // P and dS of chunk c-1 must have been consumed by its MMAs; that also
-            // means the epilogue warps are done with chunk c-2, whose row-id slot
-            // is reused here
-            if (c >= 1 && !tc::warp_wait_bar(p_empty, (uint32_t)((c - 1) & 1), abort)) break;
-            if (hf == 0) {
-                ids[st * kRows + r] = dq_row;
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(&ids_full[st]);
-            }
             tc::fence_after_sync();
             float rowsum = 0.f;
             {
@@ -363,6 +354,15 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                     __nv_bfloat162 hd = __floats2bfloat162_rn(d0, d1);
                     pk[k / 2] = *reinterpret_cast<uint32_t*>(&hp);
                     dk2[k / 2] = *reinterpret_cast<uint32_t*>(&hd);
+                }
+                // P and dS of chunk c-1 must have been consumed by its MMAs before
+                // they are overwritten; that also means the epilogue warps are done
+                // with chunk c-2, whose row-id slot is reused here
+                if (c >= 1 && !tc::warp_wait_bar(p_empty, (uint32_t)((c - 1) & 1), abort)) break;
+                if (hf == 0) {
+                    ids[st * kRows + r] = dq_row;
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(&ids_full[st]);
                 }
 #pragma unroll
                 for (int cb = 0; cb < 4; ++cb) {

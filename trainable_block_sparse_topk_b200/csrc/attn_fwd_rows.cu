@@ -387,28 +387,42 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 }
 
 // M = scale log2e q_t.k_t for each of the G query heads of a (b, kv head, t)
-// row, one warp per row (lane l holds dims 4l .. 4l+3).
+// row, one warp per row: half a warp reads a 256-byte row (16 bytes a lane),
+// both halves read k_t and heads 2u and 2u + 1 go to the two halves; the
+// loads of all heads are issued before any sum.
 __global__ void __launch_bounds__(256)
 fwd_rows_shift_kernel(Shape sh, const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                       float* __restrict__ shift) {
-    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);   // (b * Hkv + g) * T + t
-    const int lane = threadIdx.x & 31;
+    const int row = (int)(blockIdx.x * 8 + (threadIdx.x >> 5));   // (b * Hkv + g) * T + t
+    const int lane = threadIdx.x & 31, sub = lane >> 4, li = lane & 15;
     if (row >= sh.rows()) return;
-    const int64_t bg = row / sh.T;
-    const int t = (int)(row % sh.T);
-    const int b = (int)(bg / sh.Hkv), g = (int)(bg % sh.Hkv);
-    float kv[4];
-    load_vec<__nv_bfloat16, 4>(k + row * kD + lane * 4, kv);
+    const int bg = row / sh.T;
+    const int t = row - bg * sh.T;
+    const int b = bg / sh.Hkv, g = bg - b * sh.Hkv;
+    const uint4 kv = *reinterpret_cast<const uint4*>(k + (int64_t)row * kD + li * 8);
+    uint4 x[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {                      // G <= 8
+        const int h = 2 * u + sub;
+        x[u] = make_uint4(0u, 0u, 0u, 0u);
+        if (h < sh.G)
+            x[u] = *reinterpret_cast<const uint4*>(q + (((int64_t)b * sh.Hq + g * sh.G + h) * sh.T + t) * kD + li * 8);
+    }
+    float c[8];
+    load_vec<__nv_bfloat16, 8>(reinterpret_cast<const __nv_bfloat16*>(&kv), c);
     const float qk = sh.scale * kLog2e;
-    for (int h = 0; h < sh.G; ++h) {
-        const int64_t qrow = ((int64_t)b * sh.Hq + g * sh.G + h) * sh.T + t;
-        float qv[4];
-        load_vec<__nv_bfloat16, 4>(q + qrow * kD + lane * 4, qv);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        if (2 * u >= sh.G) break;                      // warp-uniform
+        float a[8];
+        load_vec<__nv_bfloat16, 8>(reinterpret_cast<const __nv_bfloat16*>(&x[u]), a);
         float d = 0.f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) d = fmaf(qv[e], kv[e], d);
-        d = warp_sum(d);
-        if (lane == 0) shift[qrow] = d * qk;
+        for (int e = 0; e < 8; ++e) d = fmaf(a[e], c[e], d);
+#pragma unroll
+        for (int m = 8; m > 0; m >>= 1) d += __shfl_xor_sync(0xffffffffu, d, m);
+        const int h = 2 * u + sub;
+        if (li == 0 && h < sh.G) shift[((int64_t)b * sh.Hq + g * sh.G + h) * sh.T + t] = d * qk;
     }
 }
 

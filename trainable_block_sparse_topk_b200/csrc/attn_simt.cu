@@ -176,21 +176,53 @@ __device__ __forceinline__ void fwd_simt_row(const Shape& sh, const T* __restric
 
 // ---------------------------------------------------------- D = rowsum(dO*O) ---
 
+// D = rowsum(o * dO) per query-head row. A row is read by D / V lanes with
+// 16-byte loads (V elements each), so one warp instruction covers 32 V / D
+// rows; each warp issues kU such instructions for both tensors before it
+// reduces any, keeping 32 16-byte loads per thread in flight.
+template <typename T>
+__device__ __forceinline__ float dot16(const uint4& x, const uint4& y) {
+    float ax[vec16<T>()], ay[vec16<T>()];
+    load_vec<T, vec16<T>()>(reinterpret_cast<const T*>(&x), ax);
+    load_vec<T, vec16<T>()>(reinterpret_cast<const T*>(&y), ay);
+    float s = 0.f;
+#pragma unroll
+    for (int e = 0; e < vec16<T>(); ++e) s = fmaf(ax[e], ay[e], s);
+    return s;
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
 rowdot_kernel(int64_t rows, const T* __restrict__ o, const T* __restrict__ dO, float* __restrict__ Dd) {
-    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    constexpr int V = vec16<T>();
+    constexpr int LPR = D / V;          // lanes per row
+    constexpr int RPI = 32 / LPR;       // rows per warp instruction
+    constexpr int kU = 4;
+    constexpr int RW = RPI * kU;        // rows per warp pass
     const int lane = threadIdx.x & 31;
-    if (row >= rows) return;
-    constexpr int DPL = D / 32;
-    float a[DPL], b[DPL];
-    load_vec<T, DPL>(o + row * D + lane * DPL, a);
-    load_vec<T, DPL>(dO + row * D + lane * DPL, b);
-    float s = 0.f;
+    const int sub = lane / LPR, li = lane % LPR;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t r0 = warp * RW; r0 < rows; r0 += nwarps * RW) {   // warp-uniform
+        uint4 x[kU], y[kU];
 #pragma unroll
-    for (int e = 0; e < DPL; ++e) s = fmaf(a[e], b[e], s);
-    s = warp_sum(s);
-    if (lane == 0) Dd[row] = s;
+        for (int u = 0; u < kU; ++u) {
+            const int64_t row = r0 + u * RPI + sub;
+            x[u] = y[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (row < rows) {
+                x[u] = *reinterpret_cast<const uint4*>(o + row * D + li * V);
+                y[u] = *reinterpret_cast<const uint4*>(dO + row * D + li * V);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            float sum = dot16<T>(x[u], y[u]);
+#pragma unroll
+            for (int m = LPR / 2; m > 0; m >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, m);
+            const int64_t row = r0 + u * RPI + sub;
+            if (li == 0 && row < rows) Dd[row] = sum;
+        }
+    }
 }
 
 // ----------------------------------------------------------------- backward ---
@@ -523,7 +555,8 @@ cudaError_t launch_fwd_simt_rows(const Shape& s, const void* q, const void* k, c
 
 cudaError_t launch_bwd_rowdot(const Shape& s, const void* o, const void* dO, float* Dd, cudaStream_t st) {
     const int64_t rows = (int64_t)s.B * s.Hq * s.T;
-    const unsigned grid = (unsigned)((rows + 7) / 8);
+    // 8 warps per CTA, at least 8 rows per warp pass; at most 16 CTAs per SM
+    const unsigned grid = (unsigned)std::min<int64_t>((rows + 63) / 64, 148 * 16);
     KernelTimer kt("rowdot", st);
     if (s.dtype == SAS_DT_FP32) {
         if (s.D == 64) rowdot_kernel<float, 64><<<grid, 256, 0, st>>>(rows, (const float*)o, (const float*)dO, Dd);

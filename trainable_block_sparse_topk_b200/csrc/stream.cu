@@ -29,6 +29,7 @@ namespace {
 
 constexpr int kBS = 64;
 constexpr int kThreads = 256;
+constexpr int kMaxRvs = 16;   // G <= 8 heads x 2 values
 
 __device__ __forceinline__ void put_rows(const Shape& sh, int b, int g, int t, const float* __restrict__ v0,
                                          const float* __restrict__ v1, int vals, float* out) {
@@ -90,8 +91,10 @@ sel_stream_index_kernel(Shape sh, const uint64_t* __restrict__ maskT, const floa
     }
 }
 
-// One warp per (b, g, t) row: its lanes load the row's per-head values once,
-// then each kept slot (one lane each) places its entry in an earlier block's run.
+// One warp per (b, g, t) row: its lanes load the row's per-head values once
+// and broadcast them to every lane, then each kept slot (one lane each) places
+// its entry and the row values (rvs <= 16 floats, 16-byte stores) in an
+// earlier block's run.
 __global__ void __launch_bounds__(kThreads)
 sel_stream_fill_kernel(Shape sh, const uint64_t* __restrict__ maskT, const int32_t* __restrict__ idx,
                        const float* __restrict__ gl, const int32_t* __restrict__ nsel, const float* __restrict__ v0,
@@ -110,6 +113,9 @@ sel_stream_fill_kernel(Shape sh, const uint64_t* __restrict__ maskT, const int32
         const int64_t qrow = ((int64_t)b * sh.Hq + g * sh.G + h) * sh.T + t;
         myv = v == 0 ? v0[qrow] : v1[qrow];
     }
+    float rowv[kMaxRvs];
+#pragma unroll
+    for (int v = 0; v < kMaxRvs; ++v) rowv[v] = __shfl_sync(0xffffffffu, myv, v);   // 0 past G * vals
     const int ns = nsel[row];
     const uint64_t below = (1ull << (t & (kBS - 1))) - 1ull;
     for (int s0 = 0; s0 < sh.K; s0 += 32) {
@@ -125,11 +131,12 @@ sel_stream_fill_kernel(Shape sh, const uint64_t* __restrict__ maskT, const int32
                 lg = gl[row * sh.K + slot];
             }
         }
-        if (pos >= 0) st.ent[pos] = make_int4(t, __float_as_int(lg), slot, 0);
-        float* out = st.rv + (pos >= 0 ? pos : 0) * st.rvs;
-        for (int v = 0; v < nv; ++v) {
-            const float x = __shfl_sync(0xffffffffu, myv, v);
-            if (pos >= 0) out[v] = x;
+        if (pos >= 0) {
+            st.ent[pos] = make_int4(t, __float_as_int(lg), slot, 0);
+            float4* out = reinterpret_cast<float4*>(st.rv + pos * st.rvs);
+#pragma unroll
+            for (int v = 0; v < kMaxRvs; v += 4)
+                if (v < st.rvs) out[v / 4] = make_float4(rowv[v], rowv[v + 1], rowv[v + 2], rowv[v + 3]);
         }
     }
 }
@@ -172,6 +179,7 @@ SelStream sel_stream_at(void* ws, const Shape& s, int vals) {
 cudaError_t launch_sel_stream(const Shape& s, const uint64_t* maskT, const int32_t* idx, const float* gl,
                               const int32_t* nsel, const float* v0, const float* v1, int vals, const SelStream& st,
                               cudaStream_t stream) {
+    if (st.rvs > kMaxRvs || st.rvs % 4 != 0) return cudaErrorInvalidValue;
     cudaError_t e = cudaMemsetAsync(st.counter, 0, sizeof(int), stream);
     if (e != cudaSuccess) return e;
     const int64_t grid = (int64_t)s.B * s.Hkv * s.NB;
