@@ -415,22 +415,56 @@ dscore_kernel(Shape sh, const float* __restrict__ scores, const float* __restric
     if (row >= sh.rows()) return;
     const int t = (int)(row % sh.T);
     const int C = (int)(((int64_t)sh.q_offset + t) / sh.bs);
-    const int n = nsel[row];
     const bool on = sh.gate == SAS_GATE_SOFTMAX;
+    const float* sr = scores + row * sh.NB;
+    float* dr = ds + row * sh.NB;
+    // every load of the row is issued before any is used: the kept list and its
+    // Gsum (masked by n afterwards), the normaliser and the first kPre chunks of
+    // 32 causal scores
+    constexpr int kPre = 8;
+    const int n = nsel[row];
+    const float lse = slse[row];
     int si[2];
     float sg[2];
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
         const int slot = lane + 32 * r;
-        si[r] = slot < n ? idx[row * sh.K + slot] : -1;
-        sg[r] = slot < n ? gsum[row * sh.K + slot] : 0.f;
+        si[r] = slot < sh.K ? idx[row * sh.K + slot] : -1;
+        sg[r] = slot < sh.K ? gsum[row * sh.K + slot] : 0.f;
     }
+    float sv[kPre];
+#pragma unroll
+    for (int q = 0; q < kPre; ++q) {
+        const int i = q * 32 + lane;
+        sv[q] = (on && i < C) ? sr[i] : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+        if (lane + 32 * r >= n) { si[r] = -1; sg[r] = 0.f; }
     const float tot = warp_sum(sg[0] + sg[1]);
-    const float lse = slse[row];
-    const float* sr = scores + row * sh.NB;
-    float* dr = ds + row * sh.NB;
     int base = 0;
-    for (int c0 = 0; c0 < sh.NB; c0 += 32) {
+#pragma unroll
+    for (int q = 0; q < kPre; ++q) {
+        const int c0 = q * 32;
+        if (c0 >= sh.NB) break;                        // warp-uniform
+        uint32_t bits = 0;
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+            if (si[r] >= c0 && si[r] < c0 + 32) bits |= 1u << (si[r] - c0);
+        const uint32_t mask = __reduce_or_sync(0xffffffffu, bits);
+        const int slot = base + __popc(mask & ((1u << lane) - 1u));
+        const float g0 = __shfl_sync(0xffffffffu, sg[0], slot & 31);
+        const float g1 = __shfl_sync(0xffffffffu, sg[1], slot & 31);
+        const int i = c0 + lane;
+        float val = 0.f;
+        if (on && i < C) {
+            val = -expf(sv[q] - lse) * tot;
+            if ((mask >> lane) & 1u) val += slot < 32 ? g0 : g1;
+        }
+        if (i < sh.NB) dr[i] = val;
+        base += __popc(mask);
+    }
+    for (int c0 = kPre * 32; c0 < sh.NB; c0 += 32) {   // long rows: the rest one chunk at a time
         uint32_t bits = 0;
 #pragma unroll
         for (int r = 0; r < 2; ++r)

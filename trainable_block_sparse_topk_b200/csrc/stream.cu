@@ -13,8 +13,8 @@
 // tokens from the column bitmap maskT[b,g,j,:], reserves a contiguous run of
 // entries with one atomic add (runs of different blocks land in any order;
 // each run's own order is fixed), stores the running token count at the start
-// of every later query tile and writes the block's own 64 tokens. Then one
-// warp per row places the row's kept (row, slot) entries: the position of token t in
+// of every later query tile and writes the block's own 64 tokens. Then a
+// group of lanes per row places the row's kept (row, slot) entries: the position of token t in
 // block j's run is the count before t's tile plus the set bits of the tile's
 // bitmap word below t -- no search. Entry e:
 //   ent[e] = {t, bits of log g_j(t), slot of j in t's ascending kept list, 0}
@@ -91,47 +91,48 @@ sel_stream_index_kernel(Shape sh, const uint64_t* __restrict__ maskT, const floa
     }
 }
 
-// One warp per (b, g, t) row: its lanes load the row's per-head values once
-// and broadcast them to every lane, then each kept slot (one lane each) places
-// its entry and the row values (rvs <= 16 floats, 16-byte stores) in an
-// earlier block's run.
+// kL lanes per (b, g, t) row (16 when K <= 16, two rows per warp, else 32):
+// they load the row's per-head values, kept blocks and log-gates together and
+// broadcast the values to the group, then each kept slot (one lane each)
+// places its entry and the row values (rvs <= 16 floats, 16-byte stores) in
+// an earlier block's run.
+template <int kL>
 __global__ void __launch_bounds__(kThreads)
 sel_stream_fill_kernel(Shape sh, const uint64_t* __restrict__ maskT, const int32_t* __restrict__ idx,
                        const float* __restrict__ gl, const int32_t* __restrict__ nsel, const float* __restrict__ v0,
                        const float* __restrict__ v1, int vals, SelStream st) {
-    const int64_t row = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (row >= sh.rows()) return;
-    const int t = (int)(row % sh.T);
+    const int sub = (threadIdx.x & 31) / kL, li = threadIdx.x & (kL - 1);
+    const int64_t row = ((int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5)) * (32 / kL) + sub;
+    const bool ok = row < sh.rows();               // no early exit: the groups shuffle
+    const int bg = ok ? (int)(row / sh.T) : 0;
+    const int t = ok ? (int)(row - (int64_t)bg * sh.T) : 0;
     const int tau = t / kBS;
-    const int64_t bg = row / sh.T;
-    const int b = (int)(bg / sh.Hkv), g = (int)(bg % sh.Hkv);
+    const int b = bg / sh.Hkv, g = bg - b * sh.Hkv;
     const int nv = sh.G * vals;                    // <= 16
     float myv = 0.f;
-    if (lane < nv) {
-        const int h = lane / vals, v = lane - h * vals;
+    if (ok && li < nv) {
+        const int h = li / vals, v = li - h * vals;
         const int64_t qrow = ((int64_t)b * sh.Hq + g * sh.G + h) * sh.T + t;
         myv = v == 0 ? v0[qrow] : v1[qrow];
     }
-    float rowv[kMaxRvs];
-#pragma unroll
-    for (int v = 0; v < kMaxRvs; ++v) rowv[v] = __shfl_sync(0xffffffffu, myv, v);   // 0 past G * vals
-    const int ns = nsel[row];
+    const int ns = ok ? nsel[row] : 0;
     const uint64_t below = (1ull << (t & (kBS - 1))) - 1ull;
-    for (int s0 = 0; s0 < sh.K; s0 += 32) {
-        const int slot = s0 + lane;
-        int64_t pos = -1;
+    for (int s0 = 0; s0 < sh.K; s0 += kL) {         // uniform across the warp
+        const int slot = s0 + li;
+        int j = -1;
         float lg = 0.f;
-        if (slot < sh.K && slot < ns) {
-            const int j = idx[row * sh.K + slot];
-            if (j >= 0 && j < tau) {                 // the own block is written by the index kernel
-                const int64_t blk = bg * sh.NB + j;
-                pos = (int64_t)st.base[blk] + st.pre[blk * sh.nT + tau] +
-                      __popcll(maskT[blk * sh.nT + tau] & below);
-                lg = gl[row * sh.K + slot];
-            }
+        if (ok && slot < sh.K) {
+            j = idx[row * sh.K + slot];
+            lg = gl[row * sh.K + slot];
         }
-        if (pos >= 0) {
+        float rowv[kMaxRvs];
+#pragma unroll
+        for (int v = 0; v < kMaxRvs; ++v) rowv[v] = __shfl_sync(0xffffffffu, myv, v, kL);   // 0 past G * vals
+        // the own block is written by the index kernel
+        if (slot < ns && j >= 0 && j < tau) {
+            const int64_t blk = (int64_t)bg * sh.NB + j;
+            const int64_t pos = (int64_t)st.base[blk] + st.pre[blk * sh.nT + tau] +
+                                __popcll(maskT[blk * sh.nT + tau] & below);
             st.ent[pos] = make_int4(t, __float_as_int(lg), slot, 0);
             float4* out = reinterpret_cast<float4*>(st.rv + pos * st.rvs);
 #pragma unroll
@@ -190,11 +191,17 @@ cudaError_t launch_sel_stream(const Shape& s, const uint64_t* maskT, const int32
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launches(1);
-    const int64_t rpb = kThreads / 32;
     {
         KernelTimer kt("sel_stream_fill", stream);
-        sel_stream_fill_kernel<<<(unsigned)((s.rows() + rpb - 1) / rpb), kThreads, 0, stream>>>(s, maskT, idx, gl, nsel,
-                                                                                                v0, v1, vals, st);
+        if (s.K <= 16) {
+            const int64_t rpb = 2 * (kThreads / 32);
+            sel_stream_fill_kernel<16><<<(unsigned)((s.rows() + rpb - 1) / rpb), kThreads, 0, stream>>>(
+                s, maskT, idx, gl, nsel, v0, v1, vals, st);
+        } else {
+            const int64_t rpb = kThreads / 32;
+            sel_stream_fill_kernel<32><<<(unsigned)((s.rows() + rpb - 1) / rpb), kThreads, 0, stream>>>(
+                s, maskT, idx, gl, nsel, v0, v1, vals, st);
+        }
     }
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
