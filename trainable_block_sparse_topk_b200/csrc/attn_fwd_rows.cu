@@ -430,7 +430,7 @@ fwd_rows_shift_kernel(Shape sh, const __nv_bfloat16* __restrict__ q, const __nv_
 // row; each warp takes kRowsU rows per pass and issues all their loads before
 // using any. Rows whose sum or output left the safe range are listed (as their
 // (b, kv head, t) row) for the exact recompute instead.
-constexpr int kRowsU = 8;
+constexpr int kRowsU = 4;
 
 __global__ void __launch_bounds__(256)
 fwd_rows_finalize_kernel(Shape sh, const float* __restrict__ shift, const float* __restrict__ l_acc,
