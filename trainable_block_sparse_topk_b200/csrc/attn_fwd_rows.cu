@@ -389,10 +389,12 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
 // M = scale log2e q_t.k_t for each of the G query heads of a (b, kv head, t)
 // row, one warp per row: half a warp reads a 256-byte row (16 bytes a lane),
 // both halves read k_t and heads 2u and 2u + 1 go to the two halves; the
-// loads of all heads are issued before any sum.
+// loads of all heads are issued before any sum. The warp also zeroes those
+// rows' l and fp32 output accumulator rows, which the gathered-row kernel
+// adds into.
 __global__ void __launch_bounds__(256)
 fwd_rows_shift_kernel(Shape sh, const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                      float* __restrict__ shift) {
+                      float* __restrict__ shift, float* __restrict__ l_acc, float* __restrict__ o_acc) {
     const int row = (int)(blockIdx.x * 8 + (threadIdx.x >> 5));   // (b * Hkv + g) * T + t
     const int lane = threadIdx.x & 31, sub = lane >> 4, li = lane & 15;
     if (row >= sh.rows()) return;
@@ -423,6 +425,11 @@ fwd_rows_shift_kernel(Shape sh, const __nv_bfloat16* __restrict__ q, const __nv_
         for (int m = 8; m > 0; m >>= 1) d += __shfl_xor_sync(0xffffffffu, d, m);
         const int h = 2 * u + sub;
         if (li == 0 && h < sh.G) shift[((int64_t)b * sh.Hq + g * sh.G + h) * sh.T + t] = d * qk;
+    }
+    for (int h = 0; h < sh.G; ++h) {
+        const int64_t qrow = ((int64_t)b * sh.Hq + g * sh.G + h) * sh.T + t;
+        reinterpret_cast<float4*>(o_acc + qrow * kD)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (lane == 0) l_acc[qrow] = 0.f;
     }
 }
 
@@ -483,14 +490,12 @@ struct RowsWs {
     float* l_acc;
     float* o_acc;
     int32_t* list_n;
-    size_t zero_bytes;   // l, O and the count are contiguous and start at zero
     RowsWs(void* ws, int64_t rows)
         : shift(static_cast<float*>(ws)),
           list(reinterpret_cast<int32_t*>(shift + rows)),
           l_acc(reinterpret_cast<float*>(list + rows)),
           o_acc(l_acc + rows),
-          list_n(reinterpret_cast<int32_t*>(o_acc + rows * kD)),
-          zero_bytes(4 * (size_t)rows + 4 * (size_t)rows * kD + 16) {}
+          list_n(reinterpret_cast<int32_t*>(o_acc + rows * kD)) {}
     static size_t head_bytes(int64_t rows) { return (12 * (size_t)rows + 4 * (size_t)rows * kD + 16 + 255) & ~(size_t)255; }
 };
 
@@ -521,12 +526,12 @@ cudaError_t launch_fwd_rows(const Shape& s, const void* q, const void* k, const 
     a.l_acc = w.l_acc;
     a.o_acc = w.o_acc;
     a.tpc = kRows / s.G;
-    cudaError_t e = cudaMemsetAsync(w.l_acc, 0, w.zero_bytes, st);
+    cudaError_t e = cudaMemsetAsync(w.list_n, 0, sizeof(int32_t), st);
     if (e != cudaSuccess) return e;
     {
         KernelTimer kt("fwd_rows_shift", st);
         fwd_rows_shift_kernel<<<(unsigned)((s.rows() + 7) / 8), 256, 0, st>>>(s, a.q, static_cast<const __nv_bfloat16*>(k),
-                                                                               w.shift);
+                                                                               w.shift, w.l_acc, w.o_acc);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -179,7 +179,9 @@ __device__ __forceinline__ void fwd_simt_row(const Shape& sh, const T* __restric
 // D = rowsum(o * dO) per query-head row. A row is read by D / V lanes with
 // 16-byte loads (V elements each), so one warp instruction covers 32 V / D
 // rows; each warp issues kU such instructions for both tensors before it
-// reduces any, keeping 32 16-byte loads per thread in flight.
+// reduces any, keeping 32 16-byte loads per thread in flight. The same lanes
+// zero the row of the fp32 dq accumulator (D floats) that the backward adds
+// into.
 template <typename T>
 __device__ __forceinline__ float dot16(const uint4& x, const uint4& y) {
     float ax[vec16<T>()], ay[vec16<T>()];
@@ -193,7 +195,8 @@ __device__ __forceinline__ float dot16(const uint4& x, const uint4& y) {
 
 template <typename T, int D>
 __global__ void __launch_bounds__(256)
-rowdot_kernel(int64_t rows, const T* __restrict__ o, const T* __restrict__ dO, float* __restrict__ Dd) {
+rowdot_kernel(int64_t rows, const T* __restrict__ o, const T* __restrict__ dO, float* __restrict__ Dd,
+              float* __restrict__ dq_acc) {
     constexpr int V = vec16<T>();
     constexpr int LPR = D / V;          // lanes per row
     constexpr int RPI = 32 / LPR;       // rows per warp instruction
@@ -221,6 +224,11 @@ rowdot_kernel(int64_t rows, const T* __restrict__ o, const T* __restrict__ dO, f
             for (int m = LPR / 2; m > 0; m >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, m);
             const int64_t row = r0 + u * RPI + sub;
             if (li == 0 && row < rows) Dd[row] = sum;
+            if (row < rows) {
+                float4* z = reinterpret_cast<float4*>(dq_acc + row * D + li * V);
+#pragma unroll
+                for (int e = 0; e < V / 4; ++e) z[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
         }
     }
 }
@@ -587,18 +595,23 @@ cudaError_t launch_fwd_simt_rows(const Shape& s, const void* q, const void* k, c
     return e;
 }
 
-cudaError_t launch_bwd_rowdot(const Shape& s, const void* o, const void* dO, float* Dd, cudaStream_t st) {
+cudaError_t launch_bwd_rowdot(const Shape& s, const void* o, const void* dO, float* Dd, float* dq_acc,
+                              cudaStream_t st) {
     const int64_t rows = (int64_t)s.B * s.Hq * s.T;
     // 8 warps per CTA, at least 8 rows per warp pass; at most 16 CTAs per SM
     const unsigned grid = (unsigned)std::min<int64_t>((rows + 63) / 64, 148 * 16);
     KernelTimer kt("rowdot", st);
     if (s.dtype == SAS_DT_FP32) {
-        if (s.D == 64) rowdot_kernel<float, 64><<<grid, 256, 0, st>>>(rows, (const float*)o, (const float*)dO, Dd);
-        else rowdot_kernel<float, 128><<<grid, 256, 0, st>>>(rows, (const float*)o, (const float*)dO, Dd);
+        if (s.D == 64) rowdot_kernel<float, 64><<<grid, 256, 0, st>>>(rows, (const float*)o, (const float*)dO, Dd,
+                                                                    dq_acc);
+        else rowdot_kernel<float, 128><<<grid, 256, 0, st>>>(rows, (const float*)o, (const float*)dO, Dd,
+                                                                    dq_acc);
     } else {
         using B16 = __nv_bfloat16;
-        if (s.D == 64) rowdot_kernel<B16, 64><<<grid, 256, 0, st>>>(rows, (const B16*)o, (const B16*)dO, Dd);
-        else rowdot_kernel<B16, 128><<<grid, 256, 0, st>>>(rows, (const B16*)o, (const B16*)dO, Dd);
+        if (s.D == 64) rowdot_kernel<B16, 64><<<grid, 256, 0, st>>>(rows, (const B16*)o, (const B16*)dO, Dd,
+                                                                    dq_acc);
+        else rowdot_kernel<B16, 128><<<grid, 256, 0, st>>>(rows, (const B16*)o, (const B16*)dO, Dd,
+                                                                    dq_acc);
     }
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);

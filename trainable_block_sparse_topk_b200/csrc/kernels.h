@@ -105,7 +105,9 @@ cudaError_t launch_fwd_tc(const Shape& s, const void* q, const void* k, const vo
                           const float* gate_logit, const int32_t* n_sel, void* o, float* attn_lse, cudaStream_t st);
 
 // Backward pieces.
-cudaError_t launch_bwd_rowdot(const Shape& s, const void* o, const void* dO, float* Dd, cudaStream_t st);
+// D = rowsum(o * dO) per query-head row; also zeroes the fp32 dq accumulator [rows, d].
+cudaError_t launch_bwd_rowdot(const Shape& s, const void* o, const void* dO, float* Dd, float* dq_acc,
+                              cudaStream_t st);
 cudaError_t launch_bwd_simt(const Shape& s, const void* q, const void* k, const void* v, const void* dO,
                             const float* attn_lse, const float* Dd, const int32_t* idx,
                             const float* gate_logit, const int32_t* n_sel, const uint64_t* maskT,

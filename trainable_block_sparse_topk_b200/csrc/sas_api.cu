@@ -288,9 +288,8 @@ sas_status sas_gated_attn_bwd(const sas_desc* desc, const void* q, const void* k
     float* gsum = reinterpret_cast<float*>(w + L.gsum);
     float* dq_acc = s.dtype == SAS_DT_FP32 ? static_cast<float*>(dq) : reinterpret_cast<float*>(w + L.dq_acc);
 
-    cudaError_t e = cudaMemsetAsync(dq_acc, 0, sizeof(float) * (size_t)s.B * s.Hq * s.T * s.D, cs);
-    if (e == cudaSuccess) e = launch_sel_bitmap_T(s, idx, n_sel, maskT, cs);
-    if (e == cudaSuccess) e = launch_bwd_rowdot(s, o, dO, Dd, cs);
+    cudaError_t e = launch_sel_bitmap_T(s, idx, n_sel, maskT, cs);
+    if (e == cudaSuccess) e = launch_bwd_rowdot(s, o, dO, Dd, dq_acc, cs);   // zeroes dq_acc too
     if (e == cudaSuccess) {
         if (bwd_tc_supported(s) && !force_simt())
             e = launch_bwd_tc(s, q, k, v, dO, attn_lse, Dd, idx, gate_logit, n_sel, maskT, w + L.stream, dq_acc, dk,

@@ -182,7 +182,7 @@ block_topk_kernel(Shape sh, const float* __restrict__ scores, int32_t* __restric
         // #{keys >= v} >= n, i.e. the n-th largest key. Invalid slots hold key
         // 0, which no candidate (>= 1) admits.
         uint32_t thr = 0;
-#pragma unroll 1
+#pragma unroll
         for (int bit = 31; bit >= 0; --bit) {
             const uint32_t cand = thr | (1u << bit);
             uint32_t c = 0;
