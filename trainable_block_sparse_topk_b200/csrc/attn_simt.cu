@@ -377,12 +377,6 @@ bwd_simt_kernel(Shape sh, const T* __restrict__ q, const T* __restrict__ k, cons
     }
 }
 
-template <typename T>
-__global__ void cast_kernel(int64_t n, const float* __restrict__ src, T* __restrict__ dst) {
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-        dst[i] = Elem<T>::from_f(src[i]);
-}
-
 // fp32 -> bf16, 8 values per thread and pass, two passes' loads in flight
 // (n8 = number of 8-value groups).
 __global__ void __launch_bounds__(256)
@@ -628,14 +622,13 @@ cudaError_t launch_bwd_simt(const Shape& s, const void* q, const void* k, const 
 }
 
 cudaError_t launch_cast_dq(const Shape& s, const float* dq_acc, void* dq, cudaStream_t st) {
-    const int64_t n = (int64_t)s.B * s.Hq * s.T * s.D;
-    const unsigned grid = (unsigned)std::min<int64_t>((n + 255) / 256, 148 * 16);
-    KernelTimer kt("cast_dq", st);
-    if (s.dtype == SAS_DT_FP32) {
-        cast_kernel<float><<<grid, 256, 0, st>>>(n, dq_acc, (float*)dq);
-    } else {   // n is a multiple of 8 (d is 64 or 128); both buffers are 16-byte aligned
-        const int64_t n8 = n / 8;
-        const unsigned g8 = (unsigned)std::min<int64_t>((n8 + 511) / 512, 148 * 8);
+    // bf16 only: fp32 accumulates dq in place. n is a multiple of 8 (d is 64 or
+    // 128); both buffers are 16-byte aligned.
+    if (s.dtype != SAS_DT_BF16) return cudaErrorInvalidValue;
+    const int64_t n8 = (int64_t)s.B * s.Hq * s.T * s.D / 8;
+    const unsigned g8 = (unsigned)std::min<int64_t>((n8 + 511) / 512, 148 * 8);
+    {
+        KernelTimer kt("cast_dq", st);
         cast_bf16x8_kernel<<<g8, 256, 0, st>>>(n8, reinterpret_cast<const float4*>(dq_acc), static_cast<uint4*>(dq));
     }
     const cudaError_t e = cudaGetLastError();

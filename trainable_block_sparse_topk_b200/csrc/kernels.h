@@ -112,6 +112,7 @@ cudaError_t launch_bwd_simt(const Shape& s, const void* q, const void* k, const 
                             const float* attn_lse, const float* Dd, const int32_t* idx,
                             const float* gate_logit, const int32_t* n_sel, const uint64_t* maskT,
                             float* dq_acc, void* dk, void* dv, float* gsum, cudaStream_t st);
+// fp32 dq accumulator -> bf16 dq (bf16 shapes only; fp32 accumulates in place).
 cudaError_t launch_cast_dq(const Shape& s, const float* dq_acc, void* dq, cudaStream_t st);
 cudaError_t launch_dscore(const Shape& s, const float* scores, const float* score_lse,
                           const int32_t* idx, const int32_t* n_sel, const float* gsum, float* dscores,
