@@ -62,6 +62,46 @@ def train_flops(w):
     return 4 * w.head_dim * per_head, 10 * w.head_dim * per_head, per_head
 
 
+def selection_stats(idx, n_sel, T, bs, G, tile=64, rows_per_chunk=128):
+    """Selection overlap and executed tensor work of one training selection.
+
+    idx [B, Hkv, T, K] (ascending kept blocks, padded), n_sel [B, Hkv, T] as
+    numpy arrays. Per (b, kv head, query tile of `tile` tokens): the number of
+    distinct kept blocks (the union a query-tile kernel would visit) and the
+    kept selections per visited block. Per (b, kv head, key block j): the
+    gathered-row kernels walk 64 own tokens plus every later token that kept
+    j, in chunks of 128 / G tokens, each chunk an M = 128 row MMA over the 64
+    keys of j; `executed_pairs` counts those row-key products (masked diagonal
+    keys and padding rows included), to set beside the kept pairs.
+    """
+    import numpy as np
+    B, Hkv, _, K = idx.shape
+    NB = (T + bs - 1) // bs
+    tpc = rows_per_chunk // G
+    slot = np.arange(K)
+    unions, visits, executed = [], [], 0
+    for b in range(B):
+        for g in range(Hkv):
+            ib = idx[b, g]
+            valid = slot[None, :] < n_sel[b, g][:, None]
+            t_of = np.broadcast_to(np.arange(T)[:, None], ib.shape)
+            hit = np.zeros((T // tile, NB), dtype=bool)
+            hit[t_of[valid] // tile, ib[valid]] = True
+            u = hit.sum(axis=1)
+            sels = np.bincount(t_of[valid] // tile, minlength=T // tile)
+            keep = u > 0
+            unions.append(u[keep])
+            visits.append(sels[keep] / u[keep])
+            count = bs + np.bincount(ib[valid], minlength=NB)[: T // bs]
+            executed += int(((count + tpc - 1) // tpc).sum()) * rows_per_chunk * bs
+    u = np.concatenate(unions) if unions else np.zeros(0)
+    v = np.concatenate(visits) if visits else np.zeros(0)
+    return {"tile_tokens": tile,
+            "union_blocks_per_tile": float(u.mean()) if u.size else 0.0,
+            "selections_per_visited_block": float(v.mean()) if v.size else 0.0,
+            "executed_pairs": executed}
+
+
 def decode_selected_bytes(w, K):
     N = w.seq
     C = (N - 1) // w.block_size
@@ -233,6 +273,9 @@ def run_ours(args, rank, world, local_rank):
     td = B.make_desc(batch=tw.batch, seq_len=tw.seq, n_q_heads=tw.n_q_heads, n_kv_heads=tw.n_kv_heads,
                      head_dim=tw.head_dim, block_size=tw.block_size, top_k=tw.top_k, dtype=tw.dtype)
     sel = api.block_topk(td, s)
+    torch.cuda.synchronize()
+    sel_stats = selection_stats(sel.idx.cpu().numpy(), sel.n_sel.cpu().numpy(), tw.seq, tw.block_size,
+                                tw.n_q_heads // tw.n_kv_heads)
     o = torch.empty_like(g["q"])
     lse = torch.empty(g["q"].shape[:-1], dtype=torch.float32, device=dev)
     dq, dk, dv = torch.empty_like(g["q"]), torch.empty_like(g["k"]), torch.empty_like(g["v"])
@@ -405,7 +448,13 @@ def run_ours(args, rank, world, local_rank):
                                f" + decode N{dw.seq} K{dw.top_k}",
                    "global_batch": tw.batch * world, "seq_len": tw.seq, "parallelism": f"replicas x{world}",
                    "l2": "flushed before every step (256 MiB memset outside the timed events)",
-                   "kept_fwd_bwd_tflop_per_step": flops / 1e12, "kept_pairs_per_head": per_head_pairs // (tw.batch * tw.n_q_heads)},
+                   "kept_fwd_bwd_tflop_per_step": flops / 1e12, "kept_pairs_per_head": per_head_pairs // (tw.batch * tw.n_q_heads),
+                   # tensor work the gathered-row kernels execute (masked diagonal keys and
+                   # chunk padding included) and the query-tile union they avoid
+                   "executed_fwd_bwd_tflop_per_step": 14 * tw.head_dim * sel_stats["executed_pairs"] / 1e12,
+                   "executed_over_kept": sel_stats["executed_pairs"] / per_head_pairs,
+                   "selection_overlap": {k: sel_stats[k] for k in ("tile_tokens", "union_blocks_per_tile",
+                                                                   "selections_per_visited_block")}},
         "parts_us": {p: mean[p] * 1e3 for p in parts},
         "kernels_us": kernels_us,
         "roofline": roof,
