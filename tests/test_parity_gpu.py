@@ -288,6 +288,38 @@ def decode_ws():
     torch.cuda.empty_cache()
 
 
+def decode_topk_check(w, s, K):
+    """sas_block_topk on the decode rows (T = 1, q_offset = N - 1) of every
+    (batch, KV head): indices and counts bit-exact, gate logits and the
+    normaliser within fp32 rounding of the oracle's brute-force sort."""
+    d = U.decode_desc(w, w.seq, top_k=K)
+    sel = api.block_topk(d, s.cuda())
+    out = {"idx": sel.idx.cpu(), "gl": sel.gate_logit.cpu(), "slse": sel.score_lse.cpu(),
+           "nsel": sel.n_sel.cpu()}
+    grp = {(b, g): [0] for b in range(w.batch) for g in range(w.n_kv_heads)}
+    wk = synth.Workload(w.name, "decode", w.batch, w.seq, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block_size,
+                        K, w.dtype, w.seed, w.qkv_std)
+    check_topk_rows(wk, s, out, grp, top_k=K, q_offset=w.seq - 1, T=1)
+    C = (w.seq - 1) // w.block_size
+    assert (out["nsel"] == min(K, C)).all()
+
+
+@pytest.mark.parametrize("K", [15, 31, 63])
+def test_decode_topk_bit_exact(decode_ws, K):
+    """The 131072-token decode workload's pooled-key scores at each budget."""
+    w, _, _, _, s = decode_ws
+    decode_topk_check(w, s, K)
+
+
+@pytest.mark.parametrize("batch", [1, 8])
+def test_long_decode_topk_bit_exact(batch):
+    """The 524288-token workload's boosted scores (8191 candidates per row),
+    every (batch, KV head) row, budget 2048 (K = 31)."""
+    w = synth.workload("long", batch=batch)
+    s = synth.decode_scores(w, synth.decode_q(w))
+    decode_topk_check(w, s, w.top_k)
+
+
 @pytest.mark.parametrize("K", [15, 31, 63])
 def test_decode_budgets(decode_ws, K):
     w, kc, vc, q, s = decode_ws
