@@ -203,3 +203,47 @@ def decode(desc: Desc, q, k_cache, v_cache, scores=None):
     if rc != 0:
         raise ValueError("oracle decode needs seq_len == 1")
     return o
+
+
+def gather_pages(pages, block_table, seq_len: int, block_size: int):
+    """Contiguous cache [Hkv, N, d] of one sequence from page pools
+    [P, Hkv, block, d]: block j of the sequence is page block_table[j]
+    (study note 3-7 inference path, step 3: blocks read from a paged cache)."""
+    nb = -(-seq_len // block_size)
+    blocks = [pages[int(block_table[j])] for j in range(nb)]        # each [Hkv, block, d]
+    return np.concatenate(blocks, axis=1)[:, :seq_len]
+
+
+def topk_varlen(desc: Desc, scores, seq_lens):
+    """Decode-row top-K (desc.seq_len == 1) with a cache length per sequence:
+    row (i, g) is the row of position seq_lens[i] - 1, with its own candidates.
+    scores [B, Hkv, 1, NB]. Returns (idx [B*Hkv, K], gate_logit, score_lse, n_sel)."""
+    s = _f32(scores)
+    out = []
+    for i, n in enumerate(seq_lens):
+        d = Desc(batch=1, seq_len=1, q_offset=int(n) - 1, n_q_heads=desc.group, n_kv_heads=1,
+                 head_dim=desc.head_dim, block_size=desc.block_size, top_k=desc.top_k, gate=desc.gate)
+        for g in range(desc.n_kv_heads):
+            row = s[i, g, 0, :d.n_blocks].reshape(1, 1, 1, -1)
+            out.append(topk(d, row))
+    return tuple(np.concatenate([o[k] for o in out]) for k in range(4))
+
+
+def decode_paged(desc: Desc, q, k_pages, v_pages, block_table, seq_lens, scores=None):
+    """Decode over paged K/V with a cache length per sequence: for each
+    sequence i, the pages of its blocks are gathered into a contiguous cache of
+    N_i = seq_lens[i] tokens and the plain decode runs at position N_i - 1 (its
+    own current block and candidates). k_pages/v_pages [P, Hkv, block, d],
+    block_table [B, max_blocks], scores [B, Hkv, 1, NB] or None (dense).
+    Returns o [B, Hq, d] f64."""
+    q = _f32(q)
+    o = np.empty((desc.batch, desc.n_q_heads, desc.head_dim), np.float64)
+    for i, n in enumerate(seq_lens):
+        n = int(n)
+        kc = gather_pages(k_pages, block_table[i], n, desc.block_size)[None]
+        vc = gather_pages(v_pages, block_table[i], n, desc.block_size)[None]
+        d = Desc(batch=1, seq_len=1, q_offset=n - 1, n_q_heads=desc.n_q_heads, n_kv_heads=desc.n_kv_heads,
+                 head_dim=desc.head_dim, block_size=desc.block_size, top_k=desc.top_k, gate=desc.gate)
+        sc = None if scores is None else _f32(scores)[i:i + 1, :, :, :d.n_blocks]
+        o[i] = decode(d, q[i:i + 1], kc, vc, sc)[0]
+    return o

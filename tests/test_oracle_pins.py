@@ -336,3 +336,47 @@ def test_decode_equals_training_row(oracle_mod):
     ro, _ = dense_causal_torch(P["q"], P["k"], P["v"], 1 / math.sqrt(P["d"]))
     np.testing.assert_allclose(dense, ro[:, :, T - 1].numpy(), atol=1e-12, rtol=0)
     assert NB == 6
+
+
+def test_paged_varlen_decode_pins(oracle_mod):
+    """Paged decode with a cache length per sequence: for every sequence the
+    oracle equals the last row of the naive [T, T] bias form (gated) and of
+    textbook causal attention (dense) over that sequence's own tokens, with
+    the pages placed in the pools through a shuffled block table; the
+    per-sequence top-K equals a stable sort of the row's own candidates."""
+    g = torch.Generator().manual_seed(23)
+    B, Hkv, Hq, d, bs, K = 3, 2, 4, 16, 8, 2
+    lens = [45, 17, 33]
+    NB = -(-max(lens) // bs)
+    k = torch.randn(B, Hkv, NB * bs, d, generator=g)
+    v = torch.randn(B, Hkv, NB * bs, d, generator=g)
+    q = torch.randn(B, Hq, d, generator=g)
+    s = torch.randn(B, Hkv, 1, NB, generator=g)
+    perm = torch.randperm(B * NB, generator=g)
+    k_pages = torch.zeros(B * NB, Hkv, bs, d)
+    v_pages = torch.zeros(B * NB, Hkv, bs, d)
+    table = np.zeros((B, NB), np.int32)
+    for i in range(B):
+        for j in range(NB):
+            pg = int(perm[i * NB + j])
+            table[i, j] = pg
+            k_pages[pg] = k[i, :, j * bs:(j + 1) * bs]
+            v_pages[pg] = v[i, :, j * bs:(j + 1) * bs]
+    desc = oracle_mod.Desc(batch=B, seq_len=1, q_offset=max(lens) - 1, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d,
+                           block_size=bs, top_k=K)
+    o = oracle_mod.decode_paged(desc, q.numpy(), k_pages.numpy(), v_pages.numpy(), table, lens, s.numpy())
+    od = oracle_mod.decode_paged(desc, q.numpy(), k_pages.numpy(), v_pages.numpy(), table, lens, None)
+    idx, _, _, nsel = oracle_mod.topk_varlen(desc, s.numpy(), lens)
+    for i, n in enumerate(lens):
+        C = (n - 1) // bs
+        for gg in range(Hkv):
+            assert stable_topk(s[i, gg, 0], C, K) == [int(x) for x in idx[i * Hkv + gg, :nsel[i * Hkv + gg]]]
+        # sequence i as a training problem of T = n rows whose last row is the decode query
+        Pi = dict(q=torch.randn(1, Hq, n, d, generator=g), k=k[i:i + 1, :, :n], v=v[i:i + 1, :, :n],
+                  s=torch.randn(1, Hkv, n, -(-n // bs), generator=g), B=1, T=n, Hq=Hq, Hkv=Hkv, d=d, bs=bs, K=K)
+        Pi["q"][0, :, n - 1] = q[i]
+        Pi["s"][0, :, n - 1] = s[i, :, 0, :-(-n // bs)]
+        ro, _ = bias_matrix_torch(Pi, Pi["s"])
+        np.testing.assert_allclose(o[i], ro[0, :, n - 1].numpy(), atol=1e-12, rtol=0)
+        rd, _ = dense_causal_torch(Pi["q"], Pi["k"], Pi["v"], 1 / math.sqrt(d))
+        np.testing.assert_allclose(od[i], rd[0, :, n - 1].numpy(), atol=1e-12, rtol=0)
