@@ -28,6 +28,10 @@ _LIB = os.path.join(_HERE, "libsas_oracle.so")
 
 GATE_SOFTMAX = 0
 GATE_NONE = 1
+GATE_SIGMOID = 2            # independent gates sigmoid(s_i)
+GATE_RAW = 3                # the raw score as the log-gate
+GATE_SOFTMAX_SELECTED = 4   # softmax over the kept blocks only
+GATE_STE = 5                # hard gate 1 on kept blocks, softmax-gate gradient (straight-through)
 
 
 def build(force: bool = False) -> str:

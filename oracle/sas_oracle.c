@@ -38,6 +38,20 @@
  * Gate mode 1 ("none") sets every log-gate to 0 and every score gradient to 0:
  * plain block-sparse attention ([note] §1-1, block-sparse eq.).
  *
+ * The other gate activations the pages compare ([paper] §4 design elements,
+ * "gate activation" and "ranking preservation"; [note] §3-3, §3-4), each with
+ * the current block left at g_0 = 1 and the same top-K selection:
+ *   2 sigmoid: independent gates g_i = sigmoid(s_i); log g_i = -log(1 + e^-s_i),
+ *     d log g_i / d s_i = 1 - sigmoid(s_i); unkept blocks get no gradient.
+ *   3 raw: the unnormalised score injected as the logit bias, log g_i = s_i,
+ *     d log g_i / d s_i = 1.
+ *   4 softmax over the kept blocks only: log g_i = s_i - log sum_{j in I} e^s_j,
+ *     d log g_i / d s_k = [i = k] - p_k for k in I (p the kept softmax), 0 else.
+ *   5 hard gate with a straight-through estimator: the forward uses g = 1 on
+ *     every kept block (log g = 0); the backward differentiates the soft
+ *     softmax gate g_i = e^(s_i - lse) as if it had been used, i.e.
+ *     dL/dg_i = dL/dlog g_i (at g = 1) and dg_i/ds_k = g_i ([i = k] - g_k).
+ *
  * All arithmetic is double precision. Inputs arrive as float32 (bf16 values are
  * exact in float32) and are widened on read.
  */
@@ -56,7 +70,7 @@ typedef struct {
     int32_t block_size;  /* bs */
     int32_t top_k;       /* K: historical blocks kept per row */
     double scale;        /* softmax scale on q.k; <= 0 means 1/sqrt(d) */
-    int32_t gate;        /* 0: softmax gate, 1: no gate */
+    int32_t gate;        /* 0 softmax, 1 none, 2 sigmoid, 3 raw, 4 softmax over the kept blocks, 5 hard (STE) */
 } sas_oracle_desc;
 
 static double eff_scale(const sas_oracle_desc* ds) {
@@ -85,6 +99,21 @@ static int cand_cmp(const void* a, const void* b) {
 static int int_cmp(const void* a, const void* b) {
     int32_t x = *(const int32_t*)a, y = *(const int32_t*)b;
     return (x > y) - (x < y);
+}
+
+/* log(1 / (1 + e^-x)), without overflow for large |x|. */
+static double log_sigmoid(double x) {
+    return x >= 0.0 ? -log1p(exp(-x)) : x - log1p(exp(x));
+}
+
+/* log sum_{j < n} e^{s[idx[j]]} (with max shift): the normaliser of the
+ * softmax over the kept blocks. */
+static double kept_lse(const float* s, const int32_t* idx, int32_t n) {
+    double m = -INFINITY, l = 0.0;
+    for (int32_t j = 0; j < n; ++j) if ((double)s[idx[j]] > m) m = (double)s[idx[j]];
+    if (m == -INFINITY) return -INFINITY;
+    for (int32_t j = 0; j < n; ++j) l += exp((double)s[idx[j]] - m);
+    return m + log(l);
 }
 
 /* One row of the selection. `s` points at the row's NB scores; C candidates.
@@ -116,8 +145,16 @@ static int32_t topk_row(const sas_oracle_desc* ds, const float* s, int64_t C,
     qsort(idx, (size_t)n, sizeof(int32_t), int_cmp);
 
     for (int32_t j = 0; j < K; ++j) logg[j] = 0.0;
-    if (ds->gate == 0)
+    if (ds->gate == 0) {
         for (int32_t j = 0; j < n; ++j) logg[j] = (double)s[idx[j]] - *lse;
+    } else if (ds->gate == 2) {
+        for (int32_t j = 0; j < n; ++j) logg[j] = log_sigmoid((double)s[idx[j]]);
+    } else if (ds->gate == 3) {
+        for (int32_t j = 0; j < n; ++j) logg[j] = (double)s[idx[j]];
+    } else if (ds->gate == 4 && n > 0) {
+        const double lk = kept_lse(s, idx, n);
+        for (int32_t j = 0; j < n; ++j) logg[j] = (double)s[idx[j]] - lk;
+    }
     return n;
 }
 
@@ -296,14 +333,31 @@ int sas_oracle_bwd(const sas_oracle_desc* ds, const float* q, const float* k,
                     for (int x = 0; x < bs; ++x) gs[jj] += dS[(int64_t)jj * bs + x];
                 for (int64_t j = (int64_t)n * bs; j < m; ++j) gsum_cur[i] += dS[j];
             }
-            /* score gradient through log g_i = s_i - lse over the C candidates */
+            /* score gradient: Gsum_i = dL/d(log g_i) through d log g_i / d s_k */
             double* dsr = dsc + i * NB;
             for (int64_t j = 0; j < NB; ++j) dsr[j] = 0.0;
             if (ds->gate == 0 && C > 0) {
+                /* log g_i = s_i - lse over the C candidates */
                 double tot = 0.0;
                 for (int32_t jj = 0; jj < n; ++jj) tot += gs[jj];
                 for (int64_t c = 0; c < C; ++c) dsr[c] = -exp((double)s[c] - lse) * tot;
                 for (int32_t jj = 0; jj < n; ++jj) dsr[idx[jj]] += gs[jj];
+            } else if (ds->gate == 2) {
+                for (int32_t jj = 0; jj < n; ++jj)
+                    dsr[idx[jj]] = gs[jj] * (1.0 - exp(log_sigmoid((double)s[idx[jj]])));
+            } else if (ds->gate == 3) {
+                for (int32_t jj = 0; jj < n; ++jj) dsr[idx[jj]] = gs[jj];
+            } else if (ds->gate == 4 && n > 0) {
+                const double lk = kept_lse(s, idx, n);
+                double tot = 0.0;
+                for (int32_t jj = 0; jj < n; ++jj) tot += gs[jj];
+                for (int32_t jj = 0; jj < n; ++jj) dsr[idx[jj]] = gs[jj] - exp((double)s[idx[jj]] - lk) * tot;
+            } else if (ds->gate == 5 && C > 0) {
+                /* dL/dg_i = Gsum_i (g = 1 in the forward), dg_i/ds_k = g_i([i = k] - g_k) */
+                double tot = 0.0;
+                for (int32_t jj = 0; jj < n; ++jj) tot += gs[jj] * exp((double)s[idx[jj]] - lse);
+                for (int64_t c = 0; c < C; ++c) dsr[c] = -tot * exp((double)s[c] - lse);
+                for (int32_t jj = 0; jj < n; ++jj) dsr[idx[jj]] += gs[jj] * exp((double)s[idx[jj]] - lse);
             }
         }
         free(idx); free(logg); free(tok); free(bias); free(P); free(dS); free(o);

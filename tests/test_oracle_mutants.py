@@ -27,6 +27,15 @@ MUTANTS = {
                                    "for (int64_t i = 1; i < C; ++i) l += exp"),
     "dv uses dS": ("dv[kv + tok[j] * d + x] += P[j] * (double)dOh[x];",
                    "dv[kv + tok[j] * d + x] += dS[j] * (double)dOh[x];"),
+    "sigmoid gate derivative uses g instead of 1 - g": (
+        "dsr[idx[jj]] = gs[jj] * (1.0 - exp(log_sigmoid((double)s[idx[jj]])));",
+        "dsr[idx[jj]] = gs[jj] * exp(log_sigmoid((double)s[idx[jj]]));"),
+    "kept-block softmax normalised over all candidates": (
+        "for (int32_t j = 0; j < n; ++j) logg[j] = (double)s[idx[j]] - lk;",
+        "for (int32_t j = 0; j < n; ++j) logg[j] = (double)s[idx[j]] - *lse;"),
+    "hard gate gradient without the gate factor": (
+        "for (int32_t jj = 0; jj < n; ++jj) dsr[idx[jj]] += gs[jj] * exp((double)s[idx[jj]] - lse);",
+        "for (int32_t jj = 0; jj < n; ++jj) dsr[idx[jj]] += gs[jj];"),
 }
 
 PIN_CALLS = [
@@ -35,6 +44,9 @@ PIN_CALLS = [
     lambda m: pins.test_golden_worked_example(m),
     lambda m: pins.test_golden_topk_ties(m),
     lambda m: pins.test_topk_bruteforce_lexsort(m),
+    lambda m: pins.test_gate_modes_forward_and_autograd(m, 2),
+    lambda m: pins.test_gate_modes_forward_and_autograd(m, 4),
+    lambda m: pins.test_gate_modes_forward_and_autograd(m, 5),
 ]
 
 

@@ -380,3 +380,91 @@ def test_paged_varlen_decode_pins(oracle_mod):
         np.testing.assert_allclose(o[i], ro[0, :, n - 1].numpy(), atol=1e-12, rtol=0)
         rd, _ = dense_causal_torch(Pi["q"], Pi["k"], Pi["v"], 1 / math.sqrt(d))
         np.testing.assert_allclose(od[i], rd[0, :, n - 1].numpy(), atol=1e-12, rtol=0)
+
+
+# ------------------------------------------------------------- gate modes ---
+
+def _logg_mode(mode, srow, C, sel, i):
+    """log g_i of kept block i under each gate activation the pages compare
+    (arXiv text, 4, design elements), written with torch ops on the row's
+    scores so that autograd differentiates it."""
+    if mode == 2:                                   # independent sigmoid gates
+        return torch.nn.functional.logsigmoid(srow[i].double())
+    if mode == 3:                                   # raw score as the logit bias
+        return srow[i].double()
+    if mode == 4:                                   # softmax over the kept blocks
+        return srow[i].double() - torch.logsumexp(srow[sel].double(), 0)
+    if mode == 5:                                   # hard gate, straight-through softmax gradient
+        g = torch.exp(srow[i].double() - torch.logsumexp(srow[:C].double(), 0))
+        return torch.log(g + (1.0 - g).detach())
+    raise ValueError(mode)
+
+
+def bias_matrix_mode(P, s, mode):
+    """The naive [T, T] bias form (as bias_matrix_torch) with the log-gate of
+    gate activation `mode`."""
+    B, T, Hq, Hkv, d, bs, K = (P[x] for x in ("B", "T", "Hq", "Hkv", "d", "bs", "K"))
+    G = Hq // Hkv
+    rows = []
+    for b in range(B):
+        per_g = []
+        for g in range(Hkv):
+            per_t = []
+            for t in range(T):
+                C = t // bs
+                sel = stable_topk(s[b, g, t].detach(), C, K)
+                row = torch.full((T,), float("-inf"), dtype=torch.float64)
+                for i in sel:
+                    logg = _logg_mode(mode, s[b, g, t], C, sel, i)
+                    row = torch.cat([row[: i * bs], logg.expand(bs), row[(i + 1) * bs:]])
+                cur = torch.zeros(t - C * bs + 1, dtype=torch.float64)
+                row = torch.cat([row[: C * bs], cur, row[t + 1:]])
+                per_t.append(row)
+            per_g.append(torch.stack(per_t))
+        rows.append(torch.stack(per_g))
+    bias = torch.stack(rows).repeat_interleave(G, 1)
+    kk = P["k"].double().repeat_interleave(G, 1)
+    vv = P["v"].double().repeat_interleave(G, 1)
+    logits = P["q"].double() @ kk.transpose(-1, -2) / math.sqrt(d) + bias
+    return torch.softmax(logits, -1) @ vv, torch.logsumexp(logits, -1)
+
+
+@pytest.mark.parametrize("mode", [2, 3, 4, 5])
+def test_gate_modes_forward_and_autograd(oracle_mod, mode):
+    """Each gate activation: the oracle's forward, log-gates and every gradient
+    (dq, dk, dv and the score gradient through the activation) equal the bias
+    form and its fp64 autograd."""
+    P = rand_problem(30 + mode, B=1, T=40, K=2, gate=mode)
+    desc = desc_of(oracle_mod, P)
+    o, lse = oracle_o_full(oracle_mod, desc, P)
+    ro, rl = bias_matrix_mode(P, P["s"], mode)
+    np.testing.assert_allclose(o, ro.detach().numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(lse, rl.detach().numpy(), atol=1e-12, rtol=0)
+    q = P["q"].double().requires_grad_()
+    k = P["k"].double().requires_grad_()
+    v = P["v"].double().requires_grad_()
+    s = P["s"].double().requires_grad_()
+    o2, _ = bias_matrix_mode(dict(P, q=q, k=k, v=v), s, mode)
+    (o2 * P["dO"].double()).sum().backward()
+    r = oracle_bwd_full(oracle_mod, desc, P)
+    np.testing.assert_allclose(r["dq"], q.grad.numpy(), atol=1e-11, rtol=0)
+    np.testing.assert_allclose(r["dk"], k.grad.numpy(), atol=1e-11, rtol=0)
+    np.testing.assert_allclose(r["dv"], v.grad.numpy(), atol=1e-11, rtol=0)
+    np.testing.assert_allclose(r["ds"], s.grad.numpy(), atol=1e-11, rtol=0)
+
+
+def test_gate_mode_closed_forms(oracle_mod):
+    """Log-gates of one row by hand: scores (0, 1, 2, 3), K = 2 keeps blocks 2
+    and 3; sigmoid gives log(1 / (1 + e^-s)), raw gives s, the kept-block
+    softmax gives s - log(e^2 + e^3), the hard gate gives 0."""
+    srow = np.array([[[[0.0, 1.0, 2.0, 3.0, 0.0]]]], np.float32)
+    for mode, exp in [(2, [-math.log1p(math.exp(-2.0)), -math.log1p(math.exp(-3.0))]),
+                      (3, [2.0, 3.0]),
+                      (4, [2.0 - math.log(math.exp(2) + math.exp(3)), 3.0 - math.log(math.exp(2) + math.exp(3))]),
+                      (5, [0.0, 0.0])]:
+        d = oracle_mod.Desc(batch=1, seq_len=1, q_offset=4 * 8, n_q_heads=1, n_kv_heads=1, head_dim=8,
+                            block_size=8, top_k=2, gate=mode)
+        idx, gl, lse, n = oracle_mod.topk(d, srow)
+        assert idx[0].tolist() == [2, 3] and n[0] == 2
+        np.testing.assert_allclose(gl[0], exp, atol=1e-12, rtol=0)
+        assert abs(lse[0] - math.log(1 + math.e + math.e ** 2 + math.e ** 3)) < 1e-12
