@@ -251,3 +251,21 @@ def decode_paged(desc: Desc, q, k_pages, v_pages, block_table, seq_lens, scores=
         sc = None if scores is None else _f32(scores)[i:i + 1, :, :, :d.n_blocks]
         o[i] = decode(d, q[i:i + 1], kc, vc, sc)[0]
     return o
+
+
+def pooled_scores(desc: Desc, q, kbar):
+    """Block scores of the decode rows from pooled keys, the fixed scorer that
+    stands in for the trained selector (study note 3-7 inference path, step 1:
+    score every cached block; 5-6: this scan dominates decode at long context):
+    s[b, g, 0, j] = qbar . kbar[b, g, j] for the C = floor(q_offset / block)
+    historical blocks, with qbar the mean of the group's G query heads; 0 for
+    j >= C. q [B, Hq, d], kbar [B, Hkv, >= C, d]. Returns [B, Hkv, 1, NB] f64."""
+    q, kb = _f32(q).astype(np.float64), _f32(kbar).astype(np.float64)
+    G, C = desc.group, desc.q_offset // desc.block_size
+    out = np.zeros((desc.batch, desc.n_kv_heads, 1, desc.n_blocks), np.float64)
+    for b in range(desc.batch):
+        for g in range(desc.n_kv_heads):
+            qbar = q[b, g * G:(g + 1) * G].sum(0) / G
+            for j in range(C):
+                out[b, g, 0, j] = float(np.dot(qbar, kb[b, g, j]))
+    return out

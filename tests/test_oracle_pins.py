@@ -468,3 +468,30 @@ def test_gate_mode_closed_forms(oracle_mod):
         assert idx[0].tolist() == [2, 3] and n[0] == 2
         np.testing.assert_allclose(gl[0], exp, atol=1e-12, rtol=0)
         assert abs(lse[0] - math.log(1 + math.e + math.e ** 2 + math.e ** 3)) < 1e-12
+
+
+def test_pooled_scores_pins(oracle_mod):
+    """The pooled-key block scores equal the seeded input recipe's own score
+    (torch float32: mean of each block's keys dotted with the mean of the
+    group's query heads) within float32 rounding, are 0 past the candidates,
+    and match a hand example."""
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    from trainable_block_sparse_topk_b200 import synth
+    w = synth.workload("decode", seq=64 * 9)
+    q = synth.decode_q(w)
+    ref = synth.decode_scores(w, q)                     # torch: kbar @ qbar per (b, g)
+    kbar = torch.stack([torch.stack([synth.decode_cache_slice(w, "k", b, g).reshape(-1, 64, w.head_dim).mean(1)
+                                     for g in range(w.n_kv_heads)]) for b in range(w.batch)])
+    d = oracle_mod.Desc(batch=w.batch, seq_len=1, q_offset=w.seq - 1, n_q_heads=w.n_q_heads,
+                        n_kv_heads=w.n_kv_heads, head_dim=w.head_dim, block_size=64, top_k=31)
+    s = oracle_mod.pooled_scores(d, q.numpy(), kbar.numpy())
+    C = (w.seq - 1) // 64
+    np.testing.assert_allclose(s[..., :C], ref[..., :C].numpy(), atol=2e-6, rtol=1e-5)
+    assert (s[..., C:] == 0).all()
+    # by hand: qbar = mean of (1, 0) and (3, 2) = (2, 1); blocks (1, 1), (0, -2)
+    d2 = oracle_mod.Desc(batch=1, seq_len=1, q_offset=2 * 4, n_q_heads=2, n_kv_heads=1, head_dim=2,
+                         block_size=4, top_k=1)
+    s2 = oracle_mod.pooled_scores(d2, np.array([[[1, 0], [3, 2]]], np.float32),
+                                  np.array([[[[1, 1], [0, -2]]]], np.float32))
+    np.testing.assert_array_equal(s2[0, 0, 0], [3.0, -2.0, 0.0])
