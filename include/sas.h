@@ -67,9 +67,30 @@ typedef enum {
 
 typedef enum { SAS_DT_BF16 = 0, SAS_DT_FP32 = 1 } sas_dtype;
 
-/* SOFTMAX: log g_i = s_i - log sum_{j<C} exp s_j (the method's normalised gate).
- * NONE: every log-gate is 0 and the score gradient is 0 (plain block-sparse). */
-typedef enum { SAS_GATE_SOFTMAX = 0, SAS_GATE_NONE = 1 } sas_gate;
+/* Gate activation: how the selector's scores become the log-gates added to
+ * the kept blocks' logits (the current block always keeps g_0 = 1), and the
+ * matching score gradient. SOFTMAX is the method's normalised gate; the others
+ * are the alternatives the method is compared against (arXiv text 4, design
+ * elements "gate activation" and "ranking preservation"; study note 3-3, 3-4).
+ *   SOFTMAX: log g_i = s_i - log sum_{j<C} exp s_j.
+ *   NONE: every log-gate is 0 and the score gradient is 0 (plain block-sparse).
+ *   SIGMOID: independent gates, log g_i = log sigmoid(s_i); kept blocks only
+ *     get a score gradient.
+ *   RAW: the unnormalised score as the logit bias, log g_i = s_i.
+ *   SOFTMAX_SELECTED: softmax over the kept blocks only,
+ *     log g_i = s_i - log sum_{j kept} exp s_j (undefined when every kept
+ *     score is -inf).
+ *   STE: hard gate, g = 1 on every kept block in the forward; the score
+ *     gradient is that of the SOFTMAX gate evaluated at g = 1
+ *     (straight-through): dL/ds_k = sum_{i kept} Gsum_i g_i ([i=k] - g_k). */
+typedef enum {
+    SAS_GATE_SOFTMAX = 0,
+    SAS_GATE_NONE = 1,
+    SAS_GATE_SIGMOID = 2,
+    SAS_GATE_RAW = 3,
+    SAS_GATE_SOFTMAX_SELECTED = 4,
+    SAS_GATE_STE = 5
+} sas_gate;
 
 typedef enum { SAS_OP_TOPK = 0, SAS_OP_FWD = 1, SAS_OP_BWD = 2, SAS_OP_DECODE = 3 } sas_op;
 
@@ -96,8 +117,8 @@ sas_status sas_workspace_size(int32_t op, const sas_desc* desc, size_t* bytes);
  * arXiv text 4, normalised gate).
  *   scores     [B, Hkv, T, NB] float32, in: block scores; row t reads [0, C).
  *   idx        [B, Hkv, T, K] int32, out: kept blocks ascending, -1 padded.
- *   gate_logit [B, Hkv, T, K] float32, out: log g of each kept block
- *              (s_i - score_lse under SOFTMAX, 0 under NONE), 0 in padding.
+ *   gate_logit [B, Hkv, T, K] float32, out: log g of each kept block under
+ *              desc.gate (s_i - score_lse under SOFTMAX), 0 in padding.
  *   score_lse  [B, Hkv, T] float32, out: log sum_{i<C} exp s_i (-inf if C = 0).
  *   n_sel      [B, Hkv, T] int32, out: min(K, C).
  * Any q_offset >= 0 is allowed (decode rows use T = 1, q_offset = N - 1). */
@@ -123,9 +144,10 @@ sas_status sas_gated_attn_fwd(const sas_desc* desc, const void* q, const void* k
  *   scores, score_lse, idx, gate_logit, n_sel: the top-K inputs/outputs, in.
  *   dq [B, Hq, T, d], dk and dv [B, Hkv, T, d] (dtype), out (overwritten).
  *   dscores [B, Hkv, T, NB] float32, out (overwritten): dL/ds; 0 for i >= C
- *   and everywhere under SAS_GATE_NONE. For i < C:
- *   dscores_i = [i kept] * Gsum_i - g_i * sum_{k kept} Gsum_k, where Gsum_i is
- *   the sum of dL/dlogit over the block's tokens and the group's G heads.
+ *   and everywhere under SAS_GATE_NONE. With Gsum_i the sum of dL/dlogit over
+ *   block i's tokens and the group's G heads, for i < C: under SOFTMAX
+ *   dscores_i = [i kept] * Gsum_i - g_i * sum_{k kept} Gsum_k; the other gate
+ *   activations apply their own derivative (see sas_gate).
  *   ws: at least sas_workspace_size(SAS_OP_BWD) bytes. */
 sas_status sas_gated_attn_bwd(const sas_desc* desc, const void* q, const void* k, const void* v,
                               const void* o, const void* dO, const float* attn_lse,
@@ -150,6 +172,65 @@ sas_status sas_sparse_decode(const sas_desc* desc, const void* q, const void* k_
                              const float* gate_logit, const int32_t* n_sel, void* o, void* ws,
                              size_t ws_bytes, void* stream);
 
+/* Paged KV cache with a cache length per sequence (study note 3-7 inference
+ * path, step 3: the kept blocks are read from the paged KV cache; 3-1 method
+ * table: paged-cache serving backend). A page holds one block (block_size
+ * tokens) of every KV head, so a kept block is one page per KV head.
+ *   q [B, Hq, d] (dtype), in.
+ *   k_pages, v_pages [num_pages, Hkv, b, d] (dtype), in: the page pools.
+ *   block_table [B, max_blocks] int32, in: page of block j of sequence i at
+ *   [i * max_blocks + j]; entries for blocks [0, ceil(N_i / b)) must be valid
+ *   pages (an entry outside [0, num_pages) makes that block be skipped).
+ *   max_blocks >= NB = ceil((q_offset + 1) / b).
+ *   seq_lens [B] int32, in: N_i, the cache length of sequence i with the new
+ *   token, in [1, q_offset + 1] (values outside are clamped); the current
+ *   block of sequence i is floor((N_i - 1) / b), causal.
+ *   desc: seq_len = 1, q_offset = max_i N_i - 1.
+ *   idx, gate_logit, n_sel: from sas_block_topk_varlen with the same desc and
+ *   seq_lens; idx == NULL selects dense decode over each sequence's [0, N_i).
+ *   o [B, Hq, d] (dtype), out.
+ *   ws: at least sas_workspace_size(SAS_OP_DECODE, desc) bytes.
+ * bf16, head_dim 128, block 64 only (SAS_ERR_UNSUPPORTED otherwise). */
+sas_status sas_sparse_decode_paged(const sas_desc* desc, const void* q, const void* k_pages,
+                                   const void* v_pages, int32_t num_pages, const int32_t* block_table,
+                                   int32_t max_blocks, const int32_t* seq_lens, const int32_t* idx,
+                                   const float* gate_logit, const int32_t* n_sel, void* o, void* ws,
+                                   size_t ws_bytes, void* stream);
+
+/* sas_block_topk for decode rows (seq_len = 1) of sequences of different
+ * lengths: row (i, g) has C_i = floor((N_i - 1) / b) candidates, N_i =
+ * seq_lens[i] (device int32 [B], clamped to [1, q_offset + 1]); desc.q_offset
+ * = max_i N_i - 1 sets NB. Outputs as sas_block_topk. */
+sas_status sas_block_topk_varlen(const sas_desc* desc, const float* scores, const int32_t* seq_lens,
+                                 int32_t* idx, float* gate_logit, float* score_lse, int32_t* n_sel,
+                                 void* stream);
+
+/* Block scores of the decode rows from pooled keys: the selector's scan over
+ * every cached block of the new token's KV group (study note 3-7 inference
+ * path, step 1; 5-6: at long context this scan, not the attention, dominates
+ * the decode step). The pages' selector is a trained network; this fixed
+ * scorer stands in for it:
+ *   scores[b, g, 0, j] = qbar . kbar[b, g, j] for j < C = floor(q_offset / b),
+ *   0 for C <= j < NB, with qbar the mean of the group's G query heads.
+ * desc: seq_len = 1, q_offset = N - 1 (as sas_sparse_decode); bf16, d 128.
+ *   q [B, Hq, d] bf16, in.
+ *   kbar [B, Hkv, kbar_stride_blocks, d] bf16, in: the mean key of each cached
+ *   block (kept by the caller beside the cache); kbar_stride_blocks >= C.
+ *   scores [B, Hkv, 1, NB] float32, out. */
+sas_status sas_block_scores_pooled(const sas_desc* desc, const void* q, const void* kbar,
+                                   int64_t kbar_stride_blocks, float* scores, void* stream);
+
+/* The serving step in one call: sas_block_scores_pooled, then sas_block_topk
+ * on those scores, then sas_sparse_decode with that selection, enqueued back
+ * to back on `stream`. Arguments as in those three calls; scores, idx,
+ * gate_logit, score_lse and n_sel are outputs the caller may inspect.
+ * ws: at least sas_workspace_size(SAS_OP_DECODE, desc) bytes. */
+sas_status sas_sparse_decode_pooled(const sas_desc* desc, const void* q, const void* k_cache,
+                                    const void* v_cache, int64_t cache_stride_tokens, const void* kbar,
+                                    int64_t kbar_stride_blocks, float* scores, int32_t* idx,
+                                    float* gate_logit, float* score_lse, int32_t* n_sel, void* o,
+                                    void* ws, size_t ws_bytes, void* stream);
+
 /* Sparse decode that allocates nothing (the paper has no counterpart: this is
  * an interface convenience, not part of the method).
  *
@@ -161,15 +242,18 @@ sas_status sas_sparse_decode(const sas_desc* desc, const void* q, const void* k_
  * device array of SAS_NOALLOC_SCRATCH_BYTES inside libsas, which every GPU
  * that loads the library holds until the process exits.
  *  - Returns SAS_ERR_WORKSPACE, launching nothing, when the shape needs more
- *    than SAS_NOALLOC_SCRATCH_BYTES of partials (4 * B * Hkv * splits * G *
- *    (d + 2) bytes; splits = K + 1 for sparse decode).
+ *    scratch than the array holds: exactly when sas_workspace_size(
+ *    SAS_OP_DECODE, desc) reports more than SAS_NOALLOC_SCRATCH_BYTES (so a
+ *    caller can test a shape in advance).
  *  - The first call on each device looks up the array's device address (a
- *    runtime call that allocates nothing); make that first call before any
- *    stream capture.
+ *    runtime call that allocates nothing) and keeps it for the life of the
+ *    process; make that first call before any stream capture, and do not use
+ *    the library across cudaDeviceReset (the kept address would be stale).
  *  - All calls share the one array and it keeps the last call's contents.
- *    Each call writes every partial it reads, so nothing needs clearing, but
- *    calls that overlap on the GPU (different streams, or different host
- *    threads on one device, with no ordering between them) race on it.
+ *    Each call writes every partial it reads and zeroes the per-group
+ *    counters it uses (with an asynchronous memset on `stream`), but calls
+ *    that overlap on the GPU (different streams, or different host threads
+ *    on one device, with no ordering between them) race on it.
  *  - No cudaMalloc, cudaFree or allocating library routine is called. */
 #define SAS_NOALLOC_SCRATCH_BYTES (8u << 20)
 sas_status sas_sparse_decode_noalloc(const sas_desc* desc, const void* q, const void* k_cache,
@@ -177,11 +261,21 @@ sas_status sas_sparse_decode_noalloc(const sas_desc* desc, const void* q, const 
                                      const int32_t* idx, const float* gate_logit,
                                      const int32_t* n_sel, void* o, void* stream);
 
-/* Diagnostics (no counterpart on the pages): number of device-side waits for
- * an asynchronous copy that gave up after their ~1 s bound since the library
- * was loaded; 0 in normal operation. A kernel whose wait gave up leaves NaN in
- * its output instead of hanging. Synchronises the current device. */
+/* Diagnostics (no counterpart on the pages): number of device-side waits
+ * that gave up at the wait limit (sas_set_wait_limit, default 1 s) since the
+ * library was loaded; 0 in normal operation. A kernel whose wait gave up
+ * leaves NaN in the call's outputs instead of hanging. Synchronises the
+ * current device. */
 sas_status sas_device_timeouts(uint32_t* count);
+
+/* Diagnostics (no counterpart on the pages): bound, in nanoseconds, on every
+ * device-side wait of a kernel for another agent's work (a copy, an MMA, the
+ * warps of another role); 0 restores the default of 1 s. A kernel whose wait
+ * gives up stops its work, lets the copies and MMAs it started finish, counts
+ * the event (sas_device_timeouts) and leaves NaN in the call's outputs
+ * instead of hanging. A tiny bound makes waits give up on purpose, to test
+ * that path. Process-wide; synchronises the current device. */
+sas_status sas_set_wait_limit(uint64_t ns);
 
 /* Diagnostics (no counterpart on the pages): number of CUDA kernels this
  * library has launched since it was loaded, counted on the host after each

@@ -71,9 +71,10 @@ def test_workspace_sizes(L):
     a = lambda p: (p + 255) // 256 * 256
     stream = lambda rvs: a(16 * cap) + a(4 * cap * rvs) + 2 * a(4 * 2 * NB) + a(4 * 2 * NB * nT) + 256
     # backward: column bitmap + D + Gsum + fp32 dq accumulator, then the
-    # streams with the lse and D of each of the G = 4 heads (rvs 8)
+    # streams with the lse and D of each of the G = 4 heads (rvs 8), then the
+    # 256-byte flag a CTA sets when it gives up on a wait
     parts = [8 * 1 * 2 * NB * nT, 4 * 8 * 256, 4 * 2 * 256 * 3, 4 * 8 * 256 * 128]
-    assert n == sum(a(p) for p in parts) + a(stream(8))
+    assert n == sum(a(p) for p in parts) + a(stream(8)) + 256
     # forward (tensor-core shapes): column bitmap, then per query-head row the
     # shift, flagged-row list, l and the fp32 output accumulator plus the
     # flagged-row count, then the streams with the shift of each head (rvs 4)
@@ -94,7 +95,7 @@ def test_workspace_sizes(L):
     (dict(batch=0), B.SAS_ERR_INVALID_ARG),
     (dict(top_k=0), B.SAS_ERR_INVALID_ARG),
     (dict(dtype=7), B.SAS_ERR_INVALID_ARG),
-    (dict(gate=3), B.SAS_ERR_INVALID_ARG),
+    (dict(gate=6), B.SAS_ERR_INVALID_ARG),
     (dict(softmax_scale=float("nan")), B.SAS_ERR_INVALID_ARG),
     (dict(head_dim=96), B.SAS_ERR_UNSUPPORTED),
     (dict(block_size=16), B.SAS_ERR_UNSUPPORTED),

@@ -27,6 +27,8 @@ GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 TOL_FP32 = 1e-4
 TOL_BF16_O = 1e-2
 TOL_BF16_GRAD = 2e-2
+ORACLE_GATE = {"softmax": oracle.GATE_SOFTMAX, "none": oracle.GATE_NONE, "sigmoid": oracle.GATE_SIGMOID,
+               "raw": oracle.GATE_RAW, "softmax_selected": oracle.GATE_SOFTMAX_SELECTED, "ste": oracle.GATE_STE}
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -267,7 +269,7 @@ def decode_check(w, kc, vc, q, s, N, K, groups, dense=False, gate="softmax"):
     for b, g in groups:
         od = oracle.Desc(batch=1, seq_len=1, q_offset=N - 1, n_q_heads=G, n_kv_heads=1, head_dim=w.head_dim,
                          block_size=w.block_size, top_k=K,
-                         gate=oracle.GATE_NONE if gate == "none" else oracle.GATE_SOFTMAX)
+                         gate=ORACLE_GATE[gate])
         kk = synth.decode_cache_slice(w, "k", b, g)[:N].numpy()[None, None]
         vv = synth.decode_cache_slice(w, "v", b, g)[:N].numpy()[None, None]
         ref = oracle.decode(od, q[b:b + 1, g * G:(g + 1) * G].numpy(), kk, vv,
@@ -375,14 +377,10 @@ def test_autograd_function_matches_abi():
     assert math.isfinite(float(o.sum()))
 
 
-@pytest.mark.parametrize("path", ["rows", "union", "simt"])
-def test_every_training_path_matches_oracle(path, monkeypatch):
-    """Each GPU implementation of the bf16 training path (gathered-row tensor
-    cores, query-tile tensor cores, CUDA cores) against the oracle, elementwise
-    on a mid-size problem with G = 5 (an odd head count pads the query-tile
-    kernel's last head pair)."""
-    monkeypatch.setenv("SAS_FORCE_SIMT", "1" if path == "simt" else "0")
-    monkeypatch.setenv("SAS_FWD_UNION", "1" if path == "union" else "0")
+def test_gqa_group_of_five_matches_oracle():
+    """The tensor-core training path (gathered-row forward and backward)
+    against the oracle, elementwise on a mid-size problem with G = 5 (128 rows
+    per chunk hold 25 tokens and 3 padding rows)."""
     w = synth.Workload("mid", "train", 2, 1024, 10, 2, 128, 64, 5, "bf16", 21, 0.5, score_noise=0.1)
     x, out = U.run_train(w)
     G = w.group
@@ -399,7 +397,7 @@ def test_every_training_path_matches_oracle(path, monkeypatch):
                    "dk": out["dk"][b:b + 1, g:g + 1].float().numpy(),
                    "dv": out["dv"][b:b + 1, g:g + 1].float().numpy(), "ds": out["ds"][b, g].numpy()}
             for key, val in got.items():
-                assert U.normwise(val, r[key]) <= TOL_BF16_GRAD, (path, key)
+                assert U.normwise(val, r[key]) <= TOL_BF16_GRAD, key
 
 
 def test_rows_beyond_the_softmax_shift_are_recomputed():
@@ -454,3 +452,130 @@ def test_kernel_timing_filter():
     B.sas_kernel_timing(None)
     assert B.sas_kernel_time("block_topk")[1] == 1
     assert B.sas_kernel_time("fwd_simt") == (0.0, 0)
+
+
+# -------------------------------------------------------------- gate modes ---
+
+GATE_MODES = {"sigmoid": oracle.GATE_SIGMOID, "raw": oracle.GATE_RAW,
+              "softmax_selected": oracle.GATE_SOFTMAX_SELECTED, "ste": oracle.GATE_STE}
+
+
+@pytest.mark.parametrize("gate", sorted(GATE_MODES))
+def test_gate_modes_fp32_elementwise(gate):
+    """Each gate activation on the tiny fp32 workload: top-K indices bit-exact,
+    log-gates within fp32 rounding, every output and gradient within 1e-4."""
+    w = synth.workload("tiny")
+    x, out = U.run_train(w, gate=gate)
+    d = U.group_desc(w, gate=GATE_MODES[gate])
+    a = U.group_arrays(x, w, 0, 0)
+    idx, gl, _, nsel = oracle.topk(d, a["s"])
+    np.testing.assert_array_equal(out["idx"][0, 0].numpy(), idx)
+    for r in range(w.seq):
+        np.testing.assert_allclose(out["gl"][0, 0, r, :nsel[r]].numpy(), gl[r, :nsel[r]], atol=2e-5, rtol=1e-6)
+    o, lse = oracle.fwd(d, a["q"], a["k"], a["v"], a["s"])
+    np.testing.assert_allclose(out["o"][0].numpy().transpose(1, 0, 2), o, atol=TOL_FP32, rtol=0)
+    r = oracle.bwd(d, a["q"], a["k"], a["v"], a["s"], a["dO"])
+    np.testing.assert_allclose(out["dq"][0].numpy().transpose(1, 0, 2), r["dq"], atol=TOL_FP32, rtol=0)
+    np.testing.assert_allclose(out["dk"].numpy(), r["dk"], atol=TOL_FP32, rtol=0)
+    np.testing.assert_allclose(out["dv"].numpy(), r["dv"], atol=TOL_FP32, rtol=0)
+    np.testing.assert_allclose(out["ds"][0, 0].numpy(), r["ds"], atol=TOL_FP32, rtol=0)
+
+
+@pytest.mark.parametrize("gate", sorted(GATE_MODES))
+def test_gate_modes_bf16_tensor_cores(gate):
+    """Each gate activation through the tensor-core path (bf16, d 128, block
+    64, G = 5): outputs within 1e-2, gradients and the score gradient within
+    2e-2 normwise of the oracle."""
+    w = synth.Workload("mid", "train", 1, 1024, 10, 2, 128, 64, 5, "bf16", 21, 0.5, score_noise=0.1)
+    x, out = U.run_train(w, gate=gate)
+    G = w.group
+    for g in range(w.n_kv_heads):
+        d = U.group_desc(w, gate=GATE_MODES[gate])
+        a = U.group_arrays(x, w, 0, g)
+        o, _ = oracle.fwd(d, a["q"], a["k"], a["v"], a["s"])
+        assert np.abs(out["o"][0, g * G:(g + 1) * G].float().numpy().transpose(1, 0, 2) - o).max() <= TOL_BF16_O
+        r = oracle.bwd(d, a["q"], a["k"], a["v"], a["s"], a["dO"])
+        got = {"dq": out["dq"][0, g * G:(g + 1) * G].float().numpy().transpose(1, 0, 2),
+               "dk": out["dk"][:, g:g + 1].float().numpy(), "dv": out["dv"][:, g:g + 1].float().numpy(),
+               "ds": out["ds"][0, g].numpy()}
+        for key, val in got.items():
+            assert U.normwise(val, r[key]) <= TOL_BF16_GRAD, (gate, key)
+
+
+@pytest.mark.parametrize("gate", sorted(GATE_MODES))
+def test_gate_modes_decode(gate, decode_ws):
+    """Each gate activation in the tensor-core decode (131072-token cache, K31)."""
+    w, kc, vc, q, s = decode_ws
+    decode_check(w, kc, vc, q, s, w.seq, 31, [(0, g) for g in (0, 4, 7)], gate=gate)
+
+
+# --------------------------------------------- pooled-key scores (serving) ---
+
+def test_pooled_scores_topk_decode(decode_ws):
+    """sas_sparse_decode_pooled on the 131072-token cache: the block scores
+    within float32 rounding of the oracle's fp64 pooled scores; the top-K of
+    those very scores bit-exact; the output within 1e-2 of the oracle's decode
+    with that selection."""
+    w, kc, vc, q, _ = decode_ws
+    kbar = kc.float().view(w.batch, w.n_kv_heads, -1, w.block_size, w.head_dim).mean(3).to(torch.bfloat16)
+    d = U.decode_desc(w, w.seq, top_k=31)
+    o, sc, sel = api.sparse_decode_pooled(d, q.to(torch.bfloat16).cuda(), kc, vc, kbar)
+    torch.cuda.synchronize()
+    od = oracle.Desc(batch=w.batch, seq_len=1, q_offset=w.seq - 1, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
+                     head_dim=w.head_dim, block_size=w.block_size, top_k=31)
+    ref_s = oracle.pooled_scores(od, q.numpy(), kbar.float().cpu().numpy())
+    got_s = sc.cpu().numpy()
+    np.testing.assert_allclose(got_s, ref_s, atol=2e-5, rtol=1e-5)
+    idx, _, _, _ = oracle.topk(od, got_s)
+    np.testing.assert_array_equal(sel.idx.cpu().numpy().reshape(idx.shape), idx)
+    G = w.group
+    got = o.float().cpu().numpy()
+    for g in (0, 3, 7):
+        og = oracle.Desc(batch=1, seq_len=1, q_offset=w.seq - 1, n_q_heads=G, n_kv_heads=1, head_dim=w.head_dim,
+                         block_size=w.block_size, top_k=31)
+        kk = synth.decode_cache_slice(w, "k", 0, g).numpy()[None, None]
+        vv = synth.decode_cache_slice(w, "v", 0, g).numpy()[None, None]
+        ref = oracle.decode(og, q[0:1, g * G:(g + 1) * G].numpy(), kk, vv, got_s[0:1, g:g + 1])
+        assert np.abs(got[0, g * G:(g + 1) * G] - ref[0]).max() <= TOL_BF16_O
+
+
+# ------------------------------------------------- sharding by (batch, KV head) ---
+
+def test_kv_head_and_batch_shards_reproduce_the_full_call():
+    """The path has no exchange step: every (batch, KV head) group is
+    independent. Running it on each half of the KV heads (training) and on
+    each half of the batch (decode) -- as the ranks of a multi-GPU run would --
+    and concatenating gives the full call's results: top-K bit-exact, the rest
+    within the bf16 tolerances (the order of floating-point additions differs)."""
+    w = synth.Workload("mid", "train", 2, 1024, 10, 2, 128, 64, 5, "bf16", 21, 0.5, score_noise=0.1)
+    x = synth.train_inputs(w)
+    _, full = U.run_train(w, inputs=x)
+    G = w.group
+    for g in range(w.n_kv_heads):
+        part = {"q": x["q"][:, g * G:(g + 1) * G].contiguous(), "k": x["k"][:, g:g + 1].contiguous(),
+                "v": x["v"][:, g:g + 1].contiguous(), "dO": x["dO"][:, g * G:(g + 1) * G].contiguous(),
+                "scores": x["scores"][:, g:g + 1].contiguous()}
+        wg = synth.Workload("mid_shard", "train", w.batch, w.seq, G, 1, w.head_dim, w.block_size, w.top_k,
+                            w.dtype, w.seed, w.qkv_std)
+        _, sh = U.run_train(wg, inputs=part)
+        assert torch.equal(sh["idx"], full["idx"][:, g:g + 1])
+        assert (sh["o"].float() - full["o"][:, g * G:(g + 1) * G].float()).abs().max() <= TOL_BF16_O
+        for key, sl in (("dq", np.s_[:, g * G:(g + 1) * G]), ("dk", np.s_[:, g:g + 1]), ("dv", np.s_[:, g:g + 1]),
+                        ("ds", np.s_[:, g:g + 1])):
+            assert U.normwise(sh[key].float().numpy(), full[key][sl].float().numpy()) <= TOL_BF16_GRAD, key
+    # decode: each half of the batch against the full batch
+    N, K = 8191, 31
+    gen = torch.Generator().manual_seed(5)
+    kc = (0.5 * torch.randn(4, 2, N, 128, generator=gen)).to(torch.bfloat16).cuda()
+    vc = (0.5 * torch.randn(4, 2, N, 128, generator=gen)).to(torch.bfloat16).cuda()
+    q = (0.5 * torch.randn(4, 8, 128, generator=gen)).to(torch.bfloat16).cuda()
+    s = torch.randn(4, 2, 1, -(-N // 64), generator=gen).cuda()
+    mk = lambda bsz: B.make_desc(batch=bsz, seq_len=1, q_offset=N - 1, n_q_heads=8, n_kv_heads=2, head_dim=128,
+                                 block_size=64, top_k=K)
+    of = api.sparse_decode(mk(4), q, kc, vc, api.block_topk(mk(4), s))
+    for h in (0, 1):
+        sl = slice(2 * h, 2 * h + 2)
+        d2 = mk(2)
+        oh = api.sparse_decode(d2, q[sl].contiguous(), kc[sl].contiguous(), vc[sl].contiguous(),
+                               api.block_topk(d2, s[sl].contiguous()))
+        assert (oh.float() - of[sl].float()).abs().max() <= 2e-3

@@ -77,6 +77,50 @@ def sparse_decode(desc, q, k_cache, v_cache, sel: Selection | None, ws=None, str
     return o
 
 
+def block_topk_varlen(desc, scores: torch.Tensor, seq_lens: torch.Tensor, stream=None) -> Selection:
+    """Decode-row top-K with a cache length per sequence (seq_lens int32 [B])."""
+    Bn, H, K = desc.batch, desc.n_kv_heads, desc.top_k
+    dev = scores.device
+    out = Selection(torch.empty(Bn, H, 1, K, dtype=torch.int32, device=dev),
+                    torch.empty(Bn, H, 1, K, dtype=torch.float32, device=dev),
+                    torch.empty(Bn, H, 1, dtype=torch.float32, device=dev),
+                    torch.empty(Bn, H, 1, dtype=torch.int32, device=dev))
+    B.sas_block_topk_varlen(desc, scores, seq_lens, out.idx, out.gate_logit, out.score_lse, out.n_sel, stream)
+    return out
+
+
+def sparse_decode_paged(desc, q, k_pages, v_pages, block_table, seq_lens, sel: Selection | None, ws=None,
+                        stream=None):
+    """Decode over page pools [num_pages, Hkv, block, d]; sel=None: dense."""
+    o = torch.empty_like(q)
+    if ws is None:
+        ws = workspace(B.SAS_OP_DECODE, desc, q.device)
+    if sel is None:
+        B.sas_sparse_decode_paged(desc, q, k_pages, v_pages, block_table, seq_lens, None, None, None, o, ws, stream)
+    else:
+        B.sas_sparse_decode_paged(desc, q, k_pages, v_pages, block_table, seq_lens, sel.idx, sel.gate_logit,
+                                  sel.n_sel, o, ws, stream)
+    return o
+
+
+def sparse_decode_pooled(desc, q, k_cache, v_cache, kbar, ws=None, stream=None):
+    """Pooled-key block scores, top-K and sparse decode in one call; returns
+    (o, scores, Selection)."""
+    Bn, H, K = desc.batch, desc.n_kv_heads, desc.top_k
+    dev = q.device
+    scores = torch.empty(Bn, H, 1, desc.n_blocks, dtype=torch.float32, device=dev)
+    sel = Selection(torch.empty(Bn, H, 1, K, dtype=torch.int32, device=dev),
+                    torch.empty(Bn, H, 1, K, dtype=torch.float32, device=dev),
+                    torch.empty(Bn, H, 1, dtype=torch.float32, device=dev),
+                    torch.empty(Bn, H, 1, dtype=torch.int32, device=dev))
+    o = torch.empty_like(q)
+    if ws is None:
+        ws = workspace(B.SAS_OP_DECODE, desc, dev)
+    B.sas_sparse_decode_pooled(desc, q, k_cache, v_cache, k_cache.shape[2], kbar, scores, sel.idx, sel.gate_logit,
+                               sel.score_lse, sel.n_sel, o, ws, stream)
+    return o, scores, sel
+
+
 class SASAttention(torch.autograd.Function):
     """o = SAS gated block-sparse attention(q, k, v; scores). Differentiable in
     q, k, v and scores (the score gradient flows through the softmax gate)."""

@@ -17,7 +17,9 @@ from .build import LIB
 
 SAS_OK, SAS_ERR_INVALID_ARG, SAS_ERR_UNSUPPORTED, SAS_ERR_MISALIGNED, SAS_ERR_WORKSPACE, SAS_ERR_CUDA = range(6)
 SAS_DT_BF16, SAS_DT_FP32 = 0, 1
-SAS_GATE_SOFTMAX, SAS_GATE_NONE = 0, 1
+SAS_GATE_SOFTMAX, SAS_GATE_NONE, SAS_GATE_SIGMOID, SAS_GATE_RAW, SAS_GATE_SOFTMAX_SELECTED, SAS_GATE_STE = range(6)
+GATES = {"softmax": SAS_GATE_SOFTMAX, "none": SAS_GATE_NONE, "sigmoid": SAS_GATE_SIGMOID, "raw": SAS_GATE_RAW,
+         "softmax_selected": SAS_GATE_SOFTMAX_SELECTED, "ste": SAS_GATE_STE}
 SAS_OP_TOPK, SAS_OP_FWD, SAS_OP_BWD, SAS_OP_DECODE = range(4)
 
 
@@ -49,7 +51,7 @@ class sas_desc(ctypes.Structure):
 def make_desc(batch, seq_len, n_q_heads, n_kv_heads, head_dim, block_size, top_k, q_offset=0,
               softmax_scale=0.0, dtype="bf16", gate="softmax") -> sas_desc:
     dt = {"bf16": SAS_DT_BF16, "fp32": SAS_DT_FP32}[dtype] if isinstance(dtype, str) else int(dtype)
-    gt = {"softmax": SAS_GATE_SOFTMAX, "none": SAS_GATE_NONE}[gate] if isinstance(gate, str) else int(gate)
+    gt = GATES[gate] if isinstance(gate, str) else int(gate)
     return sas_desc(batch, seq_len, q_offset, n_q_heads, n_kv_heads, head_dim, block_size, top_k,
                     softmax_scale, dt, gt)
 
@@ -72,16 +74,25 @@ def lib() -> ctypes.CDLL:
         L.sas_gated_attn_bwd.argtypes = [D, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.sas_sparse_decode.argtypes = [D, P, P, P, ctypes.c_int64, P, P, P, P, P, ctypes.c_size_t, P]
         L.sas_sparse_decode_noalloc.argtypes = [D, P, P, P, ctypes.c_int64, P, P, P, P, P]
+        L.sas_sparse_decode_paged.argtypes = [D, P, P, P, ctypes.c_int32, P, ctypes.c_int32, P, P, P, P, P, P,
+                                              ctypes.c_size_t, P]
+        L.sas_block_topk_varlen.argtypes = [D, P, P, P, P, P, P, P]
+        L.sas_block_scores_pooled.argtypes = [D, P, P, ctypes.c_int64, P, P]
+        L.sas_sparse_decode_pooled.argtypes = [D, P, P, P, ctypes.c_int64, P, ctypes.c_int64, P, P, P, P, P, P, P,
+                                               ctypes.c_size_t, P]
         L.sas_status_string.argtypes = [ctypes.c_int]
         L.sas_status_string.restype = ctypes.c_char_p
         L.sas_device_timeouts.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
         L.sas_kernel_launches.argtypes = []
         L.sas_kernel_launches.restype = ctypes.c_uint64
+        L.sas_set_wait_limit.argtypes = [ctypes.c_uint64]
         L.sas_kernel_timing.argtypes = [ctypes.c_char_p]
         L.sas_kernel_time.argtypes = [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint32)]
         for f in ("sas_workspace_size", "sas_block_topk", "sas_gated_attn_fwd", "sas_gated_attn_bwd",
-                  "sas_sparse_decode", "sas_sparse_decode_noalloc", "sas_device_timeouts", "sas_kernel_timing",
-                  "sas_kernel_time"):
+                  "sas_sparse_decode", "sas_sparse_decode_noalloc", "sas_sparse_decode_paged",
+                  "sas_block_topk_varlen", "sas_block_scores_pooled", "sas_sparse_decode_pooled",
+                  "sas_device_timeouts", "sas_set_wait_limit",
+                  "sas_kernel_timing", "sas_kernel_time"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -158,6 +169,46 @@ def sas_sparse_decode(desc, q, k_cache, v_cache, cache_stride_tokens, idx, gate_
         _dev(n_sel, "n_sel", i32), _dev(o, "o", dt), _dev(ws, "ws"), nbytes, _stream(stream)))
 
 
+def sas_block_topk_varlen(desc, scores, seq_lens, idx, gate_logit, score_lse, n_sel, stream=None) -> None:
+    f32, i32 = torch.float32, torch.int32
+    _check("sas_block_topk_varlen", lib().sas_block_topk_varlen(
+        ctypes.byref(desc), _dev(scores, "scores", f32), _dev(seq_lens, "seq_lens", i32), _dev(idx, "idx", i32),
+        _dev(gate_logit, "gate_logit", f32), _dev(score_lse, "score_lse", f32), _dev(n_sel, "n_sel", i32),
+        _stream(stream)))
+
+
+def sas_sparse_decode_paged(desc, q, k_pages, v_pages, block_table, seq_lens, idx, gate_logit, n_sel, o, ws,
+                            stream=None) -> None:
+    """Decode over page pools [num_pages, Hkv, block, d] through block_table
+    [B, max_blocks] (int32) with per-sequence lengths seq_lens [B] (int32)."""
+    dt, f32, i32 = desc.torch_dtype, torch.float32, torch.int32
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("sas_sparse_decode_paged", lib().sas_sparse_decode_paged(
+        ctypes.byref(desc), _dev(q, "q", dt), _dev(k_pages, "k_pages", dt), _dev(v_pages, "v_pages", dt),
+        int(k_pages.shape[0]), _dev(block_table, "block_table", i32), int(block_table.shape[1]),
+        _dev(seq_lens, "seq_lens", i32), _dev(idx, "idx", i32), _dev(gate_logit, "gate_logit", f32),
+        _dev(n_sel, "n_sel", i32), _dev(o, "o", dt), _dev(ws, "ws"), nbytes, _stream(stream)))
+
+
+def sas_block_scores_pooled(desc, q, kbar, scores, stream=None) -> None:
+    """Pooled-key block scores of the decode rows: kbar [B, Hkv, S, d] bf16."""
+    _check("sas_block_scores_pooled", lib().sas_block_scores_pooled(
+        ctypes.byref(desc), _dev(q, "q", torch.bfloat16), _dev(kbar, "kbar", torch.bfloat16), int(kbar.shape[2]),
+        _dev(scores, "scores", torch.float32), _stream(stream)))
+
+
+def sas_sparse_decode_pooled(desc, q, k_cache, v_cache, cache_stride_tokens, kbar, scores, idx, gate_logit,
+                             score_lse, n_sel, o, ws, stream=None) -> None:
+    """Pooled-key scores, top-K and sparse decode in one call."""
+    dt, f32, i32 = desc.torch_dtype, torch.float32, torch.int32
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check("sas_sparse_decode_pooled", lib().sas_sparse_decode_pooled(
+        ctypes.byref(desc), _dev(q, "q", dt), _dev(k_cache, "k_cache", dt), _dev(v_cache, "v_cache", dt),
+        int(cache_stride_tokens), _dev(kbar, "kbar", dt), int(kbar.shape[2]), _dev(scores, "scores", f32),
+        _dev(idx, "idx", i32), _dev(gate_logit, "gate_logit", f32), _dev(score_lse, "score_lse", f32),
+        _dev(n_sel, "n_sel", i32), _dev(o, "o", dt), _dev(ws, "ws"), nbytes, _stream(stream)))
+
+
 def sas_sparse_decode_noalloc(desc, q, k_cache, v_cache, cache_stride_tokens, idx, gate_logit, n_sel, o,
                               stream=None) -> None:
     """sas_sparse_decode without a workspace: the library's static scratch
@@ -173,6 +224,12 @@ def sas_device_timeouts() -> int:
     c = ctypes.c_uint32(0)
     _check("sas_device_timeouts", lib().sas_device_timeouts(ctypes.byref(c)))
     return int(c.value)
+
+
+def sas_set_wait_limit(ns: int) -> None:
+    """Bound (ns) on every device-side wait of the library's kernels; 0
+    restores the default of 1 s."""
+    _check("sas_set_wait_limit", lib().sas_set_wait_limit(int(ns)))
 
 
 def sas_kernel_launches() -> int:

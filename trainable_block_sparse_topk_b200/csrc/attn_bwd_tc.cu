@@ -62,6 +62,7 @@ struct BwdTcArgs {
     float* gsum;
     int tpc;             // tokens per chunk = 128 / G
     int meta_bytes;      // one metadata ring slot: tpc (16 + 4 rvs) bytes
+    int* aborted;        // set when a CTA gave up on a wait (the later kernels then write NaN)
 };
 
 struct BwdSmem {
@@ -169,7 +170,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             }
         }
         // chunk c's stream entries -> ring slot c & 3 (bulk copies, completion on meta_full)
+        int req_hi = -1, got_hi = -1;   // last chunk requested by this loader / whose entries have landed
         auto request = [&](int c) {
+            req_hi = c;
             if (lane == 0) {
                 const int n = min(tpc, ntok_total - c * tpc);
                 const int64_t e0 = ebase + (int64_t)c * tpc;
@@ -186,6 +189,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             // slot (c + 2) & 3 held chunk c - 2, whose readers are done with it once its stage is released
             if ((c & 1) == w && c + 2 < nc) request(c + 2);
             if (!tc::warp_wait_bar(&meta_full[c & 3], (uint32_t)((c >> 2) & 1), abort)) break;
+            got_hi = c;
             const int4* ent = ChunkMeta(sm + L::kMeta + (c & 3) * a.meta_bytes, tpc).ent;
             const int n = min(tpc, ntok_total - c * tpc);
             unsigned char* stq = sm + L::kStage + (c & 1) * L::kStageBytes;
@@ -215,6 +219,13 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             if (lane == 0) tc::mbar_arrive(&st_full[c & 1]);
         }
         tc::cp_async_wait_all();
+        if (*abort && lane == 0) {
+            // let the copies this warp started land before the CTA exits
+            int c0 = got_hi + 1;
+            if ((c0 & 1) != w) ++c0;
+            for (int c = c0; c <= req_hi; c += 2) tc::drain_wait(&meta_full[c & 3], (uint32_t)((c >> 2) & 1));
+            if (warp == 8) tc::drain_wait(kv_full, 0u);
+        }
     } else if (warp == 9) {
         // ------------------------------------------------------- MMA issuer ---
         if (lane == 0) {
@@ -289,7 +300,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                     t0 = global_ns();
                 } else if (*abort) {
                     ok = false;
-                } else if (global_ns() - t0 > 1000000000ull) {
+                } else if (global_ns() - t0 > g_sas_wait_limit_ns) {
                     *abort = 1;
                     atomicAdd(&g_sas_wait_timeouts, 1u);
                     ok = false;
@@ -307,33 +318,36 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
         const float qk = sh.scale * kLog2e;
         for (int c = 0; c < nc; ++c) {
             const int st = c & 1;
-            if (!tc::warp_wait_bar(&st_full[st], (uint32_t)((c >> 1) & 1), abort)) break;
-            const ChunkMeta meta(sm + L::kMeta + (c & 3) * a.meta_bytes, tpc);
-            const int n = min(tpc, ntok_total - c * tpc);
-            const int ti = r / G, h = r - ti * G;
-            const bool valid = ti < n;
-            int t = 0, kmax = -1;
-            float lgl = 0.f, lse2 = 0.f, Dv = 0.f;
-            bool diag = false;
-            if (valid) {
-                const int4 e = meta.ent[ti];
-                t = e.x;
-                diag = (t >> 6) == j;
-                kmax = diag ? (t & 63) : kBS - 1;
-                lgl = __int_as_float(e.y);
-                lse2 = meta.rv[ti * rvs + 2 * h];
-                Dv = meta.rv[ti * rvs + 2 * h + 1];
-            }
-            const float bias = (lgl - lse2) * kLog2e;
-            const int dq_row = valid ? (int)(((int64_t)b * sh.Hq + g * G + h) * T + t) : -1;
-            // token r of the chunk, for its Gsum (read now: the metadata slot is
-            // refilled once the chunk's last MMAs are issued)
-            const int gs_slot = r < n ? meta.ent[r].z : -1;
-            const int gs_tok = r < n ? meta.ent[r].x : 0;
-            if (!tc::warp_wait_bar(&s_full[st], (uint32_t)((c >> 1) & 1), abort)) break;
-            tc::fence_after_sync();
-            float rowsum = 0.f;
-            {
+            float* gs = tok_gs + st * kRows;
+            int n = 0, gs_slot = -1, gs_tok = 0;
+            bool fail = false;
+            do {   // a wait that gives up leaves this block, not the chunk loop
+                if (!tc::warp_wait_bar(&st_full[st], (uint32_t)((c >> 1) & 1), abort)) { fail = true; break; }
+                const ChunkMeta meta(sm + L::kMeta + (c & 3) * a.meta_bytes, tpc);
+                n = min(tpc, ntok_total - c * tpc);
+                const int ti = r / G, h = r - ti * G;
+                const bool valid = ti < n;
+                int t = 0, kmax = -1;
+                float lgl = 0.f, lse2 = 0.f, Dv = 0.f;
+                bool diag = false;
+                if (valid) {
+                    const int4 e = meta.ent[ti];
+                    t = e.x;
+                    diag = (t >> 6) == j;
+                    kmax = diag ? (t & 63) : kBS - 1;
+                    lgl = __int_as_float(e.y);
+                    lse2 = meta.rv[ti * rvs + 2 * h];
+                    Dv = meta.rv[ti * rvs + 2 * h + 1];
+                }
+                const float bias = (lgl - lse2) * kLog2e;
+                const int dq_row = valid ? (int)(((int64_t)b * sh.Hq + g * G + h) * T + t) : -1;
+                // token r of the chunk, for its Gsum (read now: the metadata slot is
+                // refilled once the chunk's last MMAs are issued)
+                gs_slot = r < n ? meta.ent[r].z : -1;
+                gs_tok = r < n ? meta.ent[r].x : 0;
+                if (!tc::warp_wait_bar(&s_full[st], (uint32_t)((c >> 1) & 1), abort)) { fail = true; break; }
+                tc::fence_after_sync();
+                float rowsum = 0.f;
                 uint32_t sv[32], pv[32];
 #pragma unroll
                 for (int cb = 0; cb < 2; ++cb) {
@@ -358,7 +372,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 // P and dS of chunk c-1 must have been consumed by its MMAs before
                 // they are overwritten; that also means the epilogue warps are done
                 // with chunk c-2, whose row-id slot is reused here
-                if (c >= 1 && !tc::warp_wait_bar(p_empty, (uint32_t)((c - 1) & 1), abort)) break;
+                if (c >= 1 && !tc::warp_wait_bar(p_empty, (uint32_t)((c - 1) & 1), abort)) { fail = true; break; }
                 if (hf == 0) {
                     ids[st * kRows + r] = dq_row;
                     __syncwarp();
@@ -374,15 +388,17 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                                  "r"(dk2[cb * 4]), "r"(dk2[cb * 4 + 1]), "r"(dk2[cb * 4 + 2]), "r"(dk2[cb * 4 + 3])
                                  : "memory");
                 }
-            }
-            tc::fence_async_shared();
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(p_full);
-            // Gsum of the token: its G rows are in this chunk
-            float* gs = tok_gs + st * kRows;
-            if (valid && !diag) atomicAdd(&gs[ti], rowsum);
-            tc::named_bar(1, 256);
+                tc::fence_async_shared();
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(p_full);
+                // Gsum of the token: its G rows are in this chunk
+                if (valid && !diag) atomicAdd(&gs[ti], rowsum);
+            } while (false);
+            // every P/dS warp takes this barrier once per chunk; it also tells them
+            // all whether any of them (or another role) gave up on a wait, so that
+            // they leave the loop together and no warp is left at a barrier
+            if (tc::bar_red_or(1, 256, fail || *abort != 0)) break;
             if (hf == 0 && r < n) {
                 if (gs_slot >= 0) a.gsum[((int64_t)bg * T + gs_tok) * K + gs_slot] = gs[r];
                 gs[r] = 0.f;
@@ -463,14 +479,27 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                     dkb[(int64_t)key * kD + r] = __float2bfloat16_rn(__uint_as_float(kv[e]) * dscale);
                 }
             }
+        } else {
+            // a wait gave up: the block's dK and dV are incomplete, mark them invalid
+            const __nv_bfloat16 nan = __float2bfloat16(__int_as_float(0x7fc00000));
+            __nv_bfloat16* dvb = a.dv + ((int64_t)bg * T + (int64_t)j * kBS) * kD;
+            __nv_bfloat16* dkb = a.dk + ((int64_t)bg * T + (int64_t)j * kBS) * kD;
+            for (int key = 0; key < kBS; ++key) {
+                dvb[(int64_t)key * kD + r] = nan;
+                dkb[(int64_t)key * kD + r] = nan;
+            }
         }
     }
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 10) {
+        // TMEM is released only after the last MMA that writes it
+        if (lane == 0) tc::drain_wait(done, 0u);
+        __syncwarp();
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, kTmemCols);
     }
+    if (tid == 0 && *abort) atomicExch(a.aborted, 1);
 }
 
 }  // namespace
@@ -485,7 +514,7 @@ size_t bwd_tc_ws_bytes(const Shape& s) { return sel_stream_bytes(s, 2); }
 cudaError_t launch_bwd_tc(const Shape& s, const void* q, const void* k, const void* v, const void* dO,
                           const float* lse, const float* Dd, const int32_t* idx, const float* gl,
                           const int32_t* nsel, const uint64_t* maskT, void* ws, float* dq_acc, void* dk, void* dv,
-                          float* gsum, cudaStream_t st) {
+                          float* gsum, int* aborted, cudaStream_t st) {
     CUtensorMap mk, mv;
     if (!encode_bf16_2d(&mk, k, (uint64_t)s.B * s.Hkv * s.T, kD, kBS) ||
         !encode_bf16_2d(&mv, v, (uint64_t)s.B * s.Hkv * s.T, kD, kBS))
@@ -499,6 +528,7 @@ cudaError_t launch_bwd_tc(const Shape& s, const void* q, const void* k, const vo
     a.dk = static_cast<__nv_bfloat16*>(dk);
     a.dv = static_cast<__nv_bfloat16*>(dv);
     a.gsum = gsum;
+    a.aborted = aborted;
     a.tpc = kRows / s.G;
     a.meta_bytes = a.tpc * (16 + 4 * a.ss.rvs);
     // the streams carry each row's lse and D
@@ -515,6 +545,10 @@ cudaError_t launch_bwd_tc(const Shape& s, const void* q, const void* k, const vo
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
     return e;
+}
+
+cudaError_t set_bwd_tc_wait_limit(unsigned long long ns) {
+    return cudaMemcpyToSymbol(g_sas_wait_limit_ns, &ns, sizeof(ns));
 }
 
 cudaError_t read_bwd_tc_timeouts(unsigned int* out) {

@@ -58,6 +58,7 @@ struct FwdRowsArgs {
     float* o_acc;         // [B*Hq*T, d]
     int tpc;              // tokens per chunk = 128 / G
     int meta_bytes;       // one metadata ring slot: tpc (16 + 4 rvs) bytes
+    int* aborted;         // set when a CTA gave up on a wait (the finalize then writes NaN)
 };
 
 // kSt Q stages (3 when shared memory allows, else 2); the metadata ring has
@@ -75,7 +76,7 @@ struct RowsSmem {
     static constexpr uint32_t kIds = kOst + kRows * kOstRow;       // i32 [4][128]: O accumulator row per chunk row
     static constexpr uint32_t kBar = kIds + 4 * kRows * 4;
     static constexpr int kMetaSlots = 2 * kSt;                     // chunk c -> slot c % kMetaSlots
-    static constexpr int kNumBars = 13 + 4 * kSt;
+    static constexpr int kNumBars = 14 + 4 * kSt;
     static constexpr uint32_t kMisc = kBar + 8 * kNumBars;         // tmem base, stream length, first entry, abort
     static constexpr uint32_t kMeta = (kMisc + 16 + 15) & ~15u;    // metadata ring, meta_bytes per slot
     static constexpr uint32_t kTmemCols = 512;                     // S double [0,128), O double [128,384)
@@ -110,6 +111,7 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     uint64_t* o_empty = o_full + 2;           // [2] 4 arrivals
     uint64_t* meta_full = o_empty + 2;        // [kMS] ring slot c % kMS holds chunk c's stream entries (tx bytes)
     uint64_t* ids_full = meta_full + kMS;     // [4] 4 arrivals: chunk c's O rows are in ids[c & 3]
+    uint64_t* mma_drain = ids_full + 4;       // every MMA of the CTA has completed
     int* ids = reinterpret_cast<int*>(sm + L::kIds);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::kMisc);
     int* ntok_slot = reinterpret_cast<int*>(sm + L::kMisc + 4);      // [2]: stream length, first entry
@@ -173,7 +175,9 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             }
         }
         // chunk c's stream entries -> ring slot c % kMS (bulk copies, completion on meta_full)
+        int req_hi = -1, got_hi = -1;   // last chunk whose entries were requested / have landed
         auto request = [&](int c) {
+            req_hi = c;
             if (lane == 0) {
                 const int n = min(tpc, ntok_total - c * tpc);
                 const int64_t e0 = ebase + (int64_t)c * tpc;
@@ -191,6 +195,7 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             // slot (c + kSt) % kMS held chunk c - kSt, whose readers are done with it once its stage is released
             if (c + kSt < nc) request(c + kSt);
             if (!tc::warp_wait_bar(&meta_full[c % kMS], (uint32_t)((c / kMS) & 1), abort)) break;
+            got_hi = c;
             const int4* ent = RowMeta(sm + L::kMeta + (c % kMS) * a.meta_bytes, tpc).ent;
             const int n = min(tpc, ntok_total - c * tpc);
             {
@@ -215,6 +220,12 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             if (lane == 0) tc::mbar_arrive(&st_full[L0]);
         }
         tc::cp_async_wait_all();
+        if (*abort && lane == 0) {
+            // let the copies this warp started land before the CTA exits
+            for (int c = got_hi < 0 ? L0 : got_hi + kSt; c <= req_hi; c += kSt)
+                tc::drain_wait(&meta_full[c % kMS], (uint32_t)((c / kMS) & 1));
+            if (warp == 8) tc::drain_wait(kv_full, 0u);
+        }
     } else if (warp == 9) {
         // ------------------------------------------------------- MMA issuer ---
         if (lane == 0) {
@@ -268,7 +279,7 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                         t0 = global_ns();
                     } else if (*abort) {
                         ok = false;
-                    } else if (global_ns() - t0 > 1000000000ull) {
+                    } else if (global_ns() - t0 > g_sas_wait_limit_ns) {
                         *abort = 1;
                         atomicAdd(&g_sas_wait_timeouts, 1u);
                         ok = false;
@@ -277,6 +288,7 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
                     }
                 }
             }
+            tc::mma_commit(mma_drain);   // arrives once every MMA issued above has completed
         }
     } else if (warp >= 4 && warp < 8) {
         // --------------------------------------------------------- P warps ---
@@ -381,9 +393,13 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 10) {
+        // TMEM is released only after the last MMA that writes it
+        if (lane == 0) tc::drain_wait(mma_drain, 0u);
+        __syncwarp();
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, L::kTmemCols);
     }
+    if (tid == 0 && *abort) atomicExch(a.aborted, 1);
 }
 
 // M = scale log2e q_t.k_t for each of the G query heads of a (b, kv head, t)
@@ -442,8 +458,18 @@ constexpr int kRowsU = 4;
 __global__ void __launch_bounds__(256)
 fwd_rows_finalize_kernel(Shape sh, const float* __restrict__ shift, const float* __restrict__ l_acc,
                          const float* __restrict__ o_acc, __nv_bfloat16* __restrict__ o, float* __restrict__ lse,
-                         int32_t* __restrict__ list, int32_t* __restrict__ list_n) {
+                         int32_t* __restrict__ list, int32_t* __restrict__ list_n, const int* __restrict__ aborted) {
     const int64_t rows = (int64_t)sh.B * sh.Hq * sh.T;
+    if (*aborted) {
+        // a CTA of the gathered-row kernel gave up on a wait: the accumulators
+        // are incomplete, so every output row is marked invalid
+        const int64_t nthr = (int64_t)gridDim.x * blockDim.x;
+        const __nv_bfloat16 nan = __float2bfloat16(__int_as_float(0x7fc00000));
+        for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < rows * kD; e += nthr) o[e] = nan;
+        for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < rows; e += nthr)
+            lse[e] = __int_as_float(0x7fc00000);
+        return;
+    }
     const int lane = threadIdx.x & 31;
     const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -483,7 +509,7 @@ fwd_rows_finalize_kernel(Shape sh, const float* __restrict__ shift, const float*
 }
 
 // Workspace: shift [rows] f32 | list [rows] i32 | l [rows] f32 | O [rows, d] f32 | list count |
-// (256-aligned) the token streams
+// abort flag | (256-aligned) the token streams
 struct RowsWs {
     float* shift;
     int32_t* list;
@@ -526,7 +552,8 @@ cudaError_t launch_fwd_rows(const Shape& s, const void* q, const void* k, const 
     a.l_acc = w.l_acc;
     a.o_acc = w.o_acc;
     a.tpc = kRows / s.G;
-    cudaError_t e = cudaMemsetAsync(w.list_n, 0, sizeof(int32_t), st);
+    a.aborted = w.list_n + 1;
+    cudaError_t e = cudaMemsetAsync(w.list_n, 0, 2 * sizeof(int32_t), st);   // list count, abort flag
     if (e != cudaSuccess) return e;
     {
         KernelTimer kt("fwd_rows_shift", st);
@@ -556,14 +583,17 @@ cudaError_t launch_fwd_rows(const Shape& s, const void* q, const void* k, const 
     {
         KernelTimer kt("fwd_rows_finalize", st);
         fwd_rows_finalize_kernel<<<(unsigned)std::min<int64_t>((rows + 8 * kRowsU - 1) / (8 * kRowsU), 148 * 16), 256, 0,
-                                   st>>>(s, w.shift, w.l_acc, w.o_acc,
-                                                                             static_cast<__nv_bfloat16*>(o), lse, w.list,
-                                                                             w.list_n);
+                                   st>>>(s, w.shift, w.l_acc, w.o_acc, static_cast<__nv_bfloat16*>(o), lse, w.list,
+                                         w.list_n, a.aborted);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     count_launches(1);
     return launch_fwd_simt_rows(s, q, k, v, idx, gl, nsel, w.list, w.list_n, o, lse, st);
+}
+
+cudaError_t set_fwd_rows_wait_limit(unsigned long long ns) {
+    return cudaMemcpyToSymbol(g_sas_wait_limit_ns, &ns, sizeof(ns));
 }
 
 cudaError_t read_fwd_rows_timeouts(unsigned int* out) {

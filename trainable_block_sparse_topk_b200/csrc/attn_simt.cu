@@ -380,8 +380,14 @@ bwd_simt_kernel(Shape sh, const T* __restrict__ q, const T* __restrict__ k, cons
 // fp32 -> bf16, 8 values per thread and pass, two passes' loads in flight
 // (n8 = number of 8-value groups).
 __global__ void __launch_bounds__(256)
-cast_bf16x8_kernel(int64_t n8, const float4* __restrict__ src, uint4* __restrict__ dst) {
+cast_bf16x8_kernel(int64_t n8, const float4* __restrict__ src, uint4* __restrict__ dst, const int* __restrict__ aborted) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    if (aborted != nullptr && *aborted) {   // the accumulator is incomplete: mark dq invalid
+        const uint32_t nan2 = 0x7fc07fc0u;
+        for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += stride)
+            dst[i] = make_uint4(nan2, nan2, nan2, nan2);
+        return;
+    }
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += 2 * stride) {
         float4 v[2][2];
 #pragma unroll
@@ -405,29 +411,39 @@ cast_bf16x8_kernel(int64_t n8, const float4* __restrict__ src, uint4* __restrict
 
 // ------------------------------------------------------- score gradient (K5) ---
 
-// ds_i = [i kept] Gsum_i - g_i sum_{k kept} Gsum_k for i < C, 0 otherwise,
-// with g_i = exp(s_i - score_lse) (arXiv text 4: d log g_i / d s_k = [i=k] - g_k).
-// One warp per (b, kv head, t) row; every column of the row is written.
+// ds_i = dL/ds_i for i < C, 0 otherwise, from Gsum_k = dL/d(log g_k) of the
+// kept blocks through the gate activation's derivative. Softmax gate
+// (arXiv text 4: d log g_i / d s_k = [i=k] - g_k, g_i = exp(s_i - score_lse)):
+// ds_i = [i kept] Gsum_i - g_i sum_{k kept} Gsum_k. The other activations of
+// the method's comparison are listed at the terms below. One warp per
+// (b, kv head, t) row; every column of the row is written.
 __global__ void __launch_bounds__(256)
 dscore_kernel(Shape sh, const float* __restrict__ scores, const float* __restrict__ slse,
               const int32_t* __restrict__ idx, const int32_t* __restrict__ nsel,
-              const float* __restrict__ gsum, float* __restrict__ ds) {
+              const float* __restrict__ gsum, float* __restrict__ ds, const int* __restrict__ aborted) {
     const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= sh.rows()) return;
+    if (aborted != nullptr && *aborted) {   // Gsum is incomplete: mark the row invalid
+        for (int i = lane; i < sh.NB; i += 32) ds[row * sh.NB + i] = __int_as_float(0x7fc00000);
+        return;
+    }
     const int t = (int)(row % sh.T);
     const int C = (int)(((int64_t)sh.q_offset + t) / sh.bs);
-    const bool on = sh.gate == SAS_GATE_SOFTMAX;
+    const int mode = sh.gate;
+    // every candidate gets -g_i * T (softmax gate and its straight-through
+    // hard form), each kept block its own term on top
+    const bool dense_term = mode == SAS_GATE_SOFTMAX || mode == SAS_GATE_STE;
     const float* sr = scores + row * sh.NB;
     float* dr = ds + row * sh.NB;
-    // every load of the row is issued before any is used: the kept list and its
-    // Gsum (masked by n afterwards), the normaliser and the first kPre chunks of
-    // 32 causal scores
+    // every load of the row is issued before any is used: the kept list, its
+    // Gsum and scores (masked by n afterwards), the normaliser and the first
+    // kPre chunks of 32 causal scores
     constexpr int kPre = 8;
     const int n = nsel[row];
     const float lse = slse[row];
     int si[2];
-    float sg[2];
+    float sg[2], sk[2];
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
         const int slot = lane + 32 * r;
@@ -438,52 +454,72 @@ dscore_kernel(Shape sh, const float* __restrict__ scores, const float* __restric
 #pragma unroll
     for (int q = 0; q < kPre; ++q) {
         const int i = q * 32 + lane;
-        sv[q] = (on && i < C) ? sr[i] : 0.f;
+        sv[q] = (dense_term && i < C) ? sr[i] : 0.f;
     }
 #pragma unroll
-    for (int r = 0; r < 2; ++r)
-        if (lane + 32 * r >= n) { si[r] = -1; sg[r] = 0.f; }
-    const float tot = warp_sum(sg[0] + sg[1]);
+    for (int r = 0; r < 2; ++r) {
+        if (lane + 32 * r >= n || (unsigned)si[r] >= (unsigned)C) { si[r] = -1; sg[r] = 0.f; }
+        sk[r] = si[r] >= 0 ? sr[si[r]] : -INFINITY;
+    }
+    // the kept blocks' own terms and the factor T of the dense term, per mode
+    // (Gsum_k = dL / d log g_k):
+    //   softmax           d log g_i/ds_k = [i=k] - g_k:  kept Gsum_k, T = sum Gsum
+    //   sigmoid           log g_k = log sigmoid(s_k):     kept Gsum_k (1 - sigmoid(s_k))
+    //   raw               log g_k = s_k:                  kept Gsum_k
+    //   softmax (kept)    log g_k = s_k - log sum_I e^s:  kept Gsum_k - p_k sum Gsum
+    //   hard (STE)        dL/dg_k = Gsum_k, dg_i/ds_k = g_i([i=k] - g_k):
+    //                                                     kept Gsum_k g_k, T = sum Gsum g
+    float kv[2] = {0.f, 0.f};
+    float T = 0.f;
+    if (mode == SAS_GATE_SOFTMAX) {
+        kv[0] = sg[0];
+        kv[1] = sg[1];
+        T = warp_sum(sg[0] + sg[1]);
+    } else if (mode == SAS_GATE_STE) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) kv[r] = si[r] >= 0 ? sg[r] * expf(sk[r] - lse) : 0.f;
+        T = warp_sum(kv[0] + kv[1]);
+    } else if (mode == SAS_GATE_SIGMOID) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) kv[r] = si[r] >= 0 ? sg[r] / (1.f + expf(sk[r])) : 0.f;   // 1 - sigmoid(s)
+    } else if (mode == SAS_GATE_RAW) {
+        kv[0] = sg[0];
+        kv[1] = sg[1];
+    } else if (mode == SAS_GATE_SOFTMAX_SELECTED) {
+        const float m = warp_max(fmaxf(sk[0], sk[1]));
+        const float l = warp_sum((si[0] >= 0 ? expf(sk[0] - m) : 0.f) + (si[1] >= 0 ? expf(sk[1] - m) : 0.f));
+        const float tot = warp_sum(sg[0] + sg[1]);
+#pragma unroll
+        for (int r = 0; r < 2; ++r) kv[r] = si[r] >= 0 ? sg[r] - expf(sk[r] - m) / l * tot : 0.f;
+    }
+    const bool any = mode != SAS_GATE_NONE;
     int base = 0;
+    auto chunk = [&](int c0, float sc) {
+        uint32_t bits = 0;
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+            if (si[r] >= c0 && si[r] < c0 + 32) bits |= 1u << (si[r] - c0);
+        const uint32_t mask = __reduce_or_sync(0xffffffffu, bits);
+        const int slot = base + __popc(mask & ((1u << lane) - 1u));
+        const float k0 = __shfl_sync(0xffffffffu, kv[0], slot & 31);
+        const float k1 = __shfl_sync(0xffffffffu, kv[1], slot & 31);
+        const int i = c0 + lane;
+        float val = 0.f;
+        if (any && i < C) {
+            if (dense_term) val = -expf(sc - lse) * T;
+            if ((mask >> lane) & 1u) val += slot < 32 ? k0 : k1;
+        }
+        if (i < sh.NB) dr[i] = val;
+        base += __popc(mask);
+    };
 #pragma unroll
     for (int q = 0; q < kPre; ++q) {
         const int c0 = q * 32;
         if (c0 >= sh.NB) break;                        // warp-uniform
-        uint32_t bits = 0;
-#pragma unroll
-        for (int r = 0; r < 2; ++r)
-            if (si[r] >= c0 && si[r] < c0 + 32) bits |= 1u << (si[r] - c0);
-        const uint32_t mask = __reduce_or_sync(0xffffffffu, bits);
-        const int slot = base + __popc(mask & ((1u << lane) - 1u));
-        const float g0 = __shfl_sync(0xffffffffu, sg[0], slot & 31);
-        const float g1 = __shfl_sync(0xffffffffu, sg[1], slot & 31);
-        const int i = c0 + lane;
-        float val = 0.f;
-        if (on && i < C) {
-            val = -expf(sv[q] - lse) * tot;
-            if ((mask >> lane) & 1u) val += slot < 32 ? g0 : g1;
-        }
-        if (i < sh.NB) dr[i] = val;
-        base += __popc(mask);
+        chunk(c0, sv[q]);
     }
-    for (int c0 = kPre * 32; c0 < sh.NB; c0 += 32) {   // long rows: the rest one chunk at a time
-        uint32_t bits = 0;
-#pragma unroll
-        for (int r = 0; r < 2; ++r)
-            if (si[r] >= c0 && si[r] < c0 + 32) bits |= 1u << (si[r] - c0);
-        const uint32_t mask = __reduce_or_sync(0xffffffffu, bits);
-        const int slot = base + __popc(mask & ((1u << lane) - 1u));
-        const float g0 = __shfl_sync(0xffffffffu, sg[0], slot & 31);
-        const float g1 = __shfl_sync(0xffffffffu, sg[1], slot & 31);
-        const int i = c0 + lane;
-        float val = 0.f;
-        if (on && i < C) {
-            val = -expf(sr[i] - lse) * tot;
-            if ((mask >> lane) & 1u) val += slot < 32 ? g0 : g1;
-        }
-        if (i < sh.NB) dr[i] = val;
-        base += __popc(mask);
-    }
+    for (int c0 = kPre * 32; c0 < sh.NB; c0 += 32)     // long rows: the rest one chunk at a time
+        chunk(c0, (dense_term && c0 + lane < C) ? sr[c0 + lane] : 0.f);
 }
 
 template <typename T, int D, int GMAX, int BS>
@@ -621,7 +657,7 @@ cudaError_t launch_bwd_simt(const Shape& s, const void* q, const void* k, const 
     return bwd_d<__nv_bfloat16>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, gsum, st);
 }
 
-cudaError_t launch_cast_dq(const Shape& s, const float* dq_acc, void* dq, cudaStream_t st) {
+cudaError_t launch_cast_dq(const Shape& s, const float* dq_acc, void* dq, const int* aborted, cudaStream_t st) {
     // bf16 only: fp32 accumulates dq in place. n is a multiple of 8 (d is 64 or
     // 128); both buffers are 16-byte aligned.
     if (s.dtype != SAS_DT_BF16) return cudaErrorInvalidValue;
@@ -629,7 +665,8 @@ cudaError_t launch_cast_dq(const Shape& s, const float* dq_acc, void* dq, cudaSt
     const unsigned g8 = (unsigned)std::min<int64_t>((n8 + 511) / 512, 148 * 8);
     {
         KernelTimer kt("cast_dq", st);
-        cast_bf16x8_kernel<<<g8, 256, 0, st>>>(n8, reinterpret_cast<const float4*>(dq_acc), static_cast<uint4*>(dq));
+        cast_bf16x8_kernel<<<g8, 256, 0, st>>>(n8, reinterpret_cast<const float4*>(dq_acc), static_cast<uint4*>(dq),
+                                               aborted);
     }
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
@@ -637,10 +674,10 @@ cudaError_t launch_cast_dq(const Shape& s, const float* dq_acc, void* dq, cudaSt
 }
 
 cudaError_t launch_dscore(const Shape& s, const float* scores, const float* slse, const int32_t* idx,
-                          const int32_t* nsel, const float* gsum, float* ds, cudaStream_t st) {
+                          const int32_t* nsel, const float* gsum, float* ds, const int* aborted, cudaStream_t st) {
     const unsigned grid = (unsigned)((s.rows() + 7) / 8);
     KernelTimer kt("dscore", st);
-    dscore_kernel<<<grid, 256, 0, st>>>(s, scores, slse, idx, nsel, gsum, ds);
+    dscore_kernel<<<grid, 256, 0, st>>>(s, scores, slse, idx, nsel, gsum, ds, aborted);
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
     return e;

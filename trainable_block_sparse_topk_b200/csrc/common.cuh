@@ -140,13 +140,22 @@ __device__ __forceinline__ uint64_t global_ns() {
 // waits; read back through sas_device_timeouts().
 static __device__ unsigned int g_sas_wait_timeouts;
 
-// Wait for phase `parity` of `bar`, giving up after ~1 s. Returns false on
-// timeout (and counts it); the caller then skips the work that needed the data.
+// Bound on every device-side wait for another agent's work (ns), one per
+// translation unit that waits; set through sas_set_wait_limit (default 1 s).
+// Waits that only let copies already in flight land before a CTA exits keep
+// a fixed 1 s bound.
+constexpr unsigned long long kDefaultWaitNs = 1000000000ull;
+static __device__ unsigned long long g_sas_wait_limit_ns = kDefaultWaitNs;
+
+// Wait for phase `parity` of `bar`, giving up after the wait limit. Returns
+// false on timeout (and counts it); the caller then skips the work that
+// needed the data.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
+    const unsigned long long lim = g_sas_wait_limit_ns;
     while (!mbar_try_wait(bar, parity)) {
-        if (global_ns() - t0 > 1000000000ull) {
+        if (global_ns() - t0 > lim) {
             atomicAdd(&g_sas_wait_timeouts, 1u);
             return false;
         }

@@ -5,12 +5,16 @@
 // (SAS study note 3-7 inference path, steps 2-4). With no selection it attends
 // every token [0, N) with no gate: the dense comparison of study note 5-6.
 //
-// Work split: the block list of each (b, kv head) is cut into `splits` chunks
-// of `bpc` blocks; one CTA per chunk streams its blocks through two shared
-// memory stages. Each block's K and V rows are contiguous in the cache, so one
-// bulk async copy per tensor moves a whole block (16 KiB at b=64, d=128, bf16)
-// with a single instruction. The CTA writes an unnormalised partial (m, l, o)
-// for the G heads, and a second kernel merges the partials by log-sum-exp.
+// bf16, d 128, block 64 (the tensor-core path, decode_flat_kernel): persistent
+// CTAs, one per SM, share out every (b, kv head)'s block list evenly, stream
+// the blocks by TMA and merge the per-CTA partials in the last CTA to finish
+// each group -- one launch per call. Other shapes and fp32 (CUDA cores,
+// decode_partial_kernel): the block list of each (b, kv head) is cut into
+// `splits` chunks of `bpc` blocks; one CTA per chunk streams its blocks
+// through two shared memory stages, one bulk async copy per tensor and block
+// (K and V rows of a block are contiguous in the cache), writes an
+// unnormalised partial (m, l, o) for the G heads, and a second kernel merges
+// the partials by log-sum-exp.
 #include <algorithm>
 #include <mutex>
 
@@ -26,6 +30,15 @@ namespace {
 
 constexpr int kDecThreads = 256;
 
+// Flat item split of the tensor-core decode: nblk items per (b, kv head)
+// group, W items in all, ncta CTAs, each owning per or per + 1 of them.
+struct FlatPlan {
+    int64_t W;
+    int nblk;
+    int ncta;
+    int64_t per, rem;
+};
+
 struct DecArgs {
     Shape sh;
     const void* q;
@@ -39,6 +52,15 @@ struct DecArgs {
     void* o;             // [B, Hq, D] output
     int bpc;
     int splits;
+    FlatPlan fp;         // tensor-core path: item split
+    int* fin;            // tensor-core path: [B*Hkv] records written per group, zeroed per call
+    // paged cache (tensor-core path): block j of sequence b is page
+    // table[b * max_blocks + j] of the pools kc/vc [num_pages, Hkv, BS, D];
+    // NULL table: the contiguous cache [B, Hkv, stride, D]
+    const int32_t* table;
+    int max_blocks;
+    int num_pages;
+    const int32_t* lens; // [B] cache length of each sequence (new token included); NULL: q_offset + 1
 };
 
 template <typename T, int D, int BS>
@@ -91,7 +113,8 @@ decode_partial_kernel(DecArgs a) {
     const int64_t N = (int64_t)sh.q_offset + 1;
     const int C = (int)(sh.q_offset / BS);
     const bool dense = a.idx == nullptr;
-    const int n = dense ? C : a.nsel[bg];
+    // a kept count outside [0, min(K, C)] would read past the row: clamp it
+    const int n = dense ? C : min(max(a.nsel[bg], 0), min(sh.K, C));
     const int nblk = n + 1;
     const int p0 = split * a.bpc;
     const int p1 = min(p0 + a.bpc, nblk);
@@ -276,10 +299,28 @@ decode_partial_kernel(DecArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// Tensor-core variant (bf16, d = 128, block 64, G <= 8). Warp 0 moves blocks
-// into a 4-stage ring by TMA (K and V as two 64-column boxes each, 128-byte
-// swizzle); warps 1 and 2 each own every other stage and run the whole block
-// on mma.sync m16n8k16 with no CTA-wide barrier:
+// Tensor-core decode (bf16, d = 128, block 64, G <= 8): persistent CTAs over a
+// flat list of work items.
+//
+// Item i is position p = i % nblk of group bg = i / nblk, the (b, kv head)
+// block lists laid end to end. Sparse: p < n is the p-th kept block, the last
+// position (nblk - 1 = min(K, C)) is the causal current block, and positions
+// in between (a row that kept fewer than min(K, C) blocks) are empty. Dense:
+// p is the block index itself, the last one being the current block.
+// CTA c takes the contiguous items [start(c), start(c + 1)), an even share of
+// all of them, so a group's list may be cut between neighbouring CTAs and a
+// CTA may finish one group and start the next. For every group it touches, a
+// CTA writes one unnormalised partial (m, l, O of the G heads) as record
+// c + bg (unique: the groups of CTA c + 1 start where those of CTA c end).
+// The CTA that completes a group last (an atomic ticket per group) merges the
+// group's records by log-sum-exp and writes o: one launch per call.
+//
+// Roles (128 threads): warp 0 resolves the items' block indices, log-gates
+// and cache rows 32 at a time and moves each block's K and V rows into a
+// kFlatStages ring by TMA (two 64-column boxes per tensor, 128-byte swizzle, no
+// multicast); warps 1-3 take every third item each (a consumer's MMA chain has
+// little parallelism of its own, so three blocks are computed at once, and
+// each consumer owns two stages) and run each block on mma.sync m16n8k16:
 //   S^T = K q^T   (M = 16 keys, N = 8 heads, K = 16 dims; 4 x 8 MMAs)
 //   online softmax per head in log2 units (scale applied in fp32 after the MMA)
 //   O^T += V^T P^T (M = 16 dims, N = 8 heads, K = 16 keys; 8 x 4 MMAs)
@@ -287,13 +328,39 @@ decode_partial_kernel(DecArgs a) {
 // (keys x heads, accumulator layout) becomes the B operand by movmatrix.trans.
 // Rows of the current block at or after the new token may hold anything in the
 // cache: their scores are replaced by -inf and their V rows zeroed in shared
-// memory before the product. The two consumers merge their (m, l, O) at the
-// end and write one partial per CTA for the same merge kernel.
-constexpr int kMmaStages = 4;
-constexpr uint32_t kMmaStage = 32768;   // K box 0 | K box 1 | V box 0 | V box 1, 8 KiB each
+// memory before the product. At the end of each group the consumers merge
+// their (m, l, O) through shared memory.
+constexpr int kFlatStages = 6;
+constexpr int kCons = 3;                 // consumer warps: item i goes to consumer i mod kCons
+constexpr int kFlatThreads = 32 * (1 + kCons);
+// Stage s always holds items of consumer s mod kCons, so each stage's barrier
+// phases are waited on by one warp, in order (a second warp could poll a phase
+// ahead of the current one and see an older phase of the same parity).
+static_assert(kFlatStages % kCons == 0, "every stage must belong to one consumer");
+constexpr uint32_t kItemBytes = 32768;   // K box 0 | K box 1 | V box 0 | V box 1, 8 KiB each
+constexpr int kMaxDecodeCtas = 160;     // grid bound (one CTA per SM)
+constexpr int kRecF = 132;              // floats per head in a record: O[128], m, l, 2 pad (16-byte rows)
+constexpr int kMaxRecs = 64;            // records of one group (CTAs sharing it), bounded by the plan
 
-struct DecMmaArgs {
-    DecArgs d;
+// Item split: CTA c owns [flat_start(c), flat_start(c + 1)).
+__host__ __device__ __forceinline__ int64_t flat_start(const FlatPlan& f, int64_t c) {
+    return c * f.per + (c < f.rem ? c : f.rem);
+}
+// The CTA that owns item i.
+__host__ __device__ __forceinline__ int64_t flat_owner(const FlatPlan& f, int64_t i) {
+    const int64_t big = f.rem * (f.per + 1);
+    return i < big ? i / (f.per + 1) : f.rem + (i - big) / f.per;
+}
+
+struct FlatSmem {
+    static constexpr uint32_t kBar = kFlatStages * kItemBytes;        // full[S], empty[S]
+    static constexpr uint32_t kMisc = kBar + 16 * kFlatStages;        // abort flag
+    static constexpr uint32_t kBlk = kMisc + 16;                      // i32 [S]: keys of the stage's item (0: none)
+    static constexpr uint32_t kLg = kBlk + 4 * kFlatStages;           // f32 [S]: its log-gate (log2 units)
+    static constexpr uint32_t kXch = (kLg + 4 * kFlatStages + 15) & ~15u;   // per consumer 1..: m[8], l[8], O^T[128][8]
+    static constexpr uint32_t kLast = kXch + 4 * (kCons - 1) * (16 + 128 * 8);   // i32: this CTA merges the group
+    static constexpr uint32_t kMerge = kLast + 16;                    // f32 m, l, weight [kMaxRecs][8] each
+    static constexpr uint32_t kTotal = kMerge + 3 * 4 * kMaxRecs * 8;
 };
 
 __device__ __forceinline__ uint32_t sw_addr(uint32_t box, int row, int chunk) {
@@ -325,43 +392,41 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__global__ void __launch_bounds__(96, 1)
-decode_mma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                  const __grid_constant__ DecMmaArgs args) {
+__global__ void __launch_bounds__(kFlatThreads, 1)
+decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const __grid_constant__ DecArgs a) {
     constexpr int D = 128, BS = 64;
-    const DecArgs& a = args.d;
+    using L = FlatSmem;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
-    uint64_t* full = reinterpret_cast<uint64_t*>(sm + kMmaStages * kMmaStage);
-    uint64_t* empty = full + kMmaStages;
-    float* xch = reinterpret_cast<float*>(empty + kMmaStages);   // consumer 1's m[8], l[8], O^T[128][8]
+    uint64_t* full = reinterpret_cast<uint64_t*>(sm + L::kBar);
+    uint64_t* empty = full + kFlatStages;
+    volatile int* abort = reinterpret_cast<volatile int*>(sm + L::kMisc);
+    int* s_ntok = reinterpret_cast<int*>(sm + L::kBlk);
+    float* s_lg = reinterpret_cast<float*>(sm + L::kLg);
+    float* xch = reinterpret_cast<float*>(sm + L::kXch);
+    volatile int* s_last = reinterpret_cast<volatile int*>(sm + L::kLast);
+    float* s_mg = reinterpret_cast<float*>(sm + L::kMerge);
+    float* s_lg2 = s_mg + kMaxRecs * 8;
+    float* s_wg = s_lg2 + kMaxRecs * 8;
 
     const Shape& sh = a.sh;
+    const FlatPlan& fp = a.fp;
     const int G = sh.G;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int split = blockIdx.x % a.splits;
-    const int64_t bg = blockIdx.x / a.splits;
-    const int b = (int)(bg / sh.Hkv), g = (int)(bg % sh.Hkv);
-    const int64_t N = (int64_t)sh.q_offset + 1;
-    const int C = (int)(sh.q_offset / BS);
+    const int64_t cta = blockIdx.x;
+    const int64_t i0 = flat_start(fp, cta), i1 = flat_start(fp, cta + 1);
+    const int nitems = (int)(i1 - i0);
+    const int64_t N = (int64_t)sh.q_offset + 1;       // the longest cache length
     const bool dense = a.idx == nullptr;
-    const int n = dense ? C : a.nsel[bg];
-    const int nblk = n + 1;
-    const int p0 = split * a.bpc;
-    const int cnt = max(min(p0 + a.bpc, nblk) - p0, 0);
-    auto block_of = [&](int pos) -> int {
-        if (dense) return pos;
-        if (pos >= n) return C;
-        const int j = a.idx[bg * sh.K + pos];
-        return ((unsigned)j < (unsigned)C) ? j : -1;
-    };
-    auto ntok_of = [&](int j) -> int { return j < 0 ? 0 : (j == C ? (int)(N - (int64_t)C * BS) : BS); };
+    const int nblk = fp.nblk;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kMmaStages; ++s) {
+        for (int s = 0; s < kFlatStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
+        *abort = 0;
         fence_mbar_init();
     }
     __syncthreads();
@@ -369,201 +434,332 @@ decode_mma_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     if (warp == 0) {
         // ---- producer ----
         if (lane == 0) {
-            for (int i = 0; i < cnt; ++i) {
-                const int s = i % kMmaStages;
-                if (i >= kMmaStages && !mbar_wait_bounded(&empty[s], (uint32_t)(((i / kMmaStages) - 1) & 1))) break;
-                const int j = block_of(p0 + i);
-                if (j < 0) {
-                    tc::mbar_arrive(&full[s]);
-                    continue;
+            tc::prefetch_tmap(&tm_k);
+            tc::prefetch_tmap(&tm_v);
+        }
+        int issued = 0;
+        bool stop = false;
+        for (int base = 0; base < nitems && !stop; base += 32) {
+            // lane l resolves item base + l: its block (-1: empty) and log-gate
+            // lane l resolves item base + l: its keys (0: nothing to load), its
+            // log-gate and the first cache row of its block
+            int ntl = 0, rowl = 0;
+            float lgl = 0.f;
+            if (base + lane < nitems) {
+                const int64_t i = i0 + base + lane;
+                const int64_t bg = i / nblk;
+                const int p = (int)(i - bg * nblk);
+                const int b = (int)(bg / sh.Hkv), g = (int)(bg - (int64_t)b * sh.Hkv);
+                const int64_t Nb = a.lens == nullptr ? N : min(max((int64_t)a.lens[b], (int64_t)1), N);
+                const int Cb = (int)((Nb - 1) / BS);   // this sequence's current block
+                int j = -1;
+                if (dense) {
+                    j = p <= Cb ? p : -1;
+                } else if (p == nblk - 1) {
+                    j = Cb;
+                } else if (p < min(max(a.nsel[bg], 0), min(sh.K, Cb))) {   // a count outside [0, min(K, C)] is clamped
+                    const int jj = a.idx[bg * sh.K + p];
+                    if ((unsigned)jj < (unsigned)Cb) {
+                        j = jj;
+                        lgl = a.gl[bg * sh.K + p] * kLog2e;
+                    }
                 }
-                mbar_arrive_expect_tx(&full[s], kMmaStage);
-                const int row = (int)(bg * a.stride + (int64_t)j * BS);
-                unsigned char* st = sm + s * kMmaStage;
-                tc::tma_load_2d(st, &tm_k, 0, row, &full[s]);
-                tc::tma_load_2d(st + 8192, &tm_k, 64, row, &full[s]);
-                tc::tma_load_2d(st + 16384, &tm_v, 0, row, &full[s]);
-                tc::tma_load_2d(st + 24576, &tm_v, 64, row, &full[s]);
+                if (j >= 0) {
+                    if (a.table == nullptr) {
+                        ntl = j == Cb ? (int)(Nb - (int64_t)Cb * BS) : BS;
+                        rowl = (int)(bg * a.stride + (int64_t)j * BS);
+                    } else {
+                        const int page = a.table[(int64_t)b * a.max_blocks + j];
+                        if ((unsigned)page < (unsigned)a.num_pages) {   // an invalid page is skipped
+                            ntl = j == Cb ? (int)(Nb - (int64_t)Cb * BS) : BS;
+                            rowl = (page * sh.Hkv + g) * BS;
+                        }
+                    }
+                }
             }
+            const int cnt = min(32, nitems - base);
+            for (int k = 0; k < cnt; ++k) {
+                const int li = base + k;
+                const int nt = __shfl_sync(0xffffffffu, ntl, k);
+                const int row = __shfl_sync(0xffffffffu, rowl, k);
+                const float lg = __shfl_sync(0xffffffffu, lgl, k);
+                int fail = 0;
+                if (lane == 0) {
+                    const int s = li % kFlatStages;
+                    if (li >= kFlatStages && !tc::wait_bar(&empty[s], (uint32_t)(((li / kFlatStages) - 1) & 1), abort)) {
+                        fail = 1;
+                    } else {
+                        s_ntok[s] = nt;
+                        s_lg[s] = lg;
+                        if (nt == 0) {
+                            tc::mbar_arrive(&full[s]);
+                        } else {
+                            mbar_arrive_expect_tx(&full[s], kItemBytes);
+                            unsigned char* st = sm + s * kItemBytes;
+                            tc::tma_load_2d(st, &tm_k, 0, row, &full[s]);
+                            tc::tma_load_2d(st + 8192, &tm_k, 64, row, &full[s]);
+                            tc::tma_load_2d(st + 16384, &tm_v, 0, row, &full[s]);
+                            tc::tma_load_2d(st + 24576, &tm_v, 64, row, &full[s]);
+                        }
+                        ++issued;
+                    }
+                }
+                if (__shfl_sync(0xffffffffu, fail, 0)) { stop = true; break; }
+            }
+        }
+        if (lane == 0 && stop) {
+            // let the copies already started land before the CTA exits
+            for (int li = max(0, issued - kFlatStages); li < issued; ++li)
+                tc::drain_wait(&full[li % kFlatStages], (uint32_t)((li / kFlatStages) & 1));
         }
         return;
     }
 
-    // ---- consumers: warp 1 takes blocks 0, 2, ...; warp 2 blocks 1, 3, ... ----
+    // ---- consumers: warp 1 + c takes the CTA-local items c, c + kCons, ... ----
     const int cw = warp - 1;
     const int gq = lane >> 2, tq = lane & 3;
     const float qk = sh.scale * kLog2e;
-    // q^T as the B operand: b0 = q[head gq][16 ks + 2 tq, +1], b1 = the same + 8
-    uint32_t qb[8][2];
-    {
-        const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q) + ((int64_t)b * sh.Hq + (int64_t)g * G) * D;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            if (gq < G) {
-                qb[ks][0] = *reinterpret_cast<const uint32_t*>(qg + gq * D + 16 * ks + 2 * tq);
-                qb[ks][1] = *reinterpret_cast<const uint32_t*>(qg + gq * D + 16 * ks + 2 * tq + 8);
-            } else {
-                qb[ks][0] = qb[ks][1] = 0u;
-            }
-        }
-    }
-    float o[8][4];          // O^T: m-tile of 16 dims, (dim gq | gq+8) x (heads 2tq, 2tq+1)
-#pragma unroll
-    for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[mt][e] = 0.f;
-    float mrun[2] = {-INFINITY, -INFINITY}, lrun[2] = {0.f, 0.f};   // heads 2tq, 2tq+1
-
     const uint32_t sbase = smem_u32(sm);
     bool ok = true;
-    for (int i = cw; i < cnt; i += 2) {
-        const int s = i % kMmaStages;
-        if (!mbar_wait_bounded(&full[s], (uint32_t)((i / kMmaStages) & 1))) { ok = false; break; }
-        const int j = block_of(p0 + i);
-        const int ntok = ntok_of(j);
-        if (ntok > 0) {
-            const uint32_t kb0 = sbase + s * kMmaStage, kb1 = kb0 + 8192, vb0 = kb0 + 16384, vb1 = kb0 + 24576;
-            if (ntok < BS) {   // the current block: clear V rows >= ntok (128 bytes per row and box)
-                unsigned char* v0p = sm + s * kMmaStage + 16384;
-                for (int e = ntok * 8 + lane; e < BS * 8; e += 32) {
-                    reinterpret_cast<uint4*>(v0p)[e] = make_uint4(0, 0, 0, 0);
-                    reinterpret_cast<uint4*>(v0p + 8192)[e] = make_uint4(0, 0, 0, 0);
-                }
-                __syncwarp();
-            }
-            const float lg = (!dense && p0 + i < n) ? a.gl[bg * sh.K + p0 + i] * kLog2e : 0.f;
-            // ---- S^T = K q^T ----
-            float sc[4][4];
+    for (int64_t seg = i0; seg < i1;) {
+        const int64_t bg = seg / nblk;
+        const int64_t seg_end = min(i1, (bg + 1) * nblk);
+        const int b = (int)(bg / sh.Hkv), g = (int)(bg % sh.Hkv);
+        // q^T as the B operand: b0 = q[head gq][16 ks + 2 tq, +1], b1 = the same + 8
+        uint32_t qb[8][2];
+        {
+            const __nv_bfloat16* qg = static_cast<const __nv_bfloat16*>(a.q) + ((int64_t)b * sh.Hq + (int64_t)g * G) * D;
 #pragma unroll
-            for (int mt = 0; mt < 4; ++mt) {
-#pragma unroll
-                for (int e = 0; e < 4; ++e) sc[mt][e] = 0.f;
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    // matrices: (keys +0..7, dims +0..7), (keys +8..15, dims +0..7), (keys +0..7, dims +8..15), (keys +8.., dims +8..)
-                    const int key = 16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8;
-                    const int chunk = 2 * ks + (lane >> 4);
-                    const uint32_t addr = sw_addr(chunk < 8 ? kb0 : kb1, key, chunk & 7);
-                    uint32_t a0, a1, a2, a3;
-                    ldsm_x4(addr, a0, a1, a2, a3);
-                    mma_bf16(sc[mt], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
-                }
-            }
-            // ---- online softmax (heads 2tq, 2tq+1; keys 16 mt + gq (+8)) ----
-            float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-            for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int key = 16 * mt + gq + (e >> 1) * 8;
-                    const float v = key < ntok ? fmaf(sc[mt][e], qk, lg) : -INFINITY;
-                    sc[mt][e] = v;
-                    mx[e & 1] = fmaxf(mx[e & 1], v);
-                }
-            float corr[2], psum[2] = {0.f, 0.f};
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 4));
-                mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 8));
-                mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 16));
-                const float mn = fmaxf(mrun[h], mx[h]);
-                corr[h] = mrun[h] == -INFINITY ? 0.f : exp2f(mrun[h] - mn);
-                mrun[h] = mn;
-            }
-            uint32_t pb[4][2];   // P^T as B operand per k-step (16 keys)
-#pragma unroll
-            for (int mt = 0; mt < 4; ++mt) {
-                float p[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float m = mrun[e & 1];
-                    p[e] = m == -INFINITY ? 0.f : exp2f(sc[mt][e] - m);
-                    psum[e & 1] += p[e];
-                }
-                pb[mt][0] = movm_t(pack_bf16(p[0], p[1]));   // keys 16 mt + 0..7
-                pb[mt][1] = movm_t(pack_bf16(p[2], p[3]));   // keys 16 mt + 8..15
-            }
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                psum[h] += __shfl_xor_sync(0xffffffffu, psum[h], 4);
-                psum[h] += __shfl_xor_sync(0xffffffffu, psum[h], 8);
-                psum[h] += __shfl_xor_sync(0xffffffffu, psum[h], 16);
-                lrun[h] = lrun[h] * corr[h] + psum[h];
-            }
-#pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {
-                o[mt][0] *= corr[0];
-                o[mt][1] *= corr[1];
-                o[mt][2] *= corr[0];
-                o[mt][3] *= corr[1];
-            }
-            // ---- O^T += V^T P^T ----
-#pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {        // dims 16 mt .. + 15
-#pragma unroll
-                for (int kst = 0; kst < 4; ++kst) { // keys 16 kst .. + 15
-                    // matrices (transposed on load): (keys +0..7, dims +0..7), (keys +0..7, dims +8..15),
-                    // (keys +8..15, dims +0..7), (keys +8..15, dims +8..15)
-                    const int key = 16 * kst + (lane & 7) + (lane >> 4) * 8;
-                    const int chunk = 2 * mt + ((lane >> 3) & 1);
-                    const uint32_t addr = sw_addr(chunk < 8 ? vb0 : vb1, key, chunk & 7);
-                    uint32_t a0, a1, a2, a3;
-                    ldsm_x4_t(addr, a0, a1, a2, a3);
-                    mma_bf16(o[mt], a0, a1, a2, a3, pb[kst][0], pb[kst][1]);
+            for (int ks = 0; ks < 8; ++ks) {
+                if (gq < G) {
+                    qb[ks][0] = *reinterpret_cast<const uint32_t*>(qg + gq * D + 16 * ks + 2 * tq);
+                    qb[ks][1] = *reinterpret_cast<const uint32_t*>(qg + gq * D + 16 * ks + 2 * tq + 8);
+                } else {
+                    qb[ks][0] = qb[ks][1] = 0u;
                 }
             }
         }
-        tc::fence_async_shared();   // the zeroed rows are rewritten by TMA next
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&empty[s]);
-    }
+        float o[8][4];          // O^T: m-tile of 16 dims, (dim gq | gq+8) x (heads 2tq, 2tq+1)
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[mt][e] = 0.f;
+        float mrun[2] = {-INFINITY, -INFINITY}, lrun[2] = {0.f, 0.f};   // heads 2tq, 2tq+1
 
-    // ---- merge the two consumers; consumer 0 writes the CTA's partial ----
-    float* rec = a.part + (bg * a.splits + split) * (int64_t)G * (D + 2);
-    if (cw == 1) {
-        if (gq == 0) {
+        for (int64_t i = seg + (cw - (int)((seg - i0) % kCons) + kCons) % kCons; i < seg_end; i += kCons) {
+            const int li = (int)(i - i0);
+            const int s = li % kFlatStages;
+            if (ok && !tc::warp_wait_bar(&full[s], (uint32_t)((li / kFlatStages) & 1), abort)) ok = false;
+            const int ntok = ok ? s_ntok[s] : 0;
+            if (ntok > 0) {
+                const uint32_t kb0 = sbase + s * kItemBytes, kb1 = kb0 + 8192, vb0 = kb0 + 16384, vb1 = kb0 + 24576;
+                if (ntok < BS) {   // the current block: clear V rows >= ntok (128 bytes per row and box)
+                    unsigned char* v0p = sm + s * kItemBytes + 16384;
+                    for (int e = ntok * 8 + lane; e < BS * 8; e += 32) {
+                        reinterpret_cast<uint4*>(v0p)[e] = make_uint4(0, 0, 0, 0);
+                        reinterpret_cast<uint4*>(v0p + 8192)[e] = make_uint4(0, 0, 0, 0);
+                    }
+                    __syncwarp();
+                }
+                const float lg = s_lg[s];
+                // ---- S^T = K q^T ----
+                float sc[4][4];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) { xch[2 * tq + h] = mrun[h]; xch[8 + 2 * tq + h] = lrun[h]; }
-        }
+                for (int mt = 0; mt < 4; ++mt) {
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt)
+                    for (int e = 0; e < 4; ++e) sc[mt][e] = 0.f;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int dim = 16 * mt + gq + (e >> 1) * 8, h = 2 * tq + (e & 1);
-                xch[16 + dim * 8 + h] = o[mt][e];
-            }
-    }
-    asm volatile("bar.sync 1, 64;" ::: "memory");
-    if (cw == 0) {
-        float m2[2], l2[2], w1[2], w2[2];
+                    for (int ks = 0; ks < 8; ++ks) {
+                        // matrices: (keys +0..7, dims +0..7), (keys +8..15, dims +0..7), (keys +0..7, dims +8..15), (keys +8.., dims +8..)
+                        const int key = 16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8;
+                        const int chunk = 2 * ks + (lane >> 4);
+                        const uint32_t addr = sw_addr(chunk < 8 ? kb0 : kb1, key, chunk & 7);
+                        uint32_t a0, a1, a2, a3;
+                        ldsm_x4(addr, a0, a1, a2, a3);
+                        mma_bf16(sc[mt], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+                    }
+                }
+                // ---- online softmax (heads 2tq, 2tq+1; keys 16 mt + gq (+8)) ----
+                float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            m2[h] = xch[2 * tq + h];
-            l2[h] = xch[8 + 2 * tq + h];
-            const float M = fmaxf(mrun[h], m2[h]);
-            w1[h] = mrun[h] == -INFINITY ? 0.f : exp2f(mrun[h] - M);
-            w2[h] = m2[h] == -INFINITY ? 0.f : exp2f(m2[h] - M);
-            mrun[h] = M;
-            lrun[h] = lrun[h] * w1[h] + l2[h] * w2[h];
-        }
+                for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
-        for (int mt = 0; mt < 8; ++mt)
+                    for (int e = 0; e < 4; ++e) {
+                        const int key = 16 * mt + gq + (e >> 1) * 8;
+                        const float v = key < ntok ? fmaf(sc[mt][e], qk, lg) : -INFINITY;
+                        sc[mt][e] = v;
+                        mx[e & 1] = fmaxf(mx[e & 1], v);
+                    }
+                float corr[2], psum[2] = {0.f, 0.f};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int dim = 16 * mt + gq + (e >> 1) * 8, h = 2 * tq + (e & 1);
-                const float v = o[mt][e] * w1[e & 1] + xch[16 + dim * 8 + h] * w2[e & 1];
-                if (h < G) rec[h * (D + 2) + dim] = ok ? v : __int_as_float(0x7fc00000);
-            }
-        if (gq == 0) {
+                for (int h = 0; h < 2; ++h) {
+                    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 4));
+                    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 8));
+                    mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 16));
+                    const float mn = fmaxf(mrun[h], mx[h]);
+                    corr[h] = mrun[h] == -INFINITY ? 0.f : exp2f(mrun[h] - mn);
+                    mrun[h] = mn;
+                }
+                uint32_t pb[4][2];   // P^T as B operand per k-step (16 keys)
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int hh = 2 * tq + h;
-                if (hh < G) {
-                    rec[hh * (D + 2) + D] = mrun[h];
-                    rec[hh * (D + 2) + D + 1] = lrun[h];
+                for (int mt = 0; mt < 4; ++mt) {
+                    float p[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float m = mrun[e & 1];
+                        p[e] = m == -INFINITY ? 0.f : exp2f(sc[mt][e] - m);
+                        psum[e & 1] += p[e];
+                    }
+                    pb[mt][0] = movm_t(pack_bf16(p[0], p[1]));   // keys 16 mt + 0..7
+                    pb[mt][1] = movm_t(pack_bf16(p[2], p[3]));   // keys 16 mt + 8..15
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    psum[h] += __shfl_xor_sync(0xffffffffu, psum[h], 4);
+                    psum[h] += __shfl_xor_sync(0xffffffffu, psum[h], 8);
+                    psum[h] += __shfl_xor_sync(0xffffffffu, psum[h], 16);
+                    lrun[h] = lrun[h] * corr[h] + psum[h];
+                }
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt) {
+                    o[mt][0] *= corr[0];
+                    o[mt][1] *= corr[1];
+                    o[mt][2] *= corr[0];
+                    o[mt][3] *= corr[1];
+                }
+                // ---- O^T += V^T P^T ----
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt) {        // dims 16 mt .. + 15
+#pragma unroll
+                    for (int kst = 0; kst < 4; ++kst) { // keys 16 kst .. + 15
+                        // matrices (transposed on load): (keys +0..7, dims +0..7), (keys +0..7, dims +8..15),
+                        // (keys +8..15, dims +0..7), (keys +8..15, dims +8..15)
+                        const int key = 16 * kst + (lane & 7) + (lane >> 4) * 8;
+                        const int chunk = 2 * mt + ((lane >> 3) & 1);
+                        const uint32_t addr = sw_addr(chunk < 8 ? vb0 : vb1, key, chunk & 7);
+                        uint32_t a0, a1, a2, a3;
+                        ldsm_x4_t(addr, a0, a1, a2, a3);
+                        mma_bf16(o[mt], a0, a1, a2, a3, pb[kst][0], pb[kst][1]);
+                    }
                 }
             }
+            tc::fence_async_shared();   // zeroed rows are rewritten by TMA next
+            __syncwarp();
+            // a stage is handed back only once its copy has landed: after a wait
+            // gave up, the producer never reuses a stage with a copy in flight
+            if (ok && lane == 0) tc::mbar_arrive(&empty[s]);
         }
+
+        // ---- merge the consumers; consumer 0 writes the CTA's record of group bg ----
+        if (cw > 0) {
+            float* x = xch + (cw - 1) * (16 + 128 * 8);
+            if (gq == 0) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) { x[2 * tq + h] = mrun[h]; x[8 + 2 * tq + h] = lrun[h]; }
+            }
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int dim = 16 * mt + gq + (e >> 1) * 8, h = 2 * tq + (e & 1);
+                    x[16 + dim * 8 + h] = o[mt][e];
+                }
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * kCons) : "memory");
+        if (cw == 0) {
+            const bool good = ok && !*abort;
+            float* rec = a.part + (cta + bg) * (int64_t)G * kRecF;
+            for (int c = 0; c < kCons - 1; ++c) {
+                const float* x = xch + c * (16 + 128 * 8);
+                float w1[2], w2[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const float m2 = x[2 * tq + h], l2 = x[8 + 2 * tq + h];
+                    const float M = fmaxf(mrun[h], m2);
+                    w1[h] = mrun[h] == -INFINITY ? 0.f : exp2f(mrun[h] - M);
+                    w2[h] = m2 == -INFINITY ? 0.f : exp2f(m2 - M);
+                    mrun[h] = M;
+                    lrun[h] = lrun[h] * w1[h] + l2 * w2[h];
+                }
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int dim = 16 * mt + gq + (e >> 1) * 8, h = 2 * tq + (e & 1);
+                        o[mt][e] = o[mt][e] * w1[e & 1] + x[16 + dim * 8 + h] * w2[e & 1];
+                    }
+            }
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int dim = 16 * mt + gq + (e >> 1) * 8, h = 2 * tq + (e & 1);
+                    if (h < G) rec[h * kRecF + dim] = good ? o[mt][e] : __int_as_float(0x7fc00000);
+                }
+            if (gq == 0) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int hh = 2 * tq + h;
+                    if (hh < G) {
+                        rec[hh * kRecF + D] = mrun[h];
+                        rec[hh * kRecF + D + 1] = lrun[h];
+                    }
+                }
+            }
+            // the last CTA of the group to get here merges its records
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) {
+                const int64_t c_first = flat_owner(fp, bg * nblk), c_last = flat_owner(fp, (bg + 1) * nblk - 1);
+                *s_last = atomicAdd(&a.fin[bg], 1) == (int)(c_last - c_first);
+            }
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * kCons) : "memory");   // xch is free; s_last is set
+        if (*s_last) {
+            // Both consumer warps merge the group's records:
+            //   o = sum_r 2^(m_r - M) O_r / sum_r 2^(m_r - M) l_r,  M = max_r m_r,
+            // staging every record's (m, l) first so that all loads are in flight together.
+            __threadfence();
+            const int t = threadIdx.x - 32;                 // 0 .. 32 kCons - 1
+            const int64_t c_first = flat_owner(fp, bg * nblk), c_last = flat_owner(fp, (bg + 1) * nblk - 1);
+            const int R = (int)(c_last - c_first + 1);      // <= kMaxRecs by the plan
+            const float* base = a.part + (c_first + bg) * (int64_t)G * kRecF;   // records are consecutive
+            for (int e = t; e < R * G; e += 32 * kCons) {
+                s_mg[e] = __ldcg(base + (int64_t)e * kRecF + D);
+                s_lg2[e] = __ldcg(base + (int64_t)e * kRecF + D + 1);
+            }
+            asm volatile("bar.sync 1, %0;" ::"n"(32 * kCons) : "memory");
+            if (t < G) {
+                float M = -INFINITY, Lsum = 0.f;
+                for (int r = 0; r < R; ++r) M = fmaxf(M, s_mg[r * G + t]);
+                for (int r = 0; r < R; ++r) {
+                    const float mr = s_mg[r * G + t];
+                    const float w = mr == -INFINITY ? 0.f : exp2f(mr - M);
+                    s_wg[r * G + t] = w;
+                    Lsum = fmaf(w, s_lg2[r * G + t], Lsum);
+                }
+                const float inv = 1.f / Lsum;
+                for (int r = 0; r < R; ++r) s_wg[r * G + t] *= inv;
+            }
+            asm volatile("bar.sync 1, %0;" ::"n"(32 * kCons) : "memory");
+            __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.o) + ((int64_t)b * sh.Hq + (int64_t)g * G) * D;
+            for (int e = t; e < G * (D / 4); e += 32 * kCons) {
+                const int h = e / (D / 4), q4 = e - h * (D / 4);
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+                for (int r = 0; r < R; ++r) {
+                    const float w = s_wg[r * G + h];
+                    const float4 v = __ldcg(reinterpret_cast<const float4*>(base + ((int64_t)r * G + h) * kRecF) + q4);
+                    acc.x = fmaf(w, v.x, acc.x);
+                    acc.y = fmaf(w, v.y, acc.y);
+                    acc.z = fmaf(w, v.z, acc.z);
+                    acc.w = fmaf(w, v.w, acc.w);
+                }
+                reinterpret_cast<uint2*>(ob + (int64_t)h * D)[q4] =
+                    make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
+            }
+        }
+        seg = seg_end;
     }
 }
 
@@ -634,26 +830,30 @@ cudaError_t run_decode(const DecArgs& a, cudaStream_t st) {
     return e;
 }
 
-cudaError_t run_decode_mma(const DecArgs& a, cudaStream_t st) {
+// SMs of the current device (148 on B200), bounded by kMaxDecodeCtas; 148 if
+// the query fails.
+int decode_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) !=
+                                                  cudaSuccess || n <= 0)
+        n = 148;
+    return std::min(n, kMaxDecodeCtas);
+}
+
+cudaError_t run_decode_flat(const DecArgs& a, cudaStream_t st) {
     CUtensorMap mk, mv;
-    const uint64_t rows = (uint64_t)a.sh.B * a.sh.Hkv * (uint64_t)a.stride;
+    const uint64_t rows = a.table == nullptr ? (uint64_t)a.sh.B * a.sh.Hkv * (uint64_t)a.stride
+                                             : (uint64_t)a.num_pages * a.sh.Hkv * 64;
     if (!encode_bf16_2d(&mk, a.kc, rows, 128, 64) || !encode_bf16_2d(&mv, a.vc, rows, 128, 64))
         return cudaErrorInvalidValue;
-    const size_t smem = (size_t)kMmaStages * kMmaStage + 2 * kMmaStages * 8 + sizeof(float) * (16 + 128 * 8) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(decode_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const size_t smem = FlatSmem::kTotal + 1024;
+    cudaError_t e = cudaFuncSetAttribute(decode_flat_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int64_t grid = (int64_t)a.sh.B * a.sh.Hkv * a.splits;
-    {
-        KernelTimer kt("decode_partial", st);
-        decode_mma_kernel<<<(unsigned)grid, 96, smem, st>>>(mk, mv, DecMmaArgs{a});
-    }
-    e = cudaGetLastError();
+    e = cudaMemsetAsync(a.fin, 0, sizeof(int) * (size_t)a.sh.B * a.sh.Hkv, st);
     if (e != cudaSuccess) return e;
-    count_launches(1);
     {
-        KernelTimer kt("decode_combine", st);
-        decode_combine_kernel<__nv_bfloat16, 128><<<(unsigned)(a.sh.B * a.sh.Hkv * a.sh.G), 128, 0, st>>>(
-            a.sh, a.part, a.splits, static_cast<__nv_bfloat16*>(a.o));
+        KernelTimer kt("decode_flat", st);
+        decode_flat_kernel<<<(unsigned)a.fp.ncta, kFlatThreads, smem, st>>>(mk, mv, a);
     }
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
@@ -678,25 +878,40 @@ cudaError_t decode_d(const DecArgs& a, cudaStream_t st) {
 
 }  // namespace
 
-static bool decode_mma_supported(const Shape& s) {
-    return s.dtype == SAS_DT_BF16 && s.D == 128 && s.bs == 64 && s.G <= 8;
+// The tensor-core path (bf16, d 128, block 64, G <= 8) with TMA row
+// coordinates that fit in int32.
+static bool decode_flat_supported(const Shape& s, int64_t stride) {
+    return s.dtype == SAS_DT_BF16 && s.D == 128 && s.bs == 64 && s.G <= 8 &&
+           (int64_t)s.B * s.Hkv * stride <= (int64_t)INT32_MAX;
 }
 
+static FlatPlan flat_plan(const Shape& s, bool dense) {
+    const int64_t C = s.q_offset / s.bs;
+    FlatPlan f;
+    f.nblk = (int)(dense ? C + 1 : std::min<int64_t>(s.K, C) + 1);
+    f.W = (int64_t)s.B * s.Hkv * f.nblk;
+    // each CTA takes >= kCons items (one per consumer warp; few records per
+    // group), and a group spans at most kMaxRecs CTAs:
+    // ceil(nblk / per) + 1 <= kMaxRecs
+    const int64_t min_per = std::max<int64_t>(kCons, (f.nblk + kMaxRecs - 3) / (kMaxRecs - 2));
+    f.ncta = (int)std::max<int64_t>(1, std::min<int64_t>(decode_sms(), f.W / min_per));
+    f.per = f.W / f.ncta;
+    f.rem = f.W % f.ncta;
+    return f;
+}
+
+// Records of the tensor-core path: at most one per (CTA, group it touches),
+// i.e. ncta - 1 + groups, numbered c + bg; then the per-group counters.
+static size_t flat_record_bytes(const Shape& s) {
+    const size_t recs = (size_t)kMaxDecodeCtas + (size_t)s.B * s.Hkv;
+    return (sizeof(float) * recs * s.G * kRecF + 255) & ~(size_t)255;
+}
+
+// CUDA-core path: `splits` CTAs of `bpc` blocks per (b, kv head), merged by a
+// second kernel.
 DecodePlan decode_plan(const Shape& s, bool dense) {
     DecodePlan p;
     const int64_t C = s.q_offset / s.bs;
-    if (decode_mma_supported(s)) {
-        // one CTA per SM (128 KiB of stages); two blocks per CTA for a
-        // selection, one wave of CTAs over every block for dense
-        const int64_t nblk = dense ? C + 1 : (int64_t)s.K + 1;
-        const int64_t groups = (int64_t)s.B * s.Hkv;
-        int64_t bpc = dense ? (groups * nblk + 147) / 148 : 2;
-        bpc = std::max<int64_t>(bpc, (nblk + kMaxSplits - 1) / kMaxSplits);
-        bpc = std::max<int64_t>(1, bpc);
-        p.bpc = (int)bpc;
-        p.splits = (int)((nblk + bpc - 1) / bpc);
-        return p;
-    }
     if (!dense) {
         p.bpc = 1;
         p.splits = s.K + 1;
@@ -716,11 +931,37 @@ DecodePlan decode_plan(const Shape& s, bool dense) {
 cudaError_t launch_decode(const Shape& s, const void* q, const void* kc, const void* vc, int64_t stride,
                           const int32_t* idx, const float* gl, const int32_t* nsel, void* o, float* part,
                           cudaStream_t st) {
-    const DecodePlan p = decode_plan(s, idx == nullptr);
-    DecArgs a{s, q, kc, vc, stride, idx, gl, nsel, part, o, p.bpc, p.splits};
-    if (decode_mma_supported(s)) return run_decode_mma(a, st);
+    const bool dense = idx == nullptr;
+    if (decode_flat_supported(s, stride)) {
+        DecArgs a{s, q, kc, vc, stride, idx, gl, nsel, part, o, 0, 0, flat_plan(s, dense), nullptr,
+                  nullptr, 0, 0, nullptr};
+        a.fin = reinterpret_cast<int*>(reinterpret_cast<unsigned char*>(part) + flat_record_bytes(s));
+        return run_decode_flat(a, st);
+    }
+    const DecodePlan p = decode_plan(s, dense);
+    DecArgs a{s, q, kc, vc, stride, idx, gl, nsel, part, o, p.bpc, p.splits, FlatPlan{}, nullptr,
+              nullptr, 0, 0, nullptr};
     if (s.dtype == SAS_DT_FP32) return decode_d<float>(a, st);
     return decode_d<__nv_bfloat16>(a, st);
+}
+
+cudaError_t set_decode_wait_limit(unsigned long long ns) {
+    return cudaMemcpyToSymbol(g_sas_wait_limit_ns, &ns, sizeof(ns));
+}
+
+bool decode_paged_supported(const Shape& s, int64_t num_pages) {
+    return s.dtype == SAS_DT_BF16 && s.D == 128 && s.bs == 64 && s.G <= 8 && num_pages >= 1 &&
+           num_pages * s.Hkv * 64 <= (int64_t)INT32_MAX;
+}
+
+cudaError_t launch_decode_paged(const Shape& s, const void* q, const void* kp, const void* vp, int num_pages,
+                                const int32_t* table, int max_blocks, const int32_t* lens, const int32_t* idx,
+                                const float* gl, const int32_t* nsel, void* o, float* part, cudaStream_t st) {
+    const bool dense = idx == nullptr;
+    DecArgs a{s, q, kp, vp, 0, idx, gl, nsel, part, o, 0, 0, flat_plan(s, dense), nullptr,
+              table, max_blocks, num_pages, lens};
+    a.fin = reinterpret_cast<int*>(reinterpret_cast<unsigned char*>(part) + flat_record_bytes(s));
+    return run_decode_flat(a, st);
 }
 
 cudaError_t read_decode_timeouts(unsigned int* out) {
@@ -728,9 +969,12 @@ cudaError_t read_decode_timeouts(unsigned int* out) {
 }
 
 size_t decode_ws_bytes(const Shape& s) {
+    // covers both layouts (the cache stride, which picks the path, is not known here)
     const DecodePlan a = decode_plan(s, false), b = decode_plan(s, true);
     const int64_t splits = std::max(a.splits, b.splits);
-    return sizeof(float) * (size_t)s.B * s.Hkv * splits * s.G * (s.D + 2);
+    const size_t simt = sizeof(float) * (size_t)s.B * s.Hkv * splits * s.G * (s.D + 2);
+    const size_t flat = flat_record_bytes(s) + sizeof(int) * (size_t)s.B * s.Hkv;
+    return std::max(simt, flat);
 }
 
 }  // namespace sas
@@ -783,13 +1027,11 @@ extern "C" sas_status sas_sparse_decode_noalloc(const sas_desc* desc, const void
     Shape s;
     sas_status st = check_decode_args(desc, q, k_cache, v_cache, cache_stride_tokens, idx, gate_logit, n_sel, o, &s);
     if (st != SAS_OK) return st;
-    const DecodePlan p = decode_plan(s, idx == nullptr);
-    const size_t need = sizeof(float) * (size_t)s.B * s.Hkv * p.splits * s.G * (s.D + 2);
-    if (need > (size_t)SAS_NOALLOC_SCRATCH_BYTES) return SAS_ERR_WORKSPACE;
+    if (decode_ws_bytes(s) > (size_t)SAS_NOALLOC_SCRATCH_BYTES) return SAS_ERR_WORKSPACE;
     float* part = nullptr;
     if (noalloc_scratch(&part) != cudaSuccess) return SAS_ERR_CUDA;
-    // Every split record is written before the merge reads it, so nothing in
-    // the shared array has to start at zero.
+    // Every split record is written before the merge reads it; the per-group
+    // counters that pick the merging CTA are zeroed by the call itself.
     const cudaError_t e = launch_decode(s, q, k_cache, v_cache, cache_stride_tokens, idx, gate_logit, n_sel, o,
                                         part, (cudaStream_t)stream);
     return e == cudaSuccess ? SAS_OK : SAS_ERR_CUDA;

@@ -39,9 +39,11 @@ struct Shape {
     __host__ __device__ int64_t rows() const { return (int64_t)B * Hkv * T; }
 };
 
-// K1: gate normaliser + hard top-K for every (b, kv head, t) row.
-cudaError_t launch_block_topk(const Shape& s, const float* scores, int32_t* idx, float* gate_logit,
-                              float* score_lse, int32_t* n_sel, cudaStream_t st);
+// K1: gate normaliser + hard top-K for every (b, kv head, t) row. `lens`
+// (device, may be NULL): per-sequence cache lengths of decode rows (T = 1);
+// row (b, g) then has floor((lens[b] - 1) / bs) candidates.
+cudaError_t launch_block_topk(const Shape& s, const float* scores, const int32_t* lens, int32_t* idx,
+                              float* gate_logit, float* score_lse, int32_t* n_sel, cudaStream_t st);
 bool topk_row_supported(int64_t max_candidates);
 
 // K1b: column-major selection bitmap maskT[b, g, j, tau] (bit r: query
@@ -90,7 +92,7 @@ size_t bwd_tc_ws_bytes(const Shape& s);
 cudaError_t launch_bwd_tc(const Shape& s, const void* q, const void* k, const void* v, const void* dO,
                           const float* attn_lse, const float* Dd, const int32_t* idx, const float* gate_logit,
                           const int32_t* n_sel, const uint64_t* maskT, void* ws, float* dq_acc, void* dk, void* dv,
-                          float* gsum, cudaStream_t st);
+                          float* gsum, int* aborted, cudaStream_t st);
 
 // Tensor-core forward over gathered rows (two passes + finalize): bf16, d = 128, block 64.
 bool fwd_rows_supported(const Shape& s);
@@ -98,11 +100,6 @@ size_t fwd_rows_ws_bytes(const Shape& s);
 cudaError_t launch_fwd_rows(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
                             const float* gate_logit, const int32_t* n_sel, const uint64_t* maskT, void* ws, void* o,
                             float* attn_lse, cudaStream_t st);
-
-// Tensor-core forward over query tiles (union of the tile's selections): bf16, d = 128, block 64.
-bool fwd_tc_supported(const Shape& s);
-cudaError_t launch_fwd_tc(const Shape& s, const void* q, const void* k, const void* v, const int32_t* idx,
-                          const float* gate_logit, const int32_t* n_sel, void* o, float* attn_lse, cudaStream_t st);
 
 // Backward pieces.
 // D = rowsum(o * dO) per query-head row; also zeroes the fp32 dq accumulator [rows, d].
@@ -113,10 +110,18 @@ cudaError_t launch_bwd_simt(const Shape& s, const void* q, const void* k, const 
                             const float* gate_logit, const int32_t* n_sel, const uint64_t* maskT,
                             float* dq_acc, void* dk, void* dv, float* gsum, cudaStream_t st);
 // fp32 dq accumulator -> bf16 dq (bf16 shapes only; fp32 accumulates in place).
-cudaError_t launch_cast_dq(const Shape& s, const float* dq_acc, void* dq, cudaStream_t st);
+// `aborted` (device flag, may be NULL): when set, dq is written as NaN.
+cudaError_t launch_cast_dq(const Shape& s, const float* dq_acc, void* dq, const int* aborted, cudaStream_t st);
+// Score gradient; `aborted` (device flag, may be NULL): when set, every row is NaN.
 cudaError_t launch_dscore(const Shape& s, const float* scores, const float* score_lse,
                           const int32_t* idx, const int32_t* n_sel, const float* gsum, float* dscores,
-                          cudaStream_t st);
+                          const int* aborted, cudaStream_t st);
+
+// Pooled-key block scores of decode rows (bf16, d 128): scores[b, g, 0, j] =
+// mean_G(q) . kbar[b, g, j] for j < C, 0 for C <= j < NB; kbar [B, Hkv,
+// kstride, d].
+cudaError_t launch_pooled_scores(const Shape& s, const void* q, const void* kbar, int64_t kstride, float* scores,
+                                 cudaStream_t st);
 
 // Decode argument checks shared by the decode entry points (sas_api.cu).
 sas_status check_decode_args(const sas_desc* desc, const void* q, const void* k_cache, const void* v_cache,
@@ -133,5 +138,12 @@ size_t decode_ws_bytes(const Shape& s);
 cudaError_t launch_decode(const Shape& s, const void* q, const void* kc, const void* vc, int64_t stride,
                           const int32_t* idx, const float* gate_logit, const int32_t* n_sel, void* o,
                           float* part, cudaStream_t st);
+// Paged cache (bf16, d 128, block 64): pools [num_pages, Hkv, 64, d], block j
+// of sequence b in page table[b * max_blocks + j], cache length lens[b].
+bool decode_paged_supported(const Shape& s, int64_t num_pages);
+cudaError_t launch_decode_paged(const Shape& s, const void* q, const void* kp, const void* vp, int num_pages,
+                                const int32_t* table, int max_blocks, const int32_t* lens, const int32_t* idx,
+                                const float* gate_logit, const int32_t* n_sel, void* o, float* part,
+                                cudaStream_t st);
 
 }  // namespace sas

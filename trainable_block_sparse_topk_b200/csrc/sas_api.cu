@@ -6,7 +6,6 @@
 // synchronises the host.
 #include <atomic>
 #include <cmath>
-#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -19,23 +18,11 @@ namespace sas {
 
 // Readers for the wait-timeout counters of the translation units that wait.
 cudaError_t read_decode_timeouts(unsigned int* out);
-cudaError_t read_fwd_tc_timeouts(unsigned int* out);
 cudaError_t read_bwd_tc_timeouts(unsigned int* out);
 cudaError_t read_fwd_rows_timeouts(unsigned int* out);
-
-// SAS_FORCE_SIMT=1 routes bf16 training calls to the CUDA-core kernels (a
-// second GPU implementation, used to cross-check the tensor-core path).
-static bool force_simt() {
-    const char* e = std::getenv("SAS_FORCE_SIMT");
-    return e != nullptr && e[0] == '1';
-}
-
-// SAS_FWD_UNION=1 routes the bf16 forward to the query-tile kernel instead of
-// the gathered-row kernels (the two compute the same result; used to cross-check).
-static bool fwd_union() {
-    const char* e = std::getenv("SAS_FWD_UNION");
-    return e != nullptr && e[0] == '1';
-}
+cudaError_t set_decode_wait_limit(unsigned long long ns);
+cudaError_t set_bwd_tc_wait_limit(unsigned long long ns);
+cudaError_t set_fwd_rows_wait_limit(unsigned long long ns);
 
 static std::atomic<unsigned long long> g_launches{0};
 void count_launches(unsigned n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
@@ -110,7 +97,7 @@ sas_status make_shape(const sas_desc* d, Kind kind, Shape* s) {
         return SAS_ERR_INVALID_ARG;
     if (d->n_q_heads % d->n_kv_heads != 0) return SAS_ERR_INVALID_ARG;
     if (d->dtype != SAS_DT_BF16 && d->dtype != SAS_DT_FP32) return SAS_ERR_INVALID_ARG;
-    if (d->gate != SAS_GATE_SOFTMAX && d->gate != SAS_GATE_NONE) return SAS_ERR_INVALID_ARG;
+    if (d->gate < SAS_GATE_SOFTMAX || d->gate > SAS_GATE_STE) return SAS_ERR_INVALID_ARG;
     if (!(d->softmax_scale <= 0.f) && !std::isfinite(d->softmax_scale)) return SAS_ERR_INVALID_ARG;
     if (std::isnan(d->softmax_scale)) return SAS_ERR_INVALID_ARG;
     const int G = d->n_q_heads / d->n_kv_heads;
@@ -147,7 +134,7 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // Training workspace layout (each piece 256-byte aligned).
 struct TrainWs {
-    size_t maskT, Dd, gsum, dq_acc, stream, total;
+    size_t maskT, Dd, gsum, dq_acc, stream, flag, total;
 };
 
 TrainWs bwd_layout(const Shape& s) {
@@ -160,6 +147,8 @@ TrainWs bwd_layout(const Shape& s) {
     if (s.dtype != SAS_DT_FP32) off += align256(sizeof(float) * (size_t)s.B * s.Hq * s.T * s.D);
     w.stream = off;   // the tensor-core backward's per-block token streams
     if (bwd_tc_supported(s)) off += align256(bwd_tc_ws_bytes(s));
+    w.flag = off;     // set by a CTA that gave up on a wait
+    off += 256;
     w.total = off;
     return w;
 }
@@ -239,7 +228,18 @@ sas_status sas_block_topk(const sas_desc* desc, const float* scores, int32_t* id
     if (st != SAS_OK) return st;
     if (any_null(scores, idx, gate_logit, score_lse, n_sel)) return SAS_ERR_INVALID_ARG;
     if (any_misaligned(scores, idx, gate_logit, score_lse, n_sel)) return SAS_ERR_MISALIGNED;
-    return cuda_status(launch_block_topk(s, scores, idx, gate_logit, score_lse, n_sel, (cudaStream_t)stream));
+    return cuda_status(launch_block_topk(s, scores, nullptr, idx, gate_logit, score_lse, n_sel, (cudaStream_t)stream));
+}
+
+sas_status sas_block_topk_varlen(const sas_desc* desc, const float* scores, const int32_t* seq_lens, int32_t* idx,
+                                 float* gate_logit, float* score_lse, int32_t* n_sel, void* stream) {
+    Shape s;
+    sas_status st = make_shape(desc, Kind::kDecode, &s);
+    if (st != SAS_OK) return st;
+    if (any_null(scores, seq_lens, idx, gate_logit, score_lse, n_sel)) return SAS_ERR_INVALID_ARG;
+    if (any_misaligned(scores, seq_lens, idx, gate_logit, score_lse, n_sel)) return SAS_ERR_MISALIGNED;
+    return cuda_status(launch_block_topk(s, scores, seq_lens, idx, gate_logit, score_lse, n_sel,
+                                         (cudaStream_t)stream));
 }
 
 sas_status sas_gated_attn_fwd(const sas_desc* desc, const void* q, const void* k, const void* v,
@@ -254,7 +254,7 @@ sas_status sas_gated_attn_fwd(const sas_desc* desc, const void* q, const void* k
     if (need > 0 && (ws == nullptr || ws_bytes_ < need)) return SAS_ERR_WORKSPACE;
     if (ws && !aligned16(ws)) return SAS_ERR_MISALIGNED;
     cudaStream_t cs = (cudaStream_t)stream;
-    if (fwd_rows_supported(s) && !force_simt() && !fwd_union()) {
+    if (fwd_rows_supported(s)) {
         unsigned char* w = static_cast<unsigned char*>(ws);
         uint64_t* maskT = reinterpret_cast<uint64_t*>(w);
         void* rows_ws = w + align256(sizeof(uint64_t) * (size_t)s.B * s.Hkv * s.NB * s.nT);
@@ -262,8 +262,6 @@ sas_status sas_gated_attn_fwd(const sas_desc* desc, const void* q, const void* k
         if (e == cudaSuccess) e = launch_fwd_rows(s, q, k, v, idx, gate_logit, n_sel, maskT, rows_ws, o, attn_lse, cs);
         return cuda_status(e);
     }
-    if (fwd_tc_supported(s) && !force_simt())
-        return cuda_status(launch_fwd_tc(s, q, k, v, idx, gate_logit, n_sel, o, attn_lse, cs));
     return cuda_status(launch_fwd_simt(s, q, k, v, idx, gate_logit, n_sel, o, attn_lse, cs));
 }
 
@@ -288,18 +286,20 @@ sas_status sas_gated_attn_bwd(const sas_desc* desc, const void* q, const void* k
     float* gsum = reinterpret_cast<float*>(w + L.gsum);
     float* dq_acc = s.dtype == SAS_DT_FP32 ? static_cast<float*>(dq) : reinterpret_cast<float*>(w + L.dq_acc);
 
-    cudaError_t e = launch_sel_bitmap_T(s, idx, n_sel, maskT, cs);
+    int* aborted = reinterpret_cast<int*>(w + L.flag);
+    cudaError_t e = cudaMemsetAsync(aborted, 0, sizeof(int), cs);
+    if (e == cudaSuccess) e = launch_sel_bitmap_T(s, idx, n_sel, maskT, cs);
     if (e == cudaSuccess) e = launch_bwd_rowdot(s, o, dO, Dd, dq_acc, cs);   // zeroes dq_acc too
     if (e == cudaSuccess) {
-        if (bwd_tc_supported(s) && !force_simt())
+        if (bwd_tc_supported(s))
             e = launch_bwd_tc(s, q, k, v, dO, attn_lse, Dd, idx, gate_logit, n_sel, maskT, w + L.stream, dq_acc, dk,
-                              dv, gsum, cs);
+                              dv, gsum, aborted, cs);
         else
             e = launch_bwd_simt(s, q, k, v, dO, attn_lse, Dd, idx, gate_logit, n_sel, maskT, dq_acc, dk, dv, gsum,
                                 cs);
     }
-    if (e == cudaSuccess && s.dtype != SAS_DT_FP32) e = launch_cast_dq(s, dq_acc, dq, cs);
-    if (e == cudaSuccess) e = launch_dscore(s, scores, score_lse, idx, n_sel, gsum, dscores, cs);
+    if (e == cudaSuccess && s.dtype != SAS_DT_FP32) e = launch_cast_dq(s, dq_acc, dq, aborted, cs);
+    if (e == cudaSuccess) e = launch_dscore(s, scores, score_lse, idx, n_sel, gsum, dscores, aborted, cs);
     return cuda_status(e);
 }
 
@@ -314,6 +314,61 @@ sas_status sas_sparse_decode(const sas_desc* desc, const void* q, const void* k_
     if (!aligned16(ws)) return SAS_ERR_MISALIGNED;
     return cuda_status(launch_decode(s, q, k_cache, v_cache, cache_stride_tokens, idx, gate_logit, n_sel, o,
                                      static_cast<float*>(ws), (cudaStream_t)stream));
+}
+
+sas_status sas_sparse_decode_paged(const sas_desc* desc, const void* q, const void* k_pages, const void* v_pages,
+                                   int32_t num_pages, const int32_t* block_table, int32_t max_blocks,
+                                   const int32_t* seq_lens, const int32_t* idx, const float* gate_logit,
+                                   const int32_t* n_sel, void* o, void* ws, size_t ws_bytes_, void* stream) {
+    Shape s;
+    sas_status st = make_shape(desc, Kind::kDecode, &s);
+    if (st != SAS_OK) return st;
+    if (any_null(q, k_pages, v_pages, block_table, seq_lens, o)) return SAS_ERR_INVALID_ARG;
+    if (idx != nullptr && any_null(gate_logit, n_sel)) return SAS_ERR_INVALID_ARG;
+    if (num_pages < 1 || max_blocks < s.NB) return SAS_ERR_INVALID_ARG;
+    if (!decode_paged_supported(s, num_pages)) return SAS_ERR_UNSUPPORTED;
+    if (any_misaligned(q, k_pages, v_pages, block_table, seq_lens, o)) return SAS_ERR_MISALIGNED;
+    if (idx != nullptr && any_misaligned(idx, gate_logit, n_sel)) return SAS_ERR_MISALIGNED;
+    const size_t need = ws_bytes(SAS_OP_DECODE, s);
+    if (ws == nullptr || ws_bytes_ < need) return SAS_ERR_WORKSPACE;
+    if (!aligned16(ws)) return SAS_ERR_MISALIGNED;
+    return cuda_status(launch_decode_paged(s, q, k_pages, v_pages, num_pages, block_table, max_blocks, seq_lens, idx,
+                                           gate_logit, n_sel, o, static_cast<float*>(ws), (cudaStream_t)stream));
+}
+
+sas_status sas_block_scores_pooled(const sas_desc* desc, const void* q, const void* kbar,
+                                   int64_t kbar_stride_blocks, float* scores, void* stream) {
+    Shape s;
+    sas_status st = make_shape(desc, Kind::kDecode, &s);
+    if (st != SAS_OK) return st;
+    if (any_null(q, kbar, scores)) return SAS_ERR_INVALID_ARG;
+    if (kbar_stride_blocks < (int64_t)(s.q_offset / s.bs)) return SAS_ERR_INVALID_ARG;
+    if (s.dtype != SAS_DT_BF16 || s.D != 128) return SAS_ERR_UNSUPPORTED;
+    if (any_misaligned(q, kbar, scores)) return SAS_ERR_MISALIGNED;
+    return cuda_status(launch_pooled_scores(s, q, kbar, kbar_stride_blocks, scores, (cudaStream_t)stream));
+}
+
+sas_status sas_sparse_decode_pooled(const sas_desc* desc, const void* q, const void* k_cache, const void* v_cache,
+                                    int64_t cache_stride_tokens, const void* kbar, int64_t kbar_stride_blocks,
+                                    float* scores, int32_t* idx, float* gate_logit, float* score_lse,
+                                    int32_t* n_sel, void* o, void* ws, size_t ws_bytes_, void* stream) {
+    Shape s;
+    sas_status st = check_decode_args(desc, q, k_cache, v_cache, cache_stride_tokens, idx, gate_logit, n_sel, o, &s);
+    if (st != SAS_OK) return st;
+    if (any_null(kbar, scores, idx, score_lse)) return SAS_ERR_INVALID_ARG;
+    if (kbar_stride_blocks < (int64_t)(s.q_offset / s.bs)) return SAS_ERR_INVALID_ARG;
+    if (s.dtype != SAS_DT_BF16 || s.D != 128) return SAS_ERR_UNSUPPORTED;
+    if (any_misaligned(kbar, scores, score_lse)) return SAS_ERR_MISALIGNED;
+    const size_t need = ws_bytes(SAS_OP_DECODE, s);
+    if (ws == nullptr || ws_bytes_ < need) return SAS_ERR_WORKSPACE;
+    if (!aligned16(ws)) return SAS_ERR_MISALIGNED;
+    cudaStream_t cs = (cudaStream_t)stream;
+    cudaError_t e = launch_pooled_scores(s, q, kbar, kbar_stride_blocks, scores, cs);
+    if (e == cudaSuccess) e = launch_block_topk(s, scores, nullptr, idx, gate_logit, score_lse, n_sel, cs);
+    if (e == cudaSuccess)
+        e = launch_decode(s, q, k_cache, v_cache, cache_stride_tokens, idx, gate_logit, n_sel, o,
+                          static_cast<float*>(ws), cs);
+    return cuda_status(e);
 }
 
 // Diagnostics: kernels launched by this library since it was loaded (host
@@ -358,14 +413,21 @@ sas_status sas_kernel_time(const char* kernel, double* total_ms, uint32_t* launc
 // library was loaded (0 in normal operation). Synchronises the device.
 sas_status sas_device_timeouts(uint32_t* count) {
     if (!count) return SAS_ERR_INVALID_ARG;
-    unsigned int c0 = 0, c1 = 0, c2 = 0, c3 = 0;
+    unsigned int c0 = 0, c2 = 0, c3 = 0;
     cudaError_t e = read_decode_timeouts(&c0);
-    if (e == cudaSuccess) e = read_fwd_tc_timeouts(&c1);
     if (e == cudaSuccess) e = read_bwd_tc_timeouts(&c2);
     if (e == cudaSuccess) e = read_fwd_rows_timeouts(&c3);
     if (e != cudaSuccess) return SAS_ERR_CUDA;
-    *count = c0 + c1 + c2 + c3;
+    *count = c0 + c2 + c3;
     return SAS_OK;
+}
+
+sas_status sas_set_wait_limit(uint64_t ns) {
+    const unsigned long long v = ns == 0 ? kDefaultWaitNs : (unsigned long long)ns;
+    cudaError_t e = set_decode_wait_limit(v);
+    if (e == cudaSuccess) e = set_bwd_tc_wait_limit(v);
+    if (e == cudaSuccess) e = set_fwd_rows_wait_limit(v);
+    return e == cudaSuccess ? SAS_OK : SAS_ERR_CUDA;
 }
 
 }  // extern "C"

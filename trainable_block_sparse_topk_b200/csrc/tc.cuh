@@ -52,15 +52,16 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Bounded wait shared by all roles: gives up after ~1 s or when another role
-// has already given up, raising the CTA's abort flag.
+// Bounded wait shared by all roles: gives up after the wait limit or when
+// another role has already given up, raising the CTA's abort flag.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
+    const unsigned long long lim = g_sas_wait_limit_ns;
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
-        if (global_ns() - t0 > 1000000000ull) {
+        if (global_ns() - t0 > lim) {
             *abort = 1;
             atomicAdd(&g_sas_wait_timeouts, 1u);
             return false;
@@ -73,7 +74,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     const uint64_t t0 = global_ns();
     while (!mbar_try_wait(bar, parity))
-        if (global_ns() - t0 > 1000000000ull) return;
+        if (global_ns() - t0 > kDefaultWaitNs) return;
 }
 
 // Warp-uniform variant: lane 0 waits, the result is broadcast.
@@ -121,6 +122,18 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
 // Named barrier over `count` threads (id 1..15).
 __device__ __forceinline__ void named_bar(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// Named barrier that also ORs a predicate over its `count` threads: every
+// participant gets the same answer.
+__device__ __forceinline__ bool bar_red_or(int id, int count, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.or.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
 }
 
 // ---------------------------------------------------------------- tcgen05 ---

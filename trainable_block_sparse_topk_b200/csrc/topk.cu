@@ -7,12 +7,13 @@
 // normalised gate), and the kept blocks' log-gates are s_i minus it.
 //
 // Exactness: scores are compared through an order-preserving uint32 key, so the
-// K-th largest key is found exactly: by a 32-step bitwise search with
-// warp-wide counts when one warp owns the row, by an MSB-first radix select
-// (4 passes of 8 bits) when a whole CTA does. The elements above it are kept,
-// and the ones equal to it are kept in index order until K are chosen. Each thread owns a contiguous run of
-// SLOTS candidates, so index order is (thread, slot) order and two prefix scans
-// (one for the ties, one for output positions) place everything.
+// K-th largest key is found exactly (a bit search over the keys, MSB first,
+// narrowed first by a bound or a histogram of the top bits). The keys above it
+// are kept, and the ones equal to it are kept in index order until K are
+// chosen. Rows of up to 512 candidates take one warp, longer (decode) rows a
+// whole CTA; either way a thread owns the strided candidates thread,
+// thread + width, ..., so index order is (slot, thread) order and per-slot
+// ballots give the tie ranks and output positions.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -20,245 +21,483 @@ namespace sas {
 
 namespace {
 
-// Inverse of float_key (-0.0 comes back as +0.0, which compares equal).
-__device__ __forceinline__ float key_float(uint32_t k) {
-    uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
-    return __uint_as_float(u);
+// log g of a kept block with score x under gate activation `mode` (arXiv text
+// 4, design elements: normalised, independent and raw-logit gates; hard gate
+// with a straight-through gradient; study note 3-3, 3-4). lse is the
+// normaliser over the C candidates, lse_sel the one over the kept blocks.
+__device__ __forceinline__ float gate_logit_of(int mode, float x, float lse, float lse_sel) {
+    switch (mode) {
+        case SAS_GATE_SOFTMAX: return x - lse;
+        case SAS_GATE_SIGMOID: return x >= 0.f ? -log1pf(expf(-x)) : x - log1pf(expf(x));
+        case SAS_GATE_RAW: return x;
+        case SAS_GATE_SOFTMAX_SELECTED: return x - lse_sel;
+        default: return 0.f;   // none; hard gate: g = 1 on every kept block
+    }
 }
 
-// A row is processed by NT threads: one warp (NT == 32, several rows per CTA)
-// or the whole CTA (NT > 32, one row per CTA).
-template <int NT>
-struct RowGroup {
-    static constexpr int kWarps = NT / 32;
-    // Scratch for cross-warp reductions/scans, per group.
-    uint32_t* red;  // kWarps + 2 words
-
-    __device__ __forceinline__ void sync() const {
-        if (NT == 32) __syncwarp(); else __syncthreads();
-    }
-    __device__ __forceinline__ int tid() const { return NT == 32 ? (threadIdx.x & 31) : threadIdx.x; }
-
-    // Exclusive prefix sum over the group in thread order; *total gets the sum.
-    __device__ __forceinline__ uint32_t excl_scan(uint32_t x, uint32_t* total) const {
-        const int lane = threadIdx.x & 31;
-        uint32_t inc = x;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
-            if (lane >= o) inc += y;
-        }
-        if (NT == 32) {
-            *total = __shfl_sync(0xffffffffu, inc, 31);
-            return inc - x;
-        }
-        const int w = threadIdx.x >> 5;
-        if (lane == 31) red[w] = inc;
-        __syncthreads();
-        uint32_t before = 0, tot = 0;
-        for (int i = 0; i < kWarps; ++i) {
-            uint32_t v = red[i];
-            before += (i < w) ? v : 0u;
-            tot += v;
-        }
-        __syncthreads();
-        *total = tot;
-        return before + inc - x;
-    }
-
-    __device__ __forceinline__ float max_all(float x) const {
-        x = warp_max(x);
-        if (NT == 32) return x;
-        const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-        float* r = reinterpret_cast<float*>(red);
-        if (lane == 0) r[w] = x;
-        __syncthreads();
-        float m = -INFINITY;
-        for (int i = 0; i < kWarps; ++i) m = fmaxf(m, r[i]);
-        __syncthreads();
-        return m;
-    }
-    __device__ __forceinline__ float sum_all(float x) const {
-        x = warp_sum(x);
-        if (NT == 32) return x;
-        const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-        float* r = reinterpret_cast<float*>(red);
-        if (lane == 0) r[w] = x;
-        __syncthreads();
-        float m = 0.f;
-        for (int i = 0; i < kWarps; ++i) m += r[i];
-        __syncthreads();
-        return m;
-    }
-};
-
-// Find the digit of the `need`-th largest key (1-based) from a 256-bin
-// histogram; returns the digit and the rank of that key within its bin.
-// Executed by one full warp.
-__device__ __forceinline__ void pick_digit(const uint32_t* hist, uint32_t need, uint32_t* digit,
-                                           uint32_t* need_in_bin) {
-    const int lane = threadIdx.x & 31;
-    uint32_t h[8], s8 = 0;
-#pragma unroll
-    for (int b = 0; b < 8; ++b) { h[b] = hist[lane * 8 + b]; s8 += h[b]; }
-    // suffix sums over lanes: count in bins >= lane*8
-    uint32_t suf = s8;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        uint32_t y = __shfl_down_sync(0xffffffffu, suf, o);
-        if (lane + o < 32) suf += y;
-    }
-    const uint32_t above = suf - s8;
-    const bool mine = (above < need) && (need <= suf);
-    uint32_t d = 0, nb = 0;
-    if (mine) {
-        uint32_t c = above;
-#pragma unroll
-        for (int b = 7; b >= 0; --b) {
-            if (d == 0 && nb == 0 && c + h[b] >= need) { d = lane * 8 + b + 1; nb = need - c; }
-            c += h[b];
-        }
-    }
-    const uint32_t ball = __ballot_sync(0xffffffffu, mine);
-    const int src = __ffs(ball) - 1;
-    *digit = __shfl_sync(0xffffffffu, d, src) - 1;
-    *need_in_bin = __shfl_sync(0xffffffffu, nb, src);
+// Position of row `row` (query t): q_offset + t, or, with per-sequence cache
+// lengths (decode rows, T = 1), the new token of sequence b: lens[b] - 1.
+__device__ __forceinline__ int64_t row_position(const Shape& sh, const int32_t* lens, int64_t row, int t) {
+    if (lens == nullptr) return (int64_t)sh.q_offset + t;
+    const int64_t b = row / ((int64_t)sh.Hkv * sh.T);
+    const int64_t n = lens[b];   // clamped to [1, q_offset + 1]: the scores row holds NB blocks
+    return (n < 1 ? 1 : (n > (int64_t)sh.q_offset + 1 ? (int64_t)sh.q_offset + 1 : n)) - 1;
 }
 
-template <int NT, int SLOTS>
-__global__ void __launch_bounds__(NT == 32 ? 256 : NT)
-block_topk_kernel(Shape sh, const float* __restrict__ scores, int32_t* __restrict__ idx_out,
-                  float* __restrict__ gl_out, float* __restrict__ lse_out, int32_t* __restrict__ nsel_out) {
-    constexpr int kRowsPerCta = NT == 32 ? 8 : 1;
-    constexpr int kWarps = NT / 32;
-    __shared__ uint32_t s_hist[kRowsPerCta][256];
-    __shared__ uint32_t s_red[kRowsPerCta][kWarps + 4];
-
-    const int grp = NT == 32 ? (threadIdx.x >> 5) : 0;
-    const int64_t row = (int64_t)blockIdx.x * kRowsPerCta + grp;
-    const bool row_ok = row < sh.rows();   // uniform per group
-    RowGroup<NT> G{s_red[grp]};
-    const int tid = G.tid();
-    uint32_t* hist = s_hist[grp];
-
-    const int t = row_ok ? (int)(row % sh.T) : 0;
-    const int64_t p = (int64_t)sh.q_offset + t;
-    const int C = row_ok ? (int)(p / sh.bs) : 0;
+// One warp per row for rows of at most 32 * SLOTS candidates (several rows per
+// CTA). Lane l owns candidates l, l + 32, l + 64, ... (coalesced loads; index
+// order is (slot, lane) order, so ties and output positions come from per-slot
+// ballots). The K-th largest key is found by a bit search like the CTA path,
+// but over a short candidate list: when K <= 32, the K-th largest of the 32
+// lane maxima (a warp bitonic sort) is a key that at least K candidates reach,
+// so the answer lies between it and the row maximum; the keys at or above it
+// (normally a few dozen) are compacted into shared memory, four per lane, and
+// the search runs only over the bits below the prefix that bound and the
+// maximum share. Rows with more than 128 such keys, or K > 32, search all
+// their keys from the top bit.
+template <int SLOTS>
+__global__ void __launch_bounds__(256)
+block_topk_warp_kernel(Shape sh, const float* __restrict__ scores, const int32_t* __restrict__ lens,
+                       int32_t* __restrict__ idx_out, float* __restrict__ gl_out, float* __restrict__ lse_out,
+                       int32_t* __restrict__ nsel_out) {
+    constexpr int kCap = 128;                    // compacted keys per warp
+    __shared__ uint32_t s_cand[8][kCap];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * 8 + warp;
+    if (row >= sh.rows()) return;                // warp-uniform
+    const int t = (int)(row % sh.T);
+    const int64_t p = row_position(sh, lens, row, t);
+    const int C = (int)(p / sh.bs);
     const int K = sh.K;
     const int n = C < K ? C : K;
     const float* srow = scores + row * sh.NB;
+    const uint32_t lt = (1u << lane) - 1u;
 
-    // --- load keys (thread owns candidates [tid*SLOTS, tid*SLOTS + SLOTS)) ---
     uint32_t key[SLOTS];
-    float mloc = -INFINITY;
+    float mloc = -INFINITY, xs[SLOTS];
 #pragma unroll
-    for (int j = 0; j < SLOTS; ++j) {
-        const int i = tid * SLOTS + j;
-        if (i < C) {
-            const float f = srow[i];
-            key[j] = float_key(f);
-            mloc = fmaxf(mloc, f);
-        } else {
-            key[j] = 0u;  // below every valid key (float_key(-inf) = 0x007fffff)
-        }
+    for (int k = 0; k < SLOTS; ++k) {
+        const int i = lane + 32 * k;
+        xs[k] = i < C ? srow[i] : -INFINITY;
+        key[k] = i < C ? float_key(xs[k]) : 0u;  // below every valid key (float_key(-inf) = 0x007fffff)
+        mloc = fmaxf(mloc, xs[k]);
     }
-
-    // --- gate normaliser: lse = m + log sum exp(s - m) ---
-    const float m = G.max_all(mloc);
+    // gate normaliser: lse = m + log sum exp(s - m)
+    const float m = warp_max(mloc);
     float lsum = 0.f;
     if (m != -INFINITY) {
 #pragma unroll
-        for (int j = 0; j < SLOTS; ++j)
-            if (tid * SLOTS + j < C) lsum += expf(key_float(key[j]) - m);
+        for (int k = 0; k < SLOTS; ++k)
+            if (lane + 32 * k < C) lsum += exp2f((xs[k] - m) * kLog2e);
     }
-    lsum = G.sum_all(lsum);
+    lsum = warp_sum(lsum);
     const float lse = (C > 0 && m != -INFINITY) ? m + logf(lsum) : -INFINITY;
 
-    // --- the n-th largest key ---
-    uint32_t prefix = 0, pmask = 0, need = (uint32_t)n;
-    if (NT == 32 && n > 0) {
-        // One warp: bitwise search, MSB first. Bit b joins the answer when at
-        // least n keys are >= (answer | bit): the result is the largest v with
-        // #{keys >= v} >= n, i.e. the n-th largest key. Invalid slots hold key
-        // 0, which no candidate (>= 1) admits.
-        uint32_t thr = 0;
+    // the n-th largest key; `need` of its copies are kept
+    uint32_t thr = 0;
+    if (n > 0 && n == C) {
+        // every candidate is kept: the threshold is the smallest key
+        uint32_t mn = 0xffffffffu;
 #pragma unroll
-        for (int bit = 31; bit >= 0; --bit) {
-            const uint32_t cand = thr | (1u << bit);
-            uint32_t c = 0;
-#pragma unroll
-            for (int j = 0; j < SLOTS; ++j) c += key[j] >= cand ? 1u : 0u;
-            if (__reduce_add_sync(0xffffffffu, c) >= (uint32_t)n) thr = cand;
-        }
-        uint32_t gt = 0;
-#pragma unroll
-        for (int j = 0; j < SLOTS; ++j) gt += key[j] > thr ? 1u : 0u;
-        prefix = thr;
-        need = (uint32_t)n - __reduce_add_sync(0xffffffffu, gt);   // copies of thr to keep
+        for (int k = 0; k < SLOTS; ++k)
+            if (lane + 32 * k < C) mn = min(mn, key[k]);
+        thr = __reduce_min_sync(0xffffffffu, mn);
     } else if (n > 0) {
-        // radix select, 4 passes of 8 bits, MSB first
-#pragma unroll 1
-        for (int pass = 0; pass < 4; ++pass) {
-            const int shift = 24 - 8 * pass;
-            for (int b = tid; b < 256; b += NT) hist[b] = 0;
-            G.sync();
+        uint32_t lmax = 0;
 #pragma unroll
-            for (int j = 0; j < SLOTS; ++j) {
-                const bool act = (tid * SLOTS + j < C) && ((key[j] & pmask) == prefix);
-                const uint32_t bin = (key[j] >> shift) & 255u;
-                const uint32_t peers = __match_any_sync(0xffffffffu, act ? bin : 0xffffffffu);
-                if (act && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+        for (int k = 0; k < SLOTS; ++k) lmax = max(lmax, key[k]);
+        const uint32_t hi = __reduce_max_sync(0xffffffffu, lmax);
+        bool compact = false;
+        uint32_t lo = 0;
+        if (n <= 32) {
+            // bitonic sort of the lane maxima, descending across lanes
+            uint32_t v = lmax;
+#pragma unroll
+            for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+                for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                    const uint32_t o = __shfl_xor_sync(0xffffffffu, v, stride);
+                    const bool up = (lane & size) == 0;         // descending runs
+                    const bool lower = (lane & stride) == 0;
+                    v = (lower == up) ? max(v, o) : min(v, o);
+                }
             }
-            G.sync();
-            uint32_t dgt, nb;
-            if (NT == 32) {
-                pick_digit(hist, need, &dgt, &nb);
-            } else {
-                if (threadIdx.x < 32) {
-                    pick_digit(hist, need, &dgt, &nb);
-                    if (threadIdx.x == 0) { s_red[grp][kWarps] = dgt; s_red[grp][kWarps + 1] = nb; }
+            lo = __shfl_sync(0xffffffffu, v, n - 1);              // n lane maxima are >= lo
+            uint32_t cnt = 0;
+#pragma unroll
+            for (int k = 0; k < SLOTS; ++k) cnt += key[k] >= lo ? 1u : 0u;
+            uint32_t incl = cnt;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+            compact = total <= (uint32_t)kCap;
+            if (compact) {
+                uint32_t at = incl - cnt;
+#pragma unroll
+                for (int k = 0; k < SLOTS; ++k)
+                    if (key[k] >= lo) s_cand[warp][at++] = key[k];
+                for (uint32_t e = total + lane; e < (uint32_t)kCap; e += 32) s_cand[warp][e] = 0u;
+                __syncwarp();
+            }
+        }
+        // bit search for the largest v with #{keys >= v} >= n, starting below
+        // the prefix that lo and hi share (every v in [lo, hi] has it)
+        const uint32_t diff = lo ^ hi;
+        const int top = diff == 0u ? -1 : 31 - __clz(diff);
+        thr = top >= 31 ? 0u : (hi & ~((2u << top) - 1u));
+        if (top < 0) thr = hi;
+        if (compact) {
+            uint32_t c4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) c4[e] = s_cand[warp][4 * lane + e];
+            for (int bit = top; bit >= 0; --bit) {
+                const uint32_t cand = thr | (1u << bit);
+                uint32_t c = 0;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) c += c4[e] >= cand ? 1u : 0u;
+                if (__reduce_add_sync(0xffffffffu, c) >= (uint32_t)n) thr = cand;
+            }
+        } else {
+            for (int bit = top; bit >= 0; --bit) {
+                const uint32_t cand = thr | (1u << bit);
+                uint32_t c = 0;
+#pragma unroll
+                for (int k = 0; k < SLOTS; ++k) c += key[k] >= cand ? 1u : 0u;
+                if (__reduce_add_sync(0xffffffffu, c) >= (uint32_t)n) thr = cand;
+            }
+        }
+    }
+
+    // keep every key above thr and the first `need` copies of thr in index order
+    uint32_t gt = 0;
+#pragma unroll
+    for (int k = 0; k < SLOTS; ++k) gt += (n > 0 && lane + 32 * k < C && key[k] > thr) ? 1u : 0u;
+    const uint32_t need = (uint32_t)n - __reduce_add_sync(0xffffffffu, gt);
+    int32_t* io = idx_out + row * K;
+    float* go = gl_out + row * K;
+    uint32_t eq_run = 0, take_bits = 0;
+#pragma unroll
+    for (int k = 0; k < SLOTS; ++k) {
+        const int i = lane + 32 * k;
+        const bool valid = n > 0 && i < C;
+        const uint32_t eqb = __ballot_sync(0xffffffffu, valid && key[k] == thr);
+        if (valid && (key[k] > thr || (key[k] == thr && eq_run + __popc(eqb & lt) < need))) take_bits |= 1u << k;
+        eq_run += __popc(eqb);
+    }
+    float lse_sel = 0.f;
+    if (sh.gate == SAS_GATE_SOFTMAX_SELECTED) {      // normaliser over the kept blocks
+        float mk = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < SLOTS; ++k)
+            if ((take_bits >> k) & 1u) mk = fmaxf(mk, xs[k]);
+        mk = warp_max(mk);
+        float sk = 0.f;
+#pragma unroll
+        for (int k = 0; k < SLOTS; ++k)
+            if ((take_bits >> k) & 1u) sk += expf(xs[k] - mk);
+        lse_sel = mk + logf(warp_sum(sk));
+    }
+    uint32_t pos_run = 0;
+#pragma unroll
+    for (int k = 0; k < SLOTS; ++k) {
+        const bool take = (take_bits >> k) & 1u;
+        const uint32_t tb = __ballot_sync(0xffffffffu, take);
+        if (take) {
+            const uint32_t pos = pos_run + __popc(tb & lt);
+            io[pos] = lane + 32 * k;
+            go[pos] = gate_logit_of(sh.gate, xs[k], lse, lse_sel);
+        }
+        pos_run += __popc(tb);
+    }
+    for (int jj = n + lane; jj < K; jj += 32) { io[jj] = -1; go[jj] = 0.f; }
+    if (lane == 0) { lse_out[row] = lse; nsel_out[row] = n; }
+}
+
+template <int SLOTS>
+cudaError_t run_topk_warp(const Shape& s, const float* scores, const int32_t* lens, int32_t* idx, float* gl,
+                          float* lse, int32_t* nsel, cudaStream_t st) {
+    const int64_t grid = (s.rows() + 7) / 8;
+    KernelTimer kt("block_topk", st);
+    block_topk_warp_kernel<SLOTS><<<(unsigned)grid, 256, 0, st>>>(s, scores, lens, idx, gl, lse, nsel);
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) count_launches(1);
+    return e;
+}
+
+// One CTA of NT threads per row, for long rows (decode rows of up to NT * 8
+// candidates). Thread t owns candidates t, t + NT, ... (coalesced loads; index
+// order is (slot, thread) order). The K-th largest key: a 2048-bin histogram of
+// the keys' top 11 bits picks the bin that holds it; the keys of that bin
+// (normally a handful) are compacted into shared memory and one warp finishes
+// with a bit search over the 21 bits below. When that bin holds more keys than
+// the compaction buffer (long runs of equal scores), the search narrows by
+// further histogram passes over 11 and then 10 bits among the keys that match
+// so far. Kept keys are then placed in index order by per-slot ballots and one
+// cross-warp prefix.
+template <int NT, int SLOTS>
+__global__ void __launch_bounds__(NT)
+block_topk_cta_kernel(Shape sh, const float* __restrict__ scores, const int32_t* __restrict__ lens,
+                      int32_t* __restrict__ idx_out, float* __restrict__ gl_out, float* __restrict__ lse_out,
+                      int32_t* __restrict__ nsel_out) {
+    constexpr int kW = NT / 32;
+    constexpr int kBins = 2048;
+    constexpr int kCand = 1024;
+    __shared__ __align__(16) uint32_t s_hist[kBins];
+    __shared__ uint32_t s_cand[kCand];
+    __shared__ float s_rm[kW], s_rs[kW];
+    __shared__ uint32_t s_cnt[SLOTS][kW];
+    __shared__ uint32_t s_misc[8];       // digit, need-in-bin, candidates, thr, need, prefix, mask, overflow
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t row = blockIdx.x;
+    const int t = (int)(row % sh.T);
+    const int64_t p = row_position(sh, lens, row, t);
+    const int C = (int)(p / sh.bs);
+    const int K = sh.K;
+    const int n = C < K ? C : K;
+    const float* srow = scores + row * sh.NB;
+    const uint32_t lt = (1u << lane) - 1u;
+
+    for (int e = tid; e < kBins; e += NT) s_hist[e] = 0u;
+    if (tid == 0) s_misc[2] = 0u;
+    uint32_t key[SLOTS];
+    float xs[SLOTS], mloc = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < SLOTS; ++k) {
+        const int i = tid + NT * k;
+        xs[k] = i < C ? srow[i] : -INFINITY;
+        key[k] = i < C ? float_key(xs[k]) : 0u;
+        mloc = fmaxf(mloc, xs[k]);
+    }
+    // gate normaliser: (max, sum of exp) pairs reduced in one pass
+    float msum = mloc, ssum = 0.f;
+    if (mloc != -INFINITY) {
+#pragma unroll
+        for (int k = 0; k < SLOTS; ++k)
+            if (tid + NT * k < C) ssum += exp2f((xs[k] - mloc) * kLog2e);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float m2 = __shfl_xor_sync(0xffffffffu, msum, o), s2 = __shfl_xor_sync(0xffffffffu, ssum, o);
+        const float mm = fmaxf(msum, m2);
+        ssum = (msum == -INFINITY ? 0.f : ssum * exp2f((msum - mm) * kLog2e)) +
+               (m2 == -INFINITY ? 0.f : s2 * exp2f((m2 - mm) * kLog2e));
+        msum = mm;
+    }
+    if (lane == 0) { s_rm[warp] = msum; s_rs[warp] = ssum; }
+    // histogram of the top 11 key bits
+#pragma unroll
+    for (int k = 0; k < SLOTS; ++k)
+        if (tid + NT * k < C) atomicAdd(&s_hist[key[k] >> 21], 1u);
+    __syncthreads();
+    float m = -INFINITY;
+    for (int w = 0; w < kW; ++w) m = fmaxf(m, s_rm[w]);
+    float lsum = 0.f;
+    for (int w = 0; w < kW; ++w) lsum += s_rm[w] == -INFINITY ? 0.f : s_rs[w] * exp2f((s_rm[w] - m) * kLog2e);
+    const float lse = (C > 0 && m != -INFINITY) ? m + logf(lsum) : -INFINITY;
+
+    // ---- the n-th largest key: radix passes of 11, 11, 10 bits until its bin is small ----
+    uint32_t prefix = 0, pmask = 0, need = (uint32_t)n, thr = 0;
+    if (n > 0) {
+        int shift = 21;
+        for (int pass = 0; pass < 3; ++pass) {
+            const int bits = pass < 2 ? 11 : 10;
+            if (pass > 0) {
+                for (int e = tid; e < kBins; e += NT) s_hist[e] = 0u;
+                __syncthreads();
+#pragma unroll
+                for (int k = 0; k < SLOTS; ++k)
+                    if (tid + NT * k < C && (key[k] & pmask) == prefix)
+                        atomicAdd(&s_hist[(key[k] >> shift) & ((1u << bits) - 1u)], 1u);
+                __syncthreads();
+            }
+            if (warp == 0) {
+                // lane l sums bins [64 l, 64 l + 64); suffix sums over lanes; the
+                // lane holding the need-th largest scans its bins from the top
+                const int nb = 1 << bits, per = nb / 32;
+                uint32_t sl = 0;
+                const uint4* h4 = reinterpret_cast<const uint4*>(s_hist + lane * per);
+#pragma unroll 4
+                for (int e = 0; e < per / 4; ++e) {
+                    const uint4 v = h4[e];
+                    sl += v.x + v.y + v.z + v.w;
+                }
+                uint32_t suf = sl;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t y = __shfl_down_sync(0xffffffffu, suf, o);
+                    if (lane + o < 32) suf += y;
+                }
+                // the lane whose bins hold the need-th largest key; then the whole
+                // warp scans that lane's bins (per / 32 each, from the top)
+                const uint32_t mine = __ballot_sync(0xffffffffu, suf - sl < need && need <= suf);
+                const int L = __ffs(mine) - 1;
+                const uint32_t above = __shfl_sync(0xffffffffu, suf - sl, L);   // keys in higher lanes' bins
+                const int sub = per / 32;                  // 2 bins per lane (11 bits) or 1 (10 bits)
+                const int hi_bin = L * per + per - 1 - lane * sub;   // lane 0 takes the top bins
+                uint32_t hs = 0, hb[2] = {0u, 0u};
+                for (int e = 0; e < sub; ++e) { hb[e] = s_hist[hi_bin - e]; hs += hb[e]; }
+                uint32_t inc = hs;                         // keys in bins >= this lane's lowest bin
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+                    if (lane >= o) inc += y;
+                }
+                const uint32_t before = above + inc - hs;  // keys in bins above this lane's
+                const uint32_t hit = __ballot_sync(0xffffffffu, before < need && need <= before + hs);
+                if (lane == __ffs(hit) - 1) {
+                    uint32_t c = before;
+                    for (int e = 0; e < sub; ++e) {
+                        if (c + hb[e] >= need) {
+                            s_misc[0] = (uint32_t)(hi_bin - e);
+                            s_misc[1] = need - c;
+                            s_misc[7] = hb[e];           // keys in the chosen bin
+                            break;
+                        }
+                        c += hb[e];
+                    }
+                }
+            }
+            __syncthreads();
+            prefix |= s_misc[0] << shift;
+            pmask |= ((1u << bits) - 1u) << shift;
+            need = s_misc[1];
+            const uint32_t inbin = s_misc[7];
+            if (inbin <= (uint32_t)kCand || shift == 0) {
+                if (shift == 0) { thr = prefix; break; }   // every bit decided
+                // compact the bin's keys (one atomic per warp and slot); one warp
+                // searches the bits below
+#pragma unroll
+                for (int k = 0; k < SLOTS; ++k) {
+                    const bool in = tid + NT * k < C && (key[k] & pmask) == prefix;
+                    const uint32_t m = __ballot_sync(0xffffffffu, in);
+                    if (m == 0u) continue;               // warp-uniform
+                    uint32_t at = 0;
+                    if (lane == __ffs(m) - 1) at = atomicAdd(&s_misc[2], (uint32_t)__popc(m));
+                    at = __shfl_sync(0xffffffffu, at, __ffs(m) - 1);
+                    if (in) s_cand[at + __popc(m & lt)] = key[k];
                 }
                 __syncthreads();
-                dgt = s_red[grp][kWarps];
-                nb = s_red[grp][kWarps + 1];
+                if (warp == 0) {
+                    const uint32_t nc = s_misc[2];
+                    uint32_t th = prefix;
+                    if (nc <= 128) {                     // four keys per lane, in registers
+                        uint32_t c4[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) c4[e] = (uint32_t)(lane + 32 * e) < nc ? s_cand[lane + 32 * e] : 0u;
+                        for (int bit = shift - 1; bit >= 0; --bit) {
+                            const uint32_t cand = th | (1u << bit);
+                            uint32_t c = 0;
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) c += c4[e] >= cand ? 1u : 0u;
+                            if (__reduce_add_sync(0xffffffffu, c) >= need) th = cand;
+                        }
+                    } else {
+                        for (int bit = shift - 1; bit >= 0; --bit) {
+                            const uint32_t cand = th | (1u << bit);
+                            uint32_t c = 0;
+                            for (uint32_t e = lane; e < nc; e += 32) c += s_cand[e] >= cand ? 1u : 0u;
+                            if (__reduce_add_sync(0xffffffffu, c) >= need) th = cand;
+                        }
+                    }
+                    if (lane == 0) s_misc[3] = th;
+                }
                 __syncthreads();
+                thr = s_misc[3];
+                break;
             }
-            prefix |= dgt << shift;
-            pmask |= 255u << shift;
-            need = nb;
+            shift -= pass == 0 ? 11 : 10;
         }
     }
-    const uint32_t thr = prefix;   // the n-th largest key; `need` of its copies are kept
 
-    // --- ties: keep the first `need` elements equal to thr, in index order ---
-    uint32_t eq_loc = 0;
+    // ---- keep the keys above thr and the first copies of thr, in index order ----
+    // Index order is (slot, warp, lane): per-slot ballots within a warp, and
+    // one warp scans the per-(slot, warp) counts into exclusive prefixes.
+    uint32_t eqb[SLOTS], tkb[SLOTS];
 #pragma unroll
-    for (int j = 0; j < SLOTS; ++j) eq_loc += (n > 0 && tid * SLOTS + j < C && key[j] == thr) ? 1u : 0u;
-    uint32_t tot;
-    uint32_t eq_before = G.excl_scan(eq_loc, &tot);
-    uint32_t take_mask = 0, take_loc = 0;
-#pragma unroll
-    for (int j = 0; j < SLOTS; ++j) {
-        const bool valid = n > 0 && tid * SLOTS + j < C;
-        bool take = valid && key[j] > thr;
-        if (valid && key[j] == thr) {
-            take = eq_before < need;
-            ++eq_before;
-        }
-        if (take) { take_mask |= 1u << j; ++take_loc; }
+    for (int k = 0; k < SLOTS; ++k) {
+        const bool valid = n > 0 && tid + NT * k < C;
+        eqb[k] = __ballot_sync(0xffffffffu, valid && key[k] == thr);
+        const uint32_t gtb = __ballot_sync(0xffffffffu, valid && key[k] > thr);
+        if (lane == 0) s_cnt[k][warp] = (uint32_t)__popc(eqb[k]) | ((uint32_t)__popc(gtb) << 16);
     }
-    uint32_t pos = G.excl_scan(take_loc, &tot);
-
-    if (!row_ok) return;
+    __syncthreads();
+    // exclusive prefix over the SLOTS * kW counts in (slot, warp) order, in place;
+    // the totals land in s_misc[4]
+    auto scan_counts = [&]() {
+        if (warp == 0) {
+            constexpr int E = SLOTS * kW / 32;           // entries per lane
+            uint32_t* flat = &s_cnt[0][0];
+            uint32_t v[E], sum = 0;
+#pragma unroll
+            for (int e = 0; e < E; ++e) { v[e] = flat[lane * E + e]; sum += v[e]; }
+            uint32_t incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            uint32_t run = incl - sum;
+#pragma unroll
+            for (int e = 0; e < E; ++e) { flat[lane * E + e] = run; run += v[e]; }
+            if (lane == 31) s_misc[4] = incl;
+        }
+        __syncthreads();
+    };
+    scan_counts();
+    // ties are counted in the low 16 bits and keys above thr in the high 16
+    // bits of each count, so one scan gives both prefixes
+    const uint32_t gt_all = s_misc[4] >> 16;
+    const uint32_t need_eq = (uint32_t)n - gt_all;
+    bool take[SLOTS];
+#pragma unroll
+    for (int k = 0; k < SLOTS; ++k) {
+        const uint32_t rank = (s_cnt[k][warp] & 0xffffu) + __popc(eqb[k] & lt);
+        const bool gt = n > 0 && tid + NT * k < C && key[k] > thr;
+        take[k] = gt || (((eqb[k] >> lane) & 1u) && rank < need_eq);
+    }
+    __syncthreads();   // s_cnt is rewritten with the kept counts
+#pragma unroll
+    for (int k = 0; k < SLOTS; ++k) {
+        tkb[k] = __ballot_sync(0xffffffffu, take[k]);
+        if (lane == 0) s_cnt[k][warp] = (uint32_t)__popc(tkb[k]);
+    }
+    __syncthreads();
+    scan_counts();
+    float lse_sel = 0.f;
+    if (sh.gate == SAS_GATE_SOFTMAX_SELECTED) {      // normaliser over the kept blocks (CTA-uniform branch)
+        float mk = -INFINITY, sk = 0.f;
+#pragma unroll
+        for (int k = 0; k < SLOTS; ++k)
+            if (take[k]) mk = fmaxf(mk, xs[k]);
+#pragma unroll
+        for (int k = 0; k < SLOTS; ++k)
+            if (take[k]) sk += expf(xs[k] - mk);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, mk, o), s2 = __shfl_xor_sync(0xffffffffu, sk, o);
+            const float mm = fmaxf(mk, m2);
+            sk = (mk == -INFINITY ? 0.f : sk * expf(mk - mm)) + (m2 == -INFINITY ? 0.f : s2 * expf(m2 - mm));
+            mk = mm;
+        }
+        if (lane == 0) { s_rm[warp] = mk; s_rs[warp] = sk; }
+        __syncthreads();
+        float M = -INFINITY, L = 0.f;
+        for (int w = 0; w < kW; ++w) M = fmaxf(M, s_rm[w]);
+        for (int w = 0; w < kW; ++w) L += s_rm[w] == -INFINITY ? 0.f : s_rs[w] * expf(s_rm[w] - M);
+        lse_sel = M + logf(L);
+    }
     int32_t* io = idx_out + row * K;
     float* go = gl_out + row * K;
 #pragma unroll
-    for (int j = 0; j < SLOTS; ++j) {
-        if (take_mask & (1u << j)) {
-            const int i = tid * SLOTS + j;
-            io[pos] = i;
-            go[pos] = sh.gate == SAS_GATE_SOFTMAX ? key_float(key[j]) - lse : 0.f;
-            ++pos;
+    for (int k = 0; k < SLOTS; ++k) {
+        if (take[k]) {
+            const uint32_t pos = s_cnt[k][warp] + __popc(tkb[k] & lt);
+            io[pos] = tid + NT * k;
+            go[pos] = gate_logit_of(sh.gate, xs[k], lse, lse_sel);
         }
     }
     for (int jj = n + tid; jj < K; jj += NT) { io[jj] = -1; go[jj] = 0.f; }
@@ -266,13 +505,10 @@ block_topk_kernel(Shape sh, const float* __restrict__ scores, int32_t* __restric
 }
 
 template <int NT, int SLOTS>
-cudaError_t run_topk(const Shape& s, const float* scores, int32_t* idx, float* gl, float* lse, int32_t* nsel,
-                     cudaStream_t st) {
-    const int64_t rows = s.rows();
-    const int rpc = NT == 32 ? 8 : 1;
-    const int64_t grid = (rows + rpc - 1) / rpc;
+cudaError_t run_topk_cta(const Shape& s, const float* scores, const int32_t* lens, int32_t* idx, float* gl,
+                         float* lse, int32_t* nsel, cudaStream_t st) {
     KernelTimer kt("block_topk", st);
-    block_topk_kernel<NT, SLOTS><<<(unsigned)grid, NT == 32 ? 256 : NT, 0, st>>>(s, scores, idx, gl, lse, nsel);
+    block_topk_cta_kernel<NT, SLOTS><<<(unsigned)s.rows(), NT, 0, st>>>(s, scores, lens, idx, gl, lse, nsel);
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
     return e;
@@ -309,14 +545,14 @@ sel_bitmap_T_kernel(Shape sh, const int32_t* __restrict__ idx, const int32_t* __
 
 bool topk_row_supported(int64_t max_candidates) { return max_candidates <= 8192; }
 
-cudaError_t launch_block_topk(const Shape& s, const float* scores, int32_t* idx, float* gl, float* lse,
-                              int32_t* nsel, cudaStream_t st) {
+cudaError_t launch_block_topk(const Shape& s, const float* scores, const int32_t* lens, int32_t* idx, float* gl,
+                              float* lse, int32_t* nsel, cudaStream_t st) {
     const int64_t cmax = ((int64_t)s.q_offset + s.T - 1) / s.bs;
-    if (cmax <= 32) return run_topk<32, 1>(s, scores, idx, gl, lse, nsel, st);
-    if (cmax <= 128) return run_topk<32, 4>(s, scores, idx, gl, lse, nsel, st);
-    if (cmax <= 512) return run_topk<32, 16>(s, scores, idx, gl, lse, nsel, st);
-    if (cmax <= 2048) return run_topk<256, 8>(s, scores, idx, gl, lse, nsel, st);
-    return run_topk<1024, 8>(s, scores, idx, gl, lse, nsel, st);
+    if (cmax <= 32) return run_topk_warp<1>(s, scores, lens, idx, gl, lse, nsel, st);
+    if (cmax <= 128) return run_topk_warp<4>(s, scores, lens, idx, gl, lse, nsel, st);
+    if (cmax <= 512) return run_topk_warp<16>(s, scores, lens, idx, gl, lse, nsel, st);
+    if (cmax <= 2048) return run_topk_cta<256, 8>(s, scores, lens, idx, gl, lse, nsel, st);
+    return run_topk_cta<1024, 8>(s, scores, lens, idx, gl, lse, nsel, st);
 }
 
 cudaError_t launch_sel_bitmap_T(const Shape& s, const int32_t* idx, const int32_t* nsel, uint64_t* maskT,
