@@ -315,15 +315,16 @@ decode_partial_kernel(DecArgs a) {
 // The CTA that completes a group last (an atomic ticket per group) merges the
 // group's records by log-sum-exp and writes o: one launch per call.
 //
-// Roles (128 threads): warp 0 resolves the items' block indices, log-gates
+// Roles (224 threads): warp 0 resolves the items' block indices, log-gates
 // and cache rows 32 at a time and moves each block's K and V rows into a
 // kFlatStages ring by TMA (two 64-column boxes per tensor, 128-byte swizzle, no
-// multicast); warps 1-3 take every third item each (a consumer's MMA chain has
-// little parallelism of its own, so three blocks are computed at once, and
-// each consumer owns two stages) and run each block on mma.sync m16n8k16:
-//   S^T = K q^T   (M = 16 keys, N = 8 heads, K = 16 dims; 4 x 8 MMAs)
+// multicast); warps 1-6 form three pairs, each pair taking every third item
+// and owning two stages, each warp of a pair taking 32 of the block's 64 keys
+// (an mma.sync chain has little parallelism of its own, so six half-blocks are
+// computed at once) and running them on mma.sync m16n8k16:
+//   S^T = K q^T   (M = 16 keys, N = 8 heads, K = 16 dims; 2 x 8 MMAs per warp)
 //   online softmax per head in log2 units (scale applied in fp32 after the MMA)
-//   O^T += V^T P^T (M = 16 dims, N = 8 heads, K = 16 keys; 8 x 4 MMAs)
+//   O^T += V^T P^T (M = 16 dims, N = 8 heads, K = 16 keys; 8 x 2 MMAs per warp)
 // K rows come through ldmatrix, V rows through ldmatrix.trans, and the P tile
 // (keys x heads, accumulator layout) becomes the B operand by movmatrix.trans.
 // Rows of the current block at or after the new token may hold anything in the
@@ -331,12 +332,14 @@ decode_partial_kernel(DecArgs a) {
 // memory before the product. At the end of each group the consumers merge
 // their (m, l, O) through shared memory.
 constexpr int kFlatStages = 6;
-constexpr int kCons = 3;                 // consumer warps: item i goes to consumer i mod kCons
-constexpr int kFlatThreads = 32 * (1 + kCons);
-// Stage s always holds items of consumer s mod kCons, so each stage's barrier
-// phases are waited on by one warp, in order (a second warp could poll a phase
-// ahead of the current one and see an older phase of the same parity).
-static_assert(kFlatStages % kCons == 0, "every stage must belong to one consumer");
+constexpr int kCons = 3;                 // consumer pairs: item i goes to pair i mod kCons
+constexpr int kConsWarps = 2 * kCons;    // each pair splits a block's 64 keys, 32 per warp
+constexpr int kFlatThreads = 32 * (1 + kConsWarps);
+// Stage s always holds items of pair s mod kCons, so each stage's barrier
+// phases are waited on by the same two warps, each in order (a warp of another
+// pair could poll a phase ahead of the current one and see an older phase of
+// the same parity).
+static_assert(kFlatStages % kCons == 0, "every stage must belong to one consumer pair");
 constexpr uint32_t kItemBytes = 32768;   // K box 0 | K box 1 | V box 0 | V box 1, 8 KiB each
 constexpr int kMaxDecodeCtas = 160;     // grid bound (one CTA per SM)
 constexpr int kRecF = 132;              // floats per head in a record: O[128], m, l, 2 pad (16-byte rows)
@@ -358,7 +361,7 @@ struct FlatSmem {
     static constexpr uint32_t kBlk = kMisc + 16;                      // i32 [S]: keys of the stage's item (0: none)
     static constexpr uint32_t kLg = kBlk + 4 * kFlatStages;           // f32 [S]: its log-gate (log2 units)
     static constexpr uint32_t kXch = (kLg + 4 * kFlatStages + 15) & ~15u;   // per consumer 1..: m[8], l[8], O^T[128][8]
-    static constexpr uint32_t kLast = kXch + 4 * (kCons - 1) * (16 + 128 * 8);   // i32: this CTA merges the group
+    static constexpr uint32_t kLast = kXch + 4 * (kConsWarps - 1) * (16 + 128 * 8);   // i32: this CTA merges the group
     static constexpr uint32_t kMerge = kLast + 16;                    // f32 m, l, weight [kMaxRecs][8] each
     static constexpr uint32_t kTotal = kMerge + 3 * 4 * kMaxRecs * 8;
 };
@@ -424,7 +427,7 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     if (threadIdx.x == 0) {
         for (int s = 0; s < kFlatStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], 2);   // both warps of the owning pair
         }
         *abort = 0;
         fence_mbar_init();
@@ -453,16 +456,23 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 const int64_t Nb = a.lens == nullptr ? N : min(max((int64_t)a.lens[b], (int64_t)1), N);
                 const int Cb = (int)((Nb - 1) / BS);   // this sequence's current block
                 int j = -1;
+                // the kept index, its log-gate and the kept count are loaded together
+                // (p < nblk - 1 <= K keeps the first two inside the row)
+                int jj = -1, ns = 0;
+                float gv = 0.f;
+                if (!dense && p < nblk - 1) {
+                    jj = a.idx[bg * sh.K + p];
+                    gv = a.gl[bg * sh.K + p];
+                    ns = a.nsel[bg];
+                }
                 if (dense) {
                     j = p <= Cb ? p : -1;
                 } else if (p == nblk - 1) {
                     j = Cb;
-                } else if (p < min(max(a.nsel[bg], 0), min(sh.K, Cb))) {   // a count outside [0, min(K, C)] is clamped
-                    const int jj = a.idx[bg * sh.K + p];
-                    if ((unsigned)jj < (unsigned)Cb) {
-                        j = jj;
-                        lgl = a.gl[bg * sh.K + p] * kLog2e;
-                    }
+                } else if (p < min(max(ns, 0), min(sh.K, Cb)) && (unsigned)jj < (unsigned)Cb) {
+                    // a count outside [0, min(K, C)] is clamped; an index outside [0, C) skipped
+                    j = jj;
+                    lgl = gv * kLog2e;
                 }
                 if (j >= 0) {
                     if (a.table == nullptr) {
@@ -515,8 +525,11 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         return;
     }
 
-    // ---- consumers: warp 1 + c takes the CTA-local items c, c + kCons, ... ----
+    // ---- consumers: warps 1 + 2c and 2 + 2c (pair c) take the CTA-local items
+    // c, c + kCons, ...; the first warp of a pair takes keys 0-31 of each
+    // block, the second keys 32-63, each with its own online-softmax state ----
     const int cw = warp - 1;
+    const int pair = cw >> 1, hf = cw & 1;
     const int gq = lane >> 2, tq = lane & 3;
     const float qk = sh.scale * kLog2e;
     const uint32_t sbase = smem_u32(sm);
@@ -546,28 +559,29 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             for (int e = 0; e < 4; ++e) o[mt][e] = 0.f;
         float mrun[2] = {-INFINITY, -INFINITY}, lrun[2] = {0.f, 0.f};   // heads 2tq, 2tq+1
 
-        for (int64_t i = seg + (cw - (int)((seg - i0) % kCons) + kCons) % kCons; i < seg_end; i += kCons) {
+        for (int64_t i = seg + (pair - (int)((seg - i0) % kCons) + kCons) % kCons; i < seg_end; i += kCons) {
             const int li = (int)(i - i0);
             const int s = li % kFlatStages;
             if (ok && !tc::warp_wait_bar(&full[s], (uint32_t)((li / kFlatStages) & 1), abort)) ok = false;
             const int ntok = ok ? s_ntok[s] : 0;
             if (ntok > 0) {
                 const uint32_t kb0 = sbase + s * kItemBytes, kb1 = kb0 + 8192, vb0 = kb0 + 16384, vb1 = kb0 + 24576;
-                if (ntok < BS) {   // the current block: clear V rows >= ntok (128 bytes per row and box)
+                if (ntok < 32 * hf + 32) {   // the current block: clear this half's V rows >= ntok (128 bytes per row and box)
                     unsigned char* v0p = sm + s * kItemBytes + 16384;
-                    for (int e = ntok * 8 + lane; e < BS * 8; e += 32) {
+                    for (int e = max(ntok, 32 * hf) * 8 + lane; e < (32 * hf + 32) * 8; e += 32) {
                         reinterpret_cast<uint4*>(v0p)[e] = make_uint4(0, 0, 0, 0);
                         reinterpret_cast<uint4*>(v0p + 8192)[e] = make_uint4(0, 0, 0, 0);
                     }
                     __syncwarp();
                 }
                 const float lg = s_lg[s];
-                // ---- S^T = K q^T ----
-                float sc[4][4];
+                // ---- S^T = K q^T over this warp's 32 keys (m-tiles 2 hf, 2 hf + 1) ----
+                float sc[2][4];
 #pragma unroll
-                for (int mt = 0; mt < 4; ++mt) {
+                for (int m2 = 0; m2 < 2; ++m2) {
+                    const int mt = 2 * hf + m2;
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) sc[mt][e] = 0.f;
+                    for (int e = 0; e < 4; ++e) sc[m2][e] = 0.f;
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks) {
                         // matrices: (keys +0..7, dims +0..7), (keys +8..15, dims +0..7), (keys +0..7, dims +8..15), (keys +8.., dims +8..)
@@ -576,18 +590,18 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                         const uint32_t addr = sw_addr(chunk < 8 ? kb0 : kb1, key, chunk & 7);
                         uint32_t a0, a1, a2, a3;
                         ldsm_x4(addr, a0, a1, a2, a3);
-                        mma_bf16(sc[mt], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+                        mma_bf16(sc[m2], a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
                     }
                 }
                 // ---- online softmax (heads 2tq, 2tq+1; keys 16 mt + gq (+8)) ----
                 float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-                for (int mt = 0; mt < 4; ++mt)
+                for (int m2 = 0; m2 < 2; ++m2)
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int key = 16 * mt + gq + (e >> 1) * 8;
-                        const float v = key < ntok ? fmaf(sc[mt][e], qk, lg) : -INFINITY;
-                        sc[mt][e] = v;
+                        const int key = 16 * (2 * hf + m2) + gq + (e >> 1) * 8;
+                        const float v = key < ntok ? fmaf(sc[m2][e], qk, lg) : -INFINITY;
+                        sc[m2][e] = v;
                         mx[e & 1] = fmaxf(mx[e & 1], v);
                     }
                 float corr[2], psum[2] = {0.f, 0.f};
@@ -600,18 +614,18 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                     corr[h] = mrun[h] == -INFINITY ? 0.f : exp2f(mrun[h] - mn);
                     mrun[h] = mn;
                 }
-                uint32_t pb[4][2];   // P^T as B operand per k-step (16 keys)
+                uint32_t pb[2][2];   // P^T as B operand per k-step (16 keys)
 #pragma unroll
-                for (int mt = 0; mt < 4; ++mt) {
+                for (int m2 = 0; m2 < 2; ++m2) {
                     float p[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const float m = mrun[e & 1];
-                        p[e] = m == -INFINITY ? 0.f : exp2f(sc[mt][e] - m);
+                        p[e] = m == -INFINITY ? 0.f : exp2f(sc[m2][e] - m);
                         psum[e & 1] += p[e];
                     }
-                    pb[mt][0] = movm_t(pack_bf16(p[0], p[1]));   // keys 16 mt + 0..7
-                    pb[mt][1] = movm_t(pack_bf16(p[2], p[3]));   // keys 16 mt + 8..15
+                    pb[m2][0] = movm_t(pack_bf16(p[0], p[1]));   // keys 16 mt + 0..7
+                    pb[m2][1] = movm_t(pack_bf16(p[2], p[3]));   // keys 16 mt + 8..15
                 }
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
@@ -631,7 +645,8 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 #pragma unroll
                 for (int mt = 0; mt < 8; ++mt) {        // dims 16 mt .. + 15
 #pragma unroll
-                    for (int kst = 0; kst < 4; ++kst) { // keys 16 kst .. + 15
+                    for (int k2 = 0; k2 < 2; ++k2) {    // keys 16 kst .. + 15 of this warp's half
+                        const int kst = 2 * hf + k2;
                         // matrices (transposed on load): (keys +0..7, dims +0..7), (keys +0..7, dims +8..15),
                         // (keys +8..15, dims +0..7), (keys +8..15, dims +8..15)
                         const int key = 16 * kst + (lane & 7) + (lane >> 4) * 8;
@@ -639,7 +654,7 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                         const uint32_t addr = sw_addr(chunk < 8 ? vb0 : vb1, key, chunk & 7);
                         uint32_t a0, a1, a2, a3;
                         ldsm_x4_t(addr, a0, a1, a2, a3);
-                        mma_bf16(o[mt], a0, a1, a2, a3, pb[kst][0], pb[kst][1]);
+                        mma_bf16(o[mt], a0, a1, a2, a3, pb[k2][0], pb[k2][1]);
                     }
                 }
             }
@@ -665,11 +680,11 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                     x[16 + dim * 8 + h] = o[mt][e];
                 }
         }
-        asm volatile("bar.sync 1, %0;" ::"n"(32 * kCons) : "memory");
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsWarps) : "memory");
         if (cw == 0) {
             const bool good = ok && !*abort;
             float* rec = a.part + (cta + bg) * (int64_t)G * kRecF;
-            for (int c = 0; c < kCons - 1; ++c) {
+            for (int c = 0; c < kConsWarps - 1; ++c) {
                 const float* x = xch + c * (16 + 128 * 8);
                 float w1[2], w2[2];
 #pragma unroll
@@ -714,21 +729,21 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 *s_last = atomicAdd(&a.fin[bg], 1) == (int)(c_last - c_first);
             }
         }
-        asm volatile("bar.sync 1, %0;" ::"n"(32 * kCons) : "memory");   // xch is free; s_last is set
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsWarps) : "memory");   // xch is free; s_last is set
         if (*s_last) {
             // Both consumer warps merge the group's records:
             //   o = sum_r 2^(m_r - M) O_r / sum_r 2^(m_r - M) l_r,  M = max_r m_r,
             // staging every record's (m, l) first so that all loads are in flight together.
             __threadfence();
-            const int t = threadIdx.x - 32;                 // 0 .. 32 kCons - 1
+            const int t = threadIdx.x - 32;                 // 0 .. 32 kConsWarps - 1
             const int64_t c_first = flat_owner(fp, bg * nblk), c_last = flat_owner(fp, (bg + 1) * nblk - 1);
             const int R = (int)(c_last - c_first + 1);      // <= kMaxRecs by the plan
             const float* base = a.part + (c_first + bg) * (int64_t)G * kRecF;   // records are consecutive
-            for (int e = t; e < R * G; e += 32 * kCons) {
+            for (int e = t; e < R * G; e += 32 * kConsWarps) {
                 s_mg[e] = __ldcg(base + (int64_t)e * kRecF + D);
                 s_lg2[e] = __ldcg(base + (int64_t)e * kRecF + D + 1);
             }
-            asm volatile("bar.sync 1, %0;" ::"n"(32 * kCons) : "memory");
+            asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsWarps) : "memory");
             if (t < G) {
                 float M = -INFINITY, Lsum = 0.f;
                 for (int r = 0; r < R; ++r) M = fmaxf(M, s_mg[r * G + t]);
@@ -741,9 +756,9 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 const float inv = 1.f / Lsum;
                 for (int r = 0; r < R; ++r) s_wg[r * G + t] *= inv;
             }
-            asm volatile("bar.sync 1, %0;" ::"n"(32 * kCons) : "memory");
+            asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsWarps) : "memory");
             __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.o) + ((int64_t)b * sh.Hq + (int64_t)g * G) * D;
-            for (int e = t; e < G * (D / 4); e += 32 * kCons) {
+            for (int e = t; e < G * (D / 4); e += 32 * kConsWarps) {
                 const int h = e / (D / 4), q4 = e - h * (D / 4);
                 float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
