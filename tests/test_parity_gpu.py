@@ -341,6 +341,23 @@ def test_decode_ragged_lengths(decode_ws, N):
     decode_check(w, kc, vc, q, s, N, 31, groups, gate="none")
 
 
+@pytest.mark.parametrize("batch", [2, 4, 12, 24])
+def test_decode_group_splits(batch):
+    """Sparse decode at batch sizes that take each split of the block lists:
+    clusters of 8, 4 and 1 CTAs per (batch, KV head) (16, 32, 96 groups) and
+    the flat split over persistent CTAs once there are more groups than SMs
+    (192 groups)."""
+    w = synth.workload("decode", batch=batch, seq=8192 + 37)
+    kc, vc = U.build_decode_cache(w)
+    q = synth.decode_q(w)
+    s = torch.randn(batch, w.n_kv_heads, 1, w.n_blocks, generator=torch.Generator().manual_seed(batch))
+    groups = [(0, 0), (batch - 1, w.n_kv_heads - 1), (batch // 2, 3)]
+    decode_check(w, kc, vc, q, s, w.seq, 31, groups)
+    decode_check(w, kc, vc, q, s, w.seq, 15, groups[:2], gate="none")
+    del kc, vc
+    torch.cuda.empty_cache()
+
+
 def test_decode_dense(decode_ws):
     w, kc, vc, q, s = decode_ws
     decode_check(w, kc, vc, q, s, w.seq, 31, [(0, 0), (0, 5)], dense=True)

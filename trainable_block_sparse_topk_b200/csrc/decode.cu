@@ -54,6 +54,7 @@ struct DecArgs {
     int splits;
     FlatPlan fp;         // tensor-core path: item split
     int* fin;            // tensor-core path: [B*Hkv] records written per group, zeroed per call
+    int cs;              // tensor-core path: 0 = flat item split; >= 1: a cluster of cs CTAs per group
     // paged cache (tensor-core path): block j of sequence b is page
     // table[b * max_blocks + j] of the pools kc/vc [num_pages, Hkv, BS, D];
     // NULL table: the contiguous cache [B, Hkv, stride, D]
@@ -344,6 +345,8 @@ constexpr uint32_t kItemBytes = 32768;   // K box 0 | K box 1 | V box 0 | V box 
 constexpr int kMaxDecodeCtas = 160;     // grid bound (one CTA per SM)
 constexpr int kRecF = 132;              // floats per head in a record: O[128], m, l, 2 pad (16-byte rows)
 constexpr int kMaxRecs = 64;            // records of one group (CTAs sharing it), bounded by the plan
+constexpr int kXchF = 16 + 128 * 8;     // floats of one consumer's state: m[8], l[8], O^T[128][8]
+constexpr int kMaxCluster = 8;          // portable cluster size
 
 // Item split: CTA c owns [flat_start(c), flat_start(c + 1)).
 __host__ __device__ __forceinline__ int64_t flat_start(const FlatPlan& f, int64_t c) {
@@ -360,11 +363,15 @@ struct FlatSmem {
     static constexpr uint32_t kMisc = kBar + 16 * kFlatStages;        // abort flag
     static constexpr uint32_t kBlk = kMisc + 16;                      // i32 [S]: keys of the stage's item (0: none)
     static constexpr uint32_t kLg = kBlk + 4 * kFlatStages;           // f32 [S]: its log-gate (log2 units)
-    static constexpr uint32_t kXch = (kLg + 4 * kFlatStages + 15) & ~15u;   // per consumer 1..: m[8], l[8], O^T[128][8]
-    static constexpr uint32_t kLast = kXch + 4 * (kConsWarps - 1) * (16 + 128 * 8);   // i32: this CTA merges the group
-    static constexpr uint32_t kMerge = kLast + 16;                    // f32 m, l, weight [kMaxRecs][8] each
+    static constexpr uint32_t kXch = (kLg + 4 * kFlatStages + 15) & ~15u;   // per consumer: m[8], l[8], O^T[128][8]
+    static constexpr uint32_t kLast = kXch + 4 * kConsWarps * kXchF;  // i32: this CTA merges the group
+    // flat split: f32 m, l, weight [kMaxRecs][8] each (the last CTA's merge);
+    // cluster: this CTA's partial, G rows of kRecF floats (O, m, l) read by the leader
+    static constexpr uint32_t kMerge = kLast + 16;
     static constexpr uint32_t kTotal = kMerge + 3 * 4 * kMaxRecs * 8;
 };
+static_assert(3 * kMaxRecs * 8 >= 8 * kRecF, "the cluster partial fits the merge area");
+static_assert(FlatSmem::kTotal + 1024 <= 232448, "shared memory of one CTA");
 
 __device__ __forceinline__ uint32_t sw_addr(uint32_t box, int row, int chunk) {
     return box + (uint32_t)row * 128u + (uint32_t)((chunk ^ (row & 7)) << 4);
@@ -395,6 +402,36 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// The address of this CTA's shared-memory location `a` in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_shared(uint32_t a, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t a) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t a) {
+    float4 v;
+    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a) : "memory");
+    return v;
+}
+
+// kClu = false: flat item split over persistent CTAs, records merged by the
+// last CTA of each group. kClu = true: a cluster of a.cs CTAs per group, each
+// taking an even share of the group's items; the cluster's leader (rank 0)
+// reads the other CTAs' partials from their shared memory and writes o.
+template <bool kClu>
 __global__ void __launch_bounds__(kFlatThreads, 1)
 decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    const __grid_constant__ DecArgs a) {
@@ -418,11 +455,24 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     const int G = sh.G;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t cta = blockIdx.x;
-    const int64_t i0 = flat_start(fp, cta), i1 = flat_start(fp, cta + 1);
+    const int nblk = fp.nblk;
+    int64_t i0, i1;
+    uint32_t rank = 0;
+    if constexpr (kClu) {
+        // grid = groups x cs, cluster dims (cs, 1, 1): CTA rank r of cluster bg
+        // takes items [r per + min(r, rem), ...) of group bg
+        rank = cluster_rank();
+        const int64_t bg = cta / a.cs;
+        const int per = nblk / a.cs, rem = nblk % a.cs;
+        i0 = bg * nblk + (int64_t)rank * per + min((int)rank, rem);
+        i1 = i0 + per + ((int)rank < rem ? 1 : 0);
+    } else {
+        i0 = flat_start(fp, cta);
+        i1 = flat_start(fp, cta + 1);
+    }
     const int nitems = (int)(i1 - i0);
     const int64_t N = (int64_t)sh.q_offset + 1;       // the longest cache length
     const bool dense = a.idx == nullptr;
-    const int nblk = fp.nblk;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kFlatStages; ++s) {
@@ -521,6 +571,14 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             // let the copies already started land before the CTA exits
             for (int li = max(0, issued - kFlatStages); li < issued; ++li)
                 tc::drain_wait(&full[li % kFlatStages], (uint32_t)((li / kFlatStages) & 1));
+        }
+        if constexpr (kClu) {
+            if (a.cs > 1) {   // take part in both cluster barriers of the consumers
+                cluster_arrive();
+                cluster_wait();
+                cluster_arrive();
+                cluster_wait();
+            }
         }
         return;
     }
@@ -665,12 +723,16 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
             if (ok && lane == 0) tc::mbar_arrive(&empty[s]);
         }
 
-        // ---- merge the consumers; consumer 0 writes the CTA's record of group bg ----
-        if (cw > 0) {
-            float* x = xch + (cw - 1) * (16 + 128 * 8);
+        // ---- every consumer warp publishes its (m, l, O^T); a failed warp
+        // publishes l = NaN, which reaches every output it touches ----
+        {
+            float* x = xch + cw * kXchF;
             if (gq == 0) {
 #pragma unroll
-                for (int h = 0; h < 2; ++h) { x[2 * tq + h] = mrun[h]; x[8 + 2 * tq + h] = lrun[h]; }
+                for (int h = 0; h < 2; ++h) {
+                    x[2 * tq + h] = mrun[h];
+                    x[8 + 2 * tq + h] = ok ? lrun[h] : __int_as_float(0x7fc00000);
+                }
             }
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt)
@@ -681,97 +743,170 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 }
         }
         asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsWarps) : "memory");
-        if (cw == 0) {
-            const bool good = ok && !*abort;
-            float* rec = a.part + (cta + bg) * (int64_t)G * kRecF;
-            for (int c = 0; c < kConsWarps - 1; ++c) {
-                const float* x = xch + c * (16 + 128 * 8);
-                float w1[2], w2[2];
+        const int t = threadIdx.x - 32;                 // 0 .. 32 kConsWarps - 1
+        const bool bad = *abort != 0;
+        // The CTA's own merge of the six states for (head h, dims 4 q4 .. 4 q4 + 3):
+        //   m = max_w m_w,  l = sum_w 2^(m_w - m) l_w,  O = sum_w 2^(m_w - m) O_w
+        auto local_merge = [&](int h, int q4, float& m, float& l, float4& ov) {
+            m = -INFINITY;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const float m2 = x[2 * tq + h], l2 = x[8 + 2 * tq + h];
-                    const float M = fmaxf(mrun[h], m2);
-                    w1[h] = mrun[h] == -INFINITY ? 0.f : exp2f(mrun[h] - M);
-                    w2[h] = m2 == -INFINITY ? 0.f : exp2f(m2 - M);
-                    mrun[h] = M;
-                    lrun[h] = lrun[h] * w1[h] + l2 * w2[h];
-                }
+            for (int w = 0; w < kConsWarps; ++w) m = fmaxf(m, xch[w * kXchF + h]);
+            l = 0.f;
+            ov = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int dim = 16 * mt + gq + (e >> 1) * 8, h = 2 * tq + (e & 1);
-                        o[mt][e] = o[mt][e] * w1[e & 1] + x[16 + dim * 8 + h] * w2[e & 1];
-                    }
+            for (int w = 0; w < kConsWarps; ++w) {
+                const float* x = xch + w * kXchF;
+                const float mw = x[h];
+                const float wt = mw == -INFINITY ? 0.f : exp2f(mw - m);
+                l = fmaf(wt, x[8 + h], l);
+                const float* ow = x + 16 + (4 * q4) * 8 + h;
+                ov.x = fmaf(wt, ow[0], ov.x);
+                ov.y = fmaf(wt, ow[8], ov.y);
+                ov.z = fmaf(wt, ow[16], ov.z);
+                ov.w = fmaf(wt, ow[24], ov.w);
             }
-#pragma unroll
-            for (int mt = 0; mt < 8; ++mt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int dim = 16 * mt + gq + (e >> 1) * 8, h = 2 * tq + (e & 1);
-                    if (h < G) rec[h * kRecF + dim] = good ? o[mt][e] : __int_as_float(0x7fc00000);
+        };
+        __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.o) + ((int64_t)b * sh.Hq + (int64_t)g * G) * D;
+        auto store_out = [&](int h, int q4, float4 ov, float l) {
+            const float inv = 1.f / l;
+            const bool nan = bad || !(l > 0.f);
+            const float f = __int_as_float(0x7fc00000);
+            reinterpret_cast<uint2*>(ob + (int64_t)h * D)[q4] =
+                nan ? make_uint2(pack_bf16(f, f), pack_bf16(f, f))
+                    : make_uint2(pack_bf16(ov.x * inv, ov.y * inv), pack_bf16(ov.z * inv, ov.w * inv));
+        };
+        if constexpr (kClu) {
+            const int cs = a.cs;
+            float* part = reinterpret_cast<float*>(sm + L::kMerge);
+            if (cs == 1) {
+                for (int e = t; e < G * (D / 4); e += 32 * kConsWarps) {
+                    const int h = e / (D / 4), q4 = e - h * (D / 4);
+                    float m, l;
+                    float4 ov;
+                    local_merge(h, q4, m, l, ov);
+                    store_out(h, q4, ov, l);
                 }
-            if (gq == 0) {
+            } else if (rank != 0) {
+                // publish this CTA's partial in its own shared memory for the leader
+                for (int e = t; e < G * (D / 4); e += 32 * kConsWarps) {
+                    const int h = e / (D / 4), q4 = e - h * (D / 4);
+                    float m, l;
+                    float4 ov;
+                    local_merge(h, q4, m, l, ov);
+                    if (bad) l = __int_as_float(0x7fc00000);
+                    reinterpret_cast<float4*>(part + h * kRecF)[q4] = ov;
+                    if (q4 == 0) { part[h * kRecF + D] = m; part[h * kRecF + D + 1] = l; }
+                }
+                cluster_arrive();   // (1) the partial is written
+                cluster_wait();
+                cluster_arrive();   // (2) the leader has read it: this CTA may exit
+                cluster_wait();
+            } else {
+                cluster_arrive();   // (1)
+                cluster_wait();
+                const uint32_t pl = smem_u32(part);
+                for (int e = t; e < G * (D / 4); e += 32 * kConsWarps) {
+                    const int h = e / (D / 4), q4 = e - h * (D / 4);
+                    float m, l;
+                    float4 ov;
+                    local_merge(h, q4, m, l, ov);
+                    // the other CTAs' (m, l, O), loads issued together
+                    float mr[kMaxCluster], lr[kMaxCluster];
+                    float4 orr[kMaxCluster];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int hh = 2 * tq + h;
-                    if (hh < G) {
-                        rec[hh * kRecF + D] = mrun[h];
-                        rec[hh * kRecF + D + 1] = lrun[h];
+                    for (int r = 1; r < kMaxCluster; ++r) {
+                        if (r < cs) {
+                            const uint32_t ra = map_shared(pl, (uint32_t)r) + (uint32_t)(h * kRecF) * 4u;
+                            mr[r] = ld_cluster_f32(ra + 4u * D);
+                            lr[r] = ld_cluster_f32(ra + 4u * (D + 1));
+                            orr[r] = ld_cluster_f32x4(ra + 16u * q4);
+                        }
                     }
+                    float M = m;
+#pragma unroll
+                    for (int r = 1; r < kMaxCluster; ++r)
+                        if (r < cs) M = fmaxf(M, mr[r]);
+                    const float w0 = m == -INFINITY ? 0.f : exp2f(m - M);
+                    float Ls = w0 * l;
+                    float4 acc = make_float4(w0 * ov.x, w0 * ov.y, w0 * ov.z, w0 * ov.w);
+#pragma unroll
+                    for (int r = 1; r < kMaxCluster; ++r) {
+                        if (r < cs) {
+                            const float wr = mr[r] == -INFINITY ? 0.f : exp2f(mr[r] - M);
+                            Ls = fmaf(wr, lr[r], Ls);
+                            acc.x = fmaf(wr, orr[r].x, acc.x);
+                            acc.y = fmaf(wr, orr[r].y, acc.y);
+                            acc.z = fmaf(wr, orr[r].z, acc.z);
+                            acc.w = fmaf(wr, orr[r].w, acc.w);
+                        }
+                    }
+                    store_out(h, q4, acc, Ls);
                 }
+                cluster_arrive();   // (2)
+                cluster_wait();
+            }
+        } else {
+            // the CTA's record of group bg: O, m, l of each head, 16-byte rows
+            float* rec = a.part + (cta + bg) * (int64_t)G * kRecF;
+            for (int e = t; e < G * (D / 4); e += 32 * kConsWarps) {
+                const int h = e / (D / 4), q4 = e - h * (D / 4);
+                float m, l;
+                float4 ov;
+                local_merge(h, q4, m, l, ov);
+                if (bad) l = __int_as_float(0x7fc00000);
+                reinterpret_cast<float4*>(rec + h * kRecF)[q4] = ov;
+                if (q4 == 0) { rec[h * kRecF + D] = m; rec[h * kRecF + D + 1] = l; }
             }
             // the last CTA of the group to get here merges its records
             __threadfence();
-            __syncwarp();
-            if (lane == 0) {
+            asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsWarps) : "memory");   // xch is free
+            if (t == 0) {
                 const int64_t c_first = flat_owner(fp, bg * nblk), c_last = flat_owner(fp, (bg + 1) * nblk - 1);
                 *s_last = atomicAdd(&a.fin[bg], 1) == (int)(c_last - c_first);
             }
-        }
-        asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsWarps) : "memory");   // xch is free; s_last is set
-        if (*s_last) {
-            // Both consumer warps merge the group's records:
-            //   o = sum_r 2^(m_r - M) O_r / sum_r 2^(m_r - M) l_r,  M = max_r m_r,
-            // staging every record's (m, l) first so that all loads are in flight together.
-            __threadfence();
-            const int t = threadIdx.x - 32;                 // 0 .. 32 kConsWarps - 1
-            const int64_t c_first = flat_owner(fp, bg * nblk), c_last = flat_owner(fp, (bg + 1) * nblk - 1);
-            const int R = (int)(c_last - c_first + 1);      // <= kMaxRecs by the plan
-            const float* base = a.part + (c_first + bg) * (int64_t)G * kRecF;   // records are consecutive
-            for (int e = t; e < R * G; e += 32 * kConsWarps) {
-                s_mg[e] = __ldcg(base + (int64_t)e * kRecF + D);
-                s_lg2[e] = __ldcg(base + (int64_t)e * kRecF + D + 1);
-            }
-            asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsWarps) : "memory");
-            if (t < G) {
-                float M = -INFINITY, Lsum = 0.f;
-                for (int r = 0; r < R; ++r) M = fmaxf(M, s_mg[r * G + t]);
-                for (int r = 0; r < R; ++r) {
-                    const float mr = s_mg[r * G + t];
-                    const float w = mr == -INFINITY ? 0.f : exp2f(mr - M);
-                    s_wg[r * G + t] = w;
-                    Lsum = fmaf(w, s_lg2[r * G + t], Lsum);
+            asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsWarps) : "memory");   // s_last is set
+            if (*s_last) {
+                // Both consumer warps merge the group's records:
+                //   o = sum_r 2^(m_r - M) O_r / sum_r 2^(m_r - M) l_r,  M = max_r m_r,
+                // staging every record's (m, l) first so that all loads are in flight together.
+                __threadfence();
+                const int64_t c_first = flat_owner(fp, bg * nblk), c_last = flat_owner(fp, (bg + 1) * nblk - 1);
+                const int R = (int)(c_last - c_first + 1);      // <= kMaxRecs by the plan
+                const float* base = a.part + (c_first + bg) * (int64_t)G * kRecF;   // records are consecutive
+                for (int e = t; e < R * G; e += 32 * kConsWarps) {
+                    s_mg[e] = __ldcg(base + (int64_t)e * kRecF + D);
+                    s_lg2[e] = __ldcg(base + (int64_t)e * kRecF + D + 1);
                 }
-                const float inv = 1.f / Lsum;
-                for (int r = 0; r < R; ++r) s_wg[r * G + t] *= inv;
-            }
-            asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsWarps) : "memory");
-            __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.o) + ((int64_t)b * sh.Hq + (int64_t)g * G) * D;
-            for (int e = t; e < G * (D / 4); e += 32 * kConsWarps) {
-                const int h = e / (D / 4), q4 = e - h * (D / 4);
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsWarps) : "memory");
+                if (t < G) {
+                    float M = -INFINITY, Lsum = 0.f;
+                    for (int r = 0; r < R; ++r) M = fmaxf(M, s_mg[r * G + t]);
+                    for (int r = 0; r < R; ++r) {
+                        const float mr = s_mg[r * G + t];
+                        const float w = mr == -INFINITY ? 0.f : exp2f(mr - M);
+                        s_wg[r * G + t] = w;
+                        Lsum = fmaf(w, s_lg2[r * G + t], Lsum);
+                    }
+                    const float inv = 1.f / Lsum;
+                    for (int r = 0; r < R; ++r) s_wg[r * G + t] *= inv;
+                }
+                asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsWarps) : "memory");
+                for (int e = t; e < G * (D / 4); e += 32 * kConsWarps) {
+                    const int h = e / (D / 4), q4 = e - h * (D / 4);
+                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
-                for (int r = 0; r < R; ++r) {
-                    const float w = s_wg[r * G + h];
-                    const float4 v = __ldcg(reinterpret_cast<const float4*>(base + ((int64_t)r * G + h) * kRecF) + q4);
-                    acc.x = fmaf(w, v.x, acc.x);
-                    acc.y = fmaf(w, v.y, acc.y);
-                    acc.z = fmaf(w, v.z, acc.z);
-                    acc.w = fmaf(w, v.w, acc.w);
+                    for (int r = 0; r < R; ++r) {
+                        const float w = s_wg[r * G + h];
+                        const float4 v = __ldcg(reinterpret_cast<const float4*>(base + ((int64_t)r * G + h) * kRecF) + q4);
+                        acc.x = fmaf(w, v.x, acc.x);
+                        acc.y = fmaf(w, v.y, acc.y);
+                        acc.z = fmaf(w, v.z, acc.z);
+                        acc.w = fmaf(w, v.w, acc.w);
+                    }
+                    reinterpret_cast<uint2*>(ob + (int64_t)h * D)[q4] =
+                        make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
                 }
-                reinterpret_cast<uint2*>(ob + (int64_t)h * D)[q4] =
-                    make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
+                // s_mg .. s_wg are read again only after the next segment's barriers
             }
         }
         seg = seg_end;
@@ -855,20 +990,96 @@ int decode_sms() {
     return std::min(n, kMaxDecodeCtas);
 }
 
-cudaError_t run_decode_flat(const DecArgs& a, cudaStream_t st) {
+constexpr size_t kFlatSmemBytes = FlatSmem::kTotal + 1024;
+
+// Clusters of cs CTAs that the current device can hold at once (0 if the
+// query fails), looked up once per device and size.
+int max_active_clusters(int cs) {
+    constexpr int kDevs = 64;
+    static std::mutex mu;
+    static int cache[kDevs][kMaxCluster + 1];
+    static bool known[kDevs][kMaxCluster + 1];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevs || cs < 1 || cs > kMaxCluster) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!known[dev][cs]) {
+        int n = 0;
+        if (cudaFuncSetAttribute(decode_flat_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kFlatSmemBytes) == cudaSuccess) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3((unsigned)cs);
+            cfg.blockDim = dim3(kFlatThreads);
+            cfg.dynamicSmemBytes = kFlatSmemBytes;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = (unsigned)cs;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            if (cudaOccupancyMaxActiveClusters(&n, decode_flat_kernel<true>, &cfg) != cudaSuccess) n = 0;
+        }
+        (void)cudaGetLastError();
+        cache[dev][cs] = n;
+        known[dev][cs] = true;
+    }
+    return cache[dev][cs];
+}
+
+// Cluster size of the tensor-core decode, 0 for the flat split. Short block
+// lists (a sparse selection: nblk <= 128) with at most one group per SM get
+// one cluster per group, as large as every cluster stays resident at once
+// (<= 8, <= nblk, groups x cs <= SMs): the partials then meet in the leader's
+// shared memory, and no record, counter or second pass over L2 is needed.
+// Long lists (dense decode) and more groups than SMs use the flat split.
+int decode_cluster_size(int64_t groups, int nblk) {
+    if (nblk > 128 || groups > decode_sms()) return 0;
+    for (int cs = kMaxCluster; cs >= 1; cs >>= 1)
+        if (cs <= nblk && groups * cs <= decode_sms() && (cs == 1 || max_active_clusters(cs) >= groups)) return cs;
+    return 0;
+}
+
+cudaError_t run_decode_flat(DecArgs a, cudaStream_t st) {
     CUtensorMap mk, mv;
     const uint64_t rows = a.table == nullptr ? (uint64_t)a.sh.B * a.sh.Hkv * (uint64_t)a.stride
                                              : (uint64_t)a.num_pages * a.sh.Hkv * 64;
     if (!encode_bf16_2d(&mk, a.kc, rows, 128, 64) || !encode_bf16_2d(&mv, a.vc, rows, 128, 64))
         return cudaErrorInvalidValue;
-    const size_t smem = FlatSmem::kTotal + 1024;
-    cudaError_t e = cudaFuncSetAttribute(decode_flat_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const int64_t groups = (int64_t)a.sh.B * a.sh.Hkv;
+    a.cs = decode_cluster_size(groups, a.fp.nblk);
+    cudaError_t e;
+    if (a.cs > 0) {
+        e = cudaFuncSetAttribute(decode_flat_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kFlatSmemBytes);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(groups * a.cs));
+        cfg.blockDim = dim3(kFlatThreads);
+        cfg.dynamicSmemBytes = kFlatSmemBytes;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)a.cs;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        {
+            KernelTimer kt("decode_flat", st);
+            e = cudaLaunchKernelEx(&cfg, decode_flat_kernel<true>, mk, mv, a);
+        }
+        if (e == cudaSuccess) e = cudaGetLastError();
+        if (e == cudaSuccess) count_launches(1);
+        return e;
+    }
+    e = cudaFuncSetAttribute(decode_flat_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kFlatSmemBytes);
     if (e != cudaSuccess) return e;
-    e = cudaMemsetAsync(a.fin, 0, sizeof(int) * (size_t)a.sh.B * a.sh.Hkv, st);
+    e = cudaMemsetAsync(a.fin, 0, sizeof(int) * (size_t)groups, st);
     if (e != cudaSuccess) return e;
     {
         KernelTimer kt("decode_flat", st);
-        decode_flat_kernel<<<(unsigned)a.fp.ncta, kFlatThreads, smem, st>>>(mk, mv, a);
+        decode_flat_kernel<false><<<(unsigned)a.fp.ncta, kFlatThreads, kFlatSmemBytes, st>>>(mk, mv, a);
     }
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
@@ -948,13 +1159,13 @@ cudaError_t launch_decode(const Shape& s, const void* q, const void* kc, const v
                           cudaStream_t st) {
     const bool dense = idx == nullptr;
     if (decode_flat_supported(s, stride)) {
-        DecArgs a{s, q, kc, vc, stride, idx, gl, nsel, part, o, 0, 0, flat_plan(s, dense), nullptr,
+        DecArgs a{s, q, kc, vc, stride, idx, gl, nsel, part, o, 0, 0, flat_plan(s, dense), nullptr, 0,
                   nullptr, 0, 0, nullptr};
         a.fin = reinterpret_cast<int*>(reinterpret_cast<unsigned char*>(part) + flat_record_bytes(s));
         return run_decode_flat(a, st);
     }
     const DecodePlan p = decode_plan(s, dense);
-    DecArgs a{s, q, kc, vc, stride, idx, gl, nsel, part, o, p.bpc, p.splits, FlatPlan{}, nullptr,
+    DecArgs a{s, q, kc, vc, stride, idx, gl, nsel, part, o, p.bpc, p.splits, FlatPlan{}, nullptr, 0,
               nullptr, 0, 0, nullptr};
     if (s.dtype == SAS_DT_FP32) return decode_d<float>(a, st);
     return decode_d<__nv_bfloat16>(a, st);
@@ -973,7 +1184,7 @@ cudaError_t launch_decode_paged(const Shape& s, const void* q, const void* kp, c
                                 const int32_t* table, int max_blocks, const int32_t* lens, const int32_t* idx,
                                 const float* gl, const int32_t* nsel, void* o, float* part, cudaStream_t st) {
     const bool dense = idx == nullptr;
-    DecArgs a{s, q, kp, vp, 0, idx, gl, nsel, part, o, 0, 0, flat_plan(s, dense), nullptr,
+    DecArgs a{s, q, kp, vp, 0, idx, gl, nsel, part, o, 0, 0, flat_plan(s, dense), nullptr, 0,
               table, max_blocks, num_pages, lens};
     a.fin = reinterpret_cast<int*>(reinterpret_cast<unsigned char*>(part) + flat_record_bytes(s));
     return run_decode_flat(a, st);
