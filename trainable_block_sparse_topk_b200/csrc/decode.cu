@@ -345,7 +345,11 @@ constexpr uint32_t kItemBytes = 32768;   // K box 0 | K box 1 | V box 0 | V box 
 constexpr int kMaxDecodeCtas = 160;     // grid bound (one CTA per SM)
 constexpr int kRecF = 132;              // floats per head in a record: O[128], m, l, 2 pad (16-byte rows)
 constexpr int kMaxRecs = 64;            // records of one group (CTAs sharing it), bounded by the plan
-constexpr int kXchF = 16 + 128 * 8;     // floats of one consumer's state: m[8], l[8], O^T[128][8]
+// One consumer's state in shared memory: m[8], l[8], then O[8 heads][kXchRow]
+// (128 dims + 4 pad: the publishing lanes (8 dims x 4 head pairs) hit 32
+// distinct banks, and a warp reading one head's row takes whole 16-byte runs).
+constexpr int kXchRow = 132;
+constexpr int kXchF = 16 + 8 * kXchRow;
 constexpr int kMaxCluster = 8;          // portable cluster size
 
 // Item split: CTA c owns [flat_start(c), flat_start(c + 1)).
@@ -360,10 +364,10 @@ __host__ __device__ __forceinline__ int64_t flat_owner(const FlatPlan& f, int64_
 
 struct FlatSmem {
     static constexpr uint32_t kBar = kFlatStages * kItemBytes;        // full[S], empty[S]
-    static constexpr uint32_t kMisc = kBar + 16 * kFlatStages;        // abort flag
+    static constexpr uint32_t kMisc = kBar + 16 * kFlatStages;        // i32 abort flag; mbarrier rcv at + 8
     static constexpr uint32_t kBlk = kMisc + 16;                      // i32 [S]: keys of the stage's item (0: none)
     static constexpr uint32_t kLg = kBlk + 4 * kFlatStages;           // f32 [S]: its log-gate (log2 units)
-    static constexpr uint32_t kXch = (kLg + 4 * kFlatStages + 15) & ~15u;   // per consumer: m[8], l[8], O^T[128][8]
+    static constexpr uint32_t kXch = (kLg + 4 * kFlatStages + 15) & ~15u;   // per consumer: m[8], l[8], O[8][kXchRow]
     static constexpr uint32_t kLast = kXch + 4 * kConsWarps * kXchF;  // i32: this CTA merges the group
     // flat split: f32 m, l, weight [kMaxRecs][8] each (the last CTA's merge);
     // cluster: this CTA's partial, G rows of kRecF floats (O, m, l) read by the leader
@@ -402,7 +406,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire;" ::: "memory"); }
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
@@ -415,16 +418,28 @@ __device__ __forceinline__ uint32_t map_shared(uint32_t a, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
     return r;
 }
-__device__ __forceinline__ float ld_cluster_f32(uint32_t a) {
-    float v;
-    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
-    return v;
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
 }
-__device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t a) {
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(a) : "memory");
-    return v;
+// Asynchronous 16-byte store into another CTA's shared memory that counts its
+// bytes on that CTA's mbarrier (both addresses in the cluster window).
+__device__ __forceinline__ void st_async_f32x4(uint32_t a, float4 v, uint32_t bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
+                 ::"r"(a), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(bar) : "memory");
+}
+// Bounded wait, with cluster-scope acquire, for the partials that the other
+// CTAs of the cluster store into this CTA's shared memory.
+__device__ __forceinline__ bool rcv_wait(uint64_t* bar, unsigned long long lim) {
+    const uint64_t t0 = global_ns();
+    while (true) {
+        uint32_t done;
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], 0;\n"
+            " selp.u32 %0, 1, 0, p;\n}"
+            : "=r"(done) : "r"(smem_u32(bar)) : "memory");
+        if (done) return true;
+        if (global_ns() - t0 > lim) return false;
+    }
 }
 
 // kClu = false: flat item split over persistent CTAs, records merged by the
@@ -459,13 +474,22 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     int64_t i0, i1;
     uint32_t rank = 0;
     if constexpr (kClu) {
-        // grid = groups x cs, cluster dims (cs, 1, 1): CTA rank r of cluster bg
-        // takes items [r per + min(r, rem), ...) of group bg
+        // grid = groups x cs, cluster dims (cs, 1, 1). The leader (rank 0) takes
+        // the first n0 items of group bg (n0 = nblk / 2 for cs = 2, at most
+        // kCons for larger clusters, all of them for cs = 1); ranks 1 .. cs - 1
+        // share the rest evenly.
         rank = cluster_rank();
-        const int64_t bg = cta / a.cs;
-        const int per = nblk / a.cs, rem = nblk % a.cs;
-        i0 = bg * nblk + (int64_t)rank * per + min((int)rank, rem);
-        i1 = i0 + per + ((int)rank < rem ? 1 : 0);
+        const int cs = a.cs;
+        const int64_t bg = cta / cs;
+        const int n0 = cs == 1 ? nblk : cs == 2 ? nblk / 2 : min(kCons, nblk / cs);
+        if (rank == 0) {
+            i0 = bg * nblk;
+            i1 = i0 + n0;
+        } else {
+            const int rest = nblk - n0, per = rest / (cs - 1), rem = rest % (cs - 1), r = (int)rank - 1;
+            i0 = bg * nblk + n0 + (int64_t)r * per + min(r, rem);
+            i1 = i0 + per + (r < rem ? 1 : 0);
+        }
     } else {
         i0 = flat_start(fp, cta);
         i1 = flat_start(fp, cta + 1);
@@ -474,15 +498,26 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     const int64_t N = (int64_t)sh.q_offset + 1;       // the longest cache length
     const bool dense = a.idx == nullptr;
 
+    uint64_t* rcv = reinterpret_cast<uint64_t*>(sm + L::kMisc + 8);
+    const bool clu = kClu && a.cs > 1;
     if (threadIdx.x == 0) {
         for (int s = 0; s < kFlatStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 2);   // both warps of the owning pair
         }
+        mbar_init(rcv, 1);
+        // the leader expects G rows of kRecF floats from each other CTA
+        if (clu && rank == 0) mbar_arrive_expect_tx(rcv, (uint32_t)((a.cs - 1) * G * kRecF * 4));
         *abort = 0;
         fence_mbar_init();
     }
     __syncthreads();
+    // Every CTA's barriers are initialised before any CTA of the cluster
+    // stores into the leader (the senders wait on this arrival before storing).
+    if (clu) cluster_arrive_relaxed();
+    // Stage ring: a cluster leader with cs >= 4 takes at most kCons items and
+    // uses stages 0 .. kCons - 1 only; the rest receives the other partials.
+    const int nst = (clu && a.cs >= 4 && rank == 0) ? kCons : kFlatStages;
 
     if (warp == 0) {
         // ---- producer ----
@@ -545,8 +580,8 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 const float lg = __shfl_sync(0xffffffffu, lgl, k);
                 int fail = 0;
                 if (lane == 0) {
-                    const int s = li % kFlatStages;
-                    if (li >= kFlatStages && !tc::wait_bar(&empty[s], (uint32_t)(((li / kFlatStages) - 1) & 1), abort)) {
+                    const int s = li % nst;
+                    if (li >= nst && !tc::wait_bar(&empty[s], (uint32_t)(((li / nst) - 1) & 1), abort)) {
                         fail = 1;
                     } else {
                         s_ntok[s] = nt;
@@ -569,16 +604,8 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         }
         if (lane == 0 && stop) {
             // let the copies already started land before the CTA exits
-            for (int li = max(0, issued - kFlatStages); li < issued; ++li)
-                tc::drain_wait(&full[li % kFlatStages], (uint32_t)((li / kFlatStages) & 1));
-        }
-        if constexpr (kClu) {
-            if (a.cs > 1) {   // take part in both cluster barriers of the consumers
-                cluster_arrive();
-                cluster_wait();
-                cluster_arrive();
-                cluster_wait();
-            }
+            for (int li = max(0, issued - nst); li < issued; ++li)
+                tc::drain_wait(&full[li % nst], (uint32_t)((li / nst) & 1));
         }
         return;
     }
@@ -619,8 +646,8 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 
         for (int64_t i = seg + (pair - (int)((seg - i0) % kCons) + kCons) % kCons; i < seg_end; i += kCons) {
             const int li = (int)(i - i0);
-            const int s = li % kFlatStages;
-            if (ok && !tc::warp_wait_bar(&full[s], (uint32_t)((li / kFlatStages) & 1), abort)) ok = false;
+            const int s = li % nst;
+            if (ok && !tc::warp_wait_bar(&full[s], (uint32_t)((li / nst) & 1), abort)) ok = false;
             const int ntok = ok ? s_ntok[s] : 0;
             if (ntok > 0) {
                 const uint32_t kb0 = sbase + s * kItemBytes, kb1 = kb0 + 8192, vb0 = kb0 + 16384, vb1 = kb0 + 24576;
@@ -739,7 +766,7 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int dim = 16 * mt + gq + (e >> 1) * 8, h = 2 * tq + (e & 1);
-                    x[16 + dim * 8 + h] = o[mt][e];
+                    x[16 + h * kXchRow + dim] = o[mt][e];
                 }
         }
         asm volatile("bar.sync 1, %0;" ::"n"(32 * kConsWarps) : "memory");
@@ -759,11 +786,11 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 const float mw = x[h];
                 const float wt = mw == -INFINITY ? 0.f : exp2f(mw - m);
                 l = fmaf(wt, x[8 + h], l);
-                const float* ow = x + 16 + (4 * q4) * 8 + h;
-                ov.x = fmaf(wt, ow[0], ov.x);
-                ov.y = fmaf(wt, ow[8], ov.y);
-                ov.z = fmaf(wt, ow[16], ov.z);
-                ov.w = fmaf(wt, ow[24], ov.w);
+                const float4 ow = reinterpret_cast<const float4*>(x + 16 + h * kXchRow)[q4];
+                ov.x = fmaf(wt, ow.x, ov.x);
+                ov.y = fmaf(wt, ow.y, ov.y);
+                ov.z = fmaf(wt, ow.z, ov.z);
+                ov.w = fmaf(wt, ow.w, ov.w);
             }
         };
         __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.o) + ((int64_t)b * sh.Hq + (int64_t)g * G) * D;
@@ -777,7 +804,6 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
         };
         if constexpr (kClu) {
             const int cs = a.cs;
-            float* part = reinterpret_cast<float*>(sm + L::kMerge);
             if (cs == 1) {
                 for (int e = t; e < G * (D / 4); e += 32 * kConsWarps) {
                     const int h = e / (D / 4), q4 = e - h * (D / 4);
@@ -786,64 +812,54 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                     local_merge(h, q4, m, l, ov);
                     store_out(h, q4, ov, l);
                 }
-            } else if (rank != 0) {
-                // publish this CTA's partial in its own shared memory for the leader
-                for (int e = t; e < G * (D / 4); e += 32 * kConsWarps) {
-                    const int h = e / (D / 4), q4 = e - h * (D / 4);
-                    float m, l;
-                    float4 ov;
-                    local_merge(h, q4, m, l, ov);
-                    if (bad) l = __int_as_float(0x7fc00000);
-                    reinterpret_cast<float4*>(part + h * kRecF)[q4] = ov;
-                    if (q4 == 0) { part[h * kRecF + D] = m; part[h * kRecF + D + 1] = l; }
-                }
-                cluster_arrive();   // (1) the partial is written
-                cluster_wait();
-                cluster_arrive();   // (2) the leader has read it: this CTA may exit
-                cluster_wait();
             } else {
-                cluster_arrive();   // (1)
-                cluster_wait();
-                const uint32_t pl = smem_u32(part);
-                for (int e = t; e < G * (D / 4); e += 32 * kConsWarps) {
-                    const int h = e / (D / 4), q4 = e - h * (D / 4);
-                    float m, l;
-                    float4 ov;
-                    local_merge(h, q4, m, l, ov);
-                    // the other CTAs' (m, l, O), loads issued together
-                    float mr[kMaxCluster], lr[kMaxCluster];
-                    float4 orr[kMaxCluster];
-#pragma unroll
-                    for (int r = 1; r < kMaxCluster; ++r) {
-                        if (r < cs) {
-                            const uint32_t ra = map_shared(pl, (uint32_t)r) + (uint32_t)(h * kRecF) * 4u;
-                            mr[r] = ld_cluster_f32(ra + 4u * D);
-                            lr[r] = ld_cluster_f32(ra + 4u * (D + 1));
-                            orr[r] = ld_cluster_f32x4(ra + 16u * q4);
-                        }
+                // the leader's receive buffer: [cs - 1][G][kRecF] floats
+                const uint32_t recv_off = cs == 2 ? L::kMerge : (uint32_t)kCons * kItemBytes;
+                if (rank != 0) {
+                    // store this CTA's partial into the leader once its barriers exist
+                    cluster_wait();
+                    const uint32_t dst = map_shared(sbase + recv_off, 0u) + ((rank - 1) * G * kRecF) * 4u;
+                    const uint32_t rbar = map_shared(smem_u32(rcv), 0u);
+                    for (int e = t; e < G * (D / 4); e += 32 * kConsWarps) {
+                        const int h = e / (D / 4), q4 = e - h * (D / 4);
+                        float m, l;
+                        float4 ov;
+                        local_merge(h, q4, m, l, ov);
+                        if (bad) l = __int_as_float(0x7fc00000);
+                        st_async_f32x4(dst + (uint32_t)(h * kRecF + 4 * q4) * 4u, ov, rbar);
+                        if (q4 == 0) st_async_f32x4(dst + (uint32_t)(h * kRecF + D) * 4u, make_float4(m, l, 0.f, 0.f), rbar);
                     }
-                    float M = m;
-#pragma unroll
-                    for (int r = 1; r < kMaxCluster; ++r)
-                        if (r < cs) M = fmaxf(M, mr[r]);
-                    const float w0 = m == -INFINITY ? 0.f : exp2f(m - M);
-                    float Ls = w0 * l;
-                    float4 acc = make_float4(w0 * ov.x, w0 * ov.y, w0 * ov.z, w0 * ov.w);
-#pragma unroll
-                    for (int r = 1; r < kMaxCluster; ++r) {
-                        if (r < cs) {
-                            const float wr = mr[r] == -INFINITY ? 0.f : exp2f(mr[r] - M);
-                            Ls = fmaf(wr, lr[r], Ls);
-                            acc.x = fmaf(wr, orr[r].x, acc.x);
-                            acc.y = fmaf(wr, orr[r].y, acc.y);
-                            acc.z = fmaf(wr, orr[r].z, acc.z);
-                            acc.w = fmaf(wr, orr[r].w, acc.w);
+                } else {
+                    // A sender that gave up on a wait still stores (NaN) within
+                    // about one wait limit: wait three before giving up here.
+                    const bool got = rcv_wait(rcv, 3ull * g_sas_wait_limit_ns);
+                    if (!got && t == 0) atomicAdd(&g_sas_wait_timeouts, 1u);
+                    const float* rv = reinterpret_cast<const float*>(sm + recv_off);
+                    for (int e = t; e < G * (D / 4); e += 32 * kConsWarps) {
+                        const int h = e / (D / 4), q4 = e - h * (D / 4);
+                        float m, l;
+                        float4 ov;
+                        local_merge(h, q4, m, l, ov);
+                        float M = m;
+                        for (int r = 0; r < cs - 1; ++r) M = fmaxf(M, rv[(r * G + h) * kRecF + D]);
+                        const float w0 = m == -INFINITY ? 0.f : exp2f(m - M);
+                        float Ls = w0 * l;
+                        float4 acc = make_float4(w0 * ov.x, w0 * ov.y, w0 * ov.z, w0 * ov.w);
+                        for (int r = 0; r < cs - 1; ++r) {
+                            const float* x = rv + (r * G + h) * kRecF;
+                            const float mr = x[D];
+                            const float wr = mr == -INFINITY ? 0.f : exp2f(mr - M);
+                            Ls = fmaf(wr, x[D + 1], Ls);
+                            const float4 v = reinterpret_cast<const float4*>(x)[q4];
+                            acc.x = fmaf(wr, v.x, acc.x);
+                            acc.y = fmaf(wr, v.y, acc.y);
+                            acc.z = fmaf(wr, v.z, acc.z);
+                            acc.w = fmaf(wr, v.w, acc.w);
                         }
+                        if (!got) Ls = __int_as_float(0x7fc00000);
+                        store_out(h, q4, acc, Ls);
                     }
-                    store_out(h, q4, acc, Ls);
                 }
-                cluster_arrive();   // (2)
-                cluster_wait();
             }
         } else {
             // the CTA's record of group bg: O, m, l of each head, 16-byte rows
