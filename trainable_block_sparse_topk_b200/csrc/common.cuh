@@ -130,6 +130,14 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Programmatic dependent launch. A kernel launched with the programmatic
+// stream serialization attribute may start before the kernel ahead of it in
+// the stream has finished (once that kernel calls pdl_trigger, or ends); it
+// must call pdl_wait before it touches memory that earlier work writes.
+// Both are no-ops in a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ uint64_t global_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));

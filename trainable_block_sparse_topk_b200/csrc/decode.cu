@@ -518,6 +518,9 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
     // Stage ring: a cluster leader with cs >= 4 takes at most kCons items and
     // uses stages 0 .. kCons - 1 only; the rest receives the other partials.
     const int nst = (clu && a.cs >= 4 && rank == 0) ? kCons : kFlatStages;
+    // Launched right behind the top-K, this CTA may already be running:
+    // everything below reads what earlier kernels wrote.
+    pdl_wait();
 
     if (warp == 0) {
         // ---- producer ----
@@ -830,16 +833,27 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                         if (q4 == 0) st_async_f32x4(dst + (uint32_t)(h * kRecF + D) * 4u, make_float4(m, l, 0.f, 0.f), rbar);
                     }
                 } else {
+                    // the CTA's own merge first, while the other partials are on their way
+                    constexpr int kPer = (8 * (D / 4) + 32 * kConsWarps - 1) / (32 * kConsWarps);
+                    float lm[kPer], ll[kPer];
+                    float4 lo[kPer];
+#pragma unroll
+                    for (int k = 0; k < kPer; ++k) {
+                        const int e = t + k * 32 * kConsWarps;
+                        if (e < G * (D / 4)) local_merge(e / (D / 4), e % (D / 4), lm[k], ll[k], lo[k]);
+                    }
                     // A sender that gave up on a wait still stores (NaN) within
                     // about one wait limit: wait three before giving up here.
                     const bool got = rcv_wait(rcv, 3ull * g_sas_wait_limit_ns);
                     if (!got && t == 0) atomicAdd(&g_sas_wait_timeouts, 1u);
                     const float* rv = reinterpret_cast<const float*>(sm + recv_off);
-                    for (int e = t; e < G * (D / 4); e += 32 * kConsWarps) {
+#pragma unroll
+                    for (int k = 0; k < kPer; ++k) {
+                        const int e = t + k * 32 * kConsWarps;
+                        if (e >= G * (D / 4)) break;
                         const int h = e / (D / 4), q4 = e - h * (D / 4);
-                        float m, l;
-                        float4 ov;
-                        local_merge(h, q4, m, l, ov);
+                        const float m = lm[k], l = ll[k];
+                        const float4 ov = lo[k];
                         float M = m;
                         for (int r = 0; r < cs - 1; ++r) M = fmaxf(M, rv[(r * G + h) * kRecF + D]);
                         const float w0 = m == -INFINITY ? 0.f : exp2f(m - M);
@@ -1073,13 +1087,15 @@ cudaError_t run_decode_flat(DecArgs a, cudaStream_t st) {
         cfg.blockDim = dim3(kFlatThreads);
         cfg.dynamicSmemBytes = kFlatSmemBytes;
         cfg.stream = st;
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = (unsigned)a.cs;
         attr[0].val.clusterDim.y = 1;
         attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = 2;
         {
             KernelTimer kt("decode_flat", st);
             e = cudaLaunchKernelEx(&cfg, decode_flat_kernel<true>, mk, mv, a);

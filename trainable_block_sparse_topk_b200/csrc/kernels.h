@@ -28,6 +28,25 @@ private:
     void* start_;
 };
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the kernel ahead of it in the stream is still running, and waits for it
+// (pdl_wait) before it reads anything that earlier work writes.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Problem shape, validated and derived from sas_desc by the entry points.
 struct Shape {
     int B, T, q_offset, Hq, Hkv, G, D, bs, K;

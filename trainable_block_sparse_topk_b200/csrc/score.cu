@@ -26,6 +26,7 @@ constexpr int kD = 128;
 __global__ void __launch_bounds__(kThreads)
 pooled_score_kernel(Shape sh, const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ kbar,
                     int64_t kstride, float* __restrict__ scores) {
+    pdl_trigger();   // the top-K after this kernel waits for its end before reading the scores
     const int tiles = (sh.NB + kTile - 1) / kTile;
     const int64_t bg = blockIdx.x / tiles;
     const int tile = (int)(blockIdx.x - bg * tiles);

@@ -62,6 +62,8 @@ block_topk_warp_kernel(Shape sh, const float* __restrict__ scores, const int32_t
                        int32_t* __restrict__ nsel_out) {
     constexpr int kCap = 128;                    // compacted keys per warp
     __shared__ uint32_t s_cand[8][kCap];
+    pdl_trigger();
+    pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t row = (int64_t)blockIdx.x * 8 + warp;
     if (row >= sh.rows()) return;                // warp-uniform
@@ -221,8 +223,9 @@ cudaError_t run_topk_warp(const Shape& s, const float* scores, const int32_t* le
                           float* lse, int32_t* nsel, cudaStream_t st) {
     const int64_t grid = (s.rows() + 7) / 8;
     KernelTimer kt("block_topk", st);
-    block_topk_warp_kernel<SLOTS><<<(unsigned)grid, 256, 0, st>>>(s, scores, lens, idx, gl, lse, nsel);
-    const cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(block_topk_warp_kernel<SLOTS>, dim3((unsigned)grid), dim3(256), 0, st, s, scores, lens,
+                               idx, gl, lse, nsel);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
     return e;
 }
@@ -252,6 +255,8 @@ block_topk_cta_kernel(Shape sh, const float* __restrict__ scores, const int32_t*
     __shared__ uint32_t s_misc[8];       // digit, need-in-bin, candidates, thr, need, prefix, mask, overflow
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_trigger();
+    pdl_wait();
     const int64_t row = blockIdx.x;
     const int t = (int)(row % sh.T);
     const int64_t p = row_position(sh, lens, row, t);
@@ -508,8 +513,9 @@ template <int NT, int SLOTS>
 cudaError_t run_topk_cta(const Shape& s, const float* scores, const int32_t* lens, int32_t* idx, float* gl,
                          float* lse, int32_t* nsel, cudaStream_t st) {
     KernelTimer kt("block_topk", st);
-    block_topk_cta_kernel<NT, SLOTS><<<(unsigned)s.rows(), NT, 0, st>>>(s, scores, lens, idx, gl, lse, nsel);
-    const cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(block_topk_cta_kernel<NT, SLOTS>, dim3((unsigned)s.rows()), dim3(NT), 0, st, s, scores,
+                               lens, idx, gl, lse, nsel);
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
     return e;
 }
