@@ -253,6 +253,7 @@ block_topk_cta_kernel(Shape sh, const float* __restrict__ scores, const int32_t*
     __shared__ float s_rm[kW], s_rs[kW];
     __shared__ uint32_t s_cnt[SLOTS][kW];
     __shared__ uint32_t s_misc[8];       // digit, need-in-bin, candidates, thr, need, prefix, mask, overflow
+    __shared__ float s_lse;
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     pdl_trigger();
@@ -298,11 +299,20 @@ block_topk_cta_kernel(Shape sh, const float* __restrict__ scores, const int32_t*
     for (int k = 0; k < SLOTS; ++k)
         if (tid + NT * k < C) atomicAdd(&s_hist[key[k] >> 21], 1u);
     __syncthreads();
-    float m = -INFINITY;
-    for (int w = 0; w < kW; ++w) m = fmaxf(m, s_rm[w]);
-    float lsum = 0.f;
-    for (int w = 0; w < kW; ++w) lsum += s_rm[w] == -INFINITY ? 0.f : s_rs[w] * exp2f((s_rm[w] - m) * kLog2e);
-    const float lse = (C > 0 && m != -INFINITY) ? m + logf(lsum) : -INFINITY;
+    if (warp == 1) {
+        // the warps' (max, sum) pairs, one per lane, reduced by warp 1 while
+        // warp 0 scans the histogram; read by the others after the barriers below
+        float m = lane < kW ? s_rm[lane] : -INFINITY, sm = lane < kW ? s_rs[lane] : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float m2 = __shfl_xor_sync(0xffffffffu, m, o), s2 = __shfl_xor_sync(0xffffffffu, sm, o);
+            const float mm = fmaxf(m, m2);
+            sm = (m == -INFINITY ? 0.f : sm * exp2f((m - mm) * kLog2e)) +
+                 (m2 == -INFINITY ? 0.f : s2 * exp2f((m2 - mm) * kLog2e));
+            m = mm;
+        }
+        if (lane == 0) s_lse = (C > 0 && m != -INFINITY) ? m + logf(sm) : -INFINITY;
+    }
 
     // ---- the n-th largest key: radix passes of 11, 11, 10 bits until its bin is small ----
     uint32_t prefix = 0, pmask = 0, need = (uint32_t)n, thr = 0;
@@ -393,12 +403,31 @@ block_topk_cta_kernel(Shape sh, const float* __restrict__ scores, const int32_t*
                         uint32_t c4[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) c4[e] = (uint32_t)(lane + 32 * e) < nc ? s_cand[lane + 32 * e] : 0u;
-                        for (int bit = shift - 1; bit >= 0; --bit) {
+                        int bit = shift - 1;
+                        if (shift & 1) {                 // an odd bit count: one single-bit step first
                             const uint32_t cand = th | (1u << bit);
                             uint32_t c = 0;
 #pragma unroll
                             for (int e = 0; e < 4; ++e) c += c4[e] >= cand ? 1u : 0u;
                             if (__reduce_add_sync(0xffffffffu, c) >= need) th = cand;
+                            --bit;
+                        }
+                        // two bits per step: the largest of th | 11, 10, 01 (<< bit - 1)
+                        // with at least `need` keys at or above it (three independent counts)
+                        for (; bit > 0; bit -= 2) {
+                            const uint32_t c1 = th | (1u << (bit - 1)), c2 = th | (2u << (bit - 1)),
+                                           c3 = th | (3u << (bit - 1));
+                            uint32_t n1 = 0, n2 = 0, n3 = 0;
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                n1 += c4[e] >= c1 ? 1u : 0u;
+                                n2 += c4[e] >= c2 ? 1u : 0u;
+                                n3 += c4[e] >= c3 ? 1u : 0u;
+                            }
+                            n1 = __reduce_add_sync(0xffffffffu, n1);
+                            n2 = __reduce_add_sync(0xffffffffu, n2);
+                            n3 = __reduce_add_sync(0xffffffffu, n3);
+                            th = n3 >= need ? c3 : n2 >= need ? c2 : n1 >= need ? c1 : th;
                         }
                     } else {
                         for (int bit = shift - 1; bit >= 0; --bit) {
@@ -421,15 +450,16 @@ block_topk_cta_kernel(Shape sh, const float* __restrict__ scores, const int32_t*
     // ---- keep the keys above thr and the first copies of thr, in index order ----
     // Index order is (slot, warp, lane): per-slot ballots within a warp, and
     // one warp scans the per-(slot, warp) counts into exclusive prefixes.
-    uint32_t eqb[SLOTS], tkb[SLOTS];
+    uint32_t eqb[SLOTS], gtb[SLOTS], tkb[SLOTS];
 #pragma unroll
     for (int k = 0; k < SLOTS; ++k) {
         const bool valid = n > 0 && tid + NT * k < C;
         eqb[k] = __ballot_sync(0xffffffffu, valid && key[k] == thr);
-        const uint32_t gtb = __ballot_sync(0xffffffffu, valid && key[k] > thr);
-        if (lane == 0) s_cnt[k][warp] = (uint32_t)__popc(eqb[k]) | ((uint32_t)__popc(gtb) << 16);
+        gtb[k] = __ballot_sync(0xffffffffu, valid && key[k] > thr);
+        if (lane == 0) s_cnt[k][warp] = (uint32_t)__popc(eqb[k]) | ((uint32_t)__popc(gtb[k]) << 16);
     }
     __syncthreads();
+    const float lse = s_lse;
     // exclusive prefix over the SLOTS * kW counts in (slot, warp) order, in place;
     // the totals land in s_misc[4]
     auto scan_counts = [&]() {
@@ -458,20 +488,33 @@ block_topk_cta_kernel(Shape sh, const float* __restrict__ scores, const int32_t*
     const uint32_t gt_all = s_misc[4] >> 16;
     const uint32_t need_eq = (uint32_t)n - gt_all;
     bool take[SLOTS];
+    uint32_t pos0[SLOTS];   // kept keys before this (slot, warp)
+    if ((s_misc[4] & 0xffffu) == need_eq) {
+        // every copy of thr is kept (the usual case): the kept keys are those
+        // >= thr, and the one scan already counts them
 #pragma unroll
-    for (int k = 0; k < SLOTS; ++k) {
-        const uint32_t rank = (s_cnt[k][warp] & 0xffffu) + __popc(eqb[k] & lt);
-        const bool gt = n > 0 && tid + NT * k < C && key[k] > thr;
-        take[k] = gt || (((eqb[k] >> lane) & 1u) && rank < need_eq);
-    }
-    __syncthreads();   // s_cnt is rewritten with the kept counts
+        for (int k = 0; k < SLOTS; ++k) {
+            tkb[k] = eqb[k] | gtb[k];
+            take[k] = (tkb[k] >> lane) & 1u;
+            pos0[k] = (s_cnt[k][warp] & 0xffffu) + (s_cnt[k][warp] >> 16);
+        }
+    } else {
 #pragma unroll
-    for (int k = 0; k < SLOTS; ++k) {
-        tkb[k] = __ballot_sync(0xffffffffu, take[k]);
-        if (lane == 0) s_cnt[k][warp] = (uint32_t)__popc(tkb[k]);
+        for (int k = 0; k < SLOTS; ++k) {
+            const uint32_t rank = (s_cnt[k][warp] & 0xffffu) + __popc(eqb[k] & lt);
+            take[k] = ((gtb[k] >> lane) & 1u) || (((eqb[k] >> lane) & 1u) && rank < need_eq);
+        }
+        __syncthreads();   // s_cnt is rewritten with the kept counts
+#pragma unroll
+        for (int k = 0; k < SLOTS; ++k) {
+            tkb[k] = __ballot_sync(0xffffffffu, take[k]);
+            if (lane == 0) s_cnt[k][warp] = (uint32_t)__popc(tkb[k]);
+        }
+        __syncthreads();
+        scan_counts();
+#pragma unroll
+        for (int k = 0; k < SLOTS; ++k) pos0[k] = s_cnt[k][warp];
     }
-    __syncthreads();
-    scan_counts();
     float lse_sel = 0.f;
     if (sh.gate == SAS_GATE_SOFTMAX_SELECTED) {      // normaliser over the kept blocks (CTA-uniform branch)
         float mk = -INFINITY, sk = 0.f;
@@ -500,7 +543,7 @@ block_topk_cta_kernel(Shape sh, const float* __restrict__ scores, const int32_t*
 #pragma unroll
     for (int k = 0; k < SLOTS; ++k) {
         if (take[k]) {
-            const uint32_t pos = s_cnt[k][warp] + __popc(tkb[k] & lt);
+            const uint32_t pos = pos0[k] + __popc(tkb[k] & lt);
             io[pos] = tid + NT * k;
             go[pos] = gate_logit_of(sh.gate, xs[k], lse, lse_sel);
         }
