@@ -561,99 +561,101 @@ def run_ours(args, rank, world, local_rank):
             if i >= args.warmup:
                 tk.append(ev[0].elapsed_time(ev[1]) * 1e3)
                 dec.append(ev[1].elapsed_time(ev[2]) * 1e3)
-        return statistics.median(tk), statistics.median(dec)
+        # means, not medians: single event intervals of a few microseconds come
+        # in coarse steps, and only the mean over the steps resolves below one
+        return statistics.mean(tk), statistics.mean(dec)
 
     decode_recs = []
-    for name, batch, K in DECODE_RECORDS:
-        w, kc, vc, qh, sh = decode_inputs(name, batch, K, dev, dt, caches)
-        q, sc = qh.to(dt).to(dev), sh.to(dev)
-        tk_us, dec_us = time_decode(w, kc, vc, q, sc)
-        by = decode_selected_bytes(w, K)
-        rec = {"workload": f"{name} N{w.seq} B{batch} Hq{w.n_q_heads}/Hkv{w.n_kv_heads} d{w.head_dim} "
-                           f"b{w.block_size} K{K} (budget {(K + 1) * w.block_size})",
-               "selected_bytes": by, "topk_us": tk_us, "decode_us": dec_us,
-               "gbs": by / (dec_us * 1e-6) / 1e9, "frac_of_hbm": by / (dec_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
-               "topk_share": tk_us / (tk_us + dec_us)}
-        if (name, K) in (("decode", 31), ("long", 31)) and batch == 1:
-            _, dense_us = time_decode(w, kc, vc, q, sc, dense=True)
-            dense_bytes = w.batch * w.n_kv_heads * w.seq * w.head_dim * 2 * 2
-            rec.update(dense_us=dense_us, dense_gbs=dense_bytes / (dense_us * 1e-6) / 1e9,
-                       sparse_vs_dense_speedup=dense_us / (dec_us + tk_us))
-        decode_recs.append(rec)
-    # paged pools with a cache length per sequence: the batch-8 workload's
-    # blocks in shuffled pages, sequence b of length N - 4097 b
-    pw, pkc, pvc, pqh, psh = decode_inputs("long", 8, 31, dev, dt, caches)
-    kp, vp, table = paginate(pkc, pvc, pw.block_size, torch.Generator().manual_seed(43))
-    lens = torch.tensor([pw.seq - 4097 * b for b in range(pw.batch)], dtype=torch.int32, device=dev)
-    pd = decode_desc(B, pw)
-    pq, ps = pqh.to(dt).to(dev), psh.to(dev)
-    psel = api.block_topk_varlen(pd, ps, lens)
-    pws = api.workspace(B.SAS_OP_DECODE, pd, dev)
-    po = torch.empty_like(pq)
-    ptk, pdec = [], []
-    for i in range(args.warmup + args.steps):
-        feed()
-        ev = new_events(3)
-        ev[0].record(stream)
-        B.sas_block_topk_varlen(pd, ps, lens, psel.idx, psel.gate_logit, psel.score_lse, psel.n_sel)
-        ev[1].record(stream)
-        B.sas_sparse_decode_paged(pd, pq, kp, vp, table, lens, psel.idx, psel.gate_logit, psel.n_sel, po, pws)
-        ev[2].record(stream)
-        torch.cuda.synchronize()
-        if i >= args.warmup:
-            ptk.append(ev[0].elapsed_time(ev[1]) * 1e3)
-            pdec.append(ev[1].elapsed_time(ev[2]) * 1e3)
-    pby = sum(pw.n_kv_heads * (min(31, (int(n) - 1) // 64) * 64 + int(n) - (int(n) - 1) // 64 * 64) * 128 * 4
-              for n in lens.tolist())
-    tk_us, dec_us = statistics.median(ptk), statistics.median(pdec)
-    decode_recs.append({"workload": f"paged long N<={pw.seq} (N_b = N - 4097 b) B{pw.batch} Hq{pw.n_q_heads}/"
-                                    f"Hkv{pw.n_kv_heads} d128 b64 K31, shuffled pages",
-                        "selected_bytes": pby, "topk_us": tk_us, "decode_us": dec_us,
-                        "gbs": pby / (dec_us * 1e-6) / 1e9, "frac_of_hbm": pby / (dec_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
-                        "topk_share": tk_us / (tk_us + dec_us)})
-    del kp, vp
-    torch.cuda.empty_cache()
+    if not args.no_records:
+        for name, batch, K in DECODE_RECORDS:
+            w, kc, vc, qh, sh = decode_inputs(name, batch, K, dev, dt, caches)
+            q, sc = qh.to(dt).to(dev), sh.to(dev)
+            tk_us, dec_us = time_decode(w, kc, vc, q, sc)
+            by = decode_selected_bytes(w, K)
+            rec = {"workload": f"{name} N{w.seq} B{batch} Hq{w.n_q_heads}/Hkv{w.n_kv_heads} d{w.head_dim} "
+                               f"b{w.block_size} K{K} (budget {(K + 1) * w.block_size})",
+                   "selected_bytes": by, "topk_us": tk_us, "decode_us": dec_us,
+                   "gbs": by / (dec_us * 1e-6) / 1e9, "frac_of_hbm": by / (dec_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+                   "topk_share": tk_us / (tk_us + dec_us)}
+            if (name, K) in (("decode", 31), ("long", 31)) and batch == 1:
+                _, dense_us = time_decode(w, kc, vc, q, sc, dense=True)
+                dense_bytes = w.batch * w.n_kv_heads * w.seq * w.head_dim * 2 * 2
+                rec.update(dense_us=dense_us, dense_gbs=dense_bytes / (dense_us * 1e-6) / 1e9,
+                           sparse_vs_dense_speedup=dense_us / (dec_us + tk_us))
+            decode_recs.append(rec)
+        # paged pools with a cache length per sequence: the batch-8 workload's
+        # blocks in shuffled pages, sequence b of length N - 4097 b
+        pw, pkc, pvc, pqh, psh = decode_inputs("long", 8, 31, dev, dt, caches)
+        kp, vp, table = paginate(pkc, pvc, pw.block_size, torch.Generator().manual_seed(43))
+        lens = torch.tensor([pw.seq - 4097 * b for b in range(pw.batch)], dtype=torch.int32, device=dev)
+        pd = decode_desc(B, pw)
+        pq, ps = pqh.to(dt).to(dev), psh.to(dev)
+        psel = api.block_topk_varlen(pd, ps, lens)
+        pws = api.workspace(B.SAS_OP_DECODE, pd, dev)
+        po = torch.empty_like(pq)
+        ptk, pdec = [], []
+        for i in range(args.warmup + args.steps):
+            feed()
+            ev = new_events(3)
+            ev[0].record(stream)
+            B.sas_block_topk_varlen(pd, ps, lens, psel.idx, psel.gate_logit, psel.score_lse, psel.n_sel)
+            ev[1].record(stream)
+            B.sas_sparse_decode_paged(pd, pq, kp, vp, table, lens, psel.idx, psel.gate_logit, psel.n_sel, po, pws)
+            ev[2].record(stream)
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                ptk.append(ev[0].elapsed_time(ev[1]) * 1e3)
+                pdec.append(ev[1].elapsed_time(ev[2]) * 1e3)
+        pby = sum(pw.n_kv_heads * (min(31, (int(n) - 1) // 64) * 64 + int(n) - (int(n) - 1) // 64 * 64) * 128 * 4
+                  for n in lens.tolist())
+        tk_us, dec_us = statistics.mean(ptk), statistics.mean(pdec)
+        decode_recs.append({"workload": f"paged long N<={pw.seq} (N_b = N - 4097 b) B{pw.batch} Hq{pw.n_q_heads}/"
+                                        f"Hkv{pw.n_kv_heads} d128 b64 K31, shuffled pages",
+                            "selected_bytes": pby, "topk_us": tk_us, "decode_us": dec_us,
+                            "gbs": pby / (dec_us * 1e-6) / 1e9, "frac_of_hbm": pby / (dec_us * 1e-6) / 1e9 / peaks["hbm_gbs"],
+                            "topk_share": tk_us / (tk_us + dec_us)})
+        del kp, vp
+        torch.cuda.empty_cache()
 
-    # the serving step in one call: pooled-key scan of every cached block,
-    # top-K, sparse decode (batch-8 long cache; kbar = each block's mean key)
-    kbar = torch.stack([pkc[b].float().view(pw.n_kv_heads, -1, pw.block_size, pw.head_dim).mean(2).to(dt)
-                        for b in range(pw.batch)])
-    pdd = decode_desc(B, pw)
-    sc_buf = torch.empty(pw.batch, pw.n_kv_heads, 1, pw.n_blocks, dtype=torch.float32, device=dev)
-    psel2 = api.block_topk(pdd, sc_buf.zero_())
-    po2 = torch.empty_like(pq)
-    pws2 = api.workspace(B.SAS_OP_DECODE, pdd, dev)
-    scan_us, call_us = [], []
-    for i in range(args.warmup + args.steps):
-        feed()
-        ev = new_events(3)
-        ev[0].record(stream)
-        B.sas_block_scores_pooled(pdd, pq, kbar, sc_buf)
-        ev[1].record(stream)
-        B.sas_sparse_decode_pooled(pdd, pq, pkc, pvc, pw.seq, kbar, sc_buf, psel2.idx, psel2.gate_logit,
-                                   psel2.score_lse, psel2.n_sel, po2, pws2)
-        ev[2].record(stream)
-        torch.cuda.synchronize()
-        if i >= args.warmup:
-            scan_us.append(ev[0].elapsed_time(ev[1]) * 1e3)
-            call_us.append(ev[1].elapsed_time(ev[2]) * 1e3)
-    C5 = (pw.seq - 1) // pw.block_size
-    scan_bytes = pw.batch * pw.n_kv_heads * C5 * pw.head_dim * 2
-    sby = decode_selected_bytes(pw, 31)
-    su, cu = statistics.median(scan_us), statistics.median(call_us)
-    decode_recs.append({"workload": f"pooled-key scan + top-K + decode in one call, long N{pw.seq} B{pw.batch} K31",
-                        "scan_bytes": scan_bytes, "scan_us": su, "scan_gbs": scan_bytes / (su * 1e-6) / 1e9,
-                        "scan_frac_of_hbm": scan_bytes / (su * 1e-6) / 1e9 / peaks["hbm_gbs"],
-                        "selected_bytes": sby, "call_us": cu, "scan_share": su / cu,
-                        "call_gbs_scan_plus_selected": (scan_bytes + sby) / (cu * 1e-6) / 1e9})
-    del kbar
-    torch.cuda.empty_cache()
-    step_dec = next(r for r in decode_recs if r["workload"].startswith(f"{DECODE_STEP[0]} ") and
-                    f" B{DECODE_STEP[1]} " in r["workload"])
+        # the serving step in one call: pooled-key scan of every cached block,
+        # top-K, sparse decode (batch-8 long cache; kbar = each block's mean key)
+        kbar = torch.stack([pkc[b].float().view(pw.n_kv_heads, -1, pw.block_size, pw.head_dim).mean(2).to(dt)
+                            for b in range(pw.batch)])
+        pdd = decode_desc(B, pw)
+        sc_buf = torch.empty(pw.batch, pw.n_kv_heads, 1, pw.n_blocks, dtype=torch.float32, device=dev)
+        psel2 = api.block_topk(pdd, sc_buf.zero_())
+        po2 = torch.empty_like(pq)
+        pws2 = api.workspace(B.SAS_OP_DECODE, pdd, dev)
+        scan_us, call_us = [], []
+        for i in range(args.warmup + args.steps):
+            feed()
+            ev = new_events(3)
+            ev[0].record(stream)
+            B.sas_block_scores_pooled(pdd, pq, kbar, sc_buf)
+            ev[1].record(stream)
+            B.sas_sparse_decode_pooled(pdd, pq, pkc, pvc, pw.seq, kbar, sc_buf, psel2.idx, psel2.gate_logit,
+                                       psel2.score_lse, psel2.n_sel, po2, pws2)
+            ev[2].record(stream)
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                scan_us.append(ev[0].elapsed_time(ev[1]) * 1e3)
+                call_us.append(ev[1].elapsed_time(ev[2]) * 1e3)
+        C5 = (pw.seq - 1) // pw.block_size
+        scan_bytes = pw.batch * pw.n_kv_heads * C5 * pw.head_dim * 2
+        sby = decode_selected_bytes(pw, 31)
+        su, cu = statistics.mean(scan_us), statistics.mean(call_us)
+        decode_recs.append({"workload": f"pooled-key scan + top-K + decode in one call, long N{pw.seq} B{pw.batch} K31",
+                            "scan_bytes": scan_bytes, "scan_us": su, "scan_gbs": scan_bytes / (su * 1e-6) / 1e9,
+                            "scan_frac_of_hbm": scan_bytes / (su * 1e-6) / 1e9 / peaks["hbm_gbs"],
+                            "selected_bytes": sby, "call_us": cu, "scan_share": su / cu,
+                            "call_gbs_scan_plus_selected": (scan_bytes + sby) / (cu * 1e-6) / 1e9})
+        del kbar
+        torch.cuda.empty_cache()
+    step_by = decode_selected_bytes(dw, DECODE_STEP[2])
     decode_info = {"peak_hbm_gbs": peaks["hbm_gbs"], "peak_source": peak_src, "records": decode_recs,
-                   "step_part": {"workload": step_dec["workload"], "topk_us": mean["decode_topk"] * 1e3,
-                                 "decode_us": mean["decode"] * 1e3,
-                                 "gbs": step_dec["selected_bytes"] / (mean["decode"] * 1e-3) / 1e9}}
+                   "step_part": {"workload": f"{dw.name} N{dw.seq} B{dw.batch} K{DECODE_STEP[2]}",
+                                 "topk_us": mean["decode_topk"] * 1e3, "decode_us": mean["decode"] * 1e3,
+                                 "gbs": step_by / (mean["decode"] * 1e-3) / 1e9}}
 
     # ---- end to end through the public API with host buffers ----
     e2e = None
@@ -661,10 +663,11 @@ def run_ours(args, rank, world, local_rank):
         e2e = run_e2e(args, tw, x, dw, dc, vc, q1c, s1c, dev, dt, flops, world)
 
     # ---- decode pipelined: a CUDA graph of 32 calls over distinct caches (run last) ----
-    gw, gkc, gvc, gq, gs = decode_inputs("decode", 1, 31, dev, dt, caches)
-    decode_info["graph"] = decode_graph(B, api, decode_desc(B, gw), gw, gs, gq.to(dt).to(dev), gkc, gvc,
-                                        api.workspace(B.SAS_OP_DECODE, decode_desc(B, gw), dev), flush, dev)
-    decode_info["graph"]["workload"] = f"decode N{gw.seq} B1 K31"
+    if not args.no_records:
+        gw, gkc, gvc, gq, gs = decode_inputs("decode", 1, 31, dev, dt, caches)
+        decode_info["graph"] = decode_graph(B, api, decode_desc(B, gw), gw, gs, gq.to(dt).to(dev), gkc, gvc,
+                                            api.workspace(B.SAS_OP_DECODE, decode_desc(B, gw), dev), flush, dev)
+        decode_info["graph"]["workload"] = f"decode N{gw.seq} B1 K31"
 
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -786,12 +789,17 @@ def run_reference(args, rank, world):
 
 
 def main():
+    global DECODE_STEP
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen14b")
+    ap.add_argument("--decode", default=":".join(map(str, DECODE_STEP)),
+                    help="decode part of the step, workload:batch:K")
+    ap.add_argument("--no-records", action="store_true",
+                    help="skip the per-workload decode records and the decode graph (smaller runs for profiling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -801,6 +809,8 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    dn, db, dk = args.decode.split(":")
+    DECODE_STEP = (dn, int(db), int(dk))
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
