@@ -45,7 +45,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # kernels timed per launch inside the timed loop (sas_kernel_timing): the
 # candidates for the dominant kernel only -- each timed launch adds a pair of
 # event records between kernels
-TIMED_KERNELS = ("bwd_tc", "fwd_rows", "block_topk", "decode_flat")
+TIMED_KERNELS = ("bwd_tc", "fwd_rows")
 # decode part of a step, and the decode workloads reported one by one:
 # (workload, batch, K)
 DECODE_STEP = ("long", 8, 31)

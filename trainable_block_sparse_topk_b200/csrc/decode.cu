@@ -351,6 +351,7 @@ constexpr int kMaxRecs = 64;            // records of one group (CTAs sharing it
 constexpr int kXchRow = 132;
 constexpr int kXchF = 16 + 8 * kXchRow;
 constexpr int kMaxCluster = 8;          // portable cluster size
+constexpr unsigned long long kRecvFloorNs = 10000000ull;   // shortest wait of a cluster leader for the partials
 
 // Item split: CTA c owns [flat_start(c), flat_start(c + 1)).
 __host__ __device__ __forceinline__ int64_t flat_start(const FlatPlan& f, int64_t c) {
@@ -843,8 +844,12 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                         if (e < G * (D / 4)) local_merge(e / (D / 4), e % (D / 4), lm[k], ll[k], lo[k]);
                     }
                     // A sender that gave up on a wait still stores (NaN) within
-                    // about one wait limit: wait three before giving up here.
-                    const bool got = rcv_wait(rcv, 3ull * g_sas_wait_limit_ns);
+                    // about one wait limit plus its own few microseconds of work:
+                    // wait three limits, and never less than 10 ms, before giving
+                    // up here -- a store into the shared memory of a leader that
+                    // has already exited must not happen.
+                    const unsigned long long lim = 3ull * g_sas_wait_limit_ns;
+                    const bool got = rcv_wait(rcv, lim > kRecvFloorNs ? lim : kRecvFloorNs);
                     if (!got && t == 0) atomicAdd(&g_sas_wait_timeouts, 1u);
                     const float* rv = reinterpret_cast<const float*>(sm + recv_off);
 #pragma unroll

@@ -54,22 +54,18 @@ __device__ __forceinline__ int64_t row_position(const Shape& sh, const int32_t* 
 // (normally a few dozen) are compacted into shared memory, four per lane, and
 // the search runs only over the bits below the prefix that bound and the
 // maximum share. Rows with more than 128 such keys, or K > 32, search all
-// their keys from the top bit.
+// their keys from the top bit. A row takes only the slots its C candidates
+// need (4, 8, 12 or 16 per lane): causal training rows have anywhere from 0
+// to NB - 1 candidates, and every per-slot step costs instructions.
+constexpr int kWarpCap = 128;                    // compacted keys per warp
+
 template <int SLOTS>
-__global__ void __launch_bounds__(256)
-block_topk_warp_kernel(Shape sh, const float* __restrict__ scores, const int32_t* __restrict__ lens,
-                       int32_t* __restrict__ idx_out, float* __restrict__ gl_out, float* __restrict__ lse_out,
-                       int32_t* __restrict__ nsel_out) {
-    constexpr int kCap = 128;                    // compacted keys per warp
-    __shared__ uint32_t s_cand[8][kCap];
-    pdl_trigger();
-    pdl_wait();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t row = (int64_t)blockIdx.x * 8 + warp;
-    if (row >= sh.rows()) return;                // warp-uniform
-    const int t = (int)(row % sh.T);
-    const int64_t p = row_position(sh, lens, row, t);
-    const int C = (int)(p / sh.bs);
+__device__ __forceinline__ void topk_warp_row(const Shape& sh, const float* __restrict__ scores, int64_t row, int C,
+                                              uint32_t* __restrict__ s_cand, int32_t* __restrict__ idx_out,
+                                              float* __restrict__ gl_out, float* __restrict__ lse_out,
+                                              int32_t* __restrict__ nsel_out) {
+    constexpr int kCap = kWarpCap;
+    const int lane = threadIdx.x & 31;
     const int K = sh.K;
     const int n = C < K ? C : K;
     const float* srow = scores + row * sh.NB;
@@ -140,8 +136,8 @@ block_topk_warp_kernel(Shape sh, const float* __restrict__ scores, const int32_t
                 uint32_t at = incl - cnt;
 #pragma unroll
                 for (int k = 0; k < SLOTS; ++k)
-                    if (key[k] >= lo) s_cand[warp][at++] = key[k];
-                for (uint32_t e = total + lane; e < (uint32_t)kCap; e += 32) s_cand[warp][e] = 0u;
+                    if (key[k] >= lo) s_cand[at++] = key[k];
+                for (uint32_t e = total + lane; e < (uint32_t)kCap; e += 32) s_cand[e] = 0u;
                 __syncwarp();
             }
         }
@@ -154,7 +150,7 @@ block_topk_warp_kernel(Shape sh, const float* __restrict__ scores, const int32_t
         if (compact) {
             uint32_t c4[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) c4[e] = s_cand[warp][4 * lane + e];
+            for (int e = 0; e < 4; ++e) c4[e] = s_cand[4 * lane + e];
             for (int bit = top; bit >= 0; --bit) {
                 const uint32_t cand = thr | (1u << bit);
                 uint32_t c = 0;
@@ -216,6 +212,29 @@ block_topk_warp_kernel(Shape sh, const float* __restrict__ scores, const int32_t
     }
     for (int jj = n + lane; jj < K; jj += 32) { io[jj] = -1; go[jj] = 0.f; }
     if (lane == 0) { lse_out[row] = lse; nsel_out[row] = n; }
+}
+
+template <int SLOTS>
+__global__ void __launch_bounds__(256)
+block_topk_warp_kernel(Shape sh, const float* __restrict__ scores, const int32_t* __restrict__ lens,
+                       int32_t* __restrict__ idx_out, float* __restrict__ gl_out, float* __restrict__ lse_out,
+                       int32_t* __restrict__ nsel_out) {
+    __shared__ uint32_t s_cand[8][kWarpCap];
+    pdl_trigger();
+    pdl_wait();
+    const int warp = threadIdx.x >> 5;
+    const int64_t row = (int64_t)blockIdx.x * 8 + warp;
+    if (row >= sh.rows()) return;                // warp-uniform
+    const int t = (int)(row % sh.T);
+    const int C = (int)(row_position(sh, lens, row, t) / sh.bs);
+    if (SLOTS > 4 && C <= 128)
+        topk_warp_row<4>(sh, scores, row, C, s_cand[warp], idx_out, gl_out, lse_out, nsel_out);
+    else if (SLOTS > 8 && C <= 256)
+        topk_warp_row<8>(sh, scores, row, C, s_cand[warp], idx_out, gl_out, lse_out, nsel_out);
+    else if (SLOTS > 12 && C <= 384)
+        topk_warp_row<12>(sh, scores, row, C, s_cand[warp], idx_out, gl_out, lse_out, nsel_out);
+    else
+        topk_warp_row<SLOTS>(sh, scores, row, C, s_cand[warp], idx_out, gl_out, lse_out, nsel_out);
 }
 
 template <int SLOTS>
