@@ -118,9 +118,11 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
     const Shape& sh = a.sh;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = sh.G, K = sh.K, T = sh.T;
-    const int ngroups = sh.B * sh.Hkv;
-    const int j = (int)(blockIdx.x / ngroups);
-    const int bg = (int)(blockIdx.x % ngroups);
+    // group-major CTA order: the CTAs running at once share one (b, kv head)
+    // group, so its accumulator rows stay in L2 between their partial adds
+    // (14B layer: 2-3% faster than key-block-major)
+    const int j = (int)(blockIdx.x % sh.nT);
+    const int bg = (int)(blockIdx.x / sh.nT);
     const int b = bg / sh.Hkv, g = bg % sh.Hkv;
     const int tpc = a.tpc;
     const int rvs = a.ss.rvs;
