@@ -439,7 +439,7 @@ dscore_kernel(Shape sh, const float* __restrict__ scores, const float* __restric
     // every load of the row is issued before any is used: the kept list, its
     // Gsum and scores (masked by n afterwards), the normaliser and the first
     // kPre chunks of 32 causal scores
-    constexpr int kPre = 8;
+    constexpr int kPre = 16;
     const int n = nsel[row];
     const float lse = slse[row];
     int si[2];
