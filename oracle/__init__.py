@@ -269,3 +269,53 @@ def pooled_scores(desc: Desc, q, kbar):
             for j in range(C):
                 out[b, g, 0, j] = float(np.dot(qbar, kb[b, g, j]))
     return out
+
+
+# ------------------------------------------------- per-query-head selection ---
+#
+# The generalisation of the selection granularity (study note
+# 3-1 selects per query group, 3-7 scores per group): every query head h keeps
+# its own top-K blocks from its own score row s[b, h, t, :], and still reads
+# the K/V of its KV head h // G. By definition this is the per-group problem
+# with one query head per group over K/V heads repeated G times; the gradient
+# of a repeated K/V head is the sum over its copies.
+
+def per_head_desc(desc: Desc) -> Desc:
+    """The per-group problem in which each query head is its own group."""
+    return Desc(batch=desc.batch, seq_len=desc.seq_len, n_q_heads=desc.n_q_heads, n_kv_heads=desc.n_q_heads,
+                head_dim=desc.head_dim, block_size=desc.block_size, top_k=desc.top_k, q_offset=desc.q_offset,
+                scale=desc.scale, gate=desc.gate)
+
+
+def _repeat_heads(x, G: int):
+    return np.repeat(_f32(x), G, axis=1)
+
+
+def topk_per_head(desc: Desc, scores, rows=None):
+    """Top-K of every (b, query head, t) row; scores [B, Hq, T, NB]."""
+    return topk(per_head_desc(desc), scores, rows)
+
+
+def fwd_per_head(desc: Desc, q, k, v, scores, rows=None):
+    """Forward with a selection per query head; scores [B, Hq, T, NB], rows
+    over (b, query head, t). Returns (o [n,1,d], attn_lse [n,1])."""
+    G = desc.group
+    return fwd(per_head_desc(desc), q, _repeat_heads(k, G), _repeat_heads(v, G), scores, rows)
+
+
+def bwd_per_head(desc: Desc, q, k, v, scores, dO, rows=None):
+    """Backward with a selection per query head. dk/dv [B,Hkv,T,d] sum the
+    contributions of the G query heads of each KV head; gsum/ds per
+    (b, query head, t) row."""
+    G = desc.group
+    r = bwd(per_head_desc(desc), q, _repeat_heads(k, G), _repeat_heads(v, G), scores, dO, rows)
+    B, T, dh = desc.batch, desc.seq_len, desc.head_dim
+    r["dk"] = r["dk"].reshape(B, desc.n_kv_heads, G, T, dh).sum(2)
+    r["dv"] = r["dv"].reshape(B, desc.n_kv_heads, G, T, dh).sum(2)
+    return r
+
+
+def decode_per_head(desc: Desc, q, k_cache, v_cache, scores=None):
+    """Decode with a selection per query head; scores [B, Hq, 1, NB]."""
+    G = desc.group
+    return decode(per_head_desc(desc), q, _repeat_heads(k_cache, G), _repeat_heads(v_cache, G), scores)

@@ -495,3 +495,86 @@ def test_pooled_scores_pins(oracle_mod):
     s2 = oracle_mod.pooled_scores(d2, np.array([[[1, 0], [3, 2]]], np.float32),
                                   np.array([[[[1, 1], [0, -2]]]], np.float32))
     np.testing.assert_array_equal(s2[0, 0, 0], [3.0, -2.0, 0.0])
+
+
+# ------------------------------------------------- per-query-head selection ---
+
+def bias_matrix_per_head_torch(P, s, gate_on=True):
+    """The naive form with a selection per query head: head h builds its
+    [T,T] bias from its own score row s[b, h] and attends to the K/V of head
+    h // G. `s` [B, Hq, T, NB] may require grad."""
+    B, T, Hq, Hkv, d, bs, K = (P[x] for x in ("B", "T", "Hq", "Hkv", "d", "bs", "K"))
+    G = Hq // Hkv
+    out, lses = [], []
+    for b in range(B):
+        ob, lb = [], []
+        for h in range(Hq):
+            rows = []
+            for t in range(T):
+                C = t // bs
+                sel = stable_topk(s[b, h, t].detach(), C, K)
+                row = torch.full((T,), float("-inf"), dtype=torch.float64)
+                if sel:
+                    lse = torch.logsumexp(s[b, h, t, :C].double(), 0)
+                    for i in sel:
+                        logg = (s[b, h, t, i].double() - lse) if gate_on else torch.zeros((), dtype=torch.float64)
+                        row = torch.cat([row[: i * bs], logg.expand(bs), row[(i + 1) * bs:]])
+                row = torch.cat([row[: C * bs], torch.zeros(t - C * bs + 1, dtype=torch.float64), row[t + 1:]])
+                rows.append(row)
+            bias = torch.stack(rows)
+            logits = P["q"][b, h].double() @ P["k"][b, h // G].double().T / math.sqrt(d) + bias
+            ob.append(torch.softmax(logits, -1) @ P["v"][b, h // G].double())
+            lb.append(torch.logsumexp(logits, -1))
+        out.append(torch.stack(ob))
+        lses.append(torch.stack(lb))
+    return torch.stack(out), torch.stack(lses)
+
+
+@pytest.mark.parametrize("seed,K,gate", [(11, 2, 0), (12, 3, 1)])
+def test_per_head_selection_pins(oracle_mod, seed, K, gate):
+    """Per-query-head selection: the oracle's forward and every gradient
+    (dq, dk/dv summed over the heads sharing a KV head, ds per head row) equal
+    fp64 autograd of the per-head bias formulation, and with identical score
+    rows across a group the selection -- and so the result -- equals the
+    per-group oracle."""
+    P = rand_problem(seed, B=1, T=40, Hq=4, Hkv=2, K=K, gate=gate)
+    g = torch.Generator().manual_seed(seed + 100)
+    sh = torch.randn(P["B"], P["Hq"], P["T"], P["s"].shape[-1], generator=g)
+    desc = desc_of(oracle_mod, P)
+    G = P["Hq"] // P["Hkv"]
+    q = P["q"].double().requires_grad_()
+    k = P["k"].double().requires_grad_()
+    v = P["v"].double().requires_grad_()
+    s = sh.double().requires_grad_()
+    o, lse = bias_matrix_per_head_torch(dict(P, q=q, k=k, v=v), s, gate_on=(gate == 0))
+    (o * P["dO"].double()).sum().backward()
+    B, T, dh = P["B"], P["T"], P["d"]
+    of, lf = oracle_mod.fwd_per_head(desc, P["q"].numpy(), P["k"].numpy(), P["v"].numpy(), sh.numpy())
+    np.testing.assert_allclose(of.reshape(B, P["Hq"], T, dh), o.detach().numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(lf.reshape(B, P["Hq"], T), lse.detach().numpy(), atol=1e-12, rtol=0)
+    r = oracle_mod.bwd_per_head(desc, P["q"].numpy(), P["k"].numpy(), P["v"].numpy(), sh.numpy(),
+                                P["dO"].numpy())
+    np.testing.assert_allclose(r["dq"].reshape(B, P["Hq"], T, dh), q.grad.numpy(), atol=1e-11, rtol=0)
+    np.testing.assert_allclose(r["dk"], k.grad.numpy(), atol=1e-11, rtol=0)
+    np.testing.assert_allclose(r["dv"], v.grad.numpy(), atol=1e-11, rtol=0)
+    sg = s.grad.numpy() if s.grad is not None else np.zeros(s.shape)
+    np.testing.assert_allclose(r["ds"].reshape(sh.shape), sg, atol=1e-11, rtol=0)
+    # a group's heads with one shared score row reduce to the per-group selection
+    s_grp = P["s"].repeat_interleave(G, 1)
+    o_h, _ = oracle_mod.fwd_per_head(desc, P["q"].numpy(), P["k"].numpy(), P["v"].numpy(), s_grp.numpy())
+    o_g, _ = oracle_o_full(oracle_mod, desc, P)
+    np.testing.assert_allclose(o_h.reshape(B, P["Hq"], T, dh), o_g, atol=1e-12, rtol=0)
+
+
+def test_per_head_decode_pin(oracle_mod):
+    """Per-head decode equals the last row of the per-head training problem."""
+    P = rand_problem(13, B=1, T=40, Hq=4, Hkv=2, K=2)
+    g = torch.Generator().manual_seed(113)
+    sh = torch.randn(P["B"], P["Hq"], P["T"], P["s"].shape[-1], generator=g)
+    desc = desc_of(oracle_mod, P)
+    of, _ = oracle_mod.fwd_per_head(desc, P["q"].numpy(), P["k"].numpy(), P["v"].numpy(), sh.numpy())
+    N = P["T"]
+    dd = desc_of(oracle_mod, P, seq_len=1, q_offset=N - 1)
+    od = oracle_mod.decode_per_head(dd, P["q"][:, :, N - 1].numpy(), P["k"].numpy(), P["v"].numpy(),
+                                    sh[:, :, N - 1:N].numpy())
+    np.testing.assert_allclose(od, of.reshape(P["B"], P["Hq"], N, P["d"])[:, :, N - 1], atol=1e-12, rtol=0)
