@@ -106,6 +106,14 @@ typedef struct {
     float softmax_scale;   /* scale on q.k; <= 0 selects 1/sqrt(d). The log-gate is added unscaled. */
     int32_t dtype;         /* sas_dtype of q/k/v/o/dO/dq/dk/dv */
     int32_t gate;          /* sas_gate */
+    /* Selection granularity. 0: one selection per (b, KV head, t), shared by
+     * the group's G = Hq / Hkv query heads (study note 3-1: per query group).
+     * 1: one selection per (b, query head, t): every query head keeps its own
+     * top-K from its own score row and reads the K/V of its KV head h / G;
+     * the K/V gradients sum over the G heads. The selection arrays (scores,
+     * idx, gate_logit, score_lse, n_sel, dscores) then have Hq rows where the
+     * calls below say Hkv, and the workspace sizes follow. */
+    int32_t select_heads;
 } sas_desc;
 
 /* Bytes of device workspace `op` needs for this shape (0 if none). The caller

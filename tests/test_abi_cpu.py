@@ -190,3 +190,26 @@ def test_kernel_timing_records_nothing_without_launches(L):
     ms, n = ctypes.c_double(1.0), ctypes.c_uint32(7)
     assert L.sas_kernel_time(None, ctypes.byref(ms), ctypes.byref(n)) == B.SAS_ERR_INVALID_ARG
     assert L.sas_kernel_time(b"fwd_rows", None, ctypes.byref(n)) == B.SAS_ERR_INVALID_ARG
+
+
+def test_select_heads_value_checked(L):
+    d = desc()
+    d.select_heads = 2            # neither 0 nor 1
+    assert ws_size(B.SAS_OP_FWD, d)[0] == B.SAS_ERR_INVALID_ARG
+
+
+def test_per_head_selection_workspace(L):
+    """Per-query-head selection: the selection arrays and streams have Hq rows
+    per position, and the backward adds fp32 dK, dV per selection group (two
+    B*Hq*T*d float arrays) for the sum over the heads of each KV head."""
+    d0, d1 = desc(), desc(select_heads=1)
+    a = lambda p: (p + 255) // 256 * 256
+    st, n0 = ws_size(B.SAS_OP_BWD, d0)
+    st1, n1 = ws_size(B.SAS_OP_BWD, d1)
+    assert st == 0 and st1 == 0
+    Bn, Hq, Hkv, T, K, D, NB, nT = 1, 8, 2, 256, 3, 128, 4, 4
+    cap1 = Bn * Hq * T * (K + 1)
+    stream1 = a(16 * cap1) + a(4 * cap1 * 4) + 2 * a(4 * Hq * NB) + a(4 * Hq * NB * nT) + 256
+    parts = [8 * Bn * Hq * NB * nT, 4 * Bn * Hq * T, 4 * Bn * Hq * T * K, 4 * Bn * Hq * T * D]
+    assert n1 == sum(a(p) for p in parts) + 2 * a(4 * Bn * Hq * T * D) + a(stream1) + 256
+    assert n1 > n0

@@ -35,7 +35,7 @@ def workspace(op: int, desc, device=None) -> torch.Tensor | None:
 
 
 def block_topk(desc, scores: torch.Tensor, out: Selection | None = None, stream=None) -> Selection:
-    Bn, H, T, K = desc.batch, desc.n_kv_heads, desc.seq_len, desc.top_k
+    Bn, H, T, K = desc.batch, desc.n_sel_groups, desc.seq_len, desc.top_k
     dev = scores.device
     if out is None:
         out = Selection(torch.empty(Bn, H, T, K, dtype=torch.int32, device=dev),
@@ -79,7 +79,7 @@ def sparse_decode(desc, q, k_cache, v_cache, sel: Selection | None, ws=None, str
 
 def block_topk_varlen(desc, scores: torch.Tensor, seq_lens: torch.Tensor, stream=None) -> Selection:
     """Decode-row top-K with a cache length per sequence (seq_lens int32 [B])."""
-    Bn, H, K = desc.batch, desc.n_kv_heads, desc.top_k
+    Bn, H, K = desc.batch, desc.n_sel_groups, desc.top_k
     dev = scores.device
     out = Selection(torch.empty(Bn, H, 1, K, dtype=torch.int32, device=dev),
                     torch.empty(Bn, H, 1, K, dtype=torch.float32, device=dev),
@@ -106,7 +106,7 @@ def sparse_decode_paged(desc, q, k_pages, v_pages, block_table, seq_lens, sel: S
 def sparse_decode_pooled(desc, q, k_cache, v_cache, kbar, ws=None, stream=None):
     """Pooled-key block scores, top-K and sparse decode in one call; returns
     (o, scores, Selection)."""
-    Bn, H, K = desc.batch, desc.n_kv_heads, desc.top_k
+    Bn, H, K = desc.batch, desc.n_sel_groups, desc.top_k
     dev = q.device
     scores = torch.empty(Bn, H, 1, desc.n_blocks, dtype=torch.float32, device=dev)
     sel = Selection(torch.empty(Bn, H, 1, K, dtype=torch.int32, device=dev),

@@ -33,11 +33,17 @@ class sas_desc(ctypes.Structure):
     _fields_ = [("batch", ctypes.c_int32), ("seq_len", ctypes.c_int32), ("q_offset", ctypes.c_int32),
                 ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("block_size", ctypes.c_int32), ("top_k", ctypes.c_int32), ("softmax_scale", ctypes.c_float),
-                ("dtype", ctypes.c_int32), ("gate", ctypes.c_int32)]
+                ("dtype", ctypes.c_int32), ("gate", ctypes.c_int32), ("select_heads", ctypes.c_int32)]
 
     @property
     def group(self) -> int:
         return self.n_q_heads // self.n_kv_heads
+
+    @property
+    def n_sel_groups(self) -> int:
+        """Rows of the selection arrays per (batch, query position): the KV
+        heads, or the query heads when every query head selects its own blocks."""
+        return self.n_q_heads if self.select_heads else self.n_kv_heads
 
     @property
     def n_blocks(self) -> int:
@@ -49,11 +55,11 @@ class sas_desc(ctypes.Structure):
 
 
 def make_desc(batch, seq_len, n_q_heads, n_kv_heads, head_dim, block_size, top_k, q_offset=0,
-              softmax_scale=0.0, dtype="bf16", gate="softmax") -> sas_desc:
+              softmax_scale=0.0, dtype="bf16", gate="softmax", select_heads=False) -> sas_desc:
     dt = {"bf16": SAS_DT_BF16, "fp32": SAS_DT_FP32}[dtype] if isinstance(dtype, str) else int(dtype)
     gt = GATES[gate] if isinstance(gate, str) else int(gate)
     return sas_desc(batch, seq_len, q_offset, n_q_heads, n_kv_heads, head_dim, block_size, top_k,
-                    softmax_scale, dt, gt)
+                    softmax_scale, dt, gt, 1 if select_heads else 0)
 
 
 _lib = None

@@ -60,6 +60,8 @@ struct BwdTcArgs {
     __nv_bfloat16* dk;
     __nv_bfloat16* dv;
     float* gsum;
+    float* dk32;         // per-query-head selection: fp32 dK, dV of each selection group
+    float* dv32;         // ([B * Hkv, T, d], summed over the heads of a KV head later); else NULL
     int tpc;             // tokens per chunk = 128 / G
     int meta_bytes;      // one metadata ring slot: tpc (16 + 4 rvs) bytes
     int* aborted;        // set when a CTA gave up on a wait (the later kernels then write NaN)
@@ -165,7 +167,7 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             tc::prefetch_tmap(&tm_k);
             tc::prefetch_tmap(&tm_v);
             mbar_arrive_expect_tx(kv_full, 32768);
-            const int kr = (int)((int64_t)bg * T + (int64_t)j * kBS);
+            const int kr = (int)(sh.kv_index(bg) * T + (int64_t)j * kBS);
             for (int h = 0; h < 2; ++h) {
                 tc::tma_load_2d(sm + L::kK + h * 8192, &tm_k, h * 64, kr, kv_full);
                 tc::tma_load_2d(sm + L::kV + h * 8192, &tm_v, h * 64, kr, kv_full);
@@ -464,10 +466,9 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
             }
         }
         // dV^T and dK^T: TMEM lane r holds column r of d for the block's 64 keys
+        const int64_t kv0 = ((int64_t)bg * T + (int64_t)j * kBS) * kD;   // this group's block rows
         if (ok && tc::warp_wait_bar(done, 0u, abort)) {
             tc::fence_after_sync();
-            __nv_bfloat16* dvb = a.dv + ((int64_t)bg * T + (int64_t)j * kBS) * kD;
-            __nv_bfloat16* dkb = a.dk + ((int64_t)bg * T + (int64_t)j * kBS) * kD;
 #pragma unroll 1
             for (int cb = 0; cb < kBS / 16; ++cb) {
                 uint32_t vv[16], kv[16];
@@ -476,19 +477,29 @@ bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ 
                 tc::tmem_wait_ld();
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const int key = cb * 16 + e;
-                    dvb[(int64_t)key * kD + r] = __float2bfloat16_rn(__uint_as_float(vv[e]));
-                    dkb[(int64_t)key * kD + r] = __float2bfloat16_rn(__uint_as_float(kv[e]) * dscale);
+                    const int64_t at = kv0 + (int64_t)(cb * 16 + e) * kD + r;
+                    const float fv = __uint_as_float(vv[e]), fk = __uint_as_float(kv[e]) * dscale;
+                    if (a.dk32 != nullptr) {
+                        a.dv32[at] = fv;
+                        a.dk32[at] = fk;
+                    } else {
+                        a.dv[at] = __float2bfloat16_rn(fv);
+                        a.dk[at] = __float2bfloat16_rn(fk);
+                    }
                 }
             }
         } else {
             // a wait gave up: the block's dK and dV are incomplete, mark them invalid
-            const __nv_bfloat16 nan = __float2bfloat16(__int_as_float(0x7fc00000));
-            __nv_bfloat16* dvb = a.dv + ((int64_t)bg * T + (int64_t)j * kBS) * kD;
-            __nv_bfloat16* dkb = a.dk + ((int64_t)bg * T + (int64_t)j * kBS) * kD;
+            const float nan = __int_as_float(0x7fc00000);
             for (int key = 0; key < kBS; ++key) {
-                dvb[(int64_t)key * kD + r] = nan;
-                dkb[(int64_t)key * kD + r] = nan;
+                const int64_t at = kv0 + (int64_t)key * kD + r;
+                if (a.dk32 != nullptr) {
+                    a.dv32[at] = nan;
+                    a.dk32[at] = nan;
+                } else {
+                    a.dv[at] = __float2bfloat16(nan);
+                    a.dk[at] = __float2bfloat16(nan);
+                }
             }
         }
     }
@@ -516,10 +527,10 @@ size_t bwd_tc_ws_bytes(const Shape& s) { return sel_stream_bytes(s, 2); }
 cudaError_t launch_bwd_tc(const Shape& s, const void* q, const void* k, const void* v, const void* dO,
                           const float* lse, const float* Dd, const int32_t* idx, const float* gl,
                           const int32_t* nsel, const uint64_t* maskT, void* ws, float* dq_acc, void* dk, void* dv,
-                          float* gsum, int* aborted, cudaStream_t st) {
+                          float* dk32, float* dv32, float* gsum, int* aborted, cudaStream_t st) {
     CUtensorMap mk, mv;
-    if (!encode_bf16_2d(&mk, k, (uint64_t)s.B * s.Hkv * s.T, kD, kBS) ||
-        !encode_bf16_2d(&mv, v, (uint64_t)s.B * s.Hkv * s.T, kD, kBS))
+    if (!encode_bf16_2d(&mk, k, (uint64_t)s.B * s.Hkvp * s.T, kD, kBS) ||
+        !encode_bf16_2d(&mv, v, (uint64_t)s.B * s.Hkvp * s.T, kD, kBS))
         return cudaErrorInvalidValue;
     BwdTcArgs a{};
     a.sh = s;
@@ -529,6 +540,8 @@ cudaError_t launch_bwd_tc(const Shape& s, const void* q, const void* k, const vo
     a.dq_acc = dq_acc;
     a.dk = static_cast<__nv_bfloat16*>(dk);
     a.dv = static_cast<__nv_bfloat16*>(dv);
+    a.dk32 = dk32;
+    a.dv32 = dv32;
     a.gsum = gsum;
     a.aborted = aborted;
     a.tpc = kRows / s.G;

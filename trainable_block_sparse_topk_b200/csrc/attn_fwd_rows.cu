@@ -170,7 +170,7 @@ fwd_rows_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             tc::prefetch_tmap(&tm_k);
             tc::prefetch_tmap(&tm_v);
             mbar_arrive_expect_tx(kv_full, 32768u);
-            const int kr = (int)((int64_t)bg * T + (int64_t)j * kBS);
+            const int kr = (int)(sh.kv_index(bg) * T + (int64_t)j * kBS);
             for (int h = 0; h < 2; ++h) {
                 tc::tma_load_2d(sm + L::kK + h * 8192, &tm_k, h * 64, kr, kv_full);
                 tc::tma_load_2d(sm + L::kV + h * 8192, &tm_v, h * 64, kr, kv_full);
@@ -419,7 +419,7 @@ fwd_rows_shift_kernel(Shape sh, const __nv_bfloat16* __restrict__ q, const __nv_
     const int bg = row / sh.T;
     const int t = row - bg * sh.T;
     const int b = bg / sh.Hkv, g = bg - b * sh.Hkv;
-    const uint4 kv = *reinterpret_cast<const uint4*>(k + (int64_t)row * kD + li * 8);
+    const uint4 kv = *reinterpret_cast<const uint4*>(k + (sh.kv_index(bg) * sh.T + t) * kD + li * 8);
     uint4 x[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {                      // G <= 8
@@ -545,8 +545,8 @@ cudaError_t launch_fwd_rows(const Shape& s, const void* q, const void* k, const 
     const RowsWs w(ws, rows);
     CUtensorMap mk, mv;
     FwdRowsArgs a{};
-    if (!encode_bf16_2d(&mk, k, (uint64_t)s.B * s.Hkv * s.T, kD, kBS) ||
-        !encode_bf16_2d(&mv, v, (uint64_t)s.B * s.Hkv * s.T, kD, kBS))
+    if (!encode_bf16_2d(&mk, k, (uint64_t)s.B * s.Hkvp * s.T, kD, kBS) ||
+        !encode_bf16_2d(&mv, v, (uint64_t)s.B * s.Hkvp * s.T, kD, kBS))
         return cudaErrorInvalidValue;
     a.sh = s;
     a.q = static_cast<const __nv_bfloat16*>(q);

@@ -89,8 +89,8 @@ __device__ __forceinline__ void fwd_simt_row(const Shape& sh, const T* __restric
 #pragma unroll
         for (int e = 0; e < DPL; ++e) acc[h][e] = 0.f;
     }
-    const T* kb = k + bg * (int64_t)sh.T * D;
-    const T* vb = v + bg * (int64_t)sh.T * D;
+    const T* kb = k + sh.kv_index(bg) * (int64_t)sh.T * D;
+    const T* vb = v + sh.kv_index(bg) * (int64_t)sh.T * D;
 
     for (int jj = 0; jj <= n; ++jj) {
         const bool hist = jj < n;
@@ -246,7 +246,7 @@ bwd_simt_kernel(Shape sh, const T* __restrict__ q, const T* __restrict__ k, cons
                 const T* __restrict__ dO, const float* __restrict__ attn_lse, const float* __restrict__ Dd,
                 const int32_t* __restrict__ idx, const float* __restrict__ gl, const int32_t* __restrict__ nsel,
                 const uint64_t* __restrict__ maskT, float* __restrict__ dq_acc, T* __restrict__ dk,
-                T* __restrict__ dv, float* __restrict__ gsum) {
+                T* __restrict__ dv, float* __restrict__ dk32, float* __restrict__ dv32, float* __restrict__ gsum) {
     constexpr int NT = BS * 4;
     constexpr int DS = D + 4;          // padded row stride: conflict-free for (kk, qd) threads
     constexpr int DQ = D / 4;
@@ -267,8 +267,8 @@ bwd_simt_kernel(Shape sh, const T* __restrict__ q, const T* __restrict__ k, cons
     const int kk = tid >> 2, qd = tid & 3;
     const float scale = sh.scale;
 
-    const T* kb = k + (bg * sh.T + (int64_t)j * BS) * D;
-    const T* vb = v + (bg * sh.T + (int64_t)j * BS) * D;
+    const T* kb = k + (sh.kv_index(bg) * sh.T + (int64_t)j * BS) * D;
+    const T* vb = v + (sh.kv_index(bg) * sh.T + (int64_t)j * BS) * D;
     for (int e = tid; e < BS * D; e += NT) {
         Ks[(e / D) * DS + e % D] = Elem<T>::to_f(kb[e]);
         Vs[(e / D) * DS + e % D] = Elem<T>::to_f(vb[e]);
@@ -368,12 +368,46 @@ bwd_simt_kernel(Shape sh, const T* __restrict__ q, const T* __restrict__ k, cons
         }
     }
 
-    T* dkb = dk + (bg * sh.T + (int64_t)j * BS) * D;
-    T* dvb = dv + (bg * sh.T + (int64_t)j * BS) * D;
+    // per-query-head selection: fp32 partials of this selection group, summed
+    // over the heads of the KV head afterwards
+    const int64_t kv0 = (bg * sh.T + (int64_t)j * BS) * D;
 #pragma unroll
     for (int i = 0; i < DQ; ++i) {
-        dkb[kk * D + qd + 4 * i] = Elem<T>::from_f(dk_r[i]);
-        dvb[kk * D + qd + 4 * i] = Elem<T>::from_f(dv_r[i]);
+        const int64_t at = kv0 + kk * D + qd + 4 * i;
+        if (dk32 != nullptr) {
+            dk32[at] = dk_r[i];
+            dv32[at] = dv_r[i];
+        } else {
+            dk[at] = Elem<T>::from_f(dk_r[i]);
+            dv[at] = Elem<T>::from_f(dv_r[i]);
+        }
+    }
+}
+
+// Per-query-head selection: dK, dV of KV head kv = the sum of the fp32
+// partials of its kvdiv query heads (selection groups kv * kvdiv + r), one
+// float4 per thread and pass.
+template <typename T>
+__global__ void __launch_bounds__(256)
+reduce_dkv_kernel(Shape sh, const float* __restrict__ dk32, const float* __restrict__ dv32, T* __restrict__ dk,
+                  T* __restrict__ dv) {
+    const int64_t per = (int64_t)sh.T * sh.D / 4;              // float4s per (b, kv head)
+    const int64_t n = (int64_t)sh.B * sh.Hkvp * per;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t bk = i / per, e = i - bk * per;
+        const int64_t b = bk / sh.Hkvp, kv = bk - b * sh.Hkvp;
+        float4 sk = make_float4(0.f, 0.f, 0.f, 0.f), sv = sk;
+        for (int r = 0; r < sh.kvdiv; ++r) {
+            const int64_t src = (b * sh.Hkv + kv * sh.kvdiv + r) * per + e;
+            const float4 a = reinterpret_cast<const float4*>(dk32)[src];
+            const float4 c = reinterpret_cast<const float4*>(dv32)[src];
+            sk.x += a.x; sk.y += a.y; sk.z += a.z; sk.w += a.w;
+            sv.x += c.x; sv.y += c.y; sv.z += c.z; sv.w += c.w;
+        }
+        T* ok = dk + i * 4;
+        T* ov = dv + i * 4;
+        ok[0] = Elem<T>::from_f(sk.x); ok[1] = Elem<T>::from_f(sk.y); ok[2] = Elem<T>::from_f(sk.z); ok[3] = Elem<T>::from_f(sk.w);
+        ov[0] = Elem<T>::from_f(sv.x); ov[1] = Elem<T>::from_f(sv.y); ov[2] = Elem<T>::from_f(sv.z); ov[3] = Elem<T>::from_f(sv.w);
     }
 }
 
@@ -538,7 +572,7 @@ template <typename T, int D, int GMAX, int BS>
 cudaError_t run_bwd(const Shape& s, const void* q, const void* k, const void* v, const void* dO,
                     const float* lse, const float* Dd, const int32_t* idx, const float* gl,
                     const int32_t* nsel, const uint64_t* maskT, float* dq_acc, void* dk, void* dv,
-                    float* gsum, cudaStream_t st) {
+                    float* dk32, float* dv32, float* gsum, cudaStream_t st) {
     constexpr int NT = BS * 4;
     const size_t smem = sizeof(float) * (2 * BS * (D + 4) + 2 * GMAX * D + GMAX * BS + 2 * GMAX + NT / 32);
     auto kern = bwd_simt_kernel<T, D, GMAX, BS>;
@@ -548,7 +582,7 @@ cudaError_t run_bwd(const Shape& s, const void* q, const void* k, const void* v,
     {
         KernelTimer kt("bwd_simt", st);
         kern<<<(unsigned)grid, NT, smem, st>>>(s, (const T*)q, (const T*)k, (const T*)v, (const T*)dO, lse, Dd, idx,
-                                               gl, nsel, maskT, dq_acc, (T*)dk, (T*)dv, gsum);
+                                               gl, nsel, maskT, dq_acc, (T*)dk, (T*)dv, dk32, dv32, gsum);
     }
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
@@ -578,25 +612,25 @@ template <typename T, int D, int BS>
 cudaError_t bwd_g(const Shape& s, const void* q, const void* k, const void* v, const void* dO,
                   const float* lse, const float* Dd, const int32_t* idx, const float* gl,
                   const int32_t* nsel, const uint64_t* maskT, float* dq_acc, void* dk, void* dv,
-                  float* gsum, cudaStream_t st) {
-    if (s.G <= 4) return run_bwd<T, D, 4, BS>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, gsum, st);
-    return run_bwd<T, D, 8, BS>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, gsum, st);
+                  float* dk32, float* dv32, float* gsum, cudaStream_t st) {
+    if (s.G <= 4) return run_bwd<T, D, 4, BS>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, dk32, dv32, gsum, st);
+    return run_bwd<T, D, 8, BS>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, dk32, dv32, gsum, st);
 }
 template <typename T, int D>
 cudaError_t bwd_b(const Shape& s, const void* q, const void* k, const void* v, const void* dO,
                   const float* lse, const float* Dd, const int32_t* idx, const float* gl,
                   const int32_t* nsel, const uint64_t* maskT, float* dq_acc, void* dk, void* dv,
-                  float* gsum, cudaStream_t st) {
-    if (s.bs == 32) return bwd_g<T, D, 32>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, gsum, st);
-    return bwd_g<T, D, 64>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, gsum, st);
+                  float* dk32, float* dv32, float* gsum, cudaStream_t st) {
+    if (s.bs == 32) return bwd_g<T, D, 32>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, dk32, dv32, gsum, st);
+    return bwd_g<T, D, 64>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, dk32, dv32, gsum, st);
 }
 template <typename T>
 cudaError_t bwd_d(const Shape& s, const void* q, const void* k, const void* v, const void* dO,
                   const float* lse, const float* Dd, const int32_t* idx, const float* gl,
                   const int32_t* nsel, const uint64_t* maskT, float* dq_acc, void* dk, void* dv,
-                  float* gsum, cudaStream_t st) {
-    if (s.D == 64) return bwd_b<T, 64>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, gsum, st);
-    return bwd_b<T, 128>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, gsum, st);
+                  float* dk32, float* dv32, float* gsum, cudaStream_t st) {
+    if (s.D == 64) return bwd_b<T, 64>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, dk32, dv32, gsum, st);
+    return bwd_b<T, 128>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, dk32, dv32, gsum, st);
 }
 
 }  // namespace
@@ -651,10 +685,10 @@ cudaError_t launch_bwd_rowdot(const Shape& s, const void* o, const void* dO, flo
 cudaError_t launch_bwd_simt(const Shape& s, const void* q, const void* k, const void* v, const void* dO,
                             const float* lse, const float* Dd, const int32_t* idx, const float* gl,
                             const int32_t* nsel, const uint64_t* maskT, float* dq_acc, void* dk, void* dv,
-                            float* gsum, cudaStream_t st) {
+                            float* dk32, float* dv32, float* gsum, cudaStream_t st) {
     if (s.dtype == SAS_DT_FP32)
-        return bwd_d<float>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, gsum, st);
-    return bwd_d<__nv_bfloat16>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, gsum, st);
+        return bwd_d<float>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, dk32, dv32, gsum, st);
+    return bwd_d<__nv_bfloat16>(s, q, k, v, dO, lse, Dd, idx, gl, nsel, maskT, dq_acc, dk, dv, dk32, dv32, gsum, st);
 }
 
 cudaError_t launch_cast_dq(const Shape& s, const float* dq_acc, void* dq, const int* aborted, cudaStream_t st) {
@@ -678,6 +712,24 @@ cudaError_t launch_dscore(const Shape& s, const float* scores, const float* slse
     const unsigned grid = (unsigned)((s.rows() + 7) / 8);
     KernelTimer kt("dscore", st);
     dscore_kernel<<<grid, 256, 0, st>>>(s, scores, slse, idx, nsel, gsum, ds, aborted);
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) count_launches(1);
+    return e;
+}
+
+}  // namespace sas
+
+namespace sas {
+
+cudaError_t launch_reduce_dkv(const Shape& s, const float* dk32, const float* dv32, void* dk, void* dv,
+                              cudaStream_t st) {
+    const int64_t n = (int64_t)s.B * s.Hkvp * s.T * s.D / 4;
+    const unsigned grid = (unsigned)std::min<int64_t>((n + 255) / 256, 148 * 8);
+    KernelTimer kt("reduce_dkv", st);
+    if (s.dtype == SAS_DT_FP32)
+        reduce_dkv_kernel<float><<<grid, 256, 0, st>>>(s, dk32, dv32, (float*)dk, (float*)dv);
+    else
+        reduce_dkv_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(s, dk32, dv32, (__nv_bfloat16*)dk, (__nv_bfloat16*)dv);
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
     return e;

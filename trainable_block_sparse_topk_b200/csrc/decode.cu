@@ -121,8 +121,8 @@ decode_partial_kernel(DecArgs a) {
     const int p1 = min(p0 + a.bpc, nblk);
     const int cnt = max(p1 - p0, 0);
 
-    const T* kc = static_cast<const T*>(a.kc) + bg * a.stride * D;
-    const T* vc = static_cast<const T*>(a.vc) + bg * a.stride * D;
+    const T* kc = static_cast<const T*>(a.kc) + sh.kv_index(bg) * a.stride * D;
+    const T* vc = static_cast<const T*>(a.vc) + sh.kv_index(bg) * a.stride * D;
 
     // An index outside [0, C) is not a valid selection: such a block is
     // skipped (no copy, no keys) rather than read out of bounds.
@@ -566,12 +566,12 @@ decode_flat_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_consta
                 if (j >= 0) {
                     if (a.table == nullptr) {
                         ntl = j == Cb ? (int)(Nb - (int64_t)Cb * BS) : BS;
-                        rowl = (int)(bg * a.stride + (int64_t)j * BS);
+                        rowl = (int)(sh.kv_index(bg) * a.stride + (int64_t)j * BS);
                     } else {
                         const int page = a.table[(int64_t)b * a.max_blocks + j];
                         if ((unsigned)page < (unsigned)a.num_pages) {   // an invalid page is skipped
                             ntl = j == Cb ? (int)(Nb - (int64_t)Cb * BS) : BS;
-                            rowl = (page * sh.Hkv + g) * BS;
+                            rowl = (page * sh.Hkvp + g / sh.kvdiv) * BS;
                         }
                     }
                 }
@@ -1076,8 +1076,8 @@ int decode_cluster_size(int64_t groups, int nblk) {
 
 cudaError_t run_decode_flat(DecArgs a, cudaStream_t st) {
     CUtensorMap mk, mv;
-    const uint64_t rows = a.table == nullptr ? (uint64_t)a.sh.B * a.sh.Hkv * (uint64_t)a.stride
-                                             : (uint64_t)a.num_pages * a.sh.Hkv * 64;
+    const uint64_t rows = a.table == nullptr ? (uint64_t)a.sh.B * a.sh.Hkvp * (uint64_t)a.stride
+                                             : (uint64_t)a.num_pages * a.sh.Hkvp * 64;
     if (!encode_bf16_2d(&mk, a.kc, rows, 128, 64) || !encode_bf16_2d(&mv, a.vc, rows, 128, 64))
         return cudaErrorInvalidValue;
     const int64_t groups = (int64_t)a.sh.B * a.sh.Hkv;
@@ -1145,7 +1145,7 @@ cudaError_t decode_d(const DecArgs& a, cudaStream_t st) {
 // coordinates that fit in int32.
 static bool decode_flat_supported(const Shape& s, int64_t stride) {
     return s.dtype == SAS_DT_BF16 && s.D == 128 && s.bs == 64 && s.G <= 8 &&
-           (int64_t)s.B * s.Hkv * stride <= (int64_t)INT32_MAX;
+           (int64_t)s.B * s.Hkvp * stride <= (int64_t)INT32_MAX;
 }
 
 static FlatPlan flat_plan(const Shape& s, bool dense) {
@@ -1214,7 +1214,7 @@ cudaError_t set_decode_wait_limit(unsigned long long ns) {
 
 bool decode_paged_supported(const Shape& s, int64_t num_pages) {
     return s.dtype == SAS_DT_BF16 && s.D == 128 && s.bs == 64 && s.G <= 8 && num_pages >= 1 &&
-           num_pages * s.Hkv * 64 <= (int64_t)INT32_MAX;
+           num_pages * s.Hkvp * 64 <= (int64_t)INT32_MAX;
 }
 
 cudaError_t launch_decode_paged(const Shape& s, const void* q, const void* kp, const void* vp, int num_pages,

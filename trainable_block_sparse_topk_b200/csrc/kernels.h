@@ -49,13 +49,21 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 // Problem shape, validated and derived from sas_desc by the entry points.
 struct Shape {
+    // Hkv: selection groups per batch (KV heads, or query heads under
+    // per-query-head selection), G: query heads per selection group (1 then);
+    // Hkvp: KV heads of k/v/caches; kvdiv: selection groups per KV head.
     int B, T, q_offset, Hq, Hkv, G, D, bs, K;
+    int Hkvp, kvdiv;
     int NB;        // ceil((q_offset + T) / bs): score columns per row
     int nT;        // T / bs (training only): query tiles per (b, kv head)
     float scale;   // softmax scale on q.k
     int dtype;     // sas_dtype
     int gate;      // sas_gate
     __host__ __device__ int64_t rows() const { return (int64_t)B * Hkv * T; }
+    // (b, KV head) index of the K/V that selection group bg = b * Hkv + g reads
+    __host__ __device__ int64_t kv_index(int64_t bg) const {
+        return kvdiv == 1 ? bg : (bg / Hkv) * Hkvp + (bg % Hkv) / kvdiv;
+    }
 };
 
 // K1: gate normaliser + hard top-K for every (b, kv head, t) row. `lens`
@@ -111,7 +119,7 @@ size_t bwd_tc_ws_bytes(const Shape& s);
 cudaError_t launch_bwd_tc(const Shape& s, const void* q, const void* k, const void* v, const void* dO,
                           const float* attn_lse, const float* Dd, const int32_t* idx, const float* gate_logit,
                           const int32_t* n_sel, const uint64_t* maskT, void* ws, float* dq_acc, void* dk, void* dv,
-                          float* gsum, int* aborted, cudaStream_t st);
+                          float* dk32, float* dv32, float* gsum, int* aborted, cudaStream_t st);
 
 // Tensor-core forward over gathered rows (two passes + finalize): bf16, d = 128, block 64.
 bool fwd_rows_supported(const Shape& s);
@@ -127,7 +135,13 @@ cudaError_t launch_bwd_rowdot(const Shape& s, const void* o, const void* dO, flo
 cudaError_t launch_bwd_simt(const Shape& s, const void* q, const void* k, const void* v, const void* dO,
                             const float* attn_lse, const float* Dd, const int32_t* idx,
                             const float* gate_logit, const int32_t* n_sel, const uint64_t* maskT,
-                            float* dq_acc, void* dk, void* dv, float* gsum, cudaStream_t st);
+                            float* dq_acc, void* dk, void* dv, float* dk32, float* dv32, float* gsum,
+                            cudaStream_t st);
+// Per-query-head selection (s.kvdiv > 1): the backward kernels write fp32 dK, dV
+// per selection group into dk32/dv32 [B * Hkv, T, d] (NULL otherwise); this
+// sums the kvdiv groups of each KV head into dk, dv [B, Hkvp, T, d] (s.dtype).
+cudaError_t launch_reduce_dkv(const Shape& s, const float* dk32, const float* dv32, void* dk, void* dv,
+                              cudaStream_t st);
 // fp32 dq accumulator -> bf16 dq (bf16 shapes only; fp32 accumulates in place).
 // `aborted` (device flag, may be NULL): when set, dq is written as NaN.
 cudaError_t launch_cast_dq(const Shape& s, const float* dq_acc, void* dq, const int* aborted, cudaStream_t st);

@@ -98,6 +98,7 @@ sas_status make_shape(const sas_desc* d, Kind kind, Shape* s) {
     if (d->n_q_heads % d->n_kv_heads != 0) return SAS_ERR_INVALID_ARG;
     if (d->dtype != SAS_DT_BF16 && d->dtype != SAS_DT_FP32) return SAS_ERR_INVALID_ARG;
     if (d->gate < SAS_GATE_SOFTMAX || d->gate > SAS_GATE_STE) return SAS_ERR_INVALID_ARG;
+    if (d->select_heads != 0 && d->select_heads != 1) return SAS_ERR_INVALID_ARG;
     if (!(d->softmax_scale <= 0.f) && !std::isfinite(d->softmax_scale)) return SAS_ERR_INVALID_ARG;
     if (std::isnan(d->softmax_scale)) return SAS_ERR_INVALID_ARG;
     const int G = d->n_q_heads / d->n_kv_heads;
@@ -116,8 +117,17 @@ sas_status make_shape(const sas_desc* d, Kind kind, Shape* s) {
     s->T = d->seq_len;
     s->q_offset = d->q_offset;
     s->Hq = d->n_q_heads;
-    s->Hkv = d->n_kv_heads;
-    s->G = G;
+    if (d->select_heads) {          // one selection group per query head
+        s->Hkv = d->n_q_heads;
+        s->G = 1;
+        s->Hkvp = d->n_kv_heads;
+        s->kvdiv = G;
+    } else {
+        s->Hkv = d->n_kv_heads;
+        s->G = G;
+        s->Hkvp = d->n_kv_heads;
+        s->kvdiv = 1;
+    }
     s->D = d->head_dim;
     s->bs = d->block_size;
     s->K = d->top_k;
@@ -134,7 +144,7 @@ size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // Training workspace layout (each piece 256-byte aligned).
 struct TrainWs {
-    size_t maskT, Dd, gsum, dq_acc, stream, flag, total;
+    size_t maskT, Dd, gsum, dq_acc, dkv32, stream, flag, total;
 };
 
 TrainWs bwd_layout(const Shape& s) {
@@ -145,6 +155,8 @@ TrainWs bwd_layout(const Shape& s) {
     w.gsum = off;  off += align256(sizeof(float) * (size_t)s.B * s.Hkv * s.T * s.K);
     w.dq_acc = off;
     if (s.dtype != SAS_DT_FP32) off += align256(sizeof(float) * (size_t)s.B * s.Hq * s.T * s.D);
+    w.dkv32 = off;    // per-query-head selection: fp32 dK, dV per selection group
+    if (s.kvdiv > 1) off += 2 * align256(sizeof(float) * (size_t)s.B * s.Hkv * s.T * s.D);
     w.stream = off;   // the tensor-core backward's per-block token streams
     if (bwd_tc_supported(s)) off += align256(bwd_tc_ws_bytes(s));
     w.flag = off;     // set by a CTA that gave up on a wait
@@ -290,14 +302,21 @@ sas_status sas_gated_attn_bwd(const sas_desc* desc, const void* q, const void* k
     cudaError_t e = cudaMemsetAsync(aborted, 0, sizeof(int), cs);
     if (e == cudaSuccess) e = launch_sel_bitmap_T(s, idx, n_sel, maskT, cs);
     if (e == cudaSuccess) e = launch_bwd_rowdot(s, o, dO, Dd, dq_acc, cs);   // zeroes dq_acc too
+    float* dk32 = nullptr;
+    float* dv32 = nullptr;
+    if (s.kvdiv > 1) {
+        dk32 = reinterpret_cast<float*>(w + L.dkv32);
+        dv32 = reinterpret_cast<float*>(w + L.dkv32 + align256(sizeof(float) * (size_t)s.B * s.Hkv * s.T * s.D));
+    }
     if (e == cudaSuccess) {
         if (bwd_tc_supported(s))
             e = launch_bwd_tc(s, q, k, v, dO, attn_lse, Dd, idx, gate_logit, n_sel, maskT, w + L.stream, dq_acc, dk,
-                              dv, gsum, aborted, cs);
+                              dv, dk32, dv32, gsum, aborted, cs);
         else
-            e = launch_bwd_simt(s, q, k, v, dO, attn_lse, Dd, idx, gate_logit, n_sel, maskT, dq_acc, dk, dv, gsum,
-                                cs);
+            e = launch_bwd_simt(s, q, k, v, dO, attn_lse, Dd, idx, gate_logit, n_sel, maskT, dq_acc, dk, dv, dk32,
+                                dv32, gsum, cs);
     }
+    if (e == cudaSuccess && s.kvdiv > 1) e = launch_reduce_dkv(s, dk32, dv32, dk, dv, cs);
     if (e == cudaSuccess && s.dtype != SAS_DT_FP32) e = launch_cast_dq(s, dq_acc, dq, aborted, cs);
     if (e == cudaSuccess) e = launch_dscore(s, scores, score_lse, idx, n_sel, gsum, dscores, aborted, cs);
     return cuda_status(e);

@@ -40,7 +40,7 @@ pooled_score_kernel(Shape sh, const __nv_bfloat16* __restrict__ q, const __nv_bf
     const int C = (int)(sh.q_offset / sh.bs);
     const int j0 = tile * kKeys;
     const int nk = max(0, min(kKeys, C - j0));            // keys of this tile with a score to compute
-    const __nv_bfloat16* kr = kbar + (int64_t)bg * kstride * kD;
+    const __nv_bfloat16* kr = kbar + sh.kv_index(bg) * kstride * kD;   // pooled keys of the KV head
     if (tid == 0) {
         mbar_init(&s_bar, 1);
         fence_mbar_init();
