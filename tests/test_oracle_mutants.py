@@ -68,3 +68,11 @@ def test_mutant_is_caught(tmp_path, monkeypatch, name):
         except AssertionError:
             failures += 1
     assert failures > 0, f"no pin caught the mutant '{name}'"
+
+
+def test_per_head_composition_mistake_is_caught(monkeypatch):
+    """The per-query-head composition pins catch K/V heads matched to the wrong
+    query heads (tiled instead of repeated: head h paired with KV head h mod Hkv)."""
+    monkeypatch.setattr(oracle, "_repeat_heads", lambda x, G: __import__("numpy").tile(oracle._f32(x), (1, G, 1, 1)))
+    with pytest.raises(AssertionError):
+        pins.test_per_head_selection_pins(oracle, 11, 2, 0)

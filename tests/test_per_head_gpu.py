@@ -122,3 +122,56 @@ def test_per_head_decode(batch):
     assert np.array_equal(sel.idx.cpu().numpy().reshape(idx.shape), idx)
     ref = oracle.decode_per_head(od, q.float().numpy(), kc.float().numpy(), vc.float().numpy(), s.numpy())
     assert np.abs(o - ref).max() <= TOL_BF16_O
+
+
+@pytest.mark.parametrize("gate", ["sigmoid", "ste"])
+def test_per_head_gate_modes_fp32(gate):
+    """Per-head selection under other gate activations (fp32 path, elementwise)."""
+    w = synth.workload("tiny")
+    x, s = head_scores(w, 9)
+    out = run(w, x, s, gate)
+    d = odesc(w, {"sigmoid": oracle.GATE_SIGMOID, "ste": oracle.GATE_STE}[gate])
+    B_, Hq, T, dh = w.batch, w.n_q_heads, w.seq, w.head_dim
+    o, _ = oracle.fwd_per_head(d, x["q"].numpy(), x["k"].numpy(), x["v"].numpy(), s.numpy())
+    np.testing.assert_allclose(out["o"].numpy(), o.reshape(B_, Hq, T, dh), atol=TOL_FP32, rtol=0)
+    r = oracle.bwd_per_head(d, x["q"].numpy(), x["k"].numpy(), x["v"].numpy(), s.numpy(), x["dO"].numpy())
+    np.testing.assert_allclose(out["dk"].numpy(), r["dk"], atol=TOL_FP32, rtol=0)
+    np.testing.assert_allclose(out["ds"].numpy(), r["ds"].reshape(s.shape), atol=TOL_FP32, rtol=0)
+
+
+def test_per_head_paged_varlen():
+    """Per-head selection over paged pools with a length per sequence."""
+    gen = torch.Generator().manual_seed(51)
+    Bn, Hq, Hkv, N, bs, K = 2, 8, 2, 9000, 64, 15
+    lens = [9000, 4097]
+    G = Hq // Hkv
+    kc = (0.5 * torch.randn(Bn, Hkv, N, 128, generator=gen)).to(torch.bfloat16)
+    vc = (0.5 * torch.randn(Bn, Hkv, N, 128, generator=gen)).to(torch.bfloat16)
+    q = (0.5 * torch.randn(Bn, Hq, 128, generator=gen)).to(torch.bfloat16)
+    NB = -(-N // bs)
+    s = torch.randn(Bn, Hq, 1, NB, generator=gen)
+    nb = NB
+    table = torch.randperm(Bn * nb + 5, generator=gen)[: Bn * nb].to(torch.int32).view(Bn, nb).contiguous()
+    P = Bn * nb + 5
+    kp = torch.zeros(P, Hkv, bs, 128, dtype=torch.bfloat16)
+    vp = torch.zeros_like(kp)
+    pad = nb * bs - N
+    for b in range(Bn):
+        kb = torch.nn.functional.pad(kc[b], (0, 0, 0, pad)).view(Hkv, nb, bs, 128).transpose(0, 1)
+        vb = torch.nn.functional.pad(vc[b], (0, 0, 0, pad)).view(Hkv, nb, bs, 128).transpose(0, 1)
+        kp[table[b].long()] = kb
+        vp[table[b].long()] = vb
+    d = B.make_desc(batch=Bn, seq_len=1, q_offset=N - 1, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=128,
+                    block_size=bs, top_k=K, select_heads=True)
+    ln = torch.tensor(lens, dtype=torch.int32).cuda()
+    sel = api.block_topk_varlen(d, s.cuda(), ln)
+    o = api.sparse_decode_paged(d, q.cuda(), kp.cuda(), vp.cuda(), table.cuda(), ln, sel).float().cpu().numpy()
+    od = oracle.Desc(batch=Bn, seq_len=1, q_offset=N - 1, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=128,
+                     block_size=bs, top_k=K)
+    ph = oracle.per_head_desc(od)
+    ridx, _, _, _ = oracle.topk_varlen(ph, s.numpy(), lens)
+    np.testing.assert_array_equal(sel.idx.cpu().numpy().reshape(ridx.shape), ridx)
+    kpr = np.repeat(kp.float().numpy(), G, axis=1)
+    vpr = np.repeat(vp.float().numpy(), G, axis=1)
+    ref = oracle.decode_paged(ph, q.float().numpy(), kpr, vpr, table.numpy(), lens, s.numpy())
+    assert np.abs(o - ref).max() <= TOL_BF16_O
