@@ -596,3 +596,30 @@ def test_kv_head_and_batch_shards_reproduce_the_full_call():
         oh = api.sparse_decode(d2, q[sl].contiguous(), kc[sl].contiguous(), vc[sl].contiguous(),
                                api.block_topk(d2, s[sl].contiguous()))
         assert (oh.float() - of[sl].float()).abs().max() <= 2e-3
+
+
+def test_pooled_scores_many_tiles():
+    """The block scan on the 524288-token shape at batch 8 (64 rows of 8191
+    blocks: every scan CTA walks a run of many tiles through its ring, runs
+    crossing from one (batch, KV head) row into the next), all scores against
+    the oracle within float32 rounding; with a per-query-head selection too."""
+    gen = torch.Generator().manual_seed(61)
+    Bn, Hq, Hkv, N = 8, 32, 8, 524288
+    C = (N - 1) // 64
+    q = (0.5 * torch.randn(Bn, Hq, 128, generator=gen)).to(torch.bfloat16)
+    kbar = (0.5 * torch.randn(Bn, Hkv, C, 128, generator=gen)).to(torch.bfloat16)
+    for per_head in (False, True):
+        d = B.make_desc(batch=Bn, seq_len=1, q_offset=N - 1, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=128,
+                        block_size=64, top_k=31, select_heads=per_head)
+        H = Hq if per_head else Hkv
+        sc = torch.empty(Bn, H, 1, -(-N // 64), dtype=torch.float32, device="cuda")
+        B.sas_block_scores_pooled(d, q.cuda(), kbar.cuda(), sc)
+        torch.cuda.synchronize()
+        od = oracle.Desc(batch=Bn, seq_len=1, q_offset=N - 1, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=128,
+                         block_size=64, top_k=31)
+        kb = kbar.float().numpy()
+        if per_head:
+            od = oracle.per_head_desc(od)
+            kb = np.repeat(kb, Hq // Hkv, axis=1)
+        ref = oracle.pooled_scores(od, q.float().numpy(), kb)
+        np.testing.assert_allclose(sc.cpu().numpy(), ref, atol=2e-5, rtol=1e-5)
