@@ -422,31 +422,12 @@ block_topk_cta_kernel(Shape sh, const float* __restrict__ scores, const int32_t*
                         uint32_t c4[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e) c4[e] = (uint32_t)(lane + 32 * e) < nc ? s_cand[lane + 32 * e] : 0u;
-                        int bit = shift - 1;
-                        if (shift & 1) {                 // an odd bit count: one single-bit step first
+                        for (int bit = shift - 1; bit >= 0; --bit) {
                             const uint32_t cand = th | (1u << bit);
                             uint32_t c = 0;
 #pragma unroll
                             for (int e = 0; e < 4; ++e) c += c4[e] >= cand ? 1u : 0u;
                             if (__reduce_add_sync(0xffffffffu, c) >= need) th = cand;
-                            --bit;
-                        }
-                        // two bits per step: the largest of th | 11, 10, 01 (<< bit - 1)
-                        // with at least `need` keys at or above it (three independent counts)
-                        for (; bit > 0; bit -= 2) {
-                            const uint32_t c1 = th | (1u << (bit - 1)), c2 = th | (2u << (bit - 1)),
-                                           c3 = th | (3u << (bit - 1));
-                            uint32_t n1 = 0, n2 = 0, n3 = 0;
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                n1 += c4[e] >= c1 ? 1u : 0u;
-                                n2 += c4[e] >= c2 ? 1u : 0u;
-                                n3 += c4[e] >= c3 ? 1u : 0u;
-                            }
-                            n1 = __reduce_add_sync(0xffffffffu, n1);
-                            n2 = __reduce_add_sync(0xffffffffu, n2);
-                            n3 = __reduce_add_sync(0xffffffffu, n3);
-                            th = n3 >= need ? c3 : n2 >= need ? c2 : n1 >= need ? c1 : th;
                         }
                     } else {
                         for (int bit = shift - 1; bit >= 0; --bit) {
