@@ -418,17 +418,43 @@ block_topk_cta_kernel(Shape sh, const float* __restrict__ scores, const int32_t*
                 if (warp == 0) {
                     const uint32_t nc = s_misc[2];
                     uint32_t th = prefix;
-                    if (nc <= 128) {                     // four keys per lane, in registers
-                        uint32_t c4[4];
+                    if (nc <= 128) {
+                        // four keys per lane (element i = lane + 32 e, padding 0 below
+                        // every key of the bin): a warp bitonic sort, descending,
+                        // puts the need-th largest at position need - 1 -- 25
+                        // shuffle steps instead of a dependent warp count per bit
+                        uint32_t v[4];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) c4[e] = (uint32_t)(lane + 32 * e) < nc ? s_cand[lane + 32 * e] : 0u;
-                        for (int bit = shift - 1; bit >= 0; --bit) {
-                            const uint32_t cand = th | (1u << bit);
-                            uint32_t c = 0;
+                        for (int e = 0; e < 4; ++e) v[e] = (uint32_t)(lane + 32 * e) < nc ? s_cand[lane + 32 * e] : 0u;
 #pragma unroll
-                            for (int e = 0; e < 4; ++e) c += c4[e] >= cand ? 1u : 0u;
-                            if (__reduce_add_sync(0xffffffffu, c) >= need) th = cand;
+                        for (int k = 2; k <= 128; k <<= 1) {
+#pragma unroll
+                            for (int j = k >> 1; j > 0; j >>= 1) {
+                                if (j >= 32) {           // partners in the same lane
+                                    const int js = j >> 5;
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e) {
+                                        if (e & js) continue;
+                                        const bool up = ((lane + 32 * e) & k) == 0;
+                                        const uint32_t a = v[e], b = v[e | js];
+                                        v[e] = up ? max(a, b) : min(a, b);
+                                        v[e | js] = up ? min(a, b) : max(a, b);
+                                    }
+                                } else {
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e) {
+                                        const uint32_t o = __shfl_xor_sync(0xffffffffu, v[e], j);
+                                        const bool up = ((lane + 32 * e) & k) == 0;
+                                        const bool lower = (lane & j) == 0;
+                                        v[e] = (lower == up) ? max(v[e], o) : min(v[e], o);
+                                    }
+                                }
+                            }
                         }
+                        const int pos = (int)need - 1;   // 0 <= pos < nc <= 128
+                        const int ps = pos >> 5;
+                        const uint32_t mine = ps == 0 ? v[0] : ps == 1 ? v[1] : ps == 2 ? v[2] : v[3];
+                        th = __shfl_sync(0xffffffffu, mine, pos & 31);
                     } else {
                         for (int bit = shift - 1; bit >= 0; --bit) {
                             const uint32_t cand = th | (1u << bit);
