@@ -47,14 +47,13 @@ __device__ __forceinline__ int64_t row_position(const Shape& sh, const int32_t* 
 // One warp per row for rows of at most 32 * SLOTS candidates (several rows per
 // CTA). Lane l owns candidates l, l + 32, l + 64, ... (coalesced loads; index
 // order is (slot, lane) order, so ties and output positions come from per-slot
-// ballots). The K-th largest key is found by a bit search like the CTA path,
-// but over a short candidate list: when K <= 32, the K-th largest of the 32
-// lane maxima (a warp bitonic sort) is a key that at least K candidates reach,
-// so the answer lies between it and the row maximum; the keys at or above it
-// (normally a few dozen) are compacted into shared memory, four per lane, and
-// the search runs only over the bits below the prefix that bound and the
-// maximum share. Rows with more than 128 such keys, or K > 32, search all
-// their keys from the top bit. A row takes only the slots its C candidates
+// ballots). When K <= 32, the K-th largest of the 32 lane maxima (a warp
+// bitonic sort) is a key that at least K candidates reach; the keys at or
+// above it (normally a few dozen) are compacted into shared memory, four per
+// lane, and a warp bitonic sort of those <= 128 keys gives the K-th largest
+// directly. Rows with more than 128 such keys, or K > 32, run a bit search
+// over all their keys from the highest bit where the bound and the row
+// maximum differ. A row takes only the slots its C candidates
 // need (4, 8, 12 or 16 per lane): causal training rows have anywhere from 0
 // to NB - 1 candidates, and every per-slot step costs instructions.
 constexpr int kWarpCap = 128;                    // compacted keys per warp
@@ -148,16 +147,38 @@ __device__ __forceinline__ void topk_warp_row(const Shape& sh, const float* __re
         thr = top >= 31 ? 0u : (hi & ~((2u << top) - 1u));
         if (top < 0) thr = hi;
         if (compact) {
-            uint32_t c4[4];
+            uint32_t v[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) c4[e] = s_cand[4 * lane + e];
-            for (int bit = top; bit >= 0; --bit) {
-                const uint32_t cand = thr | (1u << bit);
-                uint32_t c = 0;
+            for (int e = 0; e < 4; ++e) v[e] = s_cand[lane + 32 * e];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) c += c4[e] >= cand ? 1u : 0u;
-                if (__reduce_add_sync(0xffffffffu, c) >= (uint32_t)n) thr = cand;
+            for (int k = 2; k <= 128; k <<= 1) {
+#pragma unroll
+                for (int j = k >> 1; j > 0; j >>= 1) {
+                    if (j >= 32) {
+                        const int js = j >> 5;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            if (e & js) continue;
+                            const bool up = ((lane + 32 * e) & k) == 0;
+                            const uint32_t a = v[e], b = v[e | js];
+                            v[e] = up ? max(a, b) : min(a, b);
+                            v[e | js] = up ? min(a, b) : max(a, b);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const uint32_t o = __shfl_xor_sync(0xffffffffu, v[e], j);
+                            const bool up = ((lane + 32 * e) & k) == 0;
+                            const bool lower = (lane & j) == 0;
+                            v[e] = (lower == up) ? max(v[e], o) : min(v[e], o);
+                        }
+                    }
+                }
             }
+            const int pos = n - 1;
+            const int ps = pos >> 5;
+            const uint32_t mine = ps == 0 ? v[0] : ps == 1 ? v[1] : ps == 2 ? v[2] : v[3];
+            thr = __shfl_sync(0xffffffffu, mine, pos & 31);
         } else {
             for (int bit = top; bit >= 0; --bit) {
                 const uint32_t cand = thr | (1u << bit);
