@@ -220,6 +220,8 @@ sas_status sas_block_topk_varlen(const sas_desc* desc, const float* scores, cons
  * scorer stands in for it:
  *   scores[b, g, 0, j] = qbar . kbar[b, g, j] for j < C = floor(q_offset / b),
  *   0 for C <= j < NB, with qbar the mean of the group's G query heads.
+ *   With desc.select_heads = 1 every query head h scores with its own q_h
+ *   against the pooled keys of its KV head h / G, into scores[b, h, 0, :].
  * desc: seq_len = 1, q_offset = N - 1 (as sas_sparse_decode); bf16, d 128.
  *   q [B, Hq, d] bf16, in.
  *   kbar [B, Hkv, kbar_stride_blocks, d] bf16, in: the mean key of each cached
