@@ -273,8 +273,8 @@ def pooled_scores(desc: Desc, q, kbar):
 
 # ------------------------------------------------- per-query-head selection ---
 #
-# The generalisation of the selection granularity (study note
-# 3-1 selects per query group, 3-7 scores per group): every query head h keeps
+# A generalisation of the selection granularity (study note 3-1 selects per
+# query group, 3-7 scores per group): every query head h keeps
 # its own top-K blocks from its own score row s[b, h, t, :], and still reads
 # the K/V of its KV head h // G. By definition this is the per-group problem
 # with one query head per group over K/V heads repeated G times; the gradient
