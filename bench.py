@@ -183,8 +183,8 @@ def decode_graph(B, api, dd, dw, s1c, q1, dc, vc, ws_d, flush, dev, calls=32, ca
                 times.append(e0.elapsed_time(e1))
         del graph, ks, vs
         per_call_us = statistics.median(times) * 1e3 / calls
-        return {"calls": calls, "per_call_us": per_call_us,
-                "gbs": decode_selected_bytes(dw, dw.top_k) / (per_call_us * 1e-6) / 1e9,
+        gbs = decode_selected_bytes(dw, dw.top_k) / (per_call_us * 1e-6) / 1e9
+        return {"calls": calls, "per_call_us": per_call_us, "gbs": gbs, "frac_of_hbm": gbs / load_peaks()[0]["hbm_gbs"],
                 "inputs": f"{caches} distinct caches x {calls // caches} distinct index sets; "
                           "L2 flushed before each replay"}
     except Exception as exc:   # reported beside the other numbers, never fatal
@@ -498,6 +498,22 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     clocks = sampler.stop()
 
+    # every kernel of the step on its own (three more steps, outside the timed
+    # loop, CUDA events around each launch): per-launch mean microseconds
+    side_names = ("block_topk", "sel_stream_index", "sel_stream_fill", "fwd_rows_shift", "fwd_rows",
+                  "fwd_rows_finalize", "fwd_rows_fixup", "rowdot", "bwd_tc", "cast_dq", "dscore")
+    B.sas_kernel_timing(",".join(side_names))
+    for _ in range(3):
+        feed()
+        step(new_events())
+    torch.cuda.synchronize()
+    B.sas_kernel_timing(None)
+    step_kernels_us = {}
+    for name in side_names:
+        ms, n = B.sas_kernel_time(name)
+        if n:
+            step_kernels_us[name] = {"us_per_launch": 1e3 * ms / n, "launches_per_step": n / 3}
+
     part_ms = {p: [ev[i].elapsed_time(ev[i + 1]) for ev in evs] for i, p in enumerate(parts)}
     step_ms = [ev[0].elapsed_time(ev[5]) for ev in evs]
     total_ms = max_over_ranks(sum(step_ms), world, dev)
@@ -753,6 +769,13 @@ def run_ours(args, rank, world, local_rank):
         decode_info["graph"] = decode_graph(B, api, decode_desc(B, gw), gw, gs, gq.to(dt).to(dev), gkc, gvc,
                                             api.workspace(B.SAS_OP_DECODE, decode_desc(B, gw), dev), flush, dev)
         decode_info["graph"]["workload"] = f"decode N{gw.seq} B1 K31"
+        # the batch-8 long-cache decode the same way: 3 caches (the base one and
+        # two rotated copies, 17 GB each) x 8 index sets, 67 MB selected per call
+        lw, lkc, lvc, lq, ls = decode_inputs("long", 8, 31, dev, dt, caches)
+        decode_info["graph_long_b8"] = decode_graph(B, api, decode_desc(B, lw), lw, ls, lq.to(dt).to(dev), lkc, lvc,
+                                                    api.workspace(B.SAS_OP_DECODE, decode_desc(B, lw), dev), flush,
+                                                    dev, calls=24, caches=3)
+        decode_info["graph_long_b8"]["workload"] = f"long N{lw.seq} B8 K31"
 
     result = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -772,6 +795,7 @@ def run_ours(args, rank, world, local_rank):
                                                                    "selections_per_visited_block")}},
         "parts_us": {p: mean[p] * 1e3 for p in parts},
         "kernels_us": kernels_us,
+        "step_kernels_us": step_kernels_us,
         "kernel_frac_of_bf16_peak": kernel_frac,
         "topk": {"causal_score_bytes": causal_score_bytes, "gbs": topk_gbs, "frac_of_hbm": topk_gbs / peaks["hbm_gbs"]},
         "roofline": roof,

@@ -445,6 +445,42 @@ cast_bf16x8_kernel(int64_t n8, const float4* __restrict__ src, uint4* __restrict
 
 // ------------------------------------------------------- score gradient (K5) ---
 
+// The kept blocks' own terms kv[r] (slots lane and lane + 32; si[r] = -1 when
+// not kept) and the factor T of the dense term -g_i T, per gate activation
+// (Gsum_k = dL / d log g_k):
+//   softmax           d log g_i/ds_k = [i=k] - g_k:  kept Gsum_k, T = sum Gsum
+//   sigmoid           log g_k = log sigmoid(s_k):     kept Gsum_k (1 - sigmoid(s_k))
+//   raw               log g_k = s_k:                  kept Gsum_k
+//   softmax (kept)    log g_k = s_k - log sum_I e^s:  kept Gsum_k - p_k sum Gsum
+//   hard (STE)        dL/dg_k = Gsum_k, dg_i/ds_k = g_i([i=k] - g_k):
+//                                                     kept Gsum_k g_k, T = sum Gsum g
+__device__ __forceinline__ void dscore_kept_terms(int mode, const int (&si)[2], const float (&sg)[2],
+                                                  const float (&sk)[2], float lse, float (&kv)[2], float& T) {
+    kv[0] = kv[1] = 0.f;
+    T = 0.f;
+    if (mode == SAS_GATE_SOFTMAX) {
+        kv[0] = sg[0];
+        kv[1] = sg[1];
+        T = warp_sum(sg[0] + sg[1]);
+    } else if (mode == SAS_GATE_STE) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) kv[r] = si[r] >= 0 ? sg[r] * expf(sk[r] - lse) : 0.f;
+        T = warp_sum(kv[0] + kv[1]);
+    } else if (mode == SAS_GATE_SIGMOID) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) kv[r] = si[r] >= 0 ? sg[r] / (1.f + expf(sk[r])) : 0.f;   // 1 - sigmoid(s)
+    } else if (mode == SAS_GATE_RAW) {
+        kv[0] = sg[0];
+        kv[1] = sg[1];
+    } else if (mode == SAS_GATE_SOFTMAX_SELECTED) {
+        const float m = warp_max(fmaxf(sk[0], sk[1]));
+        const float l = warp_sum((si[0] >= 0 ? expf(sk[0] - m) : 0.f) + (si[1] >= 0 ? expf(sk[1] - m) : 0.f));
+        const float tot = warp_sum(sg[0] + sg[1]);
+#pragma unroll
+        for (int r = 0; r < 2; ++r) kv[r] = si[r] >= 0 ? sg[r] - expf(sk[r] - m) / l * tot : 0.f;
+    }
+}
+
 // ds_i = dL/ds_i for i < C, 0 otherwise, from Gsum_k = dL/d(log g_k) of the
 // kept blocks through the gate activation's derivative. Softmax gate
 // (arXiv text 4: d log g_i / d s_k = [i=k] - g_k, g_i = exp(s_i - score_lse)):
@@ -495,37 +531,8 @@ dscore_kernel(Shape sh, const float* __restrict__ scores, const float* __restric
         if (lane + 32 * r >= n || (unsigned)si[r] >= (unsigned)C) { si[r] = -1; sg[r] = 0.f; }
         sk[r] = si[r] >= 0 ? sr[si[r]] : -INFINITY;
     }
-    // the kept blocks' own terms and the factor T of the dense term, per mode
-    // (Gsum_k = dL / d log g_k):
-    //   softmax           d log g_i/ds_k = [i=k] - g_k:  kept Gsum_k, T = sum Gsum
-    //   sigmoid           log g_k = log sigmoid(s_k):     kept Gsum_k (1 - sigmoid(s_k))
-    //   raw               log g_k = s_k:                  kept Gsum_k
-    //   softmax (kept)    log g_k = s_k - log sum_I e^s:  kept Gsum_k - p_k sum Gsum
-    //   hard (STE)        dL/dg_k = Gsum_k, dg_i/ds_k = g_i([i=k] - g_k):
-    //                                                     kept Gsum_k g_k, T = sum Gsum g
-    float kv[2] = {0.f, 0.f};
-    float T = 0.f;
-    if (mode == SAS_GATE_SOFTMAX) {
-        kv[0] = sg[0];
-        kv[1] = sg[1];
-        T = warp_sum(sg[0] + sg[1]);
-    } else if (mode == SAS_GATE_STE) {
-#pragma unroll
-        for (int r = 0; r < 2; ++r) kv[r] = si[r] >= 0 ? sg[r] * expf(sk[r] - lse) : 0.f;
-        T = warp_sum(kv[0] + kv[1]);
-    } else if (mode == SAS_GATE_SIGMOID) {
-#pragma unroll
-        for (int r = 0; r < 2; ++r) kv[r] = si[r] >= 0 ? sg[r] / (1.f + expf(sk[r])) : 0.f;   // 1 - sigmoid(s)
-    } else if (mode == SAS_GATE_RAW) {
-        kv[0] = sg[0];
-        kv[1] = sg[1];
-    } else if (mode == SAS_GATE_SOFTMAX_SELECTED) {
-        const float m = warp_max(fmaxf(sk[0], sk[1]));
-        const float l = warp_sum((si[0] >= 0 ? expf(sk[0] - m) : 0.f) + (si[1] >= 0 ? expf(sk[1] - m) : 0.f));
-        const float tot = warp_sum(sg[0] + sg[1]);
-#pragma unroll
-        for (int r = 0; r < 2; ++r) kv[r] = si[r] >= 0 ? sg[r] - expf(sk[r] - m) / l * tot : 0.f;
-    }
+    float kv[2], T;
+    dscore_kept_terms(mode, si, sg, sk, lse, kv, T);
     const bool any = mode != SAS_GATE_NONE;
     int base = 0;
     auto chunk = [&](int c0, float sc) {
@@ -554,6 +561,71 @@ dscore_kernel(Shape sh, const float* __restrict__ scores, const float* __restric
     }
     for (int c0 = kPre * 32; c0 < sh.NB; c0 += 32)     // long rows: the rest one chunk at a time
         chunk(c0, (dense_term && c0 + lane < C) ? sr[c0 + lane] : 0.f);
+}
+
+// The same for rows of NB <= 1024 columns, NB % 4 == 0: lane l owns columns
+// 4l .. 4l + 3 of each 128-column piece (16-byte loads and stores). Every
+// column first gets its dense term (0 past C); after a warp barrier, which
+// orders the warp's global stores, each kept slot's lane rewrites its column
+// with the dense term plus its own term, computed as the scalar kernel does.
+constexpr int kDsVecCols = 1024;
+__global__ void __launch_bounds__(256)
+dscore_vec_kernel(Shape sh, const float* __restrict__ scores, const float* __restrict__ slse,
+                  const int32_t* __restrict__ idx, const int32_t* __restrict__ nsel,
+                  const float* __restrict__ gsum, float* __restrict__ ds, const int* __restrict__ aborted) {
+    constexpr int kPieces = kDsVecCols / 128;
+    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= sh.rows()) return;
+    float4* dr = reinterpret_cast<float4*>(ds + row * sh.NB);
+    const int nb4 = sh.NB / 4;
+    if (aborted != nullptr && *aborted) {   // Gsum is incomplete: mark the row invalid
+        const float nan = __int_as_float(0x7fc00000);
+        for (int i = lane; i < nb4; i += 32) dr[i] = make_float4(nan, nan, nan, nan);
+        return;
+    }
+    const int t = (int)(row % sh.T);
+    const int C = (int)(((int64_t)sh.q_offset + t) / sh.bs);
+    const int mode = sh.gate;
+    const bool dense_term = mode == SAS_GATE_SOFTMAX || mode == SAS_GATE_STE;
+    const bool any = mode != SAS_GATE_NONE;
+    const float* sr = scores + row * sh.NB;
+    const float4* sr4 = reinterpret_cast<const float4*>(sr);
+    const int n = nsel[row];
+    const float lse = slse[row];
+    int si[2];
+    float sg[2], sk[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int slot = lane + 32 * r;
+        si[r] = slot < sh.K ? idx[row * sh.K + slot] : -1;
+        sg[r] = slot < sh.K ? gsum[row * sh.K + slot] : 0.f;
+    }
+    float4 sv[kPieces];
+#pragma unroll
+    for (int q = 0; q < kPieces; ++q) {
+        const int i = q * 128 + 4 * lane;
+        sv[q] = (dense_term && i < C) ? sr4[i / 4] : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        if (lane + 32 * r >= n || (unsigned)si[r] >= (unsigned)C) { si[r] = -1; sg[r] = 0.f; }
+        sk[r] = si[r] >= 0 ? sr[si[r]] : -INFINITY;
+    }
+    float kv[2], T;
+    dscore_kept_terms(mode, si, sg, sk, lse, kv, T);
+    auto dense = [&](int i, float sc) { return (dense_term && i < C) ? -expf(sc - lse) * T : 0.f; };
+#pragma unroll
+    for (int q = 0; q < kPieces; ++q) {
+        const int i = q * 128 + 4 * lane;
+        if (i < sh.NB)
+            dr[i / 4] = make_float4(dense(i, sv[q].x), dense(i + 1, sv[q].y), dense(i + 2, sv[q].z),
+                                    dense(i + 3, sv[q].w));
+    }
+    __syncwarp();
+#pragma unroll
+    for (int r = 0; r < 2; ++r)
+        if (any && si[r] >= 0) ds[row * sh.NB + si[r]] = dense(si[r], sk[r]) + kv[r];
 }
 
 template <typename T, int D, int GMAX, int BS>
@@ -711,7 +783,11 @@ cudaError_t launch_dscore(const Shape& s, const float* scores, const float* slse
                           const int32_t* nsel, const float* gsum, float* ds, const int* aborted, cudaStream_t st) {
     const unsigned grid = (unsigned)((s.rows() + 7) / 8);
     KernelTimer kt("dscore", st);
-    dscore_kernel<<<grid, 256, 0, st>>>(s, scores, slse, idx, nsel, gsum, ds, aborted);
+    const bool vec = s.NB % 4 == 0 && s.NB <= kDsVecCols && ((uintptr_t)scores & 15) == 0 && ((uintptr_t)ds & 15) == 0;
+    if (vec)
+        dscore_vec_kernel<<<grid, 256, 0, st>>>(s, scores, slse, idx, nsel, gsum, ds, aborted);
+    else
+        dscore_kernel<<<grid, 256, 0, st>>>(s, scores, slse, idx, nsel, gsum, ds, aborted);
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
     return e;

@@ -58,6 +58,12 @@ __device__ __forceinline__ int64_t row_position(const Shape& sh, const int32_t* 
 // to NB - 1 candidates, and every per-slot step costs instructions.
 constexpr int kWarpCap = 128;                    // compacted keys per warp
 
+__device__ __forceinline__ uint32_t warp_sum_u32(uint32_t x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
 template <int SLOTS>
 __device__ __forceinline__ void topk_warp_row(const Shape& sh, const float* __restrict__ scores, int64_t row, int C,
                                               uint32_t* __restrict__ s_cand, int32_t* __restrict__ idx_out,
@@ -104,8 +110,8 @@ __device__ __forceinline__ void topk_warp_row(const Shape& sh, const float* __re
 #pragma unroll
         for (int k = 0; k < SLOTS; ++k) lmax = max(lmax, key[k]);
         const uint32_t hi = __reduce_max_sync(0xffffffffu, lmax);
-        bool compact = false;
-        uint32_t lo = 0;
+        bool compact = false, small = false;
+        uint32_t lo = 0, rank = (uint32_t)n;   // the threshold is the rank-th largest compacted key
         if (n <= 32) {
             // bitonic sort of the lane maxima, descending across lanes
             uint32_t v = lmax;
@@ -119,10 +125,33 @@ __device__ __forceinline__ void topk_warp_row(const Shape& sh, const float* __re
                     v = (lower == up) ? max(v, o) : min(v, o);
                 }
             }
-            lo = __shfl_sync(0xffffffffu, v, n - 1);              // n lane maxima are >= lo
-            uint32_t cnt = 0;
+            // the smallest i with #{keys >= v_i} >= n (i = n - 1 always
+            // qualifies: v_0 .. v_{n-1} are the maxima of n different lanes,
+            // valid keys since n < C); then v_{i-1} > v_i, and the n-th
+            // largest key lies in [v_i, v_{i-1})
+            int ia = 0, ib = n - 1;
+            while (ia < ib) {                                     // warp-uniform
+                const int mid = (ia + ib) >> 1;
+                const uint32_t vm = __shfl_sync(0xffffffffu, v, mid);
+                uint32_t c = 0;
 #pragma unroll
-            for (int k = 0; k < SLOTS; ++k) cnt += key[k] >= lo ? 1u : 0u;
+                for (int k = 0; k < SLOTS; ++k) c += key[k] >= vm ? 1u : 0u;
+                if (warp_sum_u32(c) >= (uint32_t)n) ib = mid; else ia = mid + 1;
+            }
+            lo = __shfl_sync(0xffffffffu, v, ia);
+            const uint32_t upv = __shfl_sync(0xffffffffu, v, ia > 0 ? ia - 1 : 0);
+            const bool has_up = ia > 0;
+            // the keys at or above v_{i-1} are all kept; the ones in
+            // [v_i, v_{i-1}) are compacted, and the threshold is the
+            // (n - #above)-th largest of them
+            uint32_t ca = 0, cnt = 0;
+#pragma unroll
+            for (int k = 0; k < SLOTS; ++k) {
+                const bool over = has_up && key[k] >= upv;
+                ca += over ? 1u : 0u;
+                cnt += (key[k] >= lo && !over) ? 1u : 0u;
+            }
+            rank = (uint32_t)n - warp_sum_u32(ca);
             uint32_t incl = cnt;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -131,22 +160,33 @@ __device__ __forceinline__ void topk_warp_row(const Shape& sh, const float* __re
             }
             const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
             compact = total <= (uint32_t)kCap;
+            small = total <= 32u;
             if (compact) {
                 uint32_t at = incl - cnt;
 #pragma unroll
                 for (int k = 0; k < SLOTS; ++k)
-                    if (key[k] >= lo) s_cand[at++] = key[k];
-                for (uint32_t e = total + lane; e < (uint32_t)kCap; e += 32) s_cand[e] = 0u;
+                    if (key[k] >= lo && !(has_up && key[k] >= upv)) s_cand[at++] = key[k];
+                const uint32_t fill = small ? 32u : (uint32_t)kCap;
+                for (uint32_t e = total + lane; e < fill; e += 32) s_cand[e] = 0u;
                 __syncwarp();
             }
         }
-        // bit search for the largest v with #{keys >= v} >= n, starting below
-        // the prefix that lo and hi share (every v in [lo, hi] has it)
-        const uint32_t diff = lo ^ hi;
-        const int top = diff == 0u ? -1 : 31 - __clz(diff);
-        thr = top >= 31 ? 0u : (hi & ~((2u << top) - 1u));
-        if (top < 0) thr = hi;
-        if (compact) {
+        if (compact && small) {
+            // at most 32 keys, one per lane: a 32-wide bitonic sort, descending
+            uint32_t w1 = s_cand[lane];
+#pragma unroll
+            for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+                for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                    const uint32_t o = __shfl_xor_sync(0xffffffffu, w1, stride);
+                    const bool up = (lane & size) == 0;
+                    const bool lower = (lane & stride) == 0;
+                    w1 = (lower == up) ? max(w1, o) : min(w1, o);
+                }
+            }
+            thr = __shfl_sync(0xffffffffu, w1, (int)rank - 1);
+        } else if (compact) {
+            // at most 128 keys, four per lane: a 128-wide bitonic sort, descending
             uint32_t v[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) v[e] = s_cand[lane + 32 * e];
@@ -175,36 +215,54 @@ __device__ __forceinline__ void topk_warp_row(const Shape& sh, const float* __re
                     }
                 }
             }
-            const int pos = n - 1;
+            const int pos = (int)rank - 1;
             const int ps = pos >> 5;
             const uint32_t mine = ps == 0 ? v[0] : ps == 1 ? v[1] : ps == 2 ? v[2] : v[3];
             thr = __shfl_sync(0xffffffffu, mine, pos & 31);
         } else {
+            // bit search for the largest v with #{keys >= v} >= n, starting
+            // below the prefix that lo and hi share (every v in [lo, hi] has it)
+            const uint32_t diff = lo ^ hi;
+            const int top = diff == 0u ? -1 : 31 - __clz(diff);
+            thr = top >= 31 ? 0u : (hi & ~((2u << top) - 1u));
+            if (top < 0) thr = hi;
             for (int bit = top; bit >= 0; --bit) {
                 const uint32_t cand = thr | (1u << bit);
                 uint32_t c = 0;
 #pragma unroll
                 for (int k = 0; k < SLOTS; ++k) c += key[k] >= cand ? 1u : 0u;
-                if (__reduce_add_sync(0xffffffffu, c) >= (uint32_t)n) thr = cand;
+                if (warp_sum_u32(c) >= (uint32_t)n) thr = cand;
             }
         }
     }
-
-    // keep every key above thr and the first `need` copies of thr in index order
-    uint32_t gt = 0;
-#pragma unroll
-    for (int k = 0; k < SLOTS; ++k) gt += (n > 0 && lane + 32 * k < C && key[k] > thr) ? 1u : 0u;
-    const uint32_t need = (uint32_t)n - __reduce_add_sync(0xffffffffu, gt);
-    int32_t* io = idx_out + row * K;
-    float* go = gl_out + row * K;
-    uint32_t eq_run = 0, take_bits = 0;
+    // keep every key above thr and the first `need` copies of thr in index
+    // order (all of them when that is every copy: no tie ranks needed)
+    uint32_t gt = 0, eq = 0;
 #pragma unroll
     for (int k = 0; k < SLOTS; ++k) {
-        const int i = lane + 32 * k;
-        const bool valid = n > 0 && i < C;
-        const uint32_t eqb = __ballot_sync(0xffffffffu, valid && key[k] == thr);
-        if (valid && (key[k] > thr || (key[k] == thr && eq_run + __popc(eqb & lt) < need))) take_bits |= 1u << k;
-        eq_run += __popc(eqb);
+        const bool valid = n > 0 && lane + 32 * k < C;
+        gt += (valid && key[k] > thr) ? 1u : 0u;
+        eq += (valid && key[k] == thr) ? 1u : 0u;
+    }
+    const uint32_t need = (uint32_t)n - warp_sum_u32(gt);
+    const bool all_eq = warp_sum_u32(eq) == need;
+    int32_t* io = idx_out + row * K;
+    float* go = gl_out + row * K;
+    uint32_t take_bits = 0;
+    if (all_eq) {
+#pragma unroll
+        for (int k = 0; k < SLOTS; ++k)
+            if (n > 0 && lane + 32 * k < C && key[k] >= thr) take_bits |= 1u << k;
+    } else {
+        uint32_t eq_run = 0;
+#pragma unroll
+        for (int k = 0; k < SLOTS; ++k) {
+            const int i = lane + 32 * k;
+            const bool valid = n > 0 && i < C;
+            const uint32_t eqb = __ballot_sync(0xffffffffu, valid && key[k] == thr);
+            if (valid && (key[k] > thr || (key[k] == thr && eq_run + __popc(eqb & lt) < need))) take_bits |= 1u << k;
+            eq_run += __popc(eqb);
+        }
     }
     float lse_sel = 0.f;
     if (sh.gate == SAS_GATE_SOFTMAX_SELECTED) {      // normaliser over the kept blocks
