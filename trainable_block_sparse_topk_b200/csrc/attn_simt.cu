@@ -498,8 +498,10 @@ dscore_kernel(Shape sh, const float* __restrict__ scores, const float* __restric
         for (int i = lane; i < sh.NB; i += 32) ds[row * sh.NB + i] = __int_as_float(0x7fc00000);
         return;
     }
-    const int t = (int)(row % sh.T);
-    const int C = (int)(((int64_t)sh.q_offset + t) / sh.bs);
+    const bool r32 = sh.rows() <= (int64_t)UINT32_MAX;
+    const int t = r32 ? (int)((uint32_t)row % (uint32_t)sh.T) : (int)(row % sh.T);
+    const int C = r32 ? (int)(((uint32_t)sh.q_offset + (uint32_t)t) / (uint32_t)sh.bs)
+                      : (int)(((int64_t)sh.q_offset + t) / sh.bs);
     const int mode = sh.gate;
     // every candidate gets -g_i * T (softmax gate and its straight-through
     // hard form), each kept block its own term on top
@@ -584,8 +586,10 @@ dscore_vec_kernel(Shape sh, const float* __restrict__ scores, const float* __res
         for (int i = lane; i < nb4; i += 32) dr[i] = make_float4(nan, nan, nan, nan);
         return;
     }
-    const int t = (int)(row % sh.T);
-    const int C = (int)(((int64_t)sh.q_offset + t) / sh.bs);
+    const bool r32 = sh.rows() <= (int64_t)UINT32_MAX;
+    const int t = r32 ? (int)((uint32_t)row % (uint32_t)sh.T) : (int)(row % sh.T);
+    const int C = r32 ? (int)(((uint32_t)sh.q_offset + (uint32_t)t) / (uint32_t)sh.bs)
+                      : (int)(((int64_t)sh.q_offset + t) / sh.bs);
     const int mode = sh.gate;
     const bool dense_term = mode == SAS_GATE_SOFTMAX || mode == SAS_GATE_STE;
     const bool any = mode != SAS_GATE_NONE;

@@ -304,8 +304,11 @@ block_topk_warp_kernel(Shape sh, const float* __restrict__ scores, const int32_t
     const int warp = threadIdx.x >> 5;
     const int64_t row = (int64_t)blockIdx.x * 8 + warp;
     if (row >= sh.rows()) return;                // warp-uniform
-    const int t = (int)(row % sh.T);
-    const int C = (int)(row_position(sh, lens, row, t) / sh.bs);
+    // 32-bit index arithmetic where it fits (training rows: a few per cent of the call)
+    const bool r32 = sh.rows() <= (int64_t)UINT32_MAX;
+    const int t = r32 ? (int)((uint32_t)row % (uint32_t)sh.T) : (int)(row % sh.T);
+    const int C = (lens == nullptr && r32) ? (int)(((uint32_t)sh.q_offset + (uint32_t)t) / (uint32_t)sh.bs)
+                                           : (int)(row_position(sh, lens, row, t) / sh.bs);
     if (SLOTS > 4 && C <= 128)
         topk_warp_row<4>(sh, scores, row, C, s_cand[warp], idx_out, gl_out, lse_out, nsel_out);
     else if (SLOTS > 8 && C <= 256)
