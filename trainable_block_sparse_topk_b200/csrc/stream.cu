@@ -13,10 +13,10 @@
 // tokens from the column bitmap maskT[b,g,j,:], reserves a contiguous run of
 // entries with one atomic add (runs of different blocks land in any order;
 // each run's own order is fixed), stores the running token count at the start
-// of every later query tile and writes the block's own 64 tokens. Then a
-// group of lanes per row places the row's kept (row, slot) entries: the position of token t in
-// block j's run is the count before t's tile plus the set bits of the tile's
-// bitmap word below t -- no search. Entry e:
+// of every later query tile and writes the block's own 64 tokens. Then one
+// CTA per query tile places the tile's kept (row, slot) entries, grouped by
+// block: the position of token t in block j's run is the count before t's
+// tile plus the set bits of the tile's bitmap word below t -- no search. Entry e:
 //   ent[e] = {t, bits of log g_j(t), slot of j in t's ascending kept list, 0}
 //            (log-gate 0 and slot -1 for the block's own tokens),
 //   rv[e * rvs + h * vals + v] = row value v of query head h of token t.
@@ -91,54 +91,97 @@ sel_stream_index_kernel(Shape sh, const uint64_t* __restrict__ maskT, const floa
     }
 }
 
-// kL lanes per (b, g, t) row (16 when K <= 16, two rows per warp, else 32):
-// they load the row's per-head values, kept blocks and log-gates together and
-// broadcast the values to the group, then each kept slot (one lane each)
-// places its entry and the row values (rvs <= 16 floats, 16-byte stores) in
-// an earlier block's run.
-template <int kL>
+// One CTA per (b, g, query tile tau) places the tile's kept (row, slot)
+// entries. The tile's kept blocks, log-gates and per-head row values are read
+// once (contiguous rows); the entries are bucketed by block in shared memory
+// (count, scan, scatter), and consecutive threads then write consecutive
+// entries of one block's segment for this tile -- the tokens of tile tau that
+// kept block j occupy positions base + pre[tau] .. + popcount(bitmap word) of
+// block j's run, so the stores coalesce instead of scattering one row's K
+// entries over K runs. Position of token t in its segment: the set bits of the
+// tile's bitmap word below t (the same for any processing order).
 __global__ void __launch_bounds__(kThreads)
-sel_stream_fill_kernel(Shape sh, const uint64_t* __restrict__ maskT, const int32_t* __restrict__ idx,
+sel_stream_tile_kernel(Shape sh, const uint64_t* __restrict__ maskT, const int32_t* __restrict__ idx,
                        const float* __restrict__ gl, const int32_t* __restrict__ nsel, const float* __restrict__ v0,
                        const float* __restrict__ v1, int vals, SelStream st) {
-    const int sub = (threadIdx.x & 31) / kL, li = threadIdx.x & (kL - 1);
-    const int64_t row = ((int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5)) * (32 / kL) + sub;
-    const bool ok = row < sh.rows();               // no early exit: the groups shuffle
-    const int bg = ok ? (int)(row / sh.T) : 0;
-    const int t = ok ? (int)(row - (int64_t)bg * sh.T) : 0;
-    const int tau = t / kBS;
+    extern __shared__ __align__(16) unsigned char smem[];
+    const int K = sh.K, tid = threadIdx.x;
+    const int bg = (int)(blockIdx.x / sh.nT);
+    const int tau = (int)(blockIdx.x - (int64_t)bg * sh.nT);
+    if (tau == 0) return;                            // tile 0 has no earlier block
     const int b = bg / sh.Hkv, g = bg - b * sh.Hkv;
-    const int nv = sh.G * vals;                    // <= 16
-    float myv = 0.f;
-    if (ok && li < nv) {
-        const int h = li / vals, v = li - h * vals;
-        const int64_t qrow = ((int64_t)b * sh.Hq + g * sh.G + h) * sh.T + t;
-        myv = v == 0 ? v0[qrow] : v1[qrow];
+    const int ne = kBS * K;                          // (token, slot) pairs of the tile
+    const int rvs = st.rvs;
+    int* s_j = reinterpret_cast<int*>(smem);                 // [ne] kept block, -1 if not placed here
+    float* s_lg = reinterpret_cast<float*>(s_j + ne);        // [ne] its log-gate
+    float* s_rv = s_lg + ne;                                 // [kBS][rvs] row values of the tile's tokens
+    int* s_cnt = reinterpret_cast<int*>(s_rv + kBS * rvs);   // [tau] entries per block, then cursors
+    uint16_t* s_ord = reinterpret_cast<uint16_t*>(s_cnt + tau);   // [ne] entry ids grouped by block
+    __shared__ int s_part[kThreads / 32];
+    const int64_t row0 = (int64_t)bg * sh.T + (int64_t)tau * kBS;   // the tile's first (b, g, t) row
+    for (int e = tid; e < ne; e += kThreads) {
+        const int tl = e / K, slot = e - tl * K;
+        const int64_t row = row0 + tl;
+        int j = slot < nsel[row] ? idx[row * K + slot] : -1;
+        if (j >= tau) j = -1;                        // the own block is written by the index kernel
+        s_j[e] = j;
+        s_lg[e] = gl[row * K + slot];
     }
-    const int ns = ok ? nsel[row] : 0;
-    const uint64_t below = (1ull << (t & (kBS - 1))) - 1ull;
-    for (int s0 = 0; s0 < sh.K; s0 += kL) {         // uniform across the warp
-        const int slot = s0 + li;
-        int j = -1;
-        float lg = 0.f;
-        if (ok && slot < sh.K) {
-            j = idx[row * sh.K + slot];
-            lg = gl[row * sh.K + slot];
+    for (int i = tid; i < kBS * rvs; i += kThreads) {   // token fastest: contiguous loads per head
+        const int tl = i % kBS, k = i / kBS;
+        const int h = k / vals, v = k - h * vals;
+        float x = 0.f;
+        if (h < sh.G) {
+            const int64_t qrow = ((int64_t)b * sh.Hq + g * sh.G + h) * sh.T + (int64_t)tau * kBS + tl;
+            x = v == 0 ? v0[qrow] : v1[qrow];
         }
-        float rowv[kMaxRvs];
+        s_rv[tl * rvs + k] = x;
+    }
+    for (int i = tid; i < tau; i += kThreads) s_cnt[i] = 0;
+    __syncthreads();
+    for (int e = tid; e < ne; e += kThreads)
+        if (s_j[e] >= 0) atomicAdd(&s_cnt[s_j[e]], 1);
+    __syncthreads();
+    // exclusive scan of the per-block counts: thread tid owns blocks
+    // [tid * per, (tid + 1) * per)
+    const int per = (tau + kThreads - 1) / kThreads;
+    int mine = 0;
+    for (int i = tid * per; i < min(tau, (tid + 1) * per); ++i) mine += s_cnt[i];
+    const int lane = tid & 31, warp = tid >> 5;
+    int inc = mine;
 #pragma unroll
-        for (int v = 0; v < kMaxRvs; ++v) rowv[v] = __shfl_sync(0xffffffffu, myv, v, kL);   // 0 past G * vals
-        // the own block is written by the index kernel
-        if (slot < ns && j >= 0 && j < tau) {
-            const int64_t blk = (int64_t)bg * sh.NB + j;
-            const int64_t pos = (int64_t)st.base[blk] + st.pre[blk * sh.nT + tau] +
-                                __popcll(maskT[blk * sh.nT + tau] & below);
-            st.ent[pos] = make_int4(t, __float_as_int(lg), slot, 0);
-            float4* out = reinterpret_cast<float4*>(st.rv + pos * st.rvs);
-#pragma unroll
-            for (int v = 0; v < kMaxRvs; v += 4)
-                if (v < st.rvs) out[v / 4] = make_float4(rowv[v], rowv[v + 1], rowv[v + 2], rowv[v + 3]);
-        }
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+    }
+    if (lane == 31) s_part[warp] = inc;
+    __syncthreads();
+    int off = inc - mine;
+    for (int w = 0; w < warp; ++w) off += s_part[w];
+    int total = 0;
+    for (int w = 0; w < kThreads / 32; ++w) total += s_part[w];
+    for (int i = tid * per; i < min(tau, (tid + 1) * per); ++i) {
+        const int c = s_cnt[i];
+        s_cnt[i] = off;                              // cursor: first slot of block i's bucket
+        off += c;
+    }
+    __syncthreads();
+    for (int e = tid; e < ne; e += kThreads) {
+        const int j = s_j[e];
+        if (j >= 0) s_ord[atomicAdd(&s_cnt[j], 1)] = (uint16_t)e;
+    }
+    __syncthreads();
+    for (int p = tid; p < total; p += kThreads) {
+        const int e = s_ord[p];
+        const int tl = e / K, slot = e - tl * K;
+        const int j = s_j[e];
+        const int64_t blk = (int64_t)bg * sh.NB + j;
+        const int64_t pos = (int64_t)st.base[blk] + st.pre[blk * sh.nT + tau] +
+                            __popcll(maskT[blk * sh.nT + tau] & ((1ull << tl) - 1ull));
+        st.ent[pos] = make_int4(tau * kBS + tl, __float_as_int(s_lg[e]), slot, 0);
+        const float4* src = reinterpret_cast<const float4*>(s_rv + tl * rvs);
+        float4* dst = reinterpret_cast<float4*>(st.rv + pos * rvs);
+        for (int v = 0; v < rvs / 4; ++v) dst[v] = src[v];
     }
 }
 
@@ -192,16 +235,15 @@ cudaError_t launch_sel_stream(const Shape& s, const uint64_t* maskT, const int32
     if (e != cudaSuccess) return e;
     count_launches(1);
     {
-        KernelTimer kt("sel_stream_fill", stream);
-        if (s.K <= 16) {
-            const int64_t rpb = 2 * (kThreads / 32);
-            sel_stream_fill_kernel<16><<<(unsigned)((s.rows() + rpb - 1) / rpb), kThreads, 0, stream>>>(
-                s, maskT, idx, gl, nsel, v0, v1, vals, st);
-        } else {
-            const int64_t rpb = kThreads / 32;
-            sel_stream_fill_kernel<32><<<(unsigned)((s.rows() + rpb - 1) / rpb), kThreads, 0, stream>>>(
-                s, maskT, idx, gl, nsel, v0, v1, vals, st);
+        // kept (row, slot) entries of query tiles 1 .. nT - 1 (tile 0 has none)
+        const size_t smem = (size_t)kBS * s.K * 8 + (size_t)kBS * st.rvs * 4 + (size_t)s.nT * 4 + (size_t)kBS * s.K * 2;
+        if (smem > 40 * 1024) {   // beside the static scan array
+            e = cudaFuncSetAttribute(sel_stream_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
         }
+        KernelTimer kt("sel_stream_fill", stream);
+        sel_stream_tile_kernel<<<(unsigned)((int64_t)s.B * s.Hkv * s.nT), kThreads, smem, stream>>>(
+            s, maskT, idx, gl, nsel, v0, v1, vals, st);
     }
     e = cudaGetLastError();
     if (e == cudaSuccess) count_launches(1);
