@@ -257,6 +257,18 @@ def test_big_key_blocks_dk_dv(big_run):
         assert U.normwise(got_dv, ref_dv) <= TOL_BF16_GRAD, (b, g, j)
 
 
+def test_score_gradient_rows_of_640_columns():
+    """Rows of 513-1024 block columns take the 16-byte score-gradient kernel
+    with eight 128-column pieces (the layers above use four): the tiny recipe
+    at T 20480, block 32 (640 columns), sampled rows' ds elementwise."""
+    w = synth.workload("tiny", seq=20480)
+    x, out = U.run_train(w)
+    ts = np.array(sorted({t for _, _, t in U.sample_rows(w, 60, seed=7)}), dtype=np.int64)
+    r = U.parallel_oracle_bwd(U.group_desc(w), U.group_arrays(x, w, 0, 0), ts)
+    np.testing.assert_allclose(out["ds"][0, 0][ts].numpy(), r["ds"], atol=TOL_FP32, rtol=0)
+    np.testing.assert_allclose(out["dq"][0][:, ts].numpy().transpose(1, 0, 2), r["dq"], atol=TOL_FP32, rtol=0)
+
+
 # ------------------------------------------------------------------ decode ---
 
 def decode_check(w, kc, vc, q, s, N, K, groups, dense=False, gate="softmax"):

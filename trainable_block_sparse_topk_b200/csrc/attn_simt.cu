@@ -565,17 +565,19 @@ dscore_kernel(Shape sh, const float* __restrict__ scores, const float* __restric
         chunk(c0, (dense_term && c0 + lane < C) ? sr[c0 + lane] : 0.f);
 }
 
-// The same for rows of NB <= 1024 columns, NB % 4 == 0: lane l owns columns
-// 4l .. 4l + 3 of each 128-column piece (16-byte loads and stores). Every
+// The same for rows of NB <= 128 * kPieces columns, NB % 4 == 0: lane l owns
+// columns 4l .. 4l + 3 of each 128-column piece (16-byte loads and stores;
+// kPieces 4 for rows of up to 512 columns, 8 up to 1024, so that the
+// prefetched pieces hold no more registers than the row needs). Every
 // column first gets its dense term (0 past C); after a warp barrier, which
 // orders the warp's global stores, each kept slot's lane rewrites its column
 // with the dense term plus its own term, computed as the scalar kernel does.
 constexpr int kDsVecCols = 1024;
+template <int kPieces>
 __global__ void __launch_bounds__(256)
 dscore_vec_kernel(Shape sh, const float* __restrict__ scores, const float* __restrict__ slse,
                   const int32_t* __restrict__ idx, const int32_t* __restrict__ nsel,
                   const float* __restrict__ gsum, float* __restrict__ ds, const int* __restrict__ aborted) {
-    constexpr int kPieces = kDsVecCols / 128;
     const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= sh.rows()) return;
@@ -788,8 +790,10 @@ cudaError_t launch_dscore(const Shape& s, const float* scores, const float* slse
     const unsigned grid = (unsigned)((s.rows() + 7) / 8);
     KernelTimer kt("dscore", st);
     const bool vec = s.NB % 4 == 0 && s.NB <= kDsVecCols && ((uintptr_t)scores & 15) == 0 && ((uintptr_t)ds & 15) == 0;
-    if (vec)
-        dscore_vec_kernel<<<grid, 256, 0, st>>>(s, scores, slse, idx, nsel, gsum, ds, aborted);
+    if (vec && s.NB <= 512)
+        dscore_vec_kernel<4><<<grid, 256, 0, st>>>(s, scores, slse, idx, nsel, gsum, ds, aborted);
+    else if (vec)
+        dscore_vec_kernel<8><<<grid, 256, 0, st>>>(s, scores, slse, idx, nsel, gsum, ds, aborted);
     else
         dscore_kernel<<<grid, 256, 0, st>>>(s, scores, slse, idx, nsel, gsum, ds, aborted);
     const cudaError_t e = cudaGetLastError();
