@@ -500,7 +500,7 @@ def run_ours(args, rank, world, local_rank):
 
     # every kernel of the step on its own (three more steps, outside the timed
     # loop, CUDA events around each launch): per-launch mean microseconds
-    side_names = ("block_topk", "sel_stream_index", "sel_stream_fill", "fwd_rows_shift", "fwd_rows",
+    side_names = ("block_topk", "sel_bitmap_T", "sel_stream_index", "sel_stream_fill", "fwd_rows_shift", "fwd_rows",
                   "fwd_rows_finalize", "fwd_rows_fixup", "rowdot", "bwd_tc", "cast_dq", "dscore")
     B.sas_kernel_timing(",".join(side_names))
     for _ in range(3):

@@ -674,15 +674,16 @@ cudaError_t run_topk_cta(const Shape& s, const float* scores, const int32_t* len
 // ------------------------------------------------------------ K1b: bitmap ---
 
 // One CTA per (b, g, tau): OR the tile's selections into a shared row of NB
-// words, then store it column-major so the backward can walk, per key block,
-// the query tiles that kept it.
+// words (as 32-bit halves: rows 0-31 and 32-63 of the tile), then store it
+// column-major so the backward can walk, per key block, the query tiles that
+// kept it.
 __global__ void __launch_bounds__(256)
 sel_bitmap_T_kernel(Shape sh, const int32_t* __restrict__ idx, const int32_t* __restrict__ nsel,
                     uint64_t* __restrict__ maskT) {
-    extern __shared__ unsigned long long s_words[];
+    extern __shared__ unsigned int s_half[];   // [NB][2]
     const int tau = blockIdx.x % sh.nT;
     const int bg = blockIdx.x / sh.nT;
-    for (int j = threadIdx.x; j < sh.NB; j += blockDim.x) s_words[j] = 0ull;
+    for (int i = threadIdx.x; i < 2 * sh.NB; i += blockDim.x) s_half[i] = 0u;
     __syncthreads();
     const int64_t row0 = (int64_t)bg * sh.T + (int64_t)tau * sh.bs;
     for (int e = threadIdx.x; e < sh.bs * sh.K; e += blockDim.x) {
@@ -690,12 +691,13 @@ sel_bitmap_T_kernel(Shape sh, const int32_t* __restrict__ idx, const int32_t* __
         const int64_t row = row0 + r;
         if (slot < nsel[row]) {
             const int j = idx[row * sh.K + slot];
-            if ((unsigned)j < (unsigned)sh.NB) atomicOr(&s_words[j], 1ull << r);
+            if ((unsigned)j < (unsigned)sh.NB) atomicOr(&s_half[2 * j + (r >> 5)], 1u << (r & 31));
         }
     }
     __syncthreads();
     uint64_t* col = maskT + (int64_t)bg * sh.NB * sh.nT;
-    for (int j = threadIdx.x; j < sh.NB; j += blockDim.x) col[(int64_t)j * sh.nT + tau] = s_words[j];
+    for (int j = threadIdx.x; j < sh.NB; j += blockDim.x)
+        col[(int64_t)j * sh.nT + tau] = ((uint64_t)s_half[2 * j + 1] << 32) | s_half[2 * j];
 }
 
 }  // namespace
